@@ -1,0 +1,401 @@
+#!/usr/bin/env python3
+"""Benchmark of the MoE-MXFP4 layer (router -> top-k -> softmax -> SwiGLU experts ->
+weighted combine) on B200, through the C ABI.
+
+Default workload: the gpt-oss-20b-shaped decode layer at T=64 tokens
+(d_model = d_ff = 2880, E = 32, top-4, bf16 activations, MXFP4 experts drawn
+N(0, 0.02) and quantised by the library).  One step = one forward of the whole
+layer over one batch of T tokens.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config dec64] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps,
+each preceded (outside its timed span) by a 256 MB L2 flush and bracketed by
+CUDA events on the forward's stream; barrier + synchronize before and after
+the timed region; the value uses the max over ranks.  Multi-GPU: independent
+replicas (the layer has no exchange step), weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["mxfp4_expert_gemm_router_b200/csrc/expert_gemm.cuh",
+                  "mxfp4_expert_gemm_router_b200/csrc/sm100_ptx.cuh",
+                  "mxfp4_expert_gemm_router_b200/csrc/routing.cuh",
+                  "mxfp4_expert_gemm_router_b200/csrc/quantize.cuh",
+                  "mxfp4_expert_gemm_router_b200/csrc/moe_mxfp4.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- per-kernel algorithmic work
+
+def algorithmic_work(cfg: mi.MoeConfig, T: int, touched: int):
+    """Bytes / flops each stage must move / do at minimum (per launch)."""
+    d, f, E, k = cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k
+    act = 2 if cfg.act_dtype == "bf16" else 4
+    mx_bytes_per_param = 17 / 32
+    gu_w = touched * 2 * d * f * mx_bytes_per_param
+    dn_w = touched * d * f * mx_bytes_per_param
+    rows = T * k
+    return {
+        "router_topk": {"bytes": T * d * act + E * d * act + rows * 8, "flops": 2.0 * T * d * E},
+        "gate_up_swiglu": {"bytes": gu_w + rows * d * 2 + rows * f * 2, "flops": 4.0 * rows * d * f},
+        "down_combine": {"bytes": dn_w + rows * f * 2 + T * d * 4, "flops": 2.0 * rows * d * f},
+        "layer": {"bytes": gu_w + dn_w + 2 * T * d * act + E * d * act, "flops": 6.0 * rows * d * f + 2.0 * T * d * E},
+    }
+
+
+# ---------------------------------------------------------------- clocks sampler
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [s.strip() for s in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def build_layer(cfg: mi.MoeConfig, max_tokens: int):
+    import torch
+    import mxfp4_expert_gemm_router_b200 as mx
+    from mxfp4_expert_gemm_router_b200 import build as mxbuild
+    mxbuild.build()
+    layer = mx.MoeMxfp4(cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k, max_tokens, cfg.act_dtype)
+    for e in range(cfg.n_experts):
+        wg, wu, wd = mi.draw_expert(cfg, e)
+        layer.quantize_expert(e, torch.from_numpy(wg).cuda(), torch.from_numpy(wu).cuda(),
+                              torch.from_numpy(wd).cuda())
+    wr = mi.draw_router(cfg)
+    bias = mi.draw_bias(cfg)
+    if cfg.act_dtype == "bf16":
+        wr_t = torch.from_numpy(mi.bf16_bits(wr).view(np.int16).copy()).cuda().view(torch.bfloat16)
+    else:
+        wr_t = torch.from_numpy(wr).cuda()
+    b_t = None if bias is None else torch.from_numpy(bias).cuda()
+    layer.set_router(wr_t, b_t)
+    torch.cuda.synchronize()
+    return layer, (wr_t, b_t)
+
+
+def act_tensor(cfg, a, device):
+    import torch
+    if cfg.act_dtype == "bf16":
+        return torch.from_numpy(mi.bf16_bits(a).view(np.int16).copy()).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T = cfg.T
+    layer, _ = build_layer(cfg, T)
+    x = act_tensor(cfg, mi.draw_x(cfg), dev)
+    y = torch.empty_like(x)
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, y, None, None, counts, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    layer.set_profiling(True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = []
+    clocks = ClockSampler(local_rank)
+    if rank == 0 and not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n_launch0 = layer.launch_count()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        stage_ms.append(layer.kernel_times())
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = layer.launch_count() - n_launch0
+    clk = clocks.stop() if rank == 0 and not args.no_clocks else None
+    layer.set_profiling(False)
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    # end-to-end through the public host-buffer entry point
+    xh = act_tensor(cfg, mi.draw_x(cfg), "cpu").pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(xh, yh, stream=stream)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e_s[i].record(stream)
+        layer.forward_host(xh, yh, stream=stream)
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t2.item())
+    touched = int((counts.cpu().numpy() > 0).sum())
+    return {"total_ms": total_ms, "e2e_ms": e2e_ms, "stage_ms": stage_ms, "launches": launches,
+            "clocks": clk, "touched": touched, "counts": counts.cpu().numpy().tolist(),
+            "h2d": xh.numel() * xh.element_size(), "d2h": yh.numel() * yh.element_size()}
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+
+def oracle_sample(cfg: mi.MoeConfig, n_tokens: int, nthreads: int):
+    """Oracle layer on the first n_tokens of the workload (router over the same
+    tokens).  Returns (seconds, tokens).  Weight quantisation by the oracle is set-up,
+    not timed."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    x = mi.draw_x(cfg)[:n_tokens]
+    wr = mi.draw_router(cfg)
+    bias = mi.draw_bias(cfg)
+    _, idx, w, _ = oracle.router(x, wr, bias, cfg.top_k)
+    q = oracle.QuantExperts(cfg.d_model, cfg.d_ff, cfg.n_experts)
+    needed = sorted(set(np.unique(idx).tolist()))
+
+    def one(e):
+        q.set_expert(e, *mi.draw_expert(cfg, e))
+
+    with ThreadPoolExecutor(max_workers=nthreads) as ex:
+        list(ex.map(one, needed))
+    t0 = time.perf_counter()
+    _, idx, w, _ = oracle.router(x, wr, bias, cfg.top_k)
+    oracle.moe_forward(x, q, idx, w, nthreads=nthreads)
+    return time.perf_counter() - t0, n_tokens
+
+
+def cpu_sample_size(cfg):
+    return min(cfg.T, 64 if cfg.d_model >= 1024 else cfg.T)
+
+
+def run_reference(args, cfg):
+    nthreads = os.cpu_count() or 1
+    n = cpu_sample_size(cfg)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample(cfg, min(n, 8), nthreads)
+    secs = 0.0
+    toks = 0
+    for _ in range(args.steps):
+        s, t = oracle_sample(cfg, n, nthreads)
+        secs += s
+        toks += t
+    value = toks / secs
+    sample = f"first {n} of {cfg.T} tokens per step (router + experts, double), {args.steps} steps"
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(cfg, args), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+METRIC = "MoE-MXFP4 layer tokens/s at 1 B200; % of HBM or FP4 tensor roofline"
+
+
+def config_dict(cfg, args):
+    return {"workload": f"gpt-oss-style MoE-MXFP4 layer '{cfg.name}': T={cfg.T}, d_model={cfg.d_model}, "
+                        f"d_ff={cfg.d_ff}, E={cfg.n_experts}, top-{cfg.top_k}, {cfg.act_dtype} activations",
+            "T": cfg.T, "d_model": cfg.d_model, "d_ff": cfg.d_ff, "n_experts": cfg.n_experts, "top_k": cfg.top_k,
+            "seed": cfg.seed, "parallelism": f"replicas x{args.gpus}",
+            "l2": "256 MB flush written between timed steps (outside each step's event span)"}
+
+
+def load_traffic_record():
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        return json.load(f)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="dec64", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    cfg = mi.CONFIGS[args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    r = run_ours(args, cfg, rank, world, local_rank)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    tokens = cfg.T * args.steps * world
+    value = tokens / (r["total_ms"] / 1e3)
+    e2e_value = tokens / (r["e2e_ms"] / 1e3)
+    stages = {}
+    for name in r["stage_ms"][0]:
+        vals = [s[name] for s in r["stage_ms"]]
+        stages[name] = sum(vals) / len(vals)
+    work = algorithmic_work(cfg, cfg.T, r["touched"])
+    peaks = measured_peaks()
+    dominant = max(("gate_up_swiglu", "down_combine", "router_topk"), key=lambda n: stages.get(n, 0.0))
+    dur_s = stages[dominant] / 1e3
+    tensor_bound = cfg.T * cfg.top_k / max(1, r["touched"]) >= 512
+    if tensor_bound:
+        achieved = work[dominant]["flops"] / dur_s / 1e12
+        # the expert MMAs use kind::f16 (f16 operands): same dense rate as bf16
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "kernel": dominant}
+    else:
+        achieved = work[dominant]["bytes"] / dur_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s", "kernel": dominant}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = peaks["source"]
+    roof["algorithmic_per_launch"] = work[dominant]["bytes"] if roof["bound"] == "hbm" else work[dominant]["flops"]
+    tr = load_traffic_record()
+    roof["traffic"] = None
+    if tr and tr.get("source_hash") == kernel_source_hash() and tr.get("config") == cfg.name:
+        roof["traffic"] = tr.get("per_launch_bytes", {}).get(dominant)
+    layer_s = r["total_ms"] / 1e3 / args.steps
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16 MMA operands (MXFP4 weights), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) experts quantised to MXFP4)",
+        "config": config_dict(cfg, args),
+        "roofline": roof,
+        "layer_hbm": {"bytes": work["layer"]["bytes"], "GB/s": work["layer"]["bytes"] / layer_s / 1e9,
+                      "frac_of_measured": work["layer"]["bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
+                      "frac_of_8TBs": work["layer"]["bytes"] / layer_s / 8e12},
+        "stage_ms": stages,
+        "experts_touched": r["touched"],
+        "gpu_launches": r["launches"],
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "clocks": r["clocks"],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        nthreads = os.cpu_count() or 1
+        n = cpu_sample_size(cfg)
+        secs, toks = oracle_sample(cfg, n, nthreads)
+        out["cpu_baseline"] = {"value": toks / secs, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                               "sample": f"first {n} of {cfg.T} tokens, router + experts in double, one pass"}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,178 @@
+/*
+ * moe_mxfp4.h -- C ABI of the MoE feed-forward layer with MXFP4 experts on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card"):
+ *   §3.1 Le Routeur: for each token h in R^d_model, scores = W_router . h
+ *        (+ an optional per-expert bias), the top_k experts by score are
+ *        selected, and a softmax over the selected scores gives weights that
+ *        sum to 1;
+ *   §3.2 Les Experts: each expert is a SwiGLU FFN
+ *        (Swish(h . W_gate) (.) (h . W_up)) . W_down, Swish(z) = z sigma(z);
+ *   §2.1: the layer output is the weighted sum of the top_k expert outputs;
+ *   §4 Quantification MXFP4: the expert weights are stored at 4.25 bits per
+ *        parameter -- FP4 E2M1 codes in blocks of 32 along the contraction
+ *        axis, each block sharing one E8M0 power-of-two scale.
+ *
+ * Conventions for every call:
+ *  - Pointers marked "device" are caller-owned CUDA device memory on the
+ *    device that was current when the handle was created; "host" pointers are
+ *    caller-owned host memory.  The library never frees caller memory.
+ *  - Calls are asynchronous on the given stream unless stated otherwise.  The
+ *    returned status reports host-detectable errors and CUDA launch errors;
+ *    device-side failures (a pipeline wait that timed out) are reported by
+ *    moe_mxfp4_get_status.
+ *  - A handle may be used by one host thread at a time.  Calls on one handle
+ *    that overlap on the GPU (different streams, no ordering) race on the
+ *    handle's internal workspace.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_mxfp4 moe_mxfp4_t; /* opaque: owns quantised weights and workspace */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, bad enum */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but outside the supported envelope  */
+    MOE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
+    MOE_ERR_NOT_QUANTIZED = 4, /* forward before quantize_weights            */
+    MOE_ERR_TIMEOUT = 5        /* a device-side pipeline wait ran out        */
+} moe_status_t;
+
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
+
+/* Test-only flag: the expert-GEMM producer skips its first copy, so a
+ * consumer wait runs out after config.wait_timeout_ms and the forward reports
+ * MOE_ERR_TIMEOUT through moe_mxfp4_get_status. */
+#define MOE_FLAG_TEST_SKIP_FIRST_COPY (1u << 30)
+
+typedef struct {
+    int32_t d_model;        /* model width; multiple of 32                    */
+    int32_t d_ff;           /* expert hidden width; multiple of 32            */
+    int32_t n_experts;      /* E, 1..256                                       */
+    int32_t top_k;          /* k, 1..min(8, E)                                 */
+    int32_t max_tokens;     /* largest T passed to forward, >= 1               */
+    int32_t act_dtype;      /* moe_dtype_t of x, y and the router weight      */
+    uint32_t flags;         /* 0, or MOE_FLAG_* test flags                     */
+    int32_t wait_timeout_ms;/* device pipeline wait limit; <= 0 selects 2000   */
+} moe_mxfp4_config_t;
+
+/* Create a handle on the current device.  Allocates every buffer the layer
+ * needs for up to cfg->max_tokens tokens, so forward allocates nothing.
+ * Errors: INVALID_ARG (null, non-positive sizes, bad dtype), UNSUPPORTED
+ * (d_model or d_ff not a multiple of 32, E > 256, k > min(8, E),
+ * d_model or d_ff above 16384), CUDA (allocation failed; nothing leaks). */
+moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out);
+
+/* Destroy a handle and free everything it owns.  NULL-safe.  Synchronises
+ * the device work the handle issued. */
+void moe_mxfp4_destroy(moe_mxfp4_t* h);
+
+/* Quantise all expert weights to MXFP4 and store the router.
+ *   w_gate, w_up: device fp32 [E][d_model][d_ff]   (expert e maps x -> x . W)
+ *   w_down:       device fp32 [E][d_ff][d_model]
+ *   w_router:     device [E][d_model] in act_dtype (scores = W_router . h)
+ *   router_bias:  device fp32 [E], or NULL for no bias
+ * Blocks of 32 run along the contraction axis (d_model for gate/up, d_ff for
+ * down).  Block rule: scale exponent floor(log2(max|w|)) - 2 clamped to
+ * [-127, 127]; elements round to the nearest E2M1 value, ties to the even
+ * code, above 6 saturating, sign kept; an all-zero block gets scale 2^0.
+ * Inputs must be finite.  May be called again to replace the weights. */
+moe_status_t moe_mxfp4_quantize_weights(moe_mxfp4_t* h, const float* w_gate,
+                                        const float* w_up, const float* w_down,
+                                        const void* w_router, const float* router_bias,
+                                        cudaStream_t stream);
+
+/* Same quantisation for one expert e (lets callers stream very large expert
+ * sets through a small fp32 staging buffer).  w_gate/w_up: device fp32
+ * [d_model][d_ff]; w_down: device fp32 [d_ff][d_model]. */
+moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w_gate,
+                                       const float* w_up, const float* w_down,
+                                       cudaStream_t stream);
+
+/* Store the router weight (device [E][d_model], act_dtype) and optional bias
+ * (device fp32 [E] or NULL).  Copies; the caller may free its buffers after
+ * the stream reaches this call. */
+moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router,
+                                  const float* router_bias, cudaStream_t stream);
+
+/* The layer for T tokens (0 <= T <= max_tokens; T == 0 launches nothing).
+ *   x:             device [T][d_model], act_dtype
+ *   y:             device [T][d_model], act_dtype (written, not accumulated)
+ *   topk_idx:      device int32 [T][k] or NULL -- selected experts, score-descending,
+ *                  ties to the lower index
+ *   topk_w:        device fp32 [T][k] or NULL -- softmax over the selected scores
+ *   expert_counts: device int32 [E] or NULL -- rows routed to each expert
+ * x and y must not overlap.  Expert matmuls run on f16 operands with fp32
+ * accumulation: x converts exactly from bf16 (saturating at +-65504), the
+ * SwiGLU output is rounded to f16.  Asynchronous; allocates nothing. */
+moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y,
+                               int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                               cudaStream_t stream);
+
+/* forward with HOST buffers: copies x (host [T][d_model], act_dtype) in,
+ * runs the layer, copies y (host [T][d_model]) and, if non-NULL, topk_idx
+ * (host int32 [T][k]) and topk_w (host fp32 [T][k]) out, and synchronises
+ * the stream before returning.  Uses handle-owned device staging buffers. */
+moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T,
+                                    void* y_host, int32_t* topk_idx_host,
+                                    float* topk_w_host, cudaStream_t stream);
+
+/* Export the quantised weights of one matrix in the canonical MXFP4 layout:
+ * which = 0 gate, 1 up, 2 down.  For contraction length K and N outputs
+ * (gate/up: K = d_model, N = d_ff; down: K = d_ff, N = d_model):
+ *   codes:  device uint8 [E][N][K/2]   element k of row n in byte k/2,
+ *                                      even k in the low nibble
+ *   scales: device uint8 [E][N][K/32]  E8M0 (value 2^(s-127))  */
+moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* h, int32_t which, uint8_t* codes,
+                                      uint8_t* scales, cudaStream_t stream);
+
+/* Grouping produced by the last forward (for inspection and tests):
+ *   offsets:    device int32 [E+1]  rows of expert e are [offsets[e], offsets[e+1])
+ *   row_token:  device int32 [T*k]  token of each grouped row (or NULL)
+ *   row_weight: device fp32  [T*k]  routing weight of each grouped row (or NULL)
+ * Rows of one expert appear in (token, slot) order. */
+moe_status_t moe_mxfp4_get_grouping(const moe_mxfp4_t* h, int32_t* offsets, int32_t* row_token,
+                                    float* row_weight, cudaStream_t stream);
+
+/* Synchronise the handle's last stream and return (and clear) the device
+ * status: MOE_OK, or MOE_ERR_TIMEOUT if a pipeline wait ran out. */
+moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h);
+
+/* Static description of a status code. */
+const char* moe_mxfp4_status_string(moe_status_t s);
+
+/* Per-stage timing of later forwards (CUDA events on the forward's stream).
+ * enable = 0 turns it off. */
+moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
+
+/* Stage names in the order moe_mxfp4_kernel_times reports them. */
+#define MOE_NUM_STAGES 7
+/* 0 router+top-k, 1 grouping schedule, 2 permute/gather, 3 gate/up+SwiGLU,
+ * 4 split-K SwiGLU finish, 5 down+combine, 6 output cast.  Synchronises;
+ * writes the last profiled forward's durations in ms (0 for stages that did
+ * not run) into ms[0..min(n, MOE_NUM_STAGES)). */
+moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n);
+const char* moe_mxfp4_stage_name(int32_t stage);
+
+/* Number of kernels this handle has launched since creation. */
+uint64_t moe_mxfp4_launch_count(const moe_mxfp4_t* h);
+
+/* Parameters of one expert: 3 * d_model * d_ff (three matrices, §3.2). */
+int64_t moe_mxfp4_expert_param_count(const moe_mxfp4_config_t* cfg);
+
+/* MXFP4 bytes of one expert: codes + scales = 17/32 byte per parameter. */
+int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,355 @@
+// expert_gemm.cuh -- grouped expert GEMMs on tcgen05 tensor cores.
+//
+// Method (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card", §3.2 Les
+// Experts): each expert is (Swish(x . W_gate) (.) (x . W_up)) . W_down with
+// Swish(z) = z sigma(z); §2.1: the k expert outputs of a token are summed with
+// the router weights.
+//
+// Orientation: the MMA computes D[feature, token] = W[feature, :] . X[token, :]^T
+// with M = 128 weight rows (output features) and N = BN grouped token rows, so
+// the weight tile is the A operand.  A lives in tensor memory: decoder warps
+// read the MXFP4 tile that a bulk copy brought into shared memory, turn each
+// byte into two f16 values in registers, scale them by the block's power of two
+// relative to the row scale, and store them to TMEM with tcgen05.st.  B, the
+// grouped f16 activations, arrives by 2-D TMA with 128-byte swizzle.  fp32
+// accumulators stay in TMEM; the epilogue warps read them back with tcgen05.ld.
+//
+//   MODE 0 (gate/up): two accumulators (gate, up) for the same 128 features;
+//     epilogue: H[row, f] = Swish(g * 2^sg) * (u * 2^su), stored as f16; with a
+//     K split, fp32 partials are added into GU instead.
+//   MODE 1 (down):   one accumulator; epilogue: y[token, f] += w_row *
+//     (d * 2^sd), red.add into the fp32 output accumulator (the weighted
+//     scatter-combine).
+//
+// Persistent kernel: one CTA per SM, units (expert, token tile, feature tile,
+// K split) taken round-robin from a device-built list.  Warp roles:
+//   warp 0      TMA producer (one thread)
+//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warps 2..9  decoders, then epilogue; warp w serves TMEM lanes 32*(w%4).. and
+//               MXFP4 block (w-2)/4 of each 64-wide chunk
+// Every mbarrier wait is bounded; on a timeout the CTA raises an abort flag,
+// all roles leave their loops, in-flight copies and MMAs are drained, TMEM is
+// freed and the status word reports the timeout.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "routing.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_MAX_STAGES = 16;
+constexpr int GEMM_A_SLOTS = 4;
+constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+
+struct GemmParams {
+    const uint8_t* wpack;     // tiled MXFP4 weights (quantize.cuh layout)
+    const uint8_t* rowscale;  // MODE 0: [E][2][N] (gate, up); MODE 1: [E][N]
+    const int4* units;        // {expert, first grouped row, valid rows, feature tile | split << 16}
+    const int32_t* sched;
+    int N;                    // output features
+    int K;                    // contraction length
+    int KC;                   // 64-wide chunks
+    int BN;                   // token rows per tile (MMA N), multiple of 16, <= 128
+    int stages;
+    uint32_t idesc;
+    __half* H;                // MODE 0 output [rows][N]
+    float* GU;                // MODE 0 split partials [rows][2N]
+    float* yacc;              // MODE 1 output accumulator [T][N]
+    const int32_t* row_token; // MODE 1
+    const float* row_weight;  // MODE 1
+    int* status;
+    uint64_t timeout_ns;
+    uint32_t skip_first_copy; // test hook: producer skips its first copy
+};
+
+template <int MODE>
+struct GemmShape {
+    static constexpr int CH = MODE == 0 ? 68 : 34;          // bytes per weight row per chunk
+    static constexpr int W_STAGE = CH * 128;                // weight bytes per stage (max)
+    static constexpr int A_COLS = MODE == 0 ? 64 : 32;      // TMEM columns per A slot
+    static constexpr int D_COL0 = GEMM_A_SLOTS * A_COLS;    // first accumulator column
+};
+
+__host__ inline size_t gemm_stage_bytes(int mode, int BN) {
+    return static_cast<size_t>(mode == 0 ? 68 * 128 : 34 * 128) + static_cast<size_t>(BN) * 128;
+}
+__host__ inline size_t gemm_smem_bytes(int mode, int BN, int stages) {
+    size_t b = 1024 + stages * gemm_stage_bytes(mode, BN) + (2 * stages + 2 * GEMM_A_SLOTS + 3) * 8 + 64;
+    return b < static_cast<size_t>(GEMM_MIN_SMEM) ? static_cast<size_t>(GEMM_MIN_SMEM) : b;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+    using Sh = GemmShape<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int S = p.stages;
+    const uint32_t b_bytes = static_cast<uint32_t>(p.BN) * 128u;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t b_sm = base;                                   // S x B tiles (1024-aligned)
+    const uint32_t w_sm = b_sm + S * b_bytes;                     // S x weight chunks
+    const uint32_t bar0 = w_sm + S * Sh::W_STAGE;                 // barriers (8-byte aligned)
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto afull_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
+    auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * S + GEMM_A_SLOTS + a); };
+    const uint32_t accf_bar = bar0 + 8u * (2 * S + 2 * GEMM_A_SLOTS);
+    const uint32_t acce_bar = accf_bar + 8u;
+    const uint32_t drain_bar = acce_bar + 8u;
+    uint8_t* ctl = smem_raw + (drain_bar + 8u - raw);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 8 + 1);  // 8 decoder warps + 1 MMA commit
+        }
+        for (int a = 0; a < GEMM_A_SLOTS; ++a) {
+            mbar_init(afull_bar(a), 8);
+            mbar_init(aempty_bar(a), 1);
+        }
+        mbar_init(accf_bar, 1);
+        mbar_init(acce_bar, 8);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), GEMM_TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_b);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int num_units = p.sched[MODE == 0 ? SCHED_UNITS_GU : SCHED_UNITS_DN];
+    const int nsplit = p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN];
+    const size_t expert_bytes = static_cast<size_t>(p.N) * p.KC * Sh::CH;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int pend_ph[GEMM_MAX_STAGES];
+            for (int i = 0; i < GEMM_MAX_STAGES; ++i) pend_ph[i] = -1;
+            bool skip = p.skip_first_copy != 0;
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                const int4 U = p.units[u];
+                const int ft = U.w & 0xFFFF, sp = U.w >> 16;
+                const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+                const int rf = min(128, p.N - ft * 128);
+                const uint32_t wb = static_cast<uint32_t>(Sh::CH * rf);
+                const uint8_t* wt = p.wpack + static_cast<size_t>(U.x) * expert_bytes +
+                                    static_cast<size_t>(ft) * 128 * p.KC * Sh::CH;
+                for (int c = c0; c < c1; ++c) {
+                    if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto producer_done;
+                    if (skip) {
+                        skip = false;  // test hook: this stage is never filled
+                    } else {
+                        mbar_arrive_expect_tx(full_bar(s), wb + b_bytes);
+                        bulk_g2s(w_sm + s * Sh::W_STAGE, wt + static_cast<size_t>(c) * wb, wb, full_bar(s));
+                        tma_load_2d(b_sm + s * b_bytes, &tmap_b, c * 64, U.y, full_bar(s));
+                        pend_ph[s] = static_cast<int>(ph);
+                    }
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                }
+            }
+        producer_done:
+            // copies still in flight must land before the CTA exits
+            for (int i = 0; i < S; ++i)
+                if (pend_ph[i] >= 0) mbar_wait_drain(full_bar(i), static_cast<uint32_t>(pend_ph[i]), 200000000ull);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int s = 0, a = 0;
+            uint32_t ph = 0, aph = 0, acc_ph = 0;
+            const uint64_t bdesc0 = sw128_kmajor_desc(b_sm);
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                const int4 U = p.units[u];
+                const int sp = U.w >> 16;
+                const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+                if (!mbar_wait_bounded(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto mma_done;
+                tc_fence_after();
+                for (int c = c0; c < c1; ++c) {
+                    if (!mbar_wait_bounded(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
+                    if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
+                    tc_fence_after();
+                    const uint64_t bd = bdesc0 + ((static_cast<uint64_t>(s) * b_bytes) >> 4);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
+                        const uint32_t acol = tmem + a * Sh::A_COLS + 8 * i;
+                        if (MODE == 0) {
+                            mma_f16_ts(tmem + Sh::D_COL0, acol, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts(tmem + Sh::D_COL0 + p.BN, acol + 32, bd + 2 * i, p.idesc, acc);
+                        } else {
+                            mma_f16_ts(tmem + Sh::D_COL0, acol, bd + 2 * i, p.idesc, acc);
+                        }
+                    }
+                    tc_commit(aempty_bar(a));
+                    tc_commit(empty_bar(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    if (++a == GEMM_A_SLOTS) { a = 0; aph ^= 1u; }
+                }
+                tc_commit(accf_bar);
+                acc_ph ^= 1u;
+            }
+        mma_done:
+            tc_commit(drain_bar);
+            mbar_wait_drain(drain_bar, 0, 200000000ull);
+        }
+    } else {
+        // ---------------------------------------------------------- decoders + epilogue
+        const int q = warp & 3;               // TMEM lane quadrant
+        const int hb = (warp - 2) >> 2;       // which 32-block of each chunk
+        const int row = 32 * q + lane;        // weight row within the feature tile
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        int s = 0, a = 0;
+        uint32_t ph = 0, aph = 0, acc_ph = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int e = U.x, row0 = U.y, nvalid = U.z;
+            const int ft = U.w & 0xFFFF, sp = U.w >> 16;
+            const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+            const int rf = min(128, p.N - ft * 128);
+            const bool warp_rows = 32 * q < rf;
+            const int n = ft * 128 + row;
+            int rs0 = 127, rs1 = 127;
+            if (warp_rows) {
+                if (MODE == 0) {
+                    rs0 = p.rowscale[(static_cast<size_t>(e) * 2 + 0) * p.N + n];
+                    rs1 = p.rowscale[(static_cast<size_t>(e) * 2 + 1) * p.N + n];
+                } else {
+                    rs0 = p.rowscale[static_cast<size_t>(e) * p.N + n];
+                }
+            }
+            for (int c = c0; c < c1; ++c) {
+                bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                uint4 cg = make_uint4(0, 0, 0, 0), cu = make_uint4(0, 0, 0, 0);
+                int sg = 127, su = 127;
+                if (warp_rows) {
+                    const uint8_t* ws = smem_raw + (w_sm + s * Sh::W_STAGE - raw);
+                    cg = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
+                    sg = ws[32 * rf + hb * rf + row];
+                    if (MODE == 0) {
+                        cu = *reinterpret_cast<const uint4*>(ws + 34 * rf + (hb * rf + row) * 16);
+                        su = ws[66 * rf + hb * rf + row];
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
+
+                w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                tc_fence_after();
+                if (warp_rows) {
+                    uint32_t r[16];
+                    const uint32_t mg = f16_pow2_bits(sg - rs0);
+                    const uint32_t mg2 = mg | (mg << 16);
+                    e2m1x8_to_f16x8(cg.x, mg2, r[0], r[1], r[2], r[3]);
+                    e2m1x8_to_f16x8(cg.y, mg2, r[4], r[5], r[6], r[7]);
+                    e2m1x8_to_f16x8(cg.z, mg2, r[8], r[9], r[10], r[11]);
+                    e2m1x8_to_f16x8(cg.w, mg2, r[12], r[13], r[14], r[15]);
+                    tmem_st16(tmem + lane_addr + a * Sh::A_COLS + 16 * hb, r);
+                    if (MODE == 0) {
+                        const uint32_t mu = f16_pow2_bits(su - rs1);
+                        const uint32_t mu2 = mu | (mu << 16);
+                        e2m1x8_to_f16x8(cu.x, mu2, r[0], r[1], r[2], r[3]);
+                        e2m1x8_to_f16x8(cu.y, mu2, r[4], r[5], r[6], r[7]);
+                        e2m1x8_to_f16x8(cu.z, mu2, r[8], r[9], r[10], r[11]);
+                        e2m1x8_to_f16x8(cu.w, mu2, r[12], r[13], r[14], r[15]);
+                        tmem_st16(tmem + lane_addr + a * Sh::A_COLS + 32 + 16 * hb, r);
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(afull_bar(a));
+                if (++a == GEMM_A_SLOTS) { a = 0; aph ^= 1u; }
+            }
+            if (!ok) break;
+
+            // ------------------------------------------------------ epilogue
+            {
+                const bool w_ok = mbar_wait_bounded(accf_bar, acc_ph, abort_flag, p.status, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+            }
+            acc_ph ^= 1u;
+            tc_fence_after();
+            if (warp_rows) {
+                const int half = p.BN / 2;
+                const int n0 = hb * half;
+                const float f0 = pow2f(rs0 - 127);
+                const float f1 = pow2f(rs1 - 127);
+                for (int j0 = 0; j0 < half; j0 += 8) {
+                    const int col = n0 + j0;
+                    uint32_t g[8];
+                    tmem_ld8(tmem + lane_addr + Sh::D_COL0 + col, g);
+                    if (MODE == 0) {
+                        uint32_t v[8];
+                        tmem_ld8(tmem + lane_addr + Sh::D_COL0 + p.BN + col, v);
+                        tmem_wait_ld();
+                        if (nsplit == 1) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                if (col + j < nvalid) {
+                                    const float gg = __uint_as_float(g[j]) * f0;
+                                    const float uu = __uint_as_float(v[j]) * f1;
+                                    p.H[static_cast<size_t>(row0 + col + j) * p.N + n] = to_half_sat(swish_f(gg) * uu);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                if (col + j < nvalid) {
+                                    float* gu = p.GU + static_cast<size_t>(row0 + col + j) * 2 * p.N;
+                                    atomicAdd(gu + n, __uint_as_float(g[j]) * f0);
+                                    atomicAdd(gu + p.N + n, __uint_as_float(v[j]) * f1);
+                                }
+                            }
+                        }
+                    } else {
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (col + j < nvalid) {
+                                const int rr = row0 + col + j;
+                                const int t = p.row_token[rr];
+                                const float wv = p.row_weight[rr];
+                                atomicAdd(p.yacc + static_cast<size_t>(t) * p.N + n, __uint_as_float(g[j]) * f0 * wv);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, GEMM_TMEM_COLS);
+    }
+}
+
+}  // namespace moe

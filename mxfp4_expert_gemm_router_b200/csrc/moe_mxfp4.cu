@@ -1,0 +1,600 @@
+// moe_mxfp4.cu -- C ABI of the MoE feed-forward layer with MXFP4 experts
+// (declarations and argument contracts in include/moe_mxfp4.h).
+//
+// One forward = up to seven launches on the caller's stream, no host sync and
+// no allocation:
+//   router_kernel        scores, top-k, softmax over the selected scores,
+//                        per-block expert histogram, zeroing of the output rows
+//   schedule_kernel      expert offsets, per-block prefixes, K splits, unit lists
+//   permute_kernel       grouped rows (token, weight) and f16 activation gather
+//   expert_gemm<0>       gate/up GEMM, SwiGLU epilogue
+//   swiglu_finish_kernel only when the gate/up GEMM split K
+//   expert_gemm<1>       down GEMM, routing-weighted scatter-combine epilogue
+//   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/moe_mxfp4.h"
+#include "expert_gemm.cuh"
+#include "quantize.cuh"
+#include "routing.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int BN_OPTIONS = 8;  // BN = 16 * (i + 1)
+constexpr int SPLIT_ROWS_CAP = 2048;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+struct moe_mxfp4 {
+    moe_mxfp4_config_t cfg;
+    int dev = 0, nsm = 0;
+    int act_bytes = 2;
+    int KC_gu = 0, KC_dn = 0, F_gu = 0, F_dn = 0;
+    int TK = 0, nblk_max = 0, max_units = 0, gu_rows = 0;
+    // weights
+    uint8_t* w_gu = nullptr;   // tiled gate+up
+    uint8_t* w_dn = nullptr;   // tiled down
+    uint8_t* rs_gu = nullptr;  // [E][2][d_ff]
+    uint8_t* rs_dn = nullptr;  // [E][d_model]
+    void* w_router = nullptr;
+    float* bias = nullptr;
+    bool has_bias = false, router_set = false;
+    int experts_quantized = 0;
+    bool* expert_done = nullptr;
+    // workspace
+    int32_t* idx_ws = nullptr;
+    float* w_ws = nullptr;
+    int32_t* hist = nullptr;
+    int32_t* offsets = nullptr;
+    int32_t* sched = nullptr;
+    int4* units_gu = nullptr;
+    int4* units_dn = nullptr;
+    int32_t* row_token = nullptr;
+    float* row_weight = nullptr;
+    __half* Xp = nullptr;
+    __half* H = nullptr;
+    float* GU = nullptr;
+    float* yacc = nullptr;
+    int* status = nullptr;
+    void* x_stage = nullptr;
+    void* y_stage = nullptr;
+    int32_t* idx_stage = nullptr;
+    float* w_stage = nullptr;
+    // tensor maps per BN
+    CUtensorMap tm_x[BN_OPTIONS];
+    CUtensorMap tm_h[BN_OPTIONS];
+    bool tm_ok[BN_OPTIONS] = {};
+    cudaStream_t last_stream = nullptr;
+    // profiling
+    bool prof = false, prof_valid = false;
+    cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
+    bool stage_ran[MOE_NUM_STAGES] = {};
+    uint64_t launches = 0;
+};
+
+static bool g_attrs_set = false;
+
+static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                                   \
+    do {                                                \
+        cudaError_t _e = (expr);                        \
+        if (_e != cudaSuccess) return MOE_ERR_CUDA;     \
+    } while (0)
+
+static void free_all(moe_mxfp4* h) {
+    void* ptrs[] = {h->w_gu, h->w_dn, h->rs_gu, h->rs_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
+                    h->offsets, h->sched, h->units_gu, h->units_dn, h->row_token, h->row_weight, h->Xp, h->H,
+                    h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
+    for (void* p : ptrs)
+        if (p) cudaFree(p);
+    for (auto& e : h->ev)
+        if (e) cudaEventDestroy(e);
+    delete[] h->expert_done;
+}
+
+static int choose_bn(int T, int k, int E) {
+    long per_expert = (static_cast<long>(T) * k + E - 1) / E;
+    long want = std::min<long>(T, std::max<long>(1, 4 * per_expert));
+    int bn = static_cast<int>((want + 15) / 16) * 16;
+    return std::max(16, std::min(128, bn));
+}
+
+static int stages_for(int mode, int BN) {
+    const size_t budget = 227 * 1024 - 1024 - 512;
+    int s = static_cast<int>(budget / gemm_stage_bytes(mode, BN));
+    return std::max(2, std::min(GEMM_MAX_STAGES, s));
+}
+
+extern "C" {
+
+const char* moe_mxfp4_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_NOT_QUANTIZED: return "weights or router not set";
+        case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* moe_mxfp4_stage_name(int32_t stage) {
+    static const char* names[MOE_NUM_STAGES] = {"router_topk", "schedule", "permute_gather", "gate_up_swiglu",
+                                                 "swiglu_finish", "down_combine", "cast_out"};
+    return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "unknown";
+}
+
+int64_t moe_mxfp4_expert_param_count(const moe_mxfp4_config_t* cfg) {
+    if (!cfg) return -1;
+    return 3LL * cfg->d_model * cfg->d_ff;
+}
+
+int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg) {
+    if (!cfg) return -1;
+    return moe_mxfp4_expert_param_count(cfg) * 17 / 32;
+}
+
+uint64_t moe_mxfp4_launch_count(const moe_mxfp4_t* h) { return h ? h->launches : 0; }
+
+moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) {
+    if (!cfg || !out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    const moe_mxfp4_config_t c = *cfg;
+    if (c.d_model <= 0 || c.d_ff <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.max_tokens <= 0)
+        return MOE_ERR_INVALID_ARG;
+    if (c.act_dtype != MOE_DTYPE_F32 && c.act_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c.d_model % 32 || c.d_ff % 32 || c.n_experts > MAX_EXPERTS || c.top_k > std::min(MAX_TOPK, c.n_experts) ||
+        c.d_model > 16384 || c.d_ff > 16384 || static_cast<long>(c.max_tokens) * c.top_k > (1L << 26))
+        return MOE_ERR_UNSUPPORTED;
+    if (!get_encode_fn()) return MOE_ERR_CUDA;
+
+    moe_mxfp4* h = new (std::nothrow) moe_mxfp4();
+    if (!h) return MOE_ERR_CUDA;
+    h->cfg = c;
+    h->act_bytes = c.act_dtype == MOE_DTYPE_BF16 ? 2 : 4;
+    auto fail = [&](moe_status_t s) {
+        free_all(h);
+        delete h;
+        return s;
+    };
+    if (cudaGetDevice(&h->dev) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    if (cudaDeviceGetAttribute(&h->nsm, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
+    h->KC_gu = (d + 63) / 64;
+    h->KC_dn = (f + 63) / 64;
+    h->F_gu = (f + 127) / 128;
+    h->F_dn = (d + 127) / 128;
+    h->TK = c.max_tokens * k;
+    h->nblk_max = (c.max_tokens + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+    {
+        const long tiles_big = static_cast<long>(h->TK) / 128 + E + 2;
+        const long tiles_small = 512 / 16 + E + 2;
+        const long F = std::max(h->F_gu, h->F_dn);
+        h->max_units = static_cast<int>(std::max(tiles_big, tiles_small) * F + 8L * h->nsm + 64);
+    }
+    h->gu_rows = std::min(h->TK, SPLIT_ROWS_CAP);
+    h->expert_done = new (std::nothrow) bool[E]();
+    if (!h->expert_done) return fail(MOE_ERR_CUDA);
+
+    const size_t gu_bytes = static_cast<size_t>(E) * f * h->KC_gu * 68;
+    const size_t dn_bytes = static_cast<size_t>(E) * d * h->KC_dn * 34;
+    const size_t TK = h->TK;
+    struct A { void** p; size_t bytes; };
+    A allocs[] = {
+        {reinterpret_cast<void**>(&h->w_gu), gu_bytes},
+        {reinterpret_cast<void**>(&h->w_dn), dn_bytes},
+        {reinterpret_cast<void**>(&h->rs_gu), static_cast<size_t>(E) * 2 * f},
+        {reinterpret_cast<void**>(&h->rs_dn), static_cast<size_t>(E) * d},
+        {&h->w_router, static_cast<size_t>(E) * d * h->act_bytes},
+        {reinterpret_cast<void**>(&h->bias), sizeof(float) * E},
+        {reinterpret_cast<void**>(&h->idx_ws), sizeof(int32_t) * TK},
+        {reinterpret_cast<void**>(&h->w_ws), sizeof(float) * TK},
+        {reinterpret_cast<void**>(&h->hist), sizeof(int32_t) * static_cast<size_t>(h->nblk_max) * E},
+        {reinterpret_cast<void**>(&h->offsets), sizeof(int32_t) * (E + 1)},
+        {reinterpret_cast<void**>(&h->sched), sizeof(int32_t) * SCHED_SLOTS},
+        {reinterpret_cast<void**>(&h->units_gu), sizeof(int4) * h->max_units},
+        {reinterpret_cast<void**>(&h->units_dn), sizeof(int4) * h->max_units},
+        {reinterpret_cast<void**>(&h->row_token), sizeof(int32_t) * TK},
+        {reinterpret_cast<void**>(&h->row_weight), sizeof(float) * TK},
+        {reinterpret_cast<void**>(&h->Xp), sizeof(__half) * TK * d},
+        {reinterpret_cast<void**>(&h->H), sizeof(__half) * TK * f},
+        {reinterpret_cast<void**>(&h->GU), sizeof(float) * h->gu_rows * 2 * f},
+        {reinterpret_cast<void**>(&h->yacc), sizeof(float) * static_cast<size_t>(c.max_tokens) * d},
+        {reinterpret_cast<void**>(&h->status), sizeof(int) * 4},
+        {&h->x_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
+        {&h->y_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
+        {reinterpret_cast<void**>(&h->idx_stage), sizeof(int32_t) * TK},
+        {reinterpret_cast<void**>(&h->w_stage), sizeof(float) * TK},
+    };
+    for (auto& a : allocs)
+        if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    // Grouped activation / hidden buffers start as zeros so rows a tile reads past
+    // its expert's segment are finite; the status word starts clear.
+    if (cudaMemset(h->Xp, 0, sizeof(__half) * TK * d) != cudaSuccess ||
+        cudaMemset(h->H, 0, sizeof(__half) * TK * f) != cudaSuccess ||
+        cudaMemset(h->status, 0, sizeof(int) * 4) != cudaSuccess ||
+        cudaMemset(h->bias, 0, sizeof(float) * E) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+
+    if (!g_attrs_set) {
+        if (cudaFuncSetAttribute(expert_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(expert_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess ||
+            cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess)
+            return fail(MOE_ERR_CUDA);
+        g_attrs_set = true;
+    }
+    for (auto& e : h->ev)
+        if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    *out = h;
+    return MOE_OK;
+}
+
+void moe_mxfp4_destroy(moe_mxfp4_t* h) {
+    if (!h) return;
+    cudaDeviceSynchronize();
+    free_all(h);
+    delete h;
+}
+
+static TiledMatrix tiled(moe_mxfp4* h, int which) {
+    const auto& c = h->cfg;
+    TiledMatrix M;
+    if (which < 2) {
+        M.base = h->w_gu;
+        M.N = c.d_ff;
+        M.K = c.d_model;
+        M.KC = h->KC_gu;
+        M.CH = 68;
+        M.sub = which;
+    } else {
+        M.base = h->w_dn;
+        M.N = c.d_model;
+        M.K = c.d_ff;
+        M.KC = h->KC_dn;
+        M.CH = 34;
+        M.sub = 0;
+    }
+    return M;
+}
+
+// Quantise experts [e0, e0+ne) of one matrix from fp32 [ne][K][N].
+static moe_status_t quantize_matrix(moe_mxfp4* h, int which, const float* W, int e0, int ne, cudaStream_t s) {
+    TiledMatrix M = tiled(h, which);
+    M.base += static_cast<size_t>(e0) * M.expert_bytes();
+    const dim3 blk(128);
+    const dim3 grid((M.N + 127) / 128, 2 * M.KC, ne);
+    quantize_kernel<<<grid, blk, 0, s>>>(W, static_cast<size_t>(M.K) * M.N, M);
+    h->launches++;
+    uint8_t* rs;
+    size_t rs_stride;
+    if (which < 2) {
+        rs = h->rs_gu + (static_cast<size_t>(e0) * 2 + which) * M.N;
+        rs_stride = 2 * static_cast<size_t>(M.N);
+    } else {
+        rs = h->rs_dn + static_cast<size_t>(e0) * M.N;
+        rs_stride = M.N;
+    }
+    rowscale_kernel<<<dim3((M.N + 127) / 128, 1, ne), blk, 0, s>>>(M, rs, rs_stride);
+    h->launches++;
+    return cuda_status(cudaGetLastError());
+}
+
+moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router, const float* router_bias,
+                                  cudaStream_t stream) {
+    if (!h || !w_router) return MOE_ERR_INVALID_ARG;
+    const auto& c = h->cfg;
+    MOE_TRY(cudaMemcpyAsync(h->w_router, w_router, static_cast<size_t>(c.n_experts) * c.d_model * h->act_bytes,
+                            cudaMemcpyDeviceToDevice, stream));
+    if (router_bias) {
+        MOE_TRY(cudaMemcpyAsync(h->bias, router_bias, sizeof(float) * c.n_experts, cudaMemcpyDeviceToDevice, stream));
+    } else {
+        MOE_TRY(cudaMemsetAsync(h->bias, 0, sizeof(float) * c.n_experts, stream));
+    }
+    h->has_bias = router_bias != nullptr;
+    h->router_set = true;
+    h->last_stream = stream;
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w_gate, const float* w_up,
+                                       const float* w_down, cudaStream_t stream) {
+    if (!h || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
+    if (e < 0 || e >= h->cfg.n_experts) return MOE_ERR_INVALID_ARG;
+    moe_status_t st;
+    if ((st = quantize_matrix(h, 0, w_gate, e, 1, stream)) != MOE_OK) return st;
+    if ((st = quantize_matrix(h, 1, w_up, e, 1, stream)) != MOE_OK) return st;
+    if ((st = quantize_matrix(h, 2, w_down, e, 1, stream)) != MOE_OK) return st;
+    if (!h->expert_done[e]) {
+        h->expert_done[e] = true;
+        h->experts_quantized++;
+    }
+    h->last_stream = stream;
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_quantize_weights(moe_mxfp4_t* h, const float* w_gate, const float* w_up,
+                                        const float* w_down, const void* w_router, const float* router_bias,
+                                        cudaStream_t stream) {
+    if (!h || !w_gate || !w_up || !w_down || !w_router) return MOE_ERR_INVALID_ARG;
+    const int E = h->cfg.n_experts;
+    moe_status_t st;
+    if ((st = quantize_matrix(h, 0, w_gate, 0, E, stream)) != MOE_OK) return st;
+    if ((st = quantize_matrix(h, 1, w_up, 0, E, stream)) != MOE_OK) return st;
+    if ((st = quantize_matrix(h, 2, w_down, 0, E, stream)) != MOE_OK) return st;
+    for (int e = 0; e < E; ++e) h->expert_done[e] = true;
+    h->experts_quantized = E;
+    return moe_mxfp4_set_router(h, w_router, router_bias, stream);
+}
+
+moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* hc, int32_t which, uint8_t* codes, uint8_t* scales,
+                                      cudaStream_t stream) {
+    if (!hc || !codes || !scales || which < 0 || which > 2) return MOE_ERR_INVALID_ARG;
+    moe_mxfp4* h = const_cast<moe_mxfp4*>(hc);
+    TiledMatrix M = tiled(h, which);
+    const dim3 grid((M.N + 127) / 128, M.K / 32, h->cfg.n_experts);
+    export_kernel<<<grid, 128, 0, stream>>>(M, codes, scales);
+    h->launches++;
+    return cuda_status(cudaGetLastError());
+}
+
+static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
+    const int i = BN / 16 - 1;
+    if (h->tm_ok[i]) return MOE_OK;
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    const auto& c = h->cfg;
+    for (int which = 0; which < 2; ++which) {
+        const cuuint64_t cols = which == 0 ? c.d_model : c.d_ff;
+        cuuint64_t dims[2] = {cols, static_cast<cuuint64_t>(h->TK)};
+        cuuint64_t strides[1] = {cols * sizeof(__half)};
+        cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         which == 0 ? static_cast<void*>(h->Xp) : static_cast<void*>(h->H), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    }
+    h->tm_ok[i] = true;
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y, int32_t* topk_idx,
+                               float* topk_w, int32_t* expert_counts, cudaStream_t stream) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    const auto& c = h->cfg;
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (T > c.max_tokens) return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+    if (!h->router_set || h->experts_quantized < c.n_experts) return MOE_ERR_NOT_QUANTIZED;
+    h->last_stream = stream;
+    if (T == 0) return MOE_OK;
+    const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
+    const int BN = choose_bn(T, k, E);
+    moe_status_t st = ensure_tmaps(h, BN);
+    if (st != MOE_OK) return st;
+    const int nblk = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+    int32_t* idx = topk_idx ? topk_idx : h->idx_ws;
+    float* wts = topk_w ? topk_w : h->w_ws;
+    const bool bf16 = c.act_dtype == MOE_DTYPE_BF16;
+    float* acc = bf16 ? h->yacc : static_cast<float*>(y);
+    const bool prof = h->prof;
+    for (int i = 0; i < MOE_NUM_STAGES; ++i) h->stage_ran[i] = false;
+    auto mark = [&](int i) {
+        if (prof) cudaEventRecord(h->ev[i], stream);
+    };
+
+    // 0: router + top-k + softmax
+    mark(0);
+    const size_t rsm = router_smem_bytes(E);
+    if (bf16)
+        router_kernel<__nv_bfloat16><<<nblk, ROUTER_THREADS, rsm, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(h->w_router), h->bias, T, d, E,
+            k, idx, wts, h->hist, acc, d);
+    else
+        router_kernel<float><<<nblk, ROUTER_THREADS, rsm, stream>>>(static_cast<const float*>(x),
+                                                                      static_cast<const float*>(h->w_router), h->bias,
+                                                                      T, d, E, k, idx, wts, h->hist, acc, d);
+    h->stage_ran[0] = true;
+    // 1: schedule
+    mark(1);
+    ScheduleArgs sa;
+    sa.hist = h->hist;
+    sa.nblk = nblk;
+    sa.E = E;
+    sa.BN = BN;
+    sa.F_gu = h->F_gu;
+    sa.F_dn = h->F_dn;
+    sa.KC_gu = h->KC_gu;
+    sa.KC_dn = h->KC_dn;
+    sa.nsm = h->nsm;
+    sa.split_rows_cap = h->gu_rows;
+    sa.max_units = h->max_units;
+    sa.offsets = h->offsets;
+    sa.counts_out = expert_counts;
+    sa.units_gu = h->units_gu;
+    sa.units_dn = h->units_dn;
+    sa.sched = h->sched;
+    schedule_kernel<<<1, 1024, 0, stream>>>(sa);
+    h->stage_ran[1] = true;
+    // 2: permute + gather
+    mark(2);
+    if (bf16)
+        permute_kernel<__nv_bfloat16><<<nblk, ROUTER_THREADS, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), idx, wts, h->hist, h->offsets, T, d, E, k, h->row_token,
+            h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+    else
+        permute_kernel<float><<<nblk, ROUTER_THREADS, 0, stream>>>(static_cast<const float*>(x), idx, wts, h->hist,
+                                                                     h->offsets, T, d, E, k, h->row_token,
+                                                                     h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+    h->stage_ran[2] = true;
+    // 3: gate/up GEMM + SwiGLU
+    mark(3);
+    const uint64_t tmo = static_cast<uint64_t>(c.wait_timeout_ms > 0 ? c.wait_timeout_ms : 2000) * 1000000ull;
+    GemmParams gp;
+    gp.wpack = h->w_gu;
+    gp.rowscale = h->rs_gu;
+    gp.units = h->units_gu;
+    gp.sched = h->sched;
+    gp.N = f;
+    gp.K = d;
+    gp.KC = h->KC_gu;
+    gp.BN = BN;
+    gp.stages = stages_for(0, BN);
+    gp.idesc = idesc_f16_f32(128, BN);
+    gp.H = h->H;
+    gp.GU = h->GU;
+    gp.yacc = nullptr;
+    gp.row_token = h->row_token;
+    gp.row_weight = h->row_weight;
+    gp.status = h->status;
+    gp.timeout_ns = tmo;
+    gp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
+    const int grid = h->nsm;
+    expert_gemm_kernel<0><<<grid, GEMM_THREADS, gemm_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
+    h->stage_ran[3] = true;
+    // 4: split-K finish (no-op unless the schedule split K)
+    mark(4);
+    const bool may_split = static_cast<long>(T) * k <= h->gu_rows;
+    if (may_split) {
+        const int blocks = std::min<long>(4L * h->nsm, (static_cast<long>(T) * k * f + 255) / 256);
+        swiglu_finish_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->GU, h->H, f, h->sched);
+        h->stage_ran[4] = true;
+    }
+    // 5: down GEMM + weighted scatter-combine
+    mark(5);
+    GemmParams dp = gp;
+    dp.wpack = h->w_dn;
+    dp.rowscale = h->rs_dn;
+    dp.units = h->units_dn;
+    dp.N = d;
+    dp.K = f;
+    dp.KC = h->KC_dn;
+    dp.stages = stages_for(1, BN);
+    dp.H = nullptr;
+    dp.GU = nullptr;
+    dp.yacc = acc;
+    dp.skip_first_copy = 0;
+    expert_gemm_kernel<1><<<grid, GEMM_THREADS, gemm_smem_bytes(1, BN, dp.stages), stream>>>(h->tm_h[BN / 16 - 1], dp);
+    h->stage_ran[5] = true;
+    // 6: output cast
+    mark(6);
+    if (bf16) {
+        const size_t n4 = static_cast<size_t>(T) * d / 4;
+        const int blocks = static_cast<int>(std::min<size_t>(4 * static_cast<size_t>(h->nsm), (n4 + 255) / 256));
+        cast_out_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->yacc, static_cast<__nv_bfloat16*>(y), n4);
+        h->stage_ran[6] = true;
+    }
+    mark(7);
+    h->prof_valid = prof;
+    for (int i = 0; i < MOE_NUM_STAGES; ++i) h->launches += h->stage_ran[i] ? 1 : 0;
+    return cuda_status(cudaGetLastError());
+}
+
+moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T, void* y_host,
+                                    int32_t* topk_idx_host, float* topk_w_host, cudaStream_t stream) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    const auto& c = h->cfg;
+    if (T < 0) return MOE_ERR_INVALID_ARG;
+    if (T > c.max_tokens) return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    const size_t act = static_cast<size_t>(T) * c.d_model * h->act_bytes;
+    MOE_TRY(cudaMemcpyAsync(h->x_stage, x_host, act, cudaMemcpyHostToDevice, stream));
+    moe_status_t st = moe_mxfp4_forward(h, h->x_stage, T, h->y_stage, h->idx_stage, h->w_stage, nullptr, stream);
+    if (st != MOE_OK) return st;
+    MOE_TRY(cudaMemcpyAsync(y_host, h->y_stage, act, cudaMemcpyDeviceToHost, stream));
+    const size_t tk = static_cast<size_t>(T) * c.top_k;
+    if (topk_idx_host)
+        MOE_TRY(cudaMemcpyAsync(topk_idx_host, h->idx_stage, tk * sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+    if (topk_w_host)
+        MOE_TRY(cudaMemcpyAsync(topk_w_host, h->w_stage, tk * sizeof(float), cudaMemcpyDeviceToHost, stream));
+    MOE_TRY(cudaStreamSynchronize(stream));
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_get_grouping(const moe_mxfp4_t* hc, int32_t* offsets, int32_t* row_token, float* row_weight,
+                                    cudaStream_t stream) {
+    if (!hc || !offsets) return MOE_ERR_INVALID_ARG;
+    moe_mxfp4* h = const_cast<moe_mxfp4*>(hc);
+    const auto& c = h->cfg;
+    MOE_TRY(cudaMemcpyAsync(offsets, h->offsets, sizeof(int32_t) * (c.n_experts + 1), cudaMemcpyDeviceToDevice, stream));
+    // rows in use = offsets[E]; copy the full capacity bound the caller sized for T*k
+    int32_t rows = 0;
+    MOE_TRY(cudaMemcpyAsync(&rows, h->sched + SCHED_ROWS, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+    MOE_TRY(cudaStreamSynchronize(stream));
+    if (row_token && rows > 0)
+        MOE_TRY(cudaMemcpyAsync(row_token, h->row_token, sizeof(int32_t) * rows, cudaMemcpyDeviceToDevice, stream));
+    if (row_weight && rows > 0)
+        MOE_TRY(cudaMemcpyAsync(row_weight, h->row_weight, sizeof(float) * rows, cudaMemcpyDeviceToDevice, stream));
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (h->last_stream) {
+        MOE_TRY(cudaStreamSynchronize(h->last_stream));
+    } else {
+        MOE_TRY(cudaDeviceSynchronize());
+    }
+    int s = 0;
+    MOE_TRY(cudaMemcpy(&s, h->status, sizeof(int), cudaMemcpyDeviceToHost));
+    MOE_TRY(cudaMemset(h->status, 0, sizeof(int)));
+    return s == DEV_OK ? MOE_OK : MOE_ERR_TIMEOUT;
+}
+
+moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    h->prof = enable != 0;
+    h->prof_valid = false;
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n) {
+    if (!h || !ms || n < 0) return MOE_ERR_INVALID_ARG;
+    if (!h->prof_valid) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cudaEventSynchronize(h->ev[MOE_NUM_STAGES]));
+    for (int i = 0; i < std::min<int>(n, MOE_NUM_STAGES); ++i) {
+        float t = 0.f;
+        if (h->stage_ran[i]) MOE_TRY(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]));
+        ms[i] = t;
+    }
+    return MOE_OK;
+}
+
+}  // extern "C"

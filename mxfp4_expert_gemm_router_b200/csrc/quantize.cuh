@@ -1,0 +1,137 @@
+// quantize.cuh -- MXFP4 quantisation of expert weights into the layout the
+// expert GEMMs stream, plus the export back to the canonical layout.
+//
+// Format (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card", §4
+// Quantification MXFP4: 4.25 bits per parameter; the Microscaling format cited
+// there): blocks of 32 weights along the contraction axis share one E8M0
+// scale 2^(s-127); each weight is an E2M1 code (sign, 2 exponent bits, 1
+// mantissa bit).  Block rule: exponent floor(log2(max|w|)) - 2 clamped to
+// [-127, 127]; elements round to the nearest E2M1 magnitude with ties to the
+// even code, magnitudes above 6 saturate, the sign bit is kept; an all-zero
+// block gets scale byte 127.
+//
+// Streamed layout ("tiled"): for a matrix with N output rows and contraction
+// length K, rows are cut into 128-row feature tiles (the last one holds
+// N - 128*floor(N/128) rows) and K into 64-wide chunks (two 32-blocks).  For each
+// (tile, chunk) the bytes are contiguous:
+//     codes  [2 blocks][rf rows][16 B]   (even element in the low nibble)
+//     scales [2 blocks][rf rows]          (E8M0 bytes)
+// i.e. 34 * rf bytes per matrix; gate and up are interleaved per chunk
+// (gate 34*rf bytes, then up 34*rf bytes).  A K that is 32 mod 64 gets one
+// zero block (codes 0, scale 127) at the end of its last chunk.  One further
+// byte per row, the largest scale over the row's non-zero blocks ("row
+// scale", 127 if none), lets the GEMM decode each block as f16 relative to
+// its row and apply 2^(row scale - 127) in fp32 after accumulation.
+#pragma once
+#include <cstdint>
+
+namespace moe {
+
+struct TiledMatrix {
+    uint8_t* base;   // expert 0 of the packed array
+    int N, K, KC;    // rows, contraction length, 64-chunks = ceil(K/64)
+    int CH;          // bytes per row per chunk of the interleaved group: 68 (gate+up) or 34
+    int sub;         // 0 (gate / down) or 1 (up): which 34*rf part of the chunk
+    __host__ __device__ size_t expert_bytes() const { return static_cast<size_t>(N) * KC * CH; }
+    // byte offset (within one expert) of the codes of block b (0..2*KC-1) of row n
+    __host__ __device__ void locate(int n, int b, size_t& code_off, size_t& scale_off) const {
+        const int ft = n >> 7, r = n & 127;
+        const int rf = min(128, N - (ft << 7));
+        const int c = b >> 1, h = b & 1;
+        const size_t chunk = static_cast<size_t>(ft) * 128 * KC * CH + static_cast<size_t>(c) * CH * rf +
+                             static_cast<size_t>(sub) * 34 * rf;
+        code_off = chunk + static_cast<size_t>(h * rf + r) * 16;
+        scale_off = chunk + 32 * static_cast<size_t>(rf) + h * rf + r;
+    }
+};
+
+__device__ __forceinline__ int floor_log2_pos(float a) {
+    const uint32_t u = __float_as_uint(a);
+    const int ex = static_cast<int>((u >> 23) & 0xFF);
+    if (ex != 0) return ex - 127;
+    return (31 - __clz(static_cast<int>(u & 0x7FFFFF))) - 149;  // subnormal
+}
+
+// E2M1 magnitude code of a >= 0: nearest of {0,.5,1,1.5,2,3,4,6}; at a midpoint
+// the even code wins; above 6 saturates.
+__device__ __forceinline__ uint32_t e2m1_code_of(float a) {
+    return a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
+         : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.0f ? 6u : 7u;
+}
+
+// One thread per (row n, block b) of expert blockIdx.z.  W is [K][N] fp32 per
+// expert (y = x . W); consecutive threads take consecutive n so the reads of
+// each of the 32 block elements are coalesced.
+__global__ void quantize_kernel(const float* __restrict__ W, size_t w_expert_stride, TiledMatrix M) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    const int e = blockIdx.z;
+    if (n >= M.N) return;
+    size_t co, so;
+    M.locate(n, b, co, so);
+    uint8_t* dst = M.base + static_cast<size_t>(e) * M.expert_bytes();
+    uint4 out = make_uint4(0, 0, 0, 0);
+    uint32_t scale = 127;
+    if (b * 32 < M.K) {
+        const float* src = W + static_cast<size_t>(e) * w_expert_stride + static_cast<size_t>(b) * 32 * M.N + n;
+        float v[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            v[i] = src[static_cast<size_t>(i) * M.N];
+            amax = fmaxf(amax, fabsf(v[i]));
+        }
+        if (amax > 0.f) {
+            int ex = floor_log2_pos(amax) - 2;
+            ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
+            scale = static_cast<uint32_t>(ex + 127);
+            const float inv = __int_as_float((127 - ex) << 23);  // 2^-ex, exact (ex in [-127, 125])
+            uint32_t words[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                uint32_t c = e2m1_code_of(fabsf(v[i] * inv));
+                if (__float_as_uint(v[i]) >> 31) c |= 8u;
+                words[i >> 3] |= c << (4 * (i & 7));
+            }
+            out = make_uint4(words[0], words[1], words[2], words[3]);
+        }
+    }
+    *reinterpret_cast<uint4*>(dst + co) = out;
+    dst[so] = static_cast<uint8_t>(scale);
+}
+
+// Row scale = largest scale byte over the row's blocks that hold a non-zero
+// code (127 when the row is all zero).
+__global__ void rowscale_kernel(TiledMatrix M, uint8_t* __restrict__ rowscale, size_t rs_expert_stride) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.z;
+    if (n >= M.N) return;
+    const uint8_t* src = M.base + static_cast<size_t>(e) * M.expert_bytes();
+    int best = -1;
+    for (int b = 0; b < (M.K + 31) / 32; ++b) {
+        size_t co, so;
+        M.locate(n, b, co, so);
+        const uint4 c = *reinterpret_cast<const uint4*>(src + co);
+        const uint32_t nz = (c.x | c.y | c.z | c.w) & 0x77777777u;
+        if (nz) best = max(best, static_cast<int>(src[so]));
+    }
+    rowscale[static_cast<size_t>(e) * rs_expert_stride + n] = static_cast<uint8_t>(best < 0 ? 127 : best);
+}
+
+// Tiled -> canonical: codes [E][N][K/2], scales [E][N][K/32].
+__global__ void export_kernel(TiledMatrix M, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    const int e = blockIdx.z;
+    const int nb = M.K / 32;
+    if (n >= M.N || b >= nb) return;
+    size_t co, so;
+    M.locate(n, b, co, so);
+    const uint8_t* src = M.base + static_cast<size_t>(e) * M.expert_bytes();
+    const size_t row = static_cast<size_t>(e) * M.N + n;
+    *reinterpret_cast<uint4*>(codes + row * (M.K / 2) + static_cast<size_t>(b) * 16) =
+        *reinterpret_cast<const uint4*>(src + co);
+    scales[row * nb + b] = src[so];
+}
+
+}  // namespace moe

@@ -83,13 +83,10 @@ def mxfp4_quantize_matrix(W: np.ndarray):
 
     Blocks run along the contraction axis K.  Returns canonical
     (codes [N, K/2], scales [N, K/32])."""
-    W = _c(W, np.float32)
+    W = np.asarray(W, dtype=np.float32)
     K, N = W.shape
     assert K % 32 == 0
-    codes = np.zeros((N, K // 2), np.uint8)
-    scales = np.zeros((N, K // 32), np.uint8)
-    lib().oracle_mxfp4_quantize(_ptr(W), N, K, 1, N, _ptr(codes), _ptr(scales))
-    return codes, scales
+    return mxfp4_quantize_rows(np.ascontiguousarray(W.T))
 
 
 def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:

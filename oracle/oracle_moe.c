@@ -45,12 +45,23 @@ double oracle_e8m0_decode(uint32_t s) {
     return ldexp(1.0, (int)(s & 0xFFu) - 127);
 }
 
+/* Lookup tables filled once from the decode functions above: the 16 E2M1 code
+ * values and the 256 E8M0 scale values (tables only avoid recomputing them). */
+static double g_code_value[16];
+static double g_scale_value[256];
+static pthread_once_t g_tables_once = PTHREAD_ONCE_INIT;
+static void fill_tables(void) {
+    for (uint32_t c = 0; c < 16; ++c) g_code_value[c] = oracle_e2m1_decode(c);
+    for (uint32_t s = 0; s < 256; ++s) g_scale_value[s] = oracle_e8m0_decode(s);
+}
+static void tables(void) { pthread_once(&g_tables_once, fill_tables); }
+
 /* Nearest E2M1 magnitude code for a >= 0; equal distances go to the even code. */
 static uint32_t e2m1_round_magnitude(double a) {
     uint32_t best = 0;
-    double best_d = fabs(a - e2m1_magnitude(0));
+    double best_d = fabs(a - g_code_value[0]);
     for (uint32_t c = 1; c < 8; ++c) {
-        double dd = fabs(a - e2m1_magnitude(c));
+        double dd = fabs(a - g_code_value[c]);
         if (dd < best_d || (dd == best_d && (c & 1u) == 0 && (best & 1u) == 1)) {
             best = c;
             best_d = dd;
@@ -63,6 +74,7 @@ void oracle_mxfp4_quantize(const float* w, int64_t rows, int64_t K,
                            int64_t s_row, int64_t s_k,
                            uint8_t* codes, uint8_t* scales) {
     const int64_t nb = K / 32;
+    tables();
     for (int64_t n = 0; n < rows; ++n) {
         for (int64_t b = 0; b < nb; ++b) {
             double v[32];
@@ -99,11 +111,12 @@ static inline double mx_value(const uint8_t* codes, const uint8_t* scales,
                               int64_t K, int64_t n, int64_t k) {
     uint8_t byte = codes[n * (K / 2) + k / 2];
     uint32_t c = (k & 1) ? (uint32_t)(byte >> 4) : (uint32_t)(byte & 15u);
-    return oracle_e2m1_decode(c) * oracle_e8m0_decode(scales[n * (K / 32) + k / 32]);
+    return g_code_value[c] * g_scale_value[scales[n * (K / 32) + k / 32]];
 }
 
 void oracle_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
                              int64_t K, int64_t row0, int64_t nrows, double* out) {
+    tables();
     for (int64_t r = 0; r < nrows; ++r)
         for (int64_t k = 0; k < K; ++k)
             out[r * K + k] = mx_value(codes, scales, K, row0 + r, k);
@@ -161,6 +174,7 @@ void oracle_expert(const double* x, int64_t d_model, int64_t d_ff,
                    const uint8_t* u_codes, const uint8_t* u_scales,
                    const uint8_t* d_codes, const uint8_t* d_scales,
                    double* out, double* h_out) {
+    tables();
     double* h = (double*)malloc(sizeof(double) * (size_t)d_ff);
     for (int64_t f = 0; f < d_ff; ++f) {
         double g = 0.0, u = 0.0;
