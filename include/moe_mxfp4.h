@@ -155,9 +155,10 @@ const char* moe_mxfp4_status_string(moe_status_t s);
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */
-#define MOE_NUM_STAGES 7
-/* 0 router+top-k, 1 grouping schedule, 2 permute/gather, 3 gate/up+SwiGLU,
- * 4 split-K SwiGLU finish, 5 down+combine, 6 output cast.  Synchronises;
+#define MOE_NUM_STAGES 6
+/* 0 router + top-k + softmax + grouping schedule, 1 gather into grouped rows,
+ * 2 gate/up + SwiGLU, 3 split-K SwiGLU finish, 4 down + weighted combine,
+ * 5 output cast.  Synchronises;
  * writes the last profiled forward's durations in ms (0 for stages that did
  * not run) into ms[0..min(n, MOE_NUM_STAGES)). */
 moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n);

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(HERE, "libmoe_mxfp4.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_NOT_QUANTIZED, MOE_ERR_TIMEOUT = range(6)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_FLAG_TEST_SKIP_FIRST_COPY = 1 << 30
-MOE_NUM_STAGES = 7
+MOE_NUM_STAGES = 6
 
 
 class moe_mxfp4_config_t(ctypes.Structure):

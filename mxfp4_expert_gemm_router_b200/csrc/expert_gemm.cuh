@@ -14,19 +14,23 @@
 // grouped f16 activations, arrives by 2-D TMA with 128-byte swizzle.  fp32
 // accumulators stay in TMEM; the epilogue warps read them back with tcgen05.ld.
 //
-//   MODE 0 (gate/up): two accumulators (gate, up) for the same 128 features;
-//     epilogue: H[row, f] = Swish(g * 2^sg) * (u * 2^su), stored as f16; with a
-//     K split, fp32 partials are added into GU instead.
-//   MODE 1 (down):   one accumulator; epilogue: y[token, f] += w_row *
-//     (d * 2^sd), red.add into the fp32 output accumulator (the weighted
-//     scatter-combine).
+//   MODE 0 (gate/up): stages of K = 64 holding gate and up; two accumulators
+//     (gate, up) for the same 128 features; epilogue: H[row, f] =
+//     Swish(g * 2^sg) * (u * 2^su), stored as f16; with a K split, fp32
+//     partials are added into GU instead.
+//   MODE 1 (down): stages of K = 128; one accumulator; epilogue: y[token, f] +=
+//     w_row * (d * 2^sd), red.add into the fp32 output accumulator (the
+//     weighted scatter-combine).
+// Both modes stream 8704 weight bytes (128 rows x 4 blocks x 17 B) per stage
+// and decode exactly one 32-block per decoder thread per stage.
 //
 // Persistent kernel: one CTA per SM, units (expert, token tile, feature tile,
 // K split) taken round-robin from a device-built list.  Warp roles:
-//   warp 0      TMA producer (one thread)
-//   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warps 2..9  decoders, then epilogue; warp w serves TMEM lanes 32*(w%4).. and
-//               MXFP4 block (w-2)/4 of each 64-wide chunk
+//   warp 0       TMA producer (one thread)
+//   warp 1       TMEM allocator and MMA issuer (one thread)
+//   warps 2..17  decoders, then epilogue.  Warp w serves TMEM lanes
+//                32*(w%4) .. +31 and role (w-2)/4 in 0..3: MODE 0 matrix
+//                role>>1, block role&1 of the stage; MODE 1 block role.
 // Every mbarrier wait is bounded; on a timeout the CTA raises an abort flag,
 // all roles leave their loops, in-flight copies and MMAs are drained, TMEM is
 // freed and the status word reports the timeout.
@@ -35,15 +39,20 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
+#include "quantize.cuh"
 #include "routing.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
 
-constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_DEC_WARPS = 16;
+constexpr int GEMM_THREADS = (2 + GEMM_DEC_WARPS) * 32;
 constexpr int GEMM_MAX_STAGES = 16;
 constexpr int GEMM_A_SLOTS = 4;
+constexpr int GEMM_A_COLS = 64;                               // TMEM columns per A slot
+constexpr int GEMM_D_COL0 = GEMM_A_SLOTS * GEMM_A_COLS;       // first accumulator column
 constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_W_STAGE = 128 * 4 * 17;                    // weight bytes per stage (max)
 constexpr int GEMM_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
 struct GemmParams {
@@ -51,10 +60,10 @@ struct GemmParams {
     const uint8_t* rowscale;  // MODE 0: [E][2][N] (gate, up); MODE 1: [E][N]
     const int4* units;        // {expert, first grouped row, valid rows, feature tile | split << 16}
     const int32_t* sched;
+    TiledMatrix M;            // geometry of the (first) matrix streamed
     int N;                    // output features
     int K;                    // contraction length
-    int KC;                   // 64-wide chunks
-    int BN;                   // token rows per tile (MMA N), multiple of 16, <= 128
+    int BN;                   // token rows per tile (MMA N), multiple of 16
     int stages;
     uint32_t idesc;
     __half* H;                // MODE 0 output [rows][N]
@@ -67,17 +76,11 @@ struct GemmParams {
     uint32_t skip_first_copy; // test hook: producer skips its first copy
 };
 
-template <int MODE>
-struct GemmShape {
-    static constexpr int CH = MODE == 0 ? 68 : 34;          // bytes per weight row per chunk
-    static constexpr int W_STAGE = CH * 128;                // weight bytes per stage (max)
-    static constexpr int A_COLS = MODE == 0 ? 64 : 32;      // TMEM columns per A slot
-    static constexpr int D_COL0 = GEMM_A_SLOTS * A_COLS;    // first accumulator column
-};
-
-__host__ inline size_t gemm_stage_bytes(int mode, int BN) {
-    return static_cast<size_t>(mode == 0 ? 68 * 128 : 34 * 128) + static_cast<size_t>(BN) * 128;
+__host__ __device__ inline int gemm_kstage(int mode) { return mode == 0 ? 64 : 128; }
+__host__ __device__ inline size_t gemm_b_stage_bytes(int mode, int BN) {
+    return static_cast<size_t>(BN) * 128 * (mode == 0 ? 1 : 2);
 }
+__host__ inline size_t gemm_stage_bytes(int mode, int BN) { return GEMM_W_STAGE + gemm_b_stage_bytes(mode, BN); }
 __host__ inline size_t gemm_smem_bytes(int mode, int BN, int stages) {
     size_t b = 1024 + stages * gemm_stage_bytes(mode, BN) + (2 * stages + 2 * GEMM_A_SLOTS + 3) * 8 + 64;
     return b < static_cast<size_t>(GEMM_MIN_SMEM) ? static_cast<size_t>(GEMM_MIN_SMEM) : b;
@@ -86,17 +89,18 @@ __host__ inline size_t gemm_smem_bytes(int mode, int BN, int stages) {
 template <int MODE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
-    using Sh = GemmShape<MODE>;
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int KSTAGE = MODE == 0 ? 64 : 128;
 
     const int S = p.stages;
-    const uint32_t b_bytes = static_cast<uint32_t>(p.BN) * 128u;
+    const uint32_t b_bytes = static_cast<uint32_t>(gemm_b_stage_bytes(MODE, p.BN));
+    const uint32_t b_sub = static_cast<uint32_t>(p.BN) * 128u;   // one 64-K sub-tile of B
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t b_sm = base;                                   // S x B tiles (1024-aligned)
     const uint32_t w_sm = b_sm + S * b_bytes;                     // S x weight chunks
-    const uint32_t bar0 = w_sm + S * Sh::W_STAGE;                 // barriers (8-byte aligned)
+    const uint32_t bar0 = w_sm + S * GEMM_W_STAGE;                // barriers (8-byte aligned)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     auto afull_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
@@ -111,14 +115,14 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 8 + 1);  // 8 decoder warps + 1 MMA commit
+            mbar_init(empty_bar(s), GEMM_DEC_WARPS + 1);  // decoder warps + 1 MMA commit
         }
         for (int a = 0; a < GEMM_A_SLOTS; ++a) {
-            mbar_init(afull_bar(a), 8);
+            mbar_init(afull_bar(a), GEMM_DEC_WARPS);
             mbar_init(aempty_bar(a), 1);
         }
         mbar_init(accf_bar, 1);
-        mbar_init(acce_bar, 8);
+        mbar_init(acce_bar, GEMM_DEC_WARPS);
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -135,7 +139,8 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
 
     const int num_units = p.sched[MODE == 0 ? SCHED_UNITS_GU : SCHED_UNITS_DN];
     const int nsplit = p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN];
-    const size_t expert_bytes = static_cast<size_t>(p.N) * p.KC * Sh::CH;
+    const int KC = p.M.chunks();
+    const size_t expert_bytes = p.M.expert_bytes();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -148,19 +153,21 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const int4 U = p.units[u];
                 const int ft = U.w & 0xFFFF, sp = U.w >> 16;
-                const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+                const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
                 const int rf = min(128, p.N - ft * 128);
-                const uint32_t wb = static_cast<uint32_t>(Sh::CH * rf);
-                const uint8_t* wt = p.wpack + static_cast<size_t>(U.x) * expert_bytes +
-                                    static_cast<size_t>(ft) * 128 * p.KC * Sh::CH;
+                const uint8_t* we = p.wpack + static_cast<size_t>(U.x) * expert_bytes;
                 for (int c = c0; c < c1; ++c) {
                     if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto producer_done;
                     if (skip) {
                         skip = false;  // test hook: this stage is never filled
                     } else {
-                        mbar_arrive_expect_tx(full_bar(s), wb + b_bytes);
-                        bulk_g2s(w_sm + s * Sh::W_STAGE, wt + static_cast<size_t>(c) * wb, wb, full_bar(s));
-                        tma_load_2d(b_sm + s * b_bytes, &tmap_b, c * 64, U.y, full_bar(s));
+                        const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
+                        const int k0 = c * KSTAGE;
+                        const bool second = (MODE == 1) && (k0 + 64 < p.K);
+                        mbar_arrive_expect_tx(full_bar(s), wb + (second ? 2u : 1u) * b_sub);
+                        bulk_g2s(w_sm + s * GEMM_W_STAGE, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
+                        tma_load_2d(b_sm + s * b_bytes, &tmap_b, k0, U.y, full_bar(s));
+                        if (second) tma_load_2d(b_sm + s * b_bytes + b_sub, &tmap_b, k0 + 64, U.y, full_bar(s));
                         pend_ph[s] = static_cast<int>(ph);
                     }
                     if (++s == S) { s = 0; ph ^= 1u; }
@@ -180,23 +187,24 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const int4 U = p.units[u];
                 const int sp = U.w >> 16;
-                const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+                const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
                 if (!mbar_wait_bounded(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto mma_done;
                 tc_fence_after();
                 for (int c = c0; c < c1; ++c) {
                     if (!mbar_wait_bounded(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
                     if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
                     tc_fence_after();
+                    const int ksteps = 2 * p.M.blocks_in_chunk(c);
                     const uint64_t bd = bdesc0 + ((static_cast<uint64_t>(s) * b_bytes) >> 4);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    const uint32_t acol = tmem + a * GEMM_A_COLS;
+                    for (int i = 0; i < ksteps; ++i) {
                         const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
-                        const uint32_t acol = tmem + a * Sh::A_COLS + 8 * i;
                         if (MODE == 0) {
-                            mma_f16_ts(tmem + Sh::D_COL0, acol, bd + 2 * i, p.idesc, acc);
-                            mma_f16_ts(tmem + Sh::D_COL0 + p.BN, acol + 32, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts(tmem + GEMM_D_COL0, acol + 8 * i, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts(tmem + GEMM_D_COL0 + p.BN, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
                         } else {
-                            mma_f16_ts(tmem + Sh::D_COL0, acol, bd + 2 * i, p.idesc, acc);
+                            const uint64_t bdi = bd + (((i >> 2) * b_sub) >> 4) + 2 * (i & 3);
+                            mma_f16_ts(tmem + GEMM_D_COL0, acol + 8 * i, bdi, p.idesc, acc);
                         }
                     }
                     tc_commit(aempty_bar(a));
@@ -213,10 +221,13 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
         }
     } else {
         // ---------------------------------------------------------- decoders + epilogue
-        const int q = warp & 3;               // TMEM lane quadrant
-        const int hb = (warp - 2) >> 2;       // which 32-block of each chunk
+        const int q = warp & 3;               // TMEM lane quadrant (hardware rule: warp % 4)
+        const int role = (warp - 2) >> 2;     // 0..3
+        const int mat = MODE == 0 ? (role >> 1) : 0;
+        const int hb = MODE == 0 ? (role & 1) : role;
         const int row = 32 * q + lane;        // weight row within the feature tile
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        const uint32_t tcol = static_cast<uint32_t>(mat * 32 + hb * 16);
         int s = 0, a = 0;
         uint32_t ph = 0, aph = 0, acc_ph = 0;
         bool ok = true;
@@ -224,32 +235,32 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             const int4 U = p.units[u];
             const int e = U.x, row0 = U.y, nvalid = U.z;
             const int ft = U.w & 0xFFFF, sp = U.w >> 16;
-            const int c0 = sp * p.KC / nsplit, c1 = (sp + 1) * p.KC / nsplit;
+            const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
             const int rf = min(128, p.N - ft * 128);
             const bool warp_rows = 32 * q < rf;
             const int n = ft * 128 + row;
-            int rs0 = 127, rs1 = 127;
+            int rs_mine = 127, rs0 = 127, rs1 = 127;
             if (warp_rows) {
                 if (MODE == 0) {
                     rs0 = p.rowscale[(static_cast<size_t>(e) * 2 + 0) * p.N + n];
                     rs1 = p.rowscale[(static_cast<size_t>(e) * 2 + 1) * p.N + n];
+                    rs_mine = mat ? rs1 : rs0;
                 } else {
                     rs0 = p.rowscale[static_cast<size_t>(e) * p.N + n];
+                    rs_mine = rs0;
                 }
             }
             for (int c = c0; c < c1; ++c) {
+                const int nbc = p.M.blocks_in_chunk(c);
+                const bool mine = warp_rows && hb < nbc;
                 bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
                 if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-                uint4 cg = make_uint4(0, 0, 0, 0), cu = make_uint4(0, 0, 0, 0);
-                int sg = 127, su = 127;
-                if (warp_rows) {
-                    const uint8_t* ws = smem_raw + (w_sm + s * Sh::W_STAGE - raw);
-                    cg = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
-                    sg = ws[32 * rf + hb * rf + row];
-                    if (MODE == 0) {
-                        cu = *reinterpret_cast<const uint4*>(ws + 34 * rf + (hb * rf + row) * 16);
-                        su = ws[66 * rf + hb * rf + row];
-                    }
+                uint4 cw = make_uint4(0, 0, 0, 0);
+                int sc = 127;
+                if (mine) {
+                    const uint8_t* ws = smem_raw + (w_sm + s * GEMM_W_STAGE - raw) + mat * 17 * nbc * rf;
+                    cw = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
+                    sc = ws[16 * nbc * rf + hb * rf + row];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty_bar(s));
@@ -258,24 +269,15 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
                 if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
                 tc_fence_after();
-                if (warp_rows) {
+                if (mine) {
                     uint32_t r[16];
-                    const uint32_t mg = f16_pow2_bits(sg - rs0);
-                    const uint32_t mg2 = mg | (mg << 16);
-                    e2m1x8_to_f16x8(cg.x, mg2, r[0], r[1], r[2], r[3]);
-                    e2m1x8_to_f16x8(cg.y, mg2, r[4], r[5], r[6], r[7]);
-                    e2m1x8_to_f16x8(cg.z, mg2, r[8], r[9], r[10], r[11]);
-                    e2m1x8_to_f16x8(cg.w, mg2, r[12], r[13], r[14], r[15]);
-                    tmem_st16(tmem + lane_addr + a * Sh::A_COLS + 16 * hb, r);
-                    if (MODE == 0) {
-                        const uint32_t mu = f16_pow2_bits(su - rs1);
-                        const uint32_t mu2 = mu | (mu << 16);
-                        e2m1x8_to_f16x8(cu.x, mu2, r[0], r[1], r[2], r[3]);
-                        e2m1x8_to_f16x8(cu.y, mu2, r[4], r[5], r[6], r[7]);
-                        e2m1x8_to_f16x8(cu.z, mu2, r[8], r[9], r[10], r[11]);
-                        e2m1x8_to_f16x8(cu.w, mu2, r[12], r[13], r[14], r[15]);
-                        tmem_st16(tmem + lane_addr + a * Sh::A_COLS + 32 + 16 * hb, r);
-                    }
+                    const uint32_t m1 = f16_pow2_bits(sc - rs_mine);
+                    const uint32_t m2 = m1 | (m1 << 16);
+                    e2m1x8_to_f16x8(cw.x, m2, r[0], r[1], r[2], r[3]);
+                    e2m1x8_to_f16x8(cw.y, m2, r[4], r[5], r[6], r[7]);
+                    e2m1x8_to_f16x8(cw.z, m2, r[8], r[9], r[10], r[11]);
+                    e2m1x8_to_f16x8(cw.w, m2, r[12], r[13], r[14], r[15]);
+                    tmem_st16(tmem + lane_addr + a * GEMM_A_COLS + tcol, r);
                     tmem_wait_st();
                 }
                 tc_fence_before();
@@ -293,17 +295,15 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             acc_ph ^= 1u;
             tc_fence_after();
             if (warp_rows) {
-                const int half = p.BN / 2;
-                const int n0 = hb * half;
                 const float f0 = pow2f(rs0 - 127);
                 const float f1 = pow2f(rs1 - 127);
-                for (int j0 = 0; j0 < half; j0 += 8) {
-                    const int col = n0 + j0;
+                for (int col = role * 8; col < p.BN; col += 32) {
+                    if (col >= nvalid) break;
                     uint32_t g[8];
-                    tmem_ld8(tmem + lane_addr + Sh::D_COL0 + col, g);
+                    tmem_ld8(tmem + lane_addr + GEMM_D_COL0 + col, g);
                     if (MODE == 0) {
                         uint32_t v[8];
-                        tmem_ld8(tmem + lane_addr + Sh::D_COL0 + p.BN + col, v);
+                        tmem_ld8(tmem + lane_addr + GEMM_D_COL0 + p.BN + col, v);
                         tmem_wait_ld();
                         if (nsplit == 1) {
 #pragma unroll

@@ -1,14 +1,15 @@
 // moe_mxfp4.cu -- C ABI of the MoE feed-forward layer with MXFP4 experts
 // (declarations and argument contracts in include/moe_mxfp4.h).
 //
-// One forward = up to seven launches on the caller's stream, no host sync and
+// One forward = up to six launches on the caller's stream, no host sync and
 // no allocation:
-//   router_kernel        scores, top-k, softmax over the selected scores,
-//                        per-block expert histogram, zeroing of the output rows
-//   schedule_kernel      expert offsets, per-block prefixes, K splits, unit lists
-//   permute_kernel       grouped rows (token, weight) and f16 activation gather
+//   router_kernel        scores (K split over the grid), top-k, softmax over the
+//                        selected scores, per-tile histogram and ranks, zeroing
+//                        of the output rows; its last CTA builds the schedule
+//                        (expert offsets, K splits, unit lists)
+//   gather_kernel        grouped rows (token, weight) and f16 activation gather
 //   expert_gemm<0>       gate/up GEMM, SwiGLU epilogue
-//   swiglu_finish_kernel only when the gate/up GEMM split K
+//   swiglu_finish_kernel only when the gate/up GEMM may split K
 //   expert_gemm<1>       down GEMM, routing-weighted scatter-combine epilogue
 //   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
 #include <cuda.h>
@@ -58,6 +59,7 @@ struct moe_mxfp4 {
     int act_bytes = 2;
     int KC_gu = 0, KC_dn = 0, F_gu = 0, F_dn = 0;
     int TK = 0, nblk_max = 0, max_units = 0, gu_rows = 0;
+    size_t part_elems = 0;
     // weights
     uint8_t* w_gu = nullptr;   // tiled gate+up
     uint8_t* w_dn = nullptr;   // tiled down
@@ -72,6 +74,9 @@ struct moe_mxfp4 {
     int32_t* idx_ws = nullptr;
     float* w_ws = nullptr;
     int32_t* hist = nullptr;
+    double* part = nullptr;
+    int* counters = nullptr;   // [nblk_max] tile counters + [1] global counter
+    int32_t* local_rank = nullptr;
     int32_t* offsets = nullptr;
     int32_t* sched = nullptr;
     int4* units_gu = nullptr;
@@ -111,6 +116,7 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 static void free_all(moe_mxfp4* h) {
     void* ptrs[] = {h->w_gu, h->w_dn, h->rs_gu, h->rs_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
+                    h->part, h->counters, h->local_rank,
                     h->offsets, h->sched, h->units_gu, h->units_dn, h->row_token, h->row_weight, h->Xp, h->H,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
     for (void* p : ptrs)
@@ -125,6 +131,13 @@ static int choose_bn(int T, int k, int E) {
     long want = std::min<long>(T, std::max<long>(1, 4 * per_expert));
     int bn = static_cast<int>((want + 15) / 16) * 16;
     return std::max(16, std::min(128, bn));
+}
+
+static int router_splits(int T, int d, int nsm) {
+    const int tiles = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+    const int kch = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
+    const int want = (2 * nsm + tiles - 1) / tiles;
+    return std::max(1, std::min(kch, want));
 }
 
 static int stages_for(int mode, int BN) {
@@ -148,7 +161,7 @@ const char* moe_mxfp4_status_string(moe_status_t s) {
 }
 
 const char* moe_mxfp4_stage_name(int32_t stage) {
-    static const char* names[MOE_NUM_STAGES] = {"router_topk", "schedule", "permute_gather", "gate_up_swiglu",
+    static const char* names[MOE_NUM_STAGES] = {"router_topk_schedule", "gather", "gate_up_swiglu",
                                                  "swiglu_finish", "down_combine", "cast_out"};
     return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "unknown";
 }
@@ -190,8 +203,8 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     if (cudaDeviceGetAttribute(&h->nsm, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
     const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
-    h->KC_gu = (d + 63) / 64;
-    h->KC_dn = (f + 63) / 64;
+    h->KC_gu = (d / 32 + 1) / 2;   // 64-wide chunks of the gate/up GEMM
+    h->KC_dn = (f / 32 + 3) / 4;   // 128-wide chunks of the down GEMM
     h->F_gu = (f + 127) / 128;
     h->F_dn = (d + 127) / 128;
     h->TK = c.max_tokens * k;
@@ -203,11 +216,12 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         h->max_units = static_cast<int>(std::max(tiles_big, tiles_small) * F + 8L * h->nsm + 64);
     }
     h->gu_rows = std::min(h->TK, SPLIT_ROWS_CAP);
+    h->part_elems = static_cast<size_t>(64 * h->nsm + ROUTER_TOKENS * h->nblk_max + ROUTER_TOKENS) * E;
     h->expert_done = new (std::nothrow) bool[E]();
     if (!h->expert_done) return fail(MOE_ERR_CUDA);
 
-    const size_t gu_bytes = static_cast<size_t>(E) * f * h->KC_gu * 68;
-    const size_t dn_bytes = static_cast<size_t>(E) * d * h->KC_dn * 34;
+    const size_t gu_bytes = static_cast<size_t>(E) * f * (d / 32) * 17 * 2;
+    const size_t dn_bytes = static_cast<size_t>(E) * d * (f / 32) * 17;
     const size_t TK = h->TK;
     struct A { void** p; size_t bytes; };
     A allocs[] = {
@@ -220,6 +234,9 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->idx_ws), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->w_ws), sizeof(float) * TK},
         {reinterpret_cast<void**>(&h->hist), sizeof(int32_t) * static_cast<size_t>(h->nblk_max) * E},
+        {reinterpret_cast<void**>(&h->part), sizeof(double) * h->part_elems},
+        {reinterpret_cast<void**>(&h->counters), sizeof(int) * (h->nblk_max + 1)},
+        {reinterpret_cast<void**>(&h->local_rank), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->offsets), sizeof(int32_t) * (E + 1)},
         {reinterpret_cast<void**>(&h->sched), sizeof(int32_t) * SCHED_SLOTS},
         {reinterpret_cast<void**>(&h->units_gu), sizeof(int4) * h->max_units},
@@ -243,6 +260,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     if (cudaMemset(h->Xp, 0, sizeof(__half) * TK * d) != cudaSuccess ||
         cudaMemset(h->H, 0, sizeof(__half) * TK * f) != cudaSuccess ||
         cudaMemset(h->status, 0, sizeof(int) * 4) != cudaSuccess ||
+        cudaMemset(h->counters, 0, sizeof(int) * (h->nblk_max + 1)) != cudaSuccess ||
         cudaMemset(h->bias, 0, sizeof(float) * E) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return fail(MOE_ERR_CUDA);
 
@@ -278,15 +296,15 @@ static TiledMatrix tiled(moe_mxfp4* h, int which) {
         M.base = h->w_gu;
         M.N = c.d_ff;
         M.K = c.d_model;
-        M.KC = h->KC_gu;
-        M.CH = 68;
+        M.BPC = 2;
+        M.NM = 2;
         M.sub = which;
     } else {
         M.base = h->w_dn;
         M.N = c.d_model;
         M.K = c.d_ff;
-        M.KC = h->KC_dn;
-        M.CH = 34;
+        M.BPC = 4;
+        M.NM = 1;
         M.sub = 0;
     }
     return M;
@@ -297,7 +315,7 @@ static moe_status_t quantize_matrix(moe_mxfp4* h, int which, const float* W, int
     TiledMatrix M = tiled(h, which);
     M.base += static_cast<size_t>(e0) * M.expert_bytes();
     const dim3 blk(128);
-    const dim3 grid((M.N + 127) / 128, 2 * M.KC, ne);
+    const dim3 grid((M.N + 127) / 128, M.nb(), ne);
     quantize_kernel<<<grid, blk, 0, s>>>(W, static_cast<size_t>(M.K) * M.N, M);
     h->launches++;
     uint8_t* rs;
@@ -419,61 +437,69 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         if (prof) cudaEventRecord(h->ev[i], stream);
     };
 
-    // 0: router + top-k + softmax
+    // 0: router + top-k + softmax + schedule
     mark(0);
+    RouterArgs ra;
+    ra.x = x;
+    ra.wr = h->w_router;
+    ra.bias = h->has_bias ? h->bias : nullptr;
+    ra.T = T;
+    ra.d = d;
+    ra.E = E;
+    ra.k = k;
+    ra.S = router_splits(T, d, h->nsm);
+    ra.part = h->part;
+    ra.tile_cnt = h->counters;
+    ra.glob_cnt = h->counters + h->nblk_max;
+    ra.idx_out = idx;
+    ra.w_out = wts;
+    ra.local_rank = h->local_rank;
+    ra.hist = h->hist;
+    ra.zero_rows = acc;
+    ra.zero_ld = d;
+    ra.BN = BN;
+    ra.F_gu = h->F_gu;
+    ra.F_dn = h->F_dn;
+    ra.KC_gu = h->KC_gu;
+    ra.KC_dn = h->KC_dn;
+    ra.nsm = h->nsm;
+    ra.split_rows_cap = h->gu_rows;
+    ra.max_units = h->max_units;
+    ra.offsets = h->offsets;
+    ra.counts_out = expert_counts;
+    ra.units_gu = h->units_gu;
+    ra.units_dn = h->units_dn;
+    ra.sched = h->sched;
     const size_t rsm = router_smem_bytes(E);
+    const dim3 rgrid(nblk, ra.S);
     if (bf16)
-        router_kernel<__nv_bfloat16><<<nblk, ROUTER_THREADS, rsm, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(h->w_router), h->bias, T, d, E,
-            k, idx, wts, h->hist, acc, d);
+        router_kernel<__nv_bfloat16><<<rgrid, ROUTER_THREADS, rsm, stream>>>(ra);
     else
-        router_kernel<float><<<nblk, ROUTER_THREADS, rsm, stream>>>(static_cast<const float*>(x),
-                                                                      static_cast<const float*>(h->w_router), h->bias,
-                                                                      T, d, E, k, idx, wts, h->hist, acc, d);
+        router_kernel<float><<<rgrid, ROUTER_THREADS, rsm, stream>>>(ra);
     h->stage_ran[0] = true;
-    // 1: schedule
+    // 1: gather into grouped rows
     mark(1);
-    ScheduleArgs sa;
-    sa.hist = h->hist;
-    sa.nblk = nblk;
-    sa.E = E;
-    sa.BN = BN;
-    sa.F_gu = h->F_gu;
-    sa.F_dn = h->F_dn;
-    sa.KC_gu = h->KC_gu;
-    sa.KC_dn = h->KC_dn;
-    sa.nsm = h->nsm;
-    sa.split_rows_cap = h->gu_rows;
-    sa.max_units = h->max_units;
-    sa.offsets = h->offsets;
-    sa.counts_out = expert_counts;
-    sa.units_gu = h->units_gu;
-    sa.units_dn = h->units_dn;
-    sa.sched = h->sched;
-    schedule_kernel<<<1, 1024, 0, stream>>>(sa);
-    h->stage_ran[1] = true;
-    // 2: permute + gather
-    mark(2);
+    const int gblocks = (T * k + GATHER_WARPS - 1) / GATHER_WARPS;
     if (bf16)
-        permute_kernel<__nv_bfloat16><<<nblk, ROUTER_THREADS, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), idx, wts, h->hist, h->offsets, T, d, E, k, h->row_token,
-            h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+        gather_kernel<__nv_bfloat16><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, T, d, E, k,
+            h->row_token, h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
     else
-        permute_kernel<float><<<nblk, ROUTER_THREADS, 0, stream>>>(static_cast<const float*>(x), idx, wts, h->hist,
-                                                                     h->offsets, T, d, E, k, h->row_token,
-                                                                     h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
-    h->stage_ran[2] = true;
-    // 3: gate/up GEMM + SwiGLU
-    mark(3);
+        gather_kernel<float><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
+            static_cast<const float*>(x), idx, wts, h->local_rank, h->hist, h->offsets, T, d, E, k, h->row_token,
+            h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+    h->stage_ran[1] = true;
+    // 2: gate/up GEMM + SwiGLU
+    mark(2);
     const uint64_t tmo = static_cast<uint64_t>(c.wait_timeout_ms > 0 ? c.wait_timeout_ms : 2000) * 1000000ull;
     GemmParams gp;
     gp.wpack = h->w_gu;
     gp.rowscale = h->rs_gu;
     gp.units = h->units_gu;
     gp.sched = h->sched;
+    gp.M = tiled(h, 0);
     gp.N = f;
     gp.K = d;
-    gp.KC = h->KC_gu;
     gp.BN = BN;
     gp.stages = stages_for(0, BN);
     gp.idesc = idesc_f16_f32(128, BN);
@@ -487,40 +513,40 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
     const int grid = h->nsm;
     expert_gemm_kernel<0><<<grid, GEMM_THREADS, gemm_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
-    h->stage_ran[3] = true;
-    // 4: split-K finish (no-op unless the schedule split K)
-    mark(4);
+    h->stage_ran[2] = true;
+    // 3: split-K finish (no-op unless the schedule split K)
+    mark(3);
     const bool may_split = static_cast<long>(T) * k <= h->gu_rows;
     if (may_split) {
         const int blocks = std::min<long>(4L * h->nsm, (static_cast<long>(T) * k * f + 255) / 256);
         swiglu_finish_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->GU, h->H, f, h->sched);
-        h->stage_ran[4] = true;
+        h->stage_ran[3] = true;
     }
-    // 5: down GEMM + weighted scatter-combine
-    mark(5);
+    // 4: down GEMM + weighted scatter-combine
+    mark(4);
     GemmParams dp = gp;
     dp.wpack = h->w_dn;
     dp.rowscale = h->rs_dn;
     dp.units = h->units_dn;
+    dp.M = tiled(h, 2);
     dp.N = d;
     dp.K = f;
-    dp.KC = h->KC_dn;
     dp.stages = stages_for(1, BN);
     dp.H = nullptr;
     dp.GU = nullptr;
     dp.yacc = acc;
     dp.skip_first_copy = 0;
     expert_gemm_kernel<1><<<grid, GEMM_THREADS, gemm_smem_bytes(1, BN, dp.stages), stream>>>(h->tm_h[BN / 16 - 1], dp);
-    h->stage_ran[5] = true;
-    // 6: output cast
-    mark(6);
+    h->stage_ran[4] = true;
+    // 5: output cast
+    mark(5);
     if (bf16) {
         const size_t n4 = static_cast<size_t>(T) * d / 4;
         const int blocks = static_cast<int>(std::min<size_t>(4 * static_cast<size_t>(h->nsm), (n4 + 255) / 256));
         cast_out_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->yacc, static_cast<__nv_bfloat16*>(y), n4);
-        h->stage_ran[6] = true;
+        h->stage_ran[5] = true;
     }
-    mark(7);
+    mark(6);
     h->prof_valid = prof;
     for (int i = 0; i < MOE_NUM_STAGES; ++i) h->launches += h->stage_ran[i] ? 1 : 0;
     return cuda_status(cudaGetLastError());

@@ -10,18 +10,18 @@
 // even code, magnitudes above 6 saturate, the sign bit is kept; an all-zero
 // block gets scale byte 127.
 //
-// Streamed layout ("tiled"): for a matrix with N output rows and contraction
-// length K, rows are cut into 128-row feature tiles (the last one holds
-// N - 128*floor(N/128) rows) and K into 64-wide chunks (two 32-blocks).  For each
-// (tile, chunk) the bytes are contiguous:
-//     codes  [2 blocks][rf rows][16 B]   (even element in the low nibble)
-//     scales [2 blocks][rf rows]          (E8M0 bytes)
-// i.e. 34 * rf bytes per matrix; gate and up are interleaved per chunk
-// (gate 34*rf bytes, then up 34*rf bytes).  A K that is 32 mod 64 gets one
-// zero block (codes 0, scale 127) at the end of its last chunk.  One further
-// byte per row, the largest scale over the row's non-zero blocks ("row
-// scale", 127 if none), lets the GEMM decode each block as f16 relative to
-// its row and apply 2^(row scale - 127) in fp32 after accumulation.
+// Streamed layout ("tiled"): rows (output features) are cut into 128-row
+// feature tiles (the last one holds the remainder rf) and each row's nb = K/32
+// blocks into chunks of BPC blocks (the last chunk may hold fewer, nb_c).  For
+// each (tile, chunk) the bytes of the NM interleaved matrices (gate and up, or
+// down alone) are contiguous, matrix after matrix:
+//     codes  [nb_c blocks][rf rows][16 B]   (even element in the low nibble)
+//     scales [nb_c blocks][rf rows]          (E8M0 bytes)
+// i.e. 17 bytes per row per block, exactly 4.25 bits per parameter with no
+// padding.  One further byte per row, the largest scale over the row's
+// non-zero blocks ("row scale", 127 if none), lets the GEMM decode each block
+// as f16 relative to its row and apply 2^(row scale - 127) in fp32 after
+// accumulation.
 #pragma once
 #include <cstdint>
 
@@ -29,19 +29,30 @@ namespace moe {
 
 struct TiledMatrix {
     uint8_t* base;   // expert 0 of the packed array
-    int N, K, KC;    // rows, contraction length, 64-chunks = ceil(K/64)
-    int CH;          // bytes per row per chunk of the interleaved group: 68 (gate+up) or 34
-    int sub;         // 0 (gate / down) or 1 (up): which 34*rf part of the chunk
-    __host__ __device__ size_t expert_bytes() const { return static_cast<size_t>(N) * KC * CH; }
-    // byte offset (within one expert) of the codes of block b (0..2*KC-1) of row n
+    int N, K;        // rows, contraction length (K % 32 == 0)
+    int BPC;         // 32-blocks per chunk
+    int NM;          // matrices interleaved per chunk (2: gate+up, 1: down)
+    int sub;         // which matrix of the chunk this one is (0 or 1)
+    __host__ __device__ int nb() const { return K / 32; }
+    __host__ __device__ int chunks() const { return (nb() + BPC - 1) / BPC; }
+    __host__ __device__ size_t expert_bytes() const { return static_cast<size_t>(N) * nb() * 17 * NM; }
+    __host__ __device__ int blocks_in_chunk(int c) const { return min(BPC, nb() - c * BPC); }
+    // byte offset, within one expert, of feature tile ft's chunk c (all NM matrices)
+    __host__ __device__ size_t chunk_offset(int ft, int c, int rf) const {
+        return static_cast<size_t>(ft) * 128 * nb() * 17 * NM + static_cast<size_t>(c) * BPC * 17 * NM * rf;
+    }
+    __host__ __device__ size_t chunk_bytes(int c, int rf) const {
+        return static_cast<size_t>(blocks_in_chunk(c)) * 17 * NM * rf;
+    }
+    // byte offsets (within one expert) of block b of row n of this matrix
     __host__ __device__ void locate(int n, int b, size_t& code_off, size_t& scale_off) const {
         const int ft = n >> 7, r = n & 127;
         const int rf = min(128, N - (ft << 7));
-        const int c = b >> 1, h = b & 1;
-        const size_t chunk = static_cast<size_t>(ft) * 128 * KC * CH + static_cast<size_t>(c) * CH * rf +
-                             static_cast<size_t>(sub) * 34 * rf;
-        code_off = chunk + static_cast<size_t>(h * rf + r) * 16;
-        scale_off = chunk + 32 * static_cast<size_t>(rf) + h * rf + r;
+        const int c = b / BPC, h = b % BPC;
+        const int nbc = blocks_in_chunk(c);
+        const size_t base_m = chunk_offset(ft, c, rf) + static_cast<size_t>(sub) * 17 * nbc * rf;
+        code_off = base_m + static_cast<size_t>(h * rf + r) * 16;
+        scale_off = base_m + 16 * static_cast<size_t>(nbc) * rf + h * rf + r;
     }
 };
 
@@ -66,35 +77,33 @@ __global__ void quantize_kernel(const float* __restrict__ W, size_t w_expert_str
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     const int b = blockIdx.y;
     const int e = blockIdx.z;
-    if (n >= M.N) return;
+    if (n >= M.N || b >= M.nb()) return;
     size_t co, so;
     M.locate(n, b, co, so);
     uint8_t* dst = M.base + static_cast<size_t>(e) * M.expert_bytes();
+    const float* src = W + static_cast<size_t>(e) * w_expert_stride + static_cast<size_t>(b) * 32 * M.N + n;
+    float v[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        v[i] = src[static_cast<size_t>(i) * M.N];
+        amax = fmaxf(amax, fabsf(v[i]));
+    }
     uint4 out = make_uint4(0, 0, 0, 0);
     uint32_t scale = 127;
-    if (b * 32 < M.K) {
-        const float* src = W + static_cast<size_t>(e) * w_expert_stride + static_cast<size_t>(b) * 32 * M.N + n;
-        float v[32];
-        float amax = 0.f;
+    if (amax > 0.f) {
+        int ex = floor_log2_pos(amax) - 2;
+        ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
+        scale = static_cast<uint32_t>(ex + 127);
+        const float inv = __int_as_float((127 - ex) << 23);  // 2^-ex, exact (ex in [-127, 125])
+        uint32_t words[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            v[i] = src[static_cast<size_t>(i) * M.N];
-            amax = fmaxf(amax, fabsf(v[i]));
+            uint32_t c = e2m1_code_of(fabsf(v[i] * inv));
+            if (__float_as_uint(v[i]) >> 31) c |= 8u;
+            words[i >> 3] |= c << (4 * (i & 7));
         }
-        if (amax > 0.f) {
-            int ex = floor_log2_pos(amax) - 2;
-            ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
-            scale = static_cast<uint32_t>(ex + 127);
-            const float inv = __int_as_float((127 - ex) << 23);  // 2^-ex, exact (ex in [-127, 125])
-            uint32_t words[4] = {0, 0, 0, 0};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                uint32_t c = e2m1_code_of(fabsf(v[i] * inv));
-                if (__float_as_uint(v[i]) >> 31) c |= 8u;
-                words[i >> 3] |= c << (4 * (i & 7));
-            }
-            out = make_uint4(words[0], words[1], words[2], words[3]);
-        }
+        out = make_uint4(words[0], words[1], words[2], words[3]);
     }
     *reinterpret_cast<uint4*>(dst + co) = out;
     dst[so] = static_cast<uint8_t>(scale);
@@ -108,7 +117,7 @@ __global__ void rowscale_kernel(TiledMatrix M, uint8_t* __restrict__ rowscale, s
     if (n >= M.N) return;
     const uint8_t* src = M.base + static_cast<size_t>(e) * M.expert_bytes();
     int best = -1;
-    for (int b = 0; b < (M.K + 31) / 32; ++b) {
+    for (int b = 0; b < M.nb(); ++b) {
         size_t co, so;
         M.locate(n, b, co, so);
         const uint4 c = *reinterpret_cast<const uint4*>(src + co);
@@ -123,7 +132,7 @@ __global__ void export_kernel(TiledMatrix M, uint8_t* __restrict__ codes, uint8_
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     const int b = blockIdx.y;
     const int e = blockIdx.z;
-    const int nb = M.K / 32;
+    const int nb = M.nb();
     if (n >= M.N || b >= nb) return;
     size_t co, so;
     M.locate(n, b, co, so);

@@ -1,6 +1,6 @@
 // routing.cuh -- router (scores, top-k, softmax over the selected scores), the
-// expert histogram / prefix-sum schedule, the permute-and-gather that groups
-// token rows by expert, and the small finishing kernels.
+// expert histogram / prefix-sum schedule, the gather that groups token rows by
+// expert, and the small finishing kernels.
 //
 // Method (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card", §3.1 Le
 // Routeur): scores = W_router . h (+ optional bias), the top-k scores are
@@ -14,7 +14,7 @@
 
 namespace moe {
 
-constexpr int ROUTER_TOKENS = 32;   // tokens per router / permute block
+constexpr int ROUTER_TOKENS = 32;   // tokens per router tile
 constexpr int ROUTER_THREADS = 256;
 constexpr int ROUTER_KCHUNK = 64;
 constexpr int MAX_EXPERTS = 256;
@@ -31,135 +31,7 @@ __host__ __device__ inline size_t router_smem_bytes(int E) {
                             static_cast<size_t>(ROUTER_KCHUNK) * E + static_cast<size_t>(ROUTER_TOKENS) * (E + 1));
 }
 
-// One block scores 32 tokens against all E experts (fp32 accumulation over
-// K-chunks staged in shared memory), then one warp per token selects the top-k
-// with k rounds of warp arg-max and applies the softmax over the k selected
-// scores.  Also writes the block's expert histogram and zeroes the rows of the
-// output accumulator that the down GEMM adds into.
-template <typename TA>
-__global__ void __launch_bounds__(ROUTER_THREADS)
-router_kernel(const TA* __restrict__ x, const TA* __restrict__ wr, const float* __restrict__ bias, int T, int d,
-              int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ hist,
-              float* __restrict__ zero_rows, int zero_ld) {
-    extern __shared__ float rsm[];
-    float* xs = rsm;                                     // [32][65]
-    float* ws = xs + ROUTER_TOKENS * (ROUTER_KCHUNK + 1); // [64][E]
-    float* lg = ws + ROUTER_KCHUNK * E;                   // [32][E+1]
-    __shared__ int hist_s[MAX_EXPERTS];
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * ROUTER_TOKENS;
-    const int ntok = min(ROUTER_TOKENS, T - t0);
-    const int EPT = (E + 31) / 32;  // experts per lane
-
-    for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
-
-    float acc[MAX_EXPERTS / 32][4];
-#pragma unroll
-    for (int i = 0; i < MAX_EXPERTS / 32; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-
-    for (int kc = 0; kc < d; kc += ROUTER_KCHUNK) {
-        __syncthreads();
-        for (int i = tid; i < ROUTER_TOKENS * ROUTER_KCHUNK; i += ROUTER_THREADS) {
-            int t = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
-            float v = 0.f;
-            if (t < ntok && kc + kk < d) v = to_f32(x[static_cast<size_t>(t0 + t) * d + kc + kk]);
-            xs[t * (ROUTER_KCHUNK + 1) + kk] = v;
-        }
-        for (int i = tid; i < E * ROUTER_KCHUNK; i += ROUTER_THREADS) {
-            int e = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
-            float v = 0.f;
-            if (kc + kk < d) v = to_f32(wr[static_cast<size_t>(e) * d + kc + kk]);
-            ws[kk * E + e] = v;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int kk = 0; kk < ROUTER_KCHUNK; ++kk) {
-            float xv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xv[j] = xs[(warp * 4 + j) * (ROUTER_KCHUNK + 1) + kk];
-#pragma unroll
-            for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-                if (i < EPT) {
-                    const int e = lane + 32 * i;
-                    const float wv = (e < E) ? ws[kk * E + e] : 0.f;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(wv, xv[j], acc[i][j]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-        if (i < EPT) {
-            const int e = lane + 32 * i;
-            if (e < E) {
-                const float b = bias ? bias[e] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) lg[(warp * 4 + j) * (E + 1) + e] = acc[i][j] + b;
-            }
-        }
-    }
-    __syncthreads();
-
-    // top-k + softmax: warp w handles tokens 4w .. 4w+3
-    for (int j = 0; j < 4; ++j) {
-        const int tl = warp * 4 + j;
-        if (tl >= ntok) break;
-        const float* row = lg + tl * (E + 1);
-        uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-        float sel_v[MAX_TOPK];
-        int sel_e[MAX_TOPK];
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int be = 0x7FFFFFFF;
-            for (int i = 0; i < EPT; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E && !((taken >> i) & 1u)) {
-                    const float v = row[e];
-                    if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            sel_v[r] = bv;
-            sel_e[r] = be;
-        }
-        if (lane == 0) {
-            const float m = sel_v[0];
-            float den = 0.f;
-            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
-            const float inv = 1.f / den;
-            const int t = t0 + tl;
-            for (int r = 0; r < k; ++r) {
-                idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
-                w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
-                atomicAdd(&hist_s[sel_e[r]], 1);
-            }
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += ROUTER_THREADS) hist[static_cast<size_t>(blockIdx.x) * E + e] = hist_s[e];
-
-    // zero the accumulator rows of this block's tokens (zero_ld % 4 == 0)
-    if (zero_rows) {
-        const int nvec = zero_ld / 4;
-        for (int i = tid; i < ntok * nvec; i += ROUTER_THREADS) {
-            const int t = i / nvec, v = i % nvec;
-            reinterpret_cast<float4*>(zero_rows + static_cast<size_t>(t0 + t) * zero_ld)[v] =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
-}
-
-// Schedule slots written by schedule_kernel.
+// Schedule slots.
 enum : int {
     SCHED_UNITS_GU = 0,   // units of the gate/up GEMM
     SCHED_UNITS_DN = 1,   // units of the down GEMM
@@ -169,16 +41,25 @@ enum : int {
     SCHED_SLOTS = 8
 };
 
-struct ScheduleArgs {
-    int32_t* hist;       // [nblk][E]: per-block counts in, per-block exclusive prefix out
-    int nblk, E, BN;
-    int F_gu, F_dn;      // 128-row feature tiles of the two GEMMs
-    int KC_gu, KC_dn;    // 64-wide K chunks of the two GEMMs
-    int nsm;
-    int split_rows_cap;  // largest T*k for which the gate/up GEMM may split K
-    int max_units;
-    int32_t* offsets;    // [E+1]
-    int32_t* counts_out; // [E] or null
+struct RouterArgs {
+    const void* x;         // [T][d] act dtype
+    const void* wr;        // [E][d] act dtype
+    const float* bias;     // [E] or null
+    int T, d, E, k;
+    int S;                 // K splits = gridDim.y
+    double* part;          // [S][T][E] partial scores
+    int* tile_cnt;         // [tiles] arrival counters (zero between launches)
+    int* glob_cnt;         // [1] arrival counter (zero between launches)
+    int32_t* idx_out;      // [T][k]
+    float* w_out;          // [T][k]
+    int32_t* local_rank;   // [T][k] rank of the pair among earlier pairs of its tile with the same expert
+    int32_t* hist;         // [tiles][E] per-tile counts, turned into per-tile prefixes by the schedule
+    float* zero_rows;      // output accumulator rows to clear, [T][zero_ld], or null
+    int zero_ld;
+    // schedule
+    int BN, F_gu, F_dn, KC_gu, KC_dn, nsm, split_rows_cap, max_units;
+    int32_t* offsets;      // [E+1]
+    int32_t* counts_out;   // [E] or null
     int4* units_gu;
     int4* units_dn;
     int32_t* sched;
@@ -187,38 +68,35 @@ struct ScheduleArgs {
 __device__ inline int pick_split(int base, int nsm, int KC) {
     if (base <= 0 || base >= nsm) return 1;
     int best = 1;
-    double best_eff = 0.0;
+    float best_eff = 0.f;
     const int smax = min(8, max(1, KC / 4));
     for (int s = 1; s <= smax; ++s) {
         const int w = base * s;
-        const double eff = static_cast<double>(w) / (static_cast<double>((w + nsm - 1) / nsm) * nsm);
-        if (eff >= 0.9) return s;
-        if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+        const float eff = static_cast<float>(w) / static_cast<float>(((w + nsm - 1) / nsm) * nsm);
+        if (eff >= 0.9f) return s;
+        if (eff > best_eff + 1e-6f) { best_eff = eff; best = s; }
     }
     return best;
 }
 
-// Single block: per-expert totals and per-block prefixes of the router
-// histogram (one warp per expert, warp scans over the blocks), exclusive scan
-// of the totals into group offsets, choice of K splits, and the unit lists of
-// both expert GEMMs ordered (expert, token tile, feature tile, split).
-__global__ void __launch_bounds__(1024) schedule_kernel(ScheduleArgs a) {
-    __shared__ int cnt[MAX_EXPERTS];
-    __shared__ int off[MAX_EXPERTS + 1];
-    __shared__ int split_s[2];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int e = warp; e < a.E; e += 32) {
+// Run by the last router CTA to finish: per-expert totals and per-tile
+// prefixes of the histogram (warp scans over tiles), group offsets, K splits,
+// and the unit lists of both expert GEMMs, ordered (expert, token tile, feature
+// tile, split).
+__device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt, int* off, int* split_s) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int e = warp; e < a.E; e += nwarps) {
         int carry = 0;
-        for (int b0 = 0; b0 < a.nblk; b0 += 32) {
+        for (int b0 = 0; b0 < ntiles; b0 += 32) {
             const int b = b0 + lane;
-            const int v = (b < a.nblk) ? a.hist[static_cast<size_t>(b) * a.E + e] : 0;
+            const int v = (b < ntiles) ? __ldcg(a.hist + static_cast<size_t>(b) * a.E + e) : 0;
             int inc = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int n = __shfl_up_sync(0xffffffffu, inc, o);
                 if (lane >= o) inc += n;
             }
-            if (b < a.nblk) a.hist[static_cast<size_t>(b) * a.E + e] = carry + inc - v;
+            if (b < ntiles) a.hist[static_cast<size_t>(b) * a.E + e] = carry + inc - v;
             carry += __shfl_sync(0xffffffffu, inc, 31);
         }
         if (lane == 0) cnt[e] = carry;
@@ -257,19 +135,200 @@ __global__ void __launch_bounds__(1024) schedule_kernel(ScheduleArgs a) {
         int ubase = 0;
         for (int e = 0; e < a.E; ++e) {
             const int n = cnt[e];
-            const int mt = (n + a.BN - 1) / a.BN;
-            const int nu = mt * F * S;
+            const int nu = ((n + a.BN - 1) / a.BN) * F * S;
             for (int i = tid; i < nu; i += blockDim.x) {
                 const int u = ubase + i;
                 if (u >= a.max_units) break;
                 const int m = i / (F * S);
-                const int rem = i % (F * S);
-                const int ft = rem / S, sp = rem % S;
+                const int rem = i - m * F * S;
+                const int ft = rem / S, sp = rem - ft * S;
                 units[u] = make_int4(e, off[e] + m * a.BN, min(a.BN, n - m * a.BN), ft | (sp << 16));
             }
             ubase += nu;
         }
     }
+}
+
+// Grid (tiles of 32 tokens, S splits of K).  Each CTA accumulates the scores of
+// its 32 tokens x E experts over its K range: fp32 within a 64-wide chunk
+// staged in shared memory (bf16 x bf16 products are exact in fp32), fp64
+// across chunks.  The last CTA of a tile to finish sums the S partials in split
+// order (deterministic), adds the bias, and with one warp per token selects
+// the top-k by k rounds of warp arg-max (ties to the lower index) and applies
+// the softmax over the k selected scores; it also ranks the tile's (token,
+// slot) pairs within their expert, writes the tile histogram and zeroes the
+// output accumulator rows of its tokens.  The last tile to finish builds the
+// schedule (schedule_block).
+template <typename TA>
+__global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
+    extern __shared__ float rsm[];
+    float* xs = rsm;                                      // [32][65]
+    float* ws = xs + ROUTER_TOKENS * (ROUTER_KCHUNK + 1);  // [64][E]
+    float* lg = ws + ROUTER_KCHUNK * a.E;                  // [32][E+1]
+    __shared__ int hist_s[MAX_EXPERTS];
+    __shared__ int es[ROUTER_TOKENS * MAX_TOPK];
+    __shared__ int cnt_s[MAX_EXPERTS];
+    __shared__ int off_s[MAX_EXPERTS + 1];
+    __shared__ int split_s[2];
+    __shared__ int last_s;
+
+    const TA* x = static_cast<const TA*>(a.x);
+    const TA* wr = static_cast<const TA*>(a.wr);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, d = a.d, k = a.k;
+    const int tile = blockIdx.x, split = blockIdx.y;
+    const int ntiles = gridDim.x;
+    const int t0 = tile * ROUTER_TOKENS;
+    const int ntok = min(ROUTER_TOKENS, a.T - t0);
+    const int EPT = (E + 31) / 32;  // experts per lane
+    const int KCH = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
+    const int kc0 = split * KCH / a.S, kc1 = (split + 1) * KCH / a.S;
+
+    double tot[MAX_EXPERTS / 32][4];
+#pragma unroll
+    for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
+
+    for (int kc = kc0 * ROUTER_KCHUNK; kc < kc1 * ROUTER_KCHUNK && kc < d; kc += ROUTER_KCHUNK) {
+        __syncthreads();
+        for (int i = tid; i < ROUTER_TOKENS * ROUTER_KCHUNK; i += ROUTER_THREADS) {
+            const int t = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
+            float v = 0.f;
+            if (t < ntok && kc + kk < d) v = to_f32(x[static_cast<size_t>(t0 + t) * d + kc + kk]);
+            xs[t * (ROUTER_KCHUNK + 1) + kk] = v;
+        }
+        for (int i = tid; i < E * ROUTER_KCHUNK; i += ROUTER_THREADS) {
+            const int e = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
+            float v = 0.f;
+            if (kc + kk < d) v = to_f32(wr[static_cast<size_t>(e) * d + kc + kk]);
+            ws[kk * E + e] = v;
+        }
+        __syncthreads();
+        float acc[MAX_EXPERTS / 32][4];
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+        for (int kk = 0; kk < ROUTER_KCHUNK; ++kk) {
+            float xv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xv[j] = xs[(warp * 4 + j) * (ROUTER_KCHUNK + 1) + kk];
+#pragma unroll
+            for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+                if (i < EPT) {
+                    const int e = lane + 32 * i;
+                    const float wv = (e < E) ? ws[kk * E + e] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(wv, xv[j], acc[i][j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tot[i][j] += static_cast<double>(acc[i][j]);
+    }
+    // partial scores of this split
+#pragma unroll
+    for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+        const int e = lane + 32 * i;
+        if (i < EPT && e < E) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int tl = warp * 4 + j;
+                if (tl < ntok) a.part[(static_cast<size_t>(split) * a.T + t0 + tl) * E + e] = tot[i][j];
+            }
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = (atomicAdd(a.tile_cnt + tile, 1) == a.S - 1);
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
+
+    for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
+    for (int i = tid; i < ntok * E; i += ROUTER_THREADS) {
+        const int tl = i / E, e = i % E;
+        double s = 0.0;
+        for (int sp = 0; sp < a.S; ++sp) s += __ldcg(a.part + (static_cast<size_t>(sp) * a.T + t0 + tl) * E + e);
+        if (a.bias) s += a.bias[e];
+        lg[tl * (E + 1) + e] = static_cast<float>(s);
+    }
+    __syncthreads();
+
+    // top-k + softmax: warp w handles tokens 4w .. 4w+3
+    for (int j = 0; j < 4; ++j) {
+        const int tl = warp * 4 + j;
+        if (tl >= ntok) break;
+        const float* row = lg + tl * (E + 1);
+        uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
+        float sel_v[MAX_TOPK];
+        int sel_e[MAX_TOPK];
+        for (int r = 0; r < k; ++r) {
+            float bv = -INFINITY;
+            int be = 0x7FFFFFFF;
+            for (int i = 0; i < EPT; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E && !((taken >> i) & 1u)) {
+                    const float v = row[e];
+                    if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+            }
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            sel_v[r] = bv;
+            sel_e[r] = be;
+        }
+        if (lane == 0) {
+            const float m = sel_v[0];
+            float den = 0.f;
+            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+            const float inv = 1.f / den;
+            const int t = t0 + tl;
+            for (int r = 0; r < k; ++r) {
+                a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
+                a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
+                es[tl * k + r] = sel_e[r];
+                atomicAdd(&hist_s[sel_e[r]], 1);
+            }
+        }
+    }
+    __syncthreads();
+    // stable rank of each pair among the tile's earlier pairs with the same expert
+    for (int p = tid; p < ntok * k; p += ROUTER_THREADS) {
+        const int e = es[p];
+        int rank = 0;
+        for (int q = 0; q < p; ++q) rank += (es[q] == e);
+        a.local_rank[static_cast<size_t>(t0) * k + p] = rank;
+    }
+    for (int e = tid; e < E; e += ROUTER_THREADS) a.hist[static_cast<size_t>(tile) * E + e] = hist_s[e];
+    if (a.zero_rows) {
+        const int nvec = a.zero_ld / 4;
+        for (int i = tid; i < ntok * nvec; i += ROUTER_THREADS) {
+            const int t = i / nvec, v = i % nvec;
+            reinterpret_cast<float4*>(a.zero_rows + static_cast<size_t>(t0 + t) * a.zero_ld)[v] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    // the last tile builds the schedule
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = (atomicAdd(a.glob_cnt, 1) == ntiles - 1);
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    if (tid == 0) *a.glob_cnt = 0;
+    schedule_block(a, ntiles, cnt_s, off_s, split_s);
 }
 
 __device__ __forceinline__ __half to_half_sat(float v) {
@@ -307,50 +366,38 @@ template <> struct RowLoader<float> {
     }
 };
 
-// Same token blocking as router_kernel.  Each (token, slot) pair of the block
-// gets its grouped row: offsets[e] + (rows of e in earlier blocks) + (rank among
-// earlier pairs of e in this block), so rows of an expert are in (token, slot)
-// order.  The block then copies its token rows into the grouped activation
-// matrix as f16 (16-byte vectors) and, when the gate/up GEMM splits K, zeroes
-// the matching rows of its fp32 partial-sum buffer.
+constexpr int GATHER_WARPS = 8;
+
+// One warp per (token, slot) pair p = t*k + j: its grouped row is
+// offsets[e] + (rows of e in earlier tiles) + (its rank within its tile), so the
+// rows of an expert are in (token, slot) order.  The warp records the row's
+// token and routing weight and copies the token's activations into the grouped
+// matrix as f16 (16-byte vectors); when the gate/up GEMM splits K it also
+// zeroes the row of the fp32 partial-sum buffer.
 template <typename TA>
-__global__ void __launch_bounds__(ROUTER_THREADS)
-permute_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
-               const int32_t* __restrict__ hist_prefix, const int32_t* __restrict__ offsets, int T, int d, int E,
-               int k, int32_t* __restrict__ row_token, float* __restrict__ row_weight, __half* __restrict__ Xp,
-               float* __restrict__ GU, int gu_ld, const int32_t* __restrict__ sched) {
-    __shared__ int es[ROUTER_TOKENS * MAX_TOPK];
-    __shared__ int pos_s[ROUTER_TOKENS * MAX_TOPK];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * ROUTER_TOKENS;
-    const int npairs = min(ROUTER_TOKENS, T - t0) * k;
-    int e = -1;
-    if (tid < npairs) {
-        e = idx[static_cast<size_t>(t0) * k + tid];
-        es[tid] = e;
+__global__ void __launch_bounds__(GATHER_WARPS * 32)
+gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
+              const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
+              const int32_t* __restrict__ offsets, int T, int d, int E, int k, int32_t* __restrict__ row_token,
+              float* __restrict__ row_weight, __half* __restrict__ Xp, float* __restrict__ GU, int gu_ld,
+              const int32_t* __restrict__ sched) {
+    const int lane = threadIdx.x & 31;
+    const int p = blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
+    if (p >= T * k) return;
+    const int t = p / k;
+    const int e = idx[p];
+    const int pos = offsets[e] + tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+    if (lane == 0) {
+        row_token[pos] = t;
+        row_weight[pos] = w[p];
     }
-    __syncthreads();
-    if (tid < npairs) {
-        int rank = 0;
-        for (int q = 0; q < tid; ++q) rank += (es[q] == e);
-        const int pos = offsets[e] + hist_prefix[static_cast<size_t>(blockIdx.x) * E + e] + rank;
-        pos_s[tid] = pos;
-        row_token[pos] = t0 + tid / k;
-        row_weight[pos] = w[static_cast<size_t>(t0) * k + tid];
-    }
-    __syncthreads();
-    const bool split = sched[SCHED_SPLIT_GU] > 1;
+    const TA* src = x + static_cast<size_t>(t) * d;
+    uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<size_t>(pos) * d);
     const int nvec = d / 8;
-    for (int r = warp; r < npairs; r += ROUTER_THREADS / 32) {
-        const int t = t0 + r / k;
-        const int pos = pos_s[r];
-        const TA* src = x + static_cast<size_t>(t) * d;
-        uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<size_t>(pos) * d);
-        for (int v = lane; v < nvec; v += 32) dst[v] = RowLoader<TA>::load8(src + v * 8);
-        if (split) {
-            float4* g = reinterpret_cast<float4*>(GU + static_cast<size_t>(pos) * gu_ld);
-            for (int v = lane; v < gu_ld / 4; v += 32) g[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    for (int v = lane; v < nvec; v += 32) dst[v] = RowLoader<TA>::load8(src + v * 8);
+    if (sched[SCHED_SPLIT_GU] > 1) {
+        float4* g = reinterpret_cast<float4*>(GU + static_cast<size_t>(pos) * gu_ld);
+        for (int v = lane; v < gu_ld / 4; v += 32) g[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 

@@ -128,7 +128,8 @@ def check_layer(cfg, x, wr, bias, y, idx, w, counts, ox: OracleExperts, n_sample
     _, idx_ref, w_ref, counts_ref = oracle.router(x, wr, bias, cfg.top_k)
     np.testing.assert_array_equal(idx, idx_ref)
     np.testing.assert_array_equal(counts, counts_ref)
-    assert np.abs(w - w_ref).max() <= W_ABS_TOL
+    w_err = np.abs(w - w_ref).max()
+    assert w_err <= W_ABS_TOL, ("routing weight error", w_err)
     tok = sample_tokens(idx_ref, counts_ref, n_sample)
     q = ox.ensure(np.unique(idx_ref[tok]))
     y_ref = oracle.moe_forward(x, q, idx_ref, w_ref, tokens=tok)
