@@ -48,10 +48,10 @@ namespace moe {
 constexpr int GEMM_DEC_WARPS = 16;
 constexpr int GEMM_THREADS = (2 + GEMM_DEC_WARPS) * 32;
 constexpr int GEMM_MAX_STAGES = 16;
-constexpr int GEMM_A_SLOTS = 4;
+constexpr int GEMM_MAX_A_SLOTS = 7;
 constexpr int GEMM_A_COLS = 64;                               // TMEM columns per A slot
-constexpr int GEMM_D_COL0 = GEMM_A_SLOTS * GEMM_A_COLS;       // first accumulator column
 constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_GROUP = 2;                                 // stages a decoder warp handles per round
 constexpr int GEMM_W_STAGE = 128 * 4 * 17;                    // weight bytes per stage (max)
 constexpr int GEMM_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
@@ -65,6 +65,7 @@ struct GemmParams {
     int K;                    // contraction length
     int BN;                   // token rows per tile (MMA N), multiple of 16
     int stages;
+    int a_slots;              // TMEM A slots (GEMM_A_COLS columns each); accumulators follow them
     uint32_t idesc;
     __half* H;                // MODE 0 output [rows][N]
     float* GU;                // MODE 0 split partials [rows][2N]
@@ -81,8 +82,14 @@ __host__ __device__ inline size_t gemm_b_stage_bytes(int mode, int BN) {
     return static_cast<size_t>(BN) * 128 * (mode == 0 ? 1 : 2);
 }
 __host__ inline size_t gemm_stage_bytes(int mode, int BN) { return GEMM_W_STAGE + gemm_b_stage_bytes(mode, BN); }
+// A slots that fit in TMEM beside the accumulators (2*BN columns for gate/up, BN for down).
+__host__ inline int gemm_a_slots(int mode, int BN) {
+    const int d_cols = mode == 0 ? 2 * BN : BN;
+    int n = (GEMM_TMEM_COLS - d_cols) / GEMM_A_COLS;
+    return n > GEMM_MAX_A_SLOTS ? GEMM_MAX_A_SLOTS : n;
+}
 __host__ inline size_t gemm_smem_bytes(int mode, int BN, int stages) {
-    size_t b = 1024 + stages * gemm_stage_bytes(mode, BN) + (2 * stages + 2 * GEMM_A_SLOTS + 3) * 8 + 64;
+    size_t b = 1024 + stages * gemm_stage_bytes(mode, BN) + (2 * stages + 2 * GEMM_MAX_A_SLOTS + 3) * 8 + 64;
     return b < static_cast<size_t>(GEMM_MIN_SMEM) ? static_cast<size_t>(GEMM_MIN_SMEM) : b;
 }
 
@@ -103,9 +110,11 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
     const uint32_t bar0 = w_sm + S * GEMM_W_STAGE;                // barriers (8-byte aligned)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    const int NA = p.a_slots;
+    const uint32_t d_col0 = static_cast<uint32_t>(NA * GEMM_A_COLS);   // first accumulator column
     auto afull_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
-    auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * S + GEMM_A_SLOTS + a); };
-    const uint32_t accf_bar = bar0 + 8u * (2 * S + 2 * GEMM_A_SLOTS);
+    auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * S + GEMM_MAX_A_SLOTS + a); };
+    const uint32_t accf_bar = bar0 + 8u * (2 * S + 2 * GEMM_MAX_A_SLOTS);
     const uint32_t acce_bar = accf_bar + 8u;
     const uint32_t drain_bar = acce_bar + 8u;
     uint8_t* ctl = smem_raw + (drain_bar + 8u - raw);
@@ -117,7 +126,7 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), GEMM_DEC_WARPS + 1);  // decoder warps + 1 MMA commit
         }
-        for (int a = 0; a < GEMM_A_SLOTS; ++a) {
+        for (int a = 0; a < NA; ++a) {
             mbar_init(afull_bar(a), GEMM_DEC_WARPS);
             mbar_init(aempty_bar(a), 1);
         }
@@ -200,17 +209,17 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                     for (int i = 0; i < ksteps; ++i) {
                         const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
                         if (MODE == 0) {
-                            mma_f16_ts(tmem + GEMM_D_COL0, acol + 8 * i, bd + 2 * i, p.idesc, acc);
-                            mma_f16_ts(tmem + GEMM_D_COL0 + p.BN, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts(tmem + d_col0, acol + 8 * i, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts(tmem + d_col0 + p.BN, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
                         } else {
                             const uint64_t bdi = bd + (((i >> 2) * b_sub) >> 4) + 2 * (i & 3);
-                            mma_f16_ts(tmem + GEMM_D_COL0, acol + 8 * i, bdi, p.idesc, acc);
+                            mma_f16_ts(tmem + d_col0, acol + 8 * i, bdi, p.idesc, acc);
                         }
                     }
                     tc_commit(aempty_bar(a));
                     tc_commit(empty_bar(s));
                     if (++s == S) { s = 0; ph ^= 1u; }
-                    if (++a == GEMM_A_SLOTS) { a = 0; aph ^= 1u; }
+                    if (++a == NA) { a = 0; aph ^= 1u; }
                 }
                 tc_commit(accf_bar);
                 acc_ph ^= 1u;
@@ -250,40 +259,65 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                     rs_mine = rs0;
                 }
             }
-            for (int c = c0; c < c1; ++c) {
-                const int nbc = p.M.blocks_in_chunk(c);
-                const bool mine = warp_rows && hb < nbc;
-                bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
-                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-                uint4 cw = make_uint4(0, 0, 0, 0);
-                int sc = 127;
-                if (mine) {
-                    const uint8_t* ws = smem_raw + (w_sm + s * GEMM_W_STAGE - raw) + mat * 17 * nbc * rf;
-                    cw = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
-                    sc = ws[16 * nbc * rf + hb * rf + row];
+            // Stages are taken GEMM_GROUP at a time so that one round of waits, shared
+            // loads and TMEM-store completion covers several stages.
+            for (int c = c0; c < c1 && ok; c += GEMM_GROUP) {
+                const int g = min(GEMM_GROUP, c1 - c);
+                uint4 cw[GEMM_GROUP];
+                int sc[GEMM_GROUP];
+                bool mine[GEMM_GROUP];
+                int aslot[GEMM_GROUP];
+#pragma unroll
+                for (int j = 0; j < GEMM_GROUP; ++j) {
+                    if (j >= g) break;
+                    const int nbc = p.M.blocks_in_chunk(c + j);
+                    mine[j] = warp_rows && hb < nbc;
+                    const bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
+                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                    cw[j] = make_uint4(0, 0, 0, 0);
+                    sc[j] = 127;
+                    if (mine[j]) {
+                        const uint8_t* ws = smem_raw + (w_sm + s * GEMM_W_STAGE - raw) + mat * 17 * nbc * rf;
+                        cw[j] = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
+                        sc[j] = ws[16 * nbc * rf + hb * rf + row];
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty_bar(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));
-                if (++s == S) { s = 0; ph ^= 1u; }
-
-                w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
-                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                if (!ok) break;
+#pragma unroll
+                for (int j = 0; j < GEMM_GROUP; ++j) {
+                    if (j >= g) break;
+                    const bool w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
+                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                    aslot[j] = a;
+                    if (++a == NA) { a = 0; aph ^= 1u; }
+                }
+                if (!ok) break;
                 tc_fence_after();
-                if (mine) {
-                    uint32_t r[16];
-                    const uint32_t m1 = f16_pow2_bits(sc - rs_mine);
-                    const uint32_t m2 = m1 | (m1 << 16);
-                    e2m1x8_to_f16x8(cw.x, m2, r[0], r[1], r[2], r[3]);
-                    e2m1x8_to_f16x8(cw.y, m2, r[4], r[5], r[6], r[7]);
-                    e2m1x8_to_f16x8(cw.z, m2, r[8], r[9], r[10], r[11]);
-                    e2m1x8_to_f16x8(cw.w, m2, r[12], r[13], r[14], r[15]);
-                    tmem_st16(tmem + lane_addr + a * GEMM_A_COLS + tcol, r);
-                    tmem_wait_st();
+#pragma unroll
+                for (int j = 0; j < GEMM_GROUP; ++j) {
+                    if (j >= g) break;
+                    if (mine[j]) {
+                        uint32_t r[16];
+                        const uint32_t m1 = f16_pow2_bits(sc[j] - rs_mine);
+                        const uint32_t m2 = m1 | (m1 << 16);
+                        e2m1x8_to_f16x8(cw[j].x, m2, r[0], r[1], r[2], r[3]);
+                        e2m1x8_to_f16x8(cw[j].y, m2, r[4], r[5], r[6], r[7]);
+                        e2m1x8_to_f16x8(cw[j].z, m2, r[8], r[9], r[10], r[11]);
+                        e2m1x8_to_f16x8(cw[j].w, m2, r[12], r[13], r[14], r[15]);
+                        tmem_st16(tmem + lane_addr + aslot[j] * GEMM_A_COLS + tcol, r);
+                    }
                 }
+                if (warp_rows) tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(afull_bar(a));
-                if (++a == GEMM_A_SLOTS) { a = 0; aph ^= 1u; }
+                if (lane == 0) {
+#pragma unroll
+                    for (int j = 0; j < GEMM_GROUP; ++j)
+                        if (j < g) mbar_arrive(afull_bar(aslot[j]));
+                }
             }
             if (!ok) break;
 
@@ -300,10 +334,10 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 for (int col = role * 8; col < p.BN; col += 32) {
                     if (col >= nvalid) break;
                     uint32_t g[8];
-                    tmem_ld8(tmem + lane_addr + GEMM_D_COL0 + col, g);
+                    tmem_ld8(tmem + lane_addr + d_col0 + col, g);
                     if (MODE == 0) {
                         uint32_t v[8];
-                        tmem_ld8(tmem + lane_addr + GEMM_D_COL0 + p.BN + col, v);
+                        tmem_ld8(tmem + lane_addr + d_col0 + p.BN + col, v);
                         tmem_wait_ld();
                         if (nsplit == 1) {
 #pragma unroll

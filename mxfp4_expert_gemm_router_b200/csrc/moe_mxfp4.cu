@@ -502,6 +502,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.K = d;
     gp.BN = BN;
     gp.stages = stages_for(0, BN);
+    gp.a_slots = gemm_a_slots(0, BN);
     gp.idesc = idesc_f16_f32(128, BN);
     gp.H = h->H;
     gp.GU = h->GU;
@@ -532,6 +533,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.N = d;
     dp.K = f;
     dp.stages = stages_for(1, BN);
+    dp.a_slots = gemm_a_slots(1, BN);
     dp.H = nullptr;
     dp.GU = nullptr;
     dp.yacc = acc;

@@ -20,9 +20,30 @@ constexpr int ROUTER_KCHUNK = 64;
 constexpr int MAX_EXPERTS = 256;
 constexpr int MAX_TOPK = 8;
 
-template <typename T> __device__ __forceinline__ float to_f32(T v);
-template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+// Eight consecutive activation-dtype elements held raw in registers.
+template <typename TA> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { v = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ float get(int i) const {
+        const uint32_t w = (&v.x)[i >> 1];
+        return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = *reinterpret_cast<const float4*>(p);
+        b = *reinterpret_cast<const float4*>(p + 4);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ float get(int i) const {
+        const float4& q = i < 4 ? a : b;
+        const int j = i & 3;
+        return j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w;
+    }
+};
 
 // Dynamic shared memory of router_kernel (floats): x chunk [32][65], router
 // chunk [64][E], scores [32][E+1].
@@ -190,21 +211,43 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
 #pragma unroll
         for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
 
-    for (int kc = kc0 * ROUTER_KCHUNK; kc < kc1 * ROUTER_KCHUNK && kc < d; kc += ROUTER_KCHUNK) {
-        __syncthreads();
-        for (int i = tid; i < ROUTER_TOKENS * ROUTER_KCHUNK; i += ROUTER_THREADS) {
-            const int t = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
-            float v = 0.f;
-            if (t < ntok && kc + kk < d) v = to_f32(x[static_cast<size_t>(t0 + t) * d + kc + kk]);
-            xs[t * (ROUTER_KCHUNK + 1) + kk] = v;
+    // Each thread owns one 8-element group of the x chunk (token tid/8) and up to
+    // EPT groups of the router chunk (expert (tid + 256 i)/8); the next chunk is
+    // loaded into registers while the current one is multiplied.
+    const int xt = tid >> 3, xv8 = (tid & 7) * 8;
+    Raw8<TA> xr, wrr[MAX_EXPERTS / 32];
+    auto load_chunk = [&](int kc) {
+        if (xt < ntok && kc + xv8 < d) xr.load(x + static_cast<size_t>(t0 + xt) * d + kc + xv8);
+        else xr.zero();
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+            if (i < EPT) {
+                const int idx = tid + ROUTER_THREADS * i;
+                const int e = idx >> 3, k8 = (idx & 7) * 8;
+                if (e < E && kc + k8 < d) wrr[i].load(wr + static_cast<size_t>(e) * d + kc + k8);
+                else wrr[i].zero();
+            }
         }
-        for (int i = tid; i < E * ROUTER_KCHUNK; i += ROUTER_THREADS) {
-            const int e = i / ROUTER_KCHUNK, kk = i % ROUTER_KCHUNK;
-            float v = 0.f;
-            if (kc + kk < d) v = to_f32(wr[static_cast<size_t>(e) * d + kc + kk]);
-            ws[kk * E + e] = v;
+    };
+    if (kc0 < kc1) load_chunk(kc0 * ROUTER_KCHUNK);
+    for (int c = kc0; c < kc1; ++c) {
+        const int kc = c * ROUTER_KCHUNK;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xs[xt * (ROUTER_KCHUNK + 1) + xv8 + j] = xr.get(j);
+#pragma unroll
+        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+            if (i < EPT) {
+                const int idx = tid + ROUTER_THREADS * i;
+                const int e = idx >> 3, k8 = (idx & 7) * 8;
+                if (e < E) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) ws[(k8 + j) * E + e] = wrr[i].get(j);
+                }
+            }
         }
         __syncthreads();
+        if (c + 1 < kc1) load_chunk(kc + ROUTER_KCHUNK);
         float acc[MAX_EXPERTS / 32][4];
 #pragma unroll
         for (int i = 0; i < MAX_EXPERTS / 32; ++i)
@@ -253,8 +296,20 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
     for (int i = tid; i < ntok * E; i += ROUTER_THREADS) {
         const int tl = i / E, e = i % E;
+        // partials summed in split order (deterministic), four loads in flight
         double s = 0.0;
-        for (int sp = 0; sp < a.S; ++sp) s += __ldcg(a.part + (static_cast<size_t>(sp) * a.T + t0 + tl) * E + e);
+        const double* pp = a.part + static_cast<size_t>(t0 + tl) * E + e;
+        const size_t pstride = static_cast<size_t>(a.T) * E;
+        int sp = 0;
+        for (; sp + 4 <= a.S; sp += 4) {
+            const double p0 = __ldcg(pp + (sp + 0) * pstride), p1 = __ldcg(pp + (sp + 1) * pstride);
+            const double p2 = __ldcg(pp + (sp + 2) * pstride), p3 = __ldcg(pp + (sp + 3) * pstride);
+            s += p0;
+            s += p1;
+            s += p2;
+            s += p3;
+        }
+        for (; sp < a.S; ++sp) s += __ldcg(pp + sp * pstride);
         if (a.bias) s += a.bias[e];
         lg[tl * (E + 1) + e] = static_cast<float>(s);
     }
