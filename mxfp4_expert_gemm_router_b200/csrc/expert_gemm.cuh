@@ -153,81 +153,99 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            int pend_ph[GEMM_MAX_STAGES];
-            for (int i = 0; i < GEMM_MAX_STAGES; ++i) pend_ph[i] = -1;
-            bool skip = p.skip_first_copy != 0;
-            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-                const int4 U = p.units[u];
-                const int ft = U.w & 0xFFFF, sp = U.w >> 16;
-                const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
-                const int rf = min(128, p.N - ft * 128);
-                const uint8_t* we = p.wpack + static_cast<size_t>(U.x) * expert_bytes;
-                for (int c = c0; c < c1; ++c) {
-                    if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto producer_done;
-                    if (skip) {
-                        skip = false;  // test hook: this stage is never filled
-                    } else {
-                        const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
-                        const int k0 = c * KSTAGE;
-                        const bool second = (MODE == 1) && (k0 + 64 < p.K);
-                        mbar_arrive_expect_tx(full_bar(s), wb + (second ? 2u : 1u) * b_sub);
-                        bulk_g2s(w_sm + s * GEMM_W_STAGE, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
-                        tma_load_2d(b_sm + s * b_bytes, &tmap_b, k0, U.y, full_bar(s));
-                        if (second) tma_load_2d(b_sm + s * b_bytes + b_sub, &tmap_b, k0 + 64, U.y, full_bar(s));
-                        pend_ph[s] = static_cast<int>(ph);
-                    }
-                    if (++s == S) { s = 0; ph ^= 1u; }
+        // Warp-uniform loop; one elected lane issues each copy.
+        int s = 0;
+        uint32_t ph = 0;
+        int pend_ph[GEMM_MAX_STAGES];
+        for (int i = 0; i < GEMM_MAX_STAGES; ++i) pend_ph[i] = -1;
+        bool skip = p.skip_first_copy != 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int ft = U.w & 0xFFFF, sp = U.w >> 16;
+            const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
+            const int rf = min(128, p.N - ft * 128);
+            const uint8_t* we = p.wpack + static_cast<size_t>(U.x) * expert_bytes;
+            for (int c = c0; c < c1; ++c) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
+                if (skip) {
+                    skip = false;  // test hook: this stage is never filled
+                } else {
+                    const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
+                    const int k0 = c * KSTAGE;
+                    const bool second = (MODE == 1) && (k0 + 64 < p.K);
+                    mbar_arrive_expect_tx_warp(full_bar(s), wb + (second ? 2u : 1u) * b_sub);
+                    bulk_g2s_warp(w_sm + s * GEMM_W_STAGE, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
+                    tma_load_2d_warp(b_sm + s * b_bytes, &tmap_b, k0, U.y, full_bar(s));
+                    if (second) tma_load_2d_warp(b_sm + s * b_bytes + b_sub, &tmap_b, k0 + 64, U.y, full_bar(s));
+                    pend_ph[s] = static_cast<int>(ph);
                 }
+                if (++s == S) { s = 0; ph ^= 1u; }
             }
-        producer_done:
-            // copies still in flight must land before the CTA exits
+        }
+        // copies still in flight must land before the CTA exits
+        if (lane == 0)
             for (int i = 0; i < S; ++i)
                 if (pend_ph[i] >= 0) mbar_wait_drain(full_bar(i), static_cast<uint32_t>(pend_ph[i]), 200000000ull);
-        }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            int s = 0, a = 0;
-            uint32_t ph = 0, aph = 0, acc_ph = 0;
-            const uint64_t bdesc0 = sw128_kmajor_desc(b_sm);
-            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-                const int4 U = p.units[u];
-                const int sp = U.w >> 16;
-                const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
-                if (!mbar_wait_bounded(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns)) goto mma_done;
+        // The whole warp runs the loop so descriptors and TMEM addresses stay
+        // warp-uniform; elect.sync inside each tcgen05 instruction picks the lane
+        // that issues it.  K steps are unrolled with compile-time offsets.
+        int s = 0, a = 0;
+        uint32_t ph = 0, aph = 0, acc_ph = 0;
+        const uint64_t bdesc0 = sw128_kmajor_desc(b_sm);
+        const uint32_t dg = tmem + d_col0;
+        const uint32_t du = dg + p.BN;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int sp = U.w >> 16;
+            const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns));
+            if (!ok) break;
+            for (int c = c0; c < c1; ++c) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
                 tc_fence_after();
-                for (int c = c0; c < c1; ++c) {
-                    if (!mbar_wait_bounded(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
-                    if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) goto mma_done;
-                    tc_fence_after();
-                    const int ksteps = 2 * p.M.blocks_in_chunk(c);
-                    const uint64_t bd = bdesc0 + ((static_cast<uint64_t>(s) * b_bytes) >> 4);
-                    const uint32_t acol = tmem + a * GEMM_A_COLS;
-                    for (int i = 0; i < ksteps; ++i) {
-                        const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
-                        if (MODE == 0) {
-                            mma_f16_ts(tmem + d_col0, acol + 8 * i, bd + 2 * i, p.idesc, acc);
-                            mma_f16_ts(tmem + d_col0 + p.BN, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
-                        } else {
-                            const uint64_t bdi = bd + (((i >> 2) * b_sub) >> 4) + 2 * (i & 3);
-                            mma_f16_ts(tmem + d_col0, acol + 8 * i, bdi, p.idesc, acc);
+                const int ksteps = 2 * p.M.blocks_in_chunk(c);
+                const uint64_t bd = bdesc0 + ((static_cast<uint64_t>(s) * b_bytes) >> 4);
+                const uint32_t acol = tmem + a * GEMM_A_COLS;
+                const uint32_t acc0 = c > c0 ? 1u : 0u;
+                if (MODE == 0) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < ksteps) {
+                            const uint32_t acc = i > 0 ? 1u : acc0;
+                            mma_f16_ts_warp(dg, acol + 8 * i, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts_warp(du, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
                         }
                     }
-                    tc_commit(aempty_bar(a));
-                    tc_commit(empty_bar(s));
-                    if (++s == S) { s = 0; ph ^= 1u; }
-                    if (++a == NA) { a = 0; aph ^= 1u; }
+                } else {
+                    const uint64_t bd1 = bd + (b_sub >> 4);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (i < ksteps) {
+                            const uint32_t acc = i > 0 ? 1u : acc0;
+                            mma_f16_ts_warp(dg, acol + 8 * i, (i < 4 ? bd : bd1) + 2 * (i & 3), p.idesc, acc);
+                        }
+                    }
                 }
-                tc_commit(accf_bar);
-                acc_ph ^= 1u;
+                tc_commit_warp(aempty_bar(a));
+                tc_commit_warp(empty_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
+                if (++a == NA) { a = 0; aph ^= 1u; }
             }
-        mma_done:
-            tc_commit(drain_bar);
-            mbar_wait_drain(drain_bar, 0, 200000000ull);
+            if (!ok) break;
+            tc_commit_warp(accf_bar);
+            acc_ph ^= 1u;
         }
+        tc_commit_warp(drain_bar);
+        if (lane == 0) mbar_wait_drain(drain_bar, 0, 200000000ull);
+        __syncwarp();
     } else {
         // ---------------------------------------------------------- decoders + epilogue
         const int q = warp & 3;               // TMEM lane quadrant (hardware rule: warp % 4)
