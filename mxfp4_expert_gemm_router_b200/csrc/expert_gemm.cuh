@@ -319,12 +319,12 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                     if (j >= g) break;
                     if (mine[j]) {
                         uint32_t r[16];
-                        const uint32_t m1 = f16_decode_mult_bits(sc[j] - rs_mine);
+                        const uint32_t m1 = f16_pow2_bits(sc[j] - rs_mine);
                         const uint32_t m2 = m1 | (m1 << 16);
-                        mxfp4_word_to_f16x8(cw[j].x, m2, r[0], r[1], r[2], r[3]);
-                        mxfp4_word_to_f16x8(cw[j].y, m2, r[4], r[5], r[6], r[7]);
-                        mxfp4_word_to_f16x8(cw[j].z, m2, r[8], r[9], r[10], r[11]);
-                        mxfp4_word_to_f16x8(cw[j].w, m2, r[12], r[13], r[14], r[15]);
+                        e2m1x8_to_f16x8(cw[j].x, m2, r[0], r[1], r[2], r[3]);
+                        e2m1x8_to_f16x8(cw[j].y, m2, r[4], r[5], r[6], r[7]);
+                        e2m1x8_to_f16x8(cw[j].z, m2, r[8], r[9], r[10], r[11]);
+                        e2m1x8_to_f16x8(cw[j].w, m2, r[12], r[13], r[14], r[15]);
                         tmem_st16(tmem + lane_addr + aslot[j] * GEMM_A_COLS + tcol, r);
                     }
                 }

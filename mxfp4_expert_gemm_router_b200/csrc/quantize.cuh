@@ -15,19 +15,13 @@
 // blocks into chunks of BPC blocks (the last chunk may hold fewer, nb_c).  For
 // each (tile, chunk) the bytes of the NM interleaved matrices (gate and up, or
 // down alone) are contiguous, matrix after matrix:
-//     codes  [nb_c blocks][rf rows][16 B]   (decode-ready bit order, below)
+//     codes  [nb_c blocks][rf rows][16 B]   (even element in the low nibble)
 //     scales [nb_c blocks][rf rows]          (E8M0 bytes)
 // i.e. 17 bytes per row per block, exactly 4.25 bits per parameter with no
-// padding.  Within each 32-bit word (elements 8w..8w+7 of the block) the four
-// code bits are placed for an in-register decode on the integer pipes rather
-// than the conversion unit: element e keeps its three magnitude bits (e1 e0 m)
-// at bits mag_pos(e)..+2 and its sign at sign_pos(e), chosen so that four
-// rotate-and-mask steps put elements (2j, 2j+1) at bits 9..11 / 15 and 25..27 /
-// 31 -- the exponent-low, mantissa-top and sign bits of an f16 pair, whose
-// value is then the E2M1 value times 2^-14 (f16 subnormals included).
-// One further byte per row, the largest scale over the row's non-zero blocks
-// ("row scale", 127 if none), lets the GEMM decode each block as f16 relative
-// to its row and apply 2^(row scale - 127) in fp32 after accumulation.
+// padding.  One further byte per row, the largest scale over the row's
+// non-zero blocks ("row scale", 127 if none), lets the GEMM decode each block
+// as f16 relative to its row and apply 2^(row scale - 127) in fp32 after
+// accumulation.
 #pragma once
 #include <cstdint>
 
@@ -61,20 +55,6 @@ struct TiledMatrix {
         scale_off = base_m + 16 * static_cast<size_t>(nbc) * rf + h * rf + r;
     }
 };
-
-// Bit positions of element e (0..7) of a 32-bit code word.
-__host__ __device__ __forceinline__ int mag_pos(int e) { return (e & 1) * 16 + 9 - 3 * (e >> 1); }
-__host__ __device__ __forceinline__ int sign_pos(int e) {
-    const int lo = (e >> 1) == 0 ? 15 : (e >> 1) == 1 ? 12 : (e >> 1) == 2 ? 14 : 13;
-    return (e & 1) * 16 + lo;
-}
-__host__ __device__ __forceinline__ uint32_t place_code(uint32_t code, int e) {
-    return ((code & 7u) << mag_pos(e)) | (((code >> 3) & 1u) << sign_pos(e));
-}
-__host__ __device__ __forceinline__ uint32_t extract_code(uint32_t word, int e) {
-    return ((word >> mag_pos(e)) & 7u) | (((word >> sign_pos(e)) & 1u) << 3);
-}
-constexpr uint32_t CODE_MAG_MASK = 0x0FFF0FFFu;  // all magnitude bits of a word
 
 __device__ __forceinline__ int floor_log2_pos(float a) {
     const uint32_t u = __float_as_uint(a);
@@ -121,7 +101,7 @@ __global__ void quantize_kernel(const float* __restrict__ W, size_t w_expert_str
         for (int i = 0; i < 32; ++i) {
             uint32_t c = e2m1_code_of(fabsf(v[i] * inv));
             if (__float_as_uint(v[i]) >> 31) c |= 8u;
-            words[i >> 3] |= place_code(c, i & 7);
+            words[i >> 3] |= c << (4 * (i & 7));
         }
         out = make_uint4(words[0], words[1], words[2], words[3]);
     }
@@ -141,14 +121,13 @@ __global__ void rowscale_kernel(TiledMatrix M, uint8_t* __restrict__ rowscale, s
         size_t co, so;
         M.locate(n, b, co, so);
         const uint4 c = *reinterpret_cast<const uint4*>(src + co);
-        const uint32_t nz = (c.x | c.y | c.z | c.w) & CODE_MAG_MASK;
+        const uint32_t nz = (c.x | c.y | c.z | c.w) & 0x77777777u;
         if (nz) best = max(best, static_cast<int>(src[so]));
     }
     rowscale[static_cast<size_t>(e) * rs_expert_stride + n] = static_cast<uint8_t>(best < 0 ? 127 : best);
 }
 
-// Tiled -> canonical: codes [E][N][K/2] (even element in the low nibble),
-// scales [E][N][K/32].
+// Tiled -> canonical: codes [E][N][K/2], scales [E][N][K/32].
 __global__ void export_kernel(TiledMatrix M, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     const int b = blockIdx.y;
@@ -159,18 +138,8 @@ __global__ void export_kernel(TiledMatrix M, uint8_t* __restrict__ codes, uint8_
     M.locate(n, b, co, so);
     const uint8_t* src = M.base + static_cast<size_t>(e) * M.expert_bytes();
     const size_t row = static_cast<size_t>(e) * M.N + n;
-    const uint4 in = *reinterpret_cast<const uint4*>(src + co);
-    const uint32_t win[4] = {in.x, in.y, in.z, in.w};
-    uint32_t wout[4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t o = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o |= extract_code(win[w], e) << (4 * e);
-        wout[w] = o;
-    }
     *reinterpret_cast<uint4*>(codes + row * (M.K / 2) + static_cast<size_t>(b) * 16) =
-        make_uint4(wout[0], wout[1], wout[2], wout[3]);
+        *reinterpret_cast<const uint4*>(src + co);
     scales[row * nb + b] = src[so];
 }
 

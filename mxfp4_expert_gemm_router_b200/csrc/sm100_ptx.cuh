@@ -230,39 +230,32 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 }
 
 // ------------------------------------------------------------------ MXFP4 decode
-// One 32-bit code word in the decode-ready order (see quantize.cuh) -> four f16x2
-// words (elements 2j, 2j+1 in word j).  Rotate-and-mask puts each code's sign at
-// f16 bit 15 and its magnitude bits (e1 e0 m) at bits 11..9, which makes the f16
-// value the E2M1 value times 2^-14; one f16x2 multiply by `mult2` = 2^(14+rel)
-// in both halves then yields value * 2^rel exactly (the product is exact while
-// it stays representable).  Only integer-pipe logic and one f16x2 multiply per
-// pair -- no conversion-unit instructions.
-__device__ __forceinline__ uint32_t rotl32(uint32_t x, int r) { return __funnelshift_l(x, x, r); }
-__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ void mxfp4_word_to_f16x8(uint32_t w, uint32_t mult2, uint32_t& o0, uint32_t& o1,
-                                                    uint32_t& o2, uint32_t& o3) {
-    constexpr uint32_t FULL = 0x8E008E00u, MAG = 0x0E000E00u, SGN = 0x80008000u;
-    const uint32_t p0 = w & FULL;
-    const uint32_t p1 = rotl32(w, 3) & FULL;
-    const uint32_t p2 = (rotl32(w, 6) & MAG) | (rotl32(w, 1) & SGN);
-    const uint32_t p3 = (rotl32(w, 9) & MAG) | (rotl32(w, 2) & SGN);
-    o0 = hmul2_bits(p0, mult2);
-    o1 = hmul2_bits(p1, mult2);
-    o2 = hmul2_bits(p2, mult2);
-    o3 = hmul2_bits(p3, mult2);
+// Four bytes = eight E2M1 codes (even element in the low nibble) -> four f16x2
+// words, each multiplied by the f16x2 block multiplier `mult2`.  The E2M1 to f16
+// conversion is exact; multiplying by a power of two is exact while the result
+// stays in the f16 range (the multiplier is at most 1).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t mult2, uint32_t& o0, uint32_t& o1,
+                                                uint32_t& o2, uint32_t& o3) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 t0, t1, t2, t3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 t0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 t1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 t2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 t3, b3;\n\t"
+        "mul.rn.f16x2 %0, t0, %5;\n\t"
+        "mul.rn.f16x2 %1, t1, %5;\n\t"
+        "mul.rn.f16x2 %2, t2, %5;\n\t"
+        "mul.rn.f16x2 %3, t3, %5;\n\t}"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(w), "r"(mult2));
 }
 
-// f16 bit pattern of 2^(14+rel) for rel <= 0 (normal down to 2^-14, subnormal
-// down to 2^-24, zero below).
-__device__ __forceinline__ uint32_t f16_decode_mult_bits(int rel) {
+// f16 bit pattern of 2^rel for rel <= 0 (normal down to 2^-14, subnormal down to
+// 2^-24, zero below).
+__device__ __forceinline__ uint32_t f16_pow2_bits(int rel) {
     rel = rel > 0 ? 0 : rel;
-    const int e = 14 + rel;
-    if (e >= -14) return static_cast<uint32_t>(e + 15) << 10;
-    if (e >= -24) return 1u << (e + 24);
+    if (rel >= -14) return static_cast<uint32_t>(rel + 15) << 10;
+    if (rel >= -24) return 1u << (rel + 24);
     return 0u;
 }
 
