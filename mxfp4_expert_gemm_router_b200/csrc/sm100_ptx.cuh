@@ -67,13 +67,14 @@ enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag, int* status,
                                                   uint64_t limit_ns) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    // One quick check, then suspend in hardware until the phase completes (or
+    // the hint expires): spinning here would take issue slots from the decoder
+    // warps that share this warp's scheduler.
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
