@@ -167,7 +167,7 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             const int rf = min(128, p.N - ft * 128);
             const uint8_t* we = p.wpack + static_cast<size_t>(U.x) * expert_bytes;
             for (int c = c0; c < c1; ++c) {
-                ok = mbar_wait_warp(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns));
                 if (!ok) break;
                 if (skip) {
                     skip = false;  // test hook: this stage is never filled
@@ -204,12 +204,11 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
             const int4 U = p.units[u];
             const int sp = U.w >> 16;
             const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
-            ok = mbar_wait_warp(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(acce_bar, acc_ph ^ 1u, abort_flag, p.status, p.timeout_ns));
             if (!ok) break;
             for (int c = c0; c < c1; ++c) {
-                // afull implies the stage's copies landed: every decoder warp waited on
-                // full_bar(s) before arriving, so the MMA warp need not wait on it.
-                ok = mbar_wait_warp(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(afull_bar(a), aph, abort_flag, p.status, p.timeout_ns));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
                 const int ksteps = 2 * p.M.blocks_in_chunk(c);
@@ -217,31 +216,22 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 const uint32_t acol = tmem + a * GEMM_A_COLS;
                 const uint32_t acc0 = c > c0 ? 1u : 0u;
                 if (MODE == 0) {
-                    mma_f16_ts_warp(dg, acol, bd, p.idesc, acc0);
-                    mma_f16_ts_warp(du, acol + 32, bd, p.idesc, acc0);
-                    mma_f16_ts_warp(dg, acol + 8, bd + 2, p.idesc, 1u);
-                    mma_f16_ts_warp(du, acol + 40, bd + 2, p.idesc, 1u);
-                    if (ksteps == 4) {
-                        mma_f16_ts_warp(dg, acol + 16, bd + 4, p.idesc, 1u);
-                        mma_f16_ts_warp(du, acol + 48, bd + 4, p.idesc, 1u);
-                        mma_f16_ts_warp(dg, acol + 24, bd + 6, p.idesc, 1u);
-                        mma_f16_ts_warp(du, acol + 56, bd + 6, p.idesc, 1u);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i < ksteps) {
+                            const uint32_t acc = i > 0 ? 1u : acc0;
+                            mma_f16_ts_warp(dg, acol + 8 * i, bd + 2 * i, p.idesc, acc);
+                            mma_f16_ts_warp(du, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
+                        }
                     }
                 } else {
                     const uint64_t bd1 = bd + (b_sub >> 4);
-                    mma_f16_ts_warp(dg, acol, bd, p.idesc, acc0);
-                    mma_f16_ts_warp(dg, acol + 8, bd + 2, p.idesc, 1u);
-                    if (ksteps >= 4) {
-                        mma_f16_ts_warp(dg, acol + 16, bd + 4, p.idesc, 1u);
-                        mma_f16_ts_warp(dg, acol + 24, bd + 6, p.idesc, 1u);
-                    }
-                    if (ksteps >= 6) {
-                        mma_f16_ts_warp(dg, acol + 32, bd1, p.idesc, 1u);
-                        mma_f16_ts_warp(dg, acol + 40, bd1 + 2, p.idesc, 1u);
-                    }
-                    if (ksteps >= 8) {
-                        mma_f16_ts_warp(dg, acol + 48, bd1 + 4, p.idesc, 1u);
-                        mma_f16_ts_warp(dg, acol + 56, bd1 + 6, p.idesc, 1u);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (i < ksteps) {
+                            const uint32_t acc = i > 0 ? 1u : acc0;
+                            mma_f16_ts_warp(dg, acol + 8 * i, (i < 4 ? bd : bd1) + 2 * (i & 3), p.idesc, acc);
+                        }
                     }
                 }
                 tc_commit_warp(aempty_bar(a));
@@ -300,7 +290,8 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                     if (j >= g) break;
                     const int nbc = p.M.blocks_in_chunk(c + j);
                     mine[j] = warp_rows && hb < nbc;
-                    if (!mbar_wait_warp(full_bar(s), ph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                    const bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
+                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
                     cw[j] = make_uint4(0, 0, 0, 0);
                     sc[j] = 127;
                     if (mine[j]) {
@@ -316,7 +307,8 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
 #pragma unroll
                 for (int j = 0; j < GEMM_GROUP; ++j) {
                     if (j >= g) break;
-                    if (!mbar_wait_warp(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                    const bool w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
+                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
                     aslot[j] = a;
                     if (++a == NA) { a = 0; aph ^= 1u; }
                 }
@@ -349,7 +341,8 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
 
             // ------------------------------------------------------ epilogue
             {
-                if (!mbar_wait_warp(accf_bar, acc_ph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                const bool w_ok = mbar_wait_bounded(accf_bar, acc_ph, abort_flag, p.status, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
             }
             acc_ph ^= 1u;
             tc_fence_after();

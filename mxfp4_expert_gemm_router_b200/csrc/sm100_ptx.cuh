@@ -84,15 +84,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// Warp form: lane 0 waits, the shuffle broadcasts the outcome and orders the
-// other lanes after lane 0's observation of the phase.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                               uint64_t limit_ns) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, abort_flag, status, limit_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 // Bounded wait that ignores the abort flag (used to drain copies in flight).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();
