@@ -14,15 +14,15 @@
 // grouped f16 activations, arrives by 2-D TMA with 128-byte swizzle.  fp32
 // accumulators stay in TMEM; the epilogue warps read them back with tcgen05.ld.
 //
-//   MODE 0 (gate/up): stages of K = 64 holding gate and up; two accumulators
-//     (gate, up) for the same 128 features; epilogue: H[row, f] =
-//     Swish(g * 2^sg) * (u * 2^su), stored as f16; with a K split, fp32
-//     partials are added into GU instead.
-//   MODE 1 (down): stages of K = 128; one accumulator; epilogue: y[token, f] +=
-//     w_row * (d * 2^sd), red.add into the fp32 output accumulator (the
-//     weighted scatter-combine).
-// Both modes stream 8704 weight bytes (128 rows x 4 blocks x 17 B) per stage
-// and decode exactly one 32-block per decoder thread per stage.
+//   MODE 0 (gate/up): stages of K = 128 holding gate and up (17408 weight
+//     bytes); two accumulators (gate, up) for the same 128 features; epilogue:
+//     H[row, f] = Swish(g * 2^sg) * (u * 2^su), stored as f16; with a K split,
+//     fp32 partials are added into GU instead.
+//   MODE 1 (down): stages of K = 128 (8704 weight bytes); one accumulator;
+//     epilogue: y[token, f] += w_row * (d * 2^sd), red.add into the fp32 output
+//     accumulator (the weighted scatter-combine).
+// Each decoder thread decodes two 32-blocks per round: MODE 0 two blocks of
+// one stage, MODE 1 one block of each of two stages.
 //
 // Persistent kernel: one CTA per SM, units (expert, token tile, feature tile,
 // K split) taken round-robin from a device-built list.  Warp roles:
@@ -49,10 +49,8 @@ constexpr int GEMM_DEC_WARPS = 16;
 constexpr int GEMM_THREADS = (2 + GEMM_DEC_WARPS) * 32;
 constexpr int GEMM_MAX_STAGES = 16;
 constexpr int GEMM_MAX_A_SLOTS = 7;
-constexpr int GEMM_A_COLS = 64;                               // TMEM columns per A slot
 constexpr int GEMM_TMEM_COLS = 512;
-constexpr int GEMM_GROUP = 2;                                 // stages a decoder warp handles per round
-constexpr int GEMM_W_STAGE = 128 * 4 * 17;                    // weight bytes per stage (max)
+constexpr int GEMM_KSTAGE = 128;                              // K per pipeline stage, both modes
 constexpr int GEMM_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
 struct GemmParams {
@@ -65,7 +63,7 @@ struct GemmParams {
     int K;                    // contraction length
     int BN;                   // token rows per tile (MMA N), multiple of 16
     int stages;
-    int a_slots;              // TMEM A slots (GEMM_A_COLS columns each); accumulators follow them
+    int a_slots;              // TMEM A slots (gemm_a_cols(MODE) columns each); accumulators follow them
     uint32_t idesc;
     __half* H;                // MODE 0 output [rows][N]
     float* GU;                // MODE 0 split partials [rows][2N]
@@ -77,15 +75,20 @@ struct GemmParams {
     uint32_t skip_first_copy; // test hook: producer skips its first copy
 };
 
-__host__ __device__ inline int gemm_kstage(int mode) { return mode == 0 ? 64 : 128; }
+// Weight bytes per stage (128 rows x 4 blocks x 17 B per matrix), TMEM columns
+// per A slot (K = 128 of f16 per matrix = 64 columns), B bytes per stage (two
+// 64-wide K sub-tiles of BN rows x 128 B).
+__host__ __device__ constexpr int gemm_w_stage(int mode) { return mode == 0 ? 2 * 128 * 4 * 17 : 128 * 4 * 17; }
+__host__ __device__ constexpr int gemm_a_cols(int mode) { return mode == 0 ? 128 : 64; }
 __host__ __device__ inline size_t gemm_b_stage_bytes(int mode, int BN) {
-    return static_cast<size_t>(BN) * 128 * (mode == 0 ? 1 : 2);
+    (void)mode;
+    return static_cast<size_t>(BN) * 128 * 2;
 }
-__host__ inline size_t gemm_stage_bytes(int mode, int BN) { return GEMM_W_STAGE + gemm_b_stage_bytes(mode, BN); }
+__host__ inline size_t gemm_stage_bytes(int mode, int BN) { return gemm_w_stage(mode) + gemm_b_stage_bytes(mode, BN); }
 // A slots that fit in TMEM beside the accumulators (2*BN columns for gate/up, BN for down).
 __host__ inline int gemm_a_slots(int mode, int BN) {
     const int d_cols = mode == 0 ? 2 * BN : BN;
-    int n = (GEMM_TMEM_COLS - d_cols) / GEMM_A_COLS;
+    int n = (GEMM_TMEM_COLS - d_cols) / gemm_a_cols(mode);
     return n > GEMM_MAX_A_SLOTS ? GEMM_MAX_A_SLOTS : n;
 }
 __host__ inline size_t gemm_smem_bytes(int mode, int BN, int stages) {
@@ -98,7 +101,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int KSTAGE = MODE == 0 ? 64 : 128;
+    constexpr int KSTAGE = GEMM_KSTAGE;
+    constexpr int W_STAGE = gemm_w_stage(MODE);
+    constexpr int A_COLS = gemm_a_cols(MODE);
 
     const int S = p.stages;
     const uint32_t b_bytes = static_cast<uint32_t>(gemm_b_stage_bytes(MODE, p.BN));
@@ -107,11 +112,11 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t b_sm = base;                                   // S x B tiles (1024-aligned)
     const uint32_t w_sm = b_sm + S * b_bytes;                     // S x weight chunks
-    const uint32_t bar0 = w_sm + S * GEMM_W_STAGE;                // barriers (8-byte aligned)
+    const uint32_t bar0 = w_sm + S * W_STAGE;                     // barriers (8-byte aligned)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     const int NA = p.a_slots;
-    const uint32_t d_col0 = static_cast<uint32_t>(NA * GEMM_A_COLS);   // first accumulator column
+    const uint32_t d_col0 = static_cast<uint32_t>(NA * A_COLS);        // first accumulator column
     auto afull_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
     auto aempty_bar = [&](int a) { return bar0 + 8u * (2 * S + GEMM_MAX_A_SLOTS + a); };
     const uint32_t accf_bar = bar0 + 8u * (2 * S + 2 * GEMM_MAX_A_SLOTS);
@@ -174,9 +179,9 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 } else {
                     const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
                     const int k0 = c * KSTAGE;
-                    const bool second = (MODE == 1) && (k0 + 64 < p.K);
+                    const bool second = k0 + 64 < p.K;
                     mbar_arrive_expect_tx_warp(full_bar(s), wb + (second ? 2u : 1u) * b_sub);
-                    bulk_g2s_warp(w_sm + s * GEMM_W_STAGE, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
+                    bulk_g2s_warp(w_sm + s * W_STAGE, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
                     tma_load_2d_warp(b_sm + s * b_bytes, &tmap_b, k0, U.y, full_bar(s));
                     if (second) tma_load_2d_warp(b_sm + s * b_bytes + b_sub, &tmap_b, k0 + 64, U.y, full_bar(s));
                     pend_ph[s] = static_cast<int>(ph);
@@ -213,25 +218,16 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 tc_fence_after();
                 const int ksteps = 2 * p.M.blocks_in_chunk(c);
                 const uint64_t bd = bdesc0 + ((static_cast<uint64_t>(s) * b_bytes) >> 4);
-                const uint32_t acol = tmem + a * GEMM_A_COLS;
+                const uint32_t acol = tmem + a * A_COLS;
                 const uint32_t acc0 = c > c0 ? 1u : 0u;
-                if (MODE == 0) {
+                const uint64_t bd1 = bd + (b_sub >> 4);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        if (i < ksteps) {
-                            const uint32_t acc = i > 0 ? 1u : acc0;
-                            mma_f16_ts_warp(dg, acol + 8 * i, bd + 2 * i, p.idesc, acc);
-                            mma_f16_ts_warp(du, acol + 32 + 8 * i, bd + 2 * i, p.idesc, acc);
-                        }
-                    }
-                } else {
-                    const uint64_t bd1 = bd + (b_sub >> 4);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (i < ksteps) {
-                            const uint32_t acc = i > 0 ? 1u : acc0;
-                            mma_f16_ts_warp(dg, acol + 8 * i, (i < 4 ? bd : bd1) + 2 * (i & 3), p.idesc, acc);
-                        }
+                for (int i = 0; i < 8; ++i) {
+                    if (i < ksteps) {
+                        const uint32_t acc = i > 0 ? 1u : acc0;
+                        const uint64_t bdi = (i < 4 ? bd : bd1) + 2 * (i & 3);
+                        mma_f16_ts_warp(dg, acol + 8 * i, bdi, p.idesc, acc);
+                        if (MODE == 0) mma_f16_ts_warp(du, acol + 64 + 8 * i, bdi, p.idesc, acc);
                     }
                 }
                 tc_commit_warp(aempty_bar(a));
@@ -250,11 +246,12 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
         // ---------------------------------------------------------- decoders + epilogue
         const int q = warp & 3;               // TMEM lane quadrant (hardware rule: warp % 4)
         const int role = (warp - 2) >> 2;     // 0..3
+        // MODE 0: matrix role>>1, blocks 2*(role&1) and 2*(role&1)+1 of each stage;
+        // MODE 1: block `role` of each of two consecutive stages.
         const int mat = MODE == 0 ? (role >> 1) : 0;
-        const int hb = MODE == 0 ? (role & 1) : role;
         const int row = 32 * q + lane;        // weight row within the feature tile
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        const uint32_t tcol = static_cast<uint32_t>(mat * 32 + hb * 16);
+        constexpr int SPR = MODE == 0 ? 1 : 2;   // stages per decoder round
         int s = 0, a = 0;
         uint32_t ph = 0, aph = 0, acc_ph = 0;
         bool ok = true;
@@ -277,55 +274,68 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                     rs_mine = rs0;
                 }
             }
-            // Stages are taken GEMM_GROUP at a time so that one round of waits, shared
-            // loads and TMEM-store completion covers several stages.
-            for (int c = c0; c < c1 && ok; c += GEMM_GROUP) {
-                const int g = min(GEMM_GROUP, c1 - c);
-                uint4 cw[GEMM_GROUP];
-                int sc[GEMM_GROUP];
-                bool mine[GEMM_GROUP];
-                int aslot[GEMM_GROUP];
+            for (int c = c0; c < c1 && ok; c += SPR) {
+                const int g = min(SPR, c1 - c);       // stages this round
+                uint4 cw[2];
+                int sc[2];
+                bool mine[2];
+                int aslot[2];
+                uint32_t tcol[2];
+                // -- read this round's two blocks from shared memory
 #pragma unroll
-                for (int j = 0; j < GEMM_GROUP; ++j) {
+                for (int j = 0; j < SPR; ++j) {
                     if (j >= g) break;
                     const int nbc = p.M.blocks_in_chunk(c + j);
-                    mine[j] = warp_rows && hb < nbc;
-                    const bool w_ok = mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns);
-                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-                    cw[j] = make_uint4(0, 0, 0, 0);
-                    sc[j] = 127;
-                    if (mine[j]) {
-                        const uint8_t* ws = smem_raw + (w_sm + s * GEMM_W_STAGE - raw) + mat * 17 * nbc * rf;
-                        cw[j] = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
-                        sc[j] = ws[16 * nbc * rf + hb * rf + row];
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t* ws = smem_raw + (w_sm + s * W_STAGE - raw) + mat * 17 * nbc * rf;
+#pragma unroll
+                    for (int t = 0; t < (MODE == 0 ? 2 : 1); ++t) {
+                        const int slot = MODE == 0 ? t : j;
+                        const int hb = MODE == 0 ? 2 * (role & 1) + t : role;
+                        mine[slot] = warp_rows && hb < nbc;
+                        cw[slot] = make_uint4(0, 0, 0, 0);
+                        sc[slot] = 127;
+                        if (mine[slot]) {
+                            cw[slot] = *reinterpret_cast<const uint4*>(ws + (hb * rf + row) * 16);
+                            sc[slot] = ws[16 * nbc * rf + hb * rf + row];
+                        }
+                        tcol[slot] = static_cast<uint32_t>(mat * 64 + hb * 16);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(empty_bar(s));
                     if (++s == S) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
+                // -- claim the A slots
 #pragma unroll
-                for (int j = 0; j < GEMM_GROUP; ++j) {
+                for (int j = 0; j < SPR; ++j) {
                     if (j >= g) break;
-                    const bool w_ok = mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns);
-                    if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+                    if (!__all_sync(0xffffffffu, mbar_wait_bounded(aempty_bar(a), aph ^ 1u, abort_flag, p.status, p.timeout_ns))) {
+                        ok = false;
+                        break;
+                    }
                     aslot[j] = a;
                     if (++a == NA) { a = 0; aph ^= 1u; }
                 }
                 if (!ok) break;
+                if (MODE == 0) aslot[1] = aslot[0];
                 tc_fence_after();
+                // -- decode and store to tensor memory
 #pragma unroll
-                for (int j = 0; j < GEMM_GROUP; ++j) {
-                    if (j >= g) break;
-                    if (mine[j]) {
+                for (int b = 0; b < 2; ++b) {
+                    if (MODE == 1 && b >= g) break;
+                    if (mine[b]) {
                         uint32_t r[16];
-                        const uint32_t m1 = f16_pow2_bits(sc[j] - rs_mine);
+                        const uint32_t m1 = f16_pow2_bits(sc[b] - rs_mine);
                         const uint32_t m2 = m1 | (m1 << 16);
-                        e2m1x8_to_f16x8(cw[j].x, m2, r[0], r[1], r[2], r[3]);
-                        e2m1x8_to_f16x8(cw[j].y, m2, r[4], r[5], r[6], r[7]);
-                        e2m1x8_to_f16x8(cw[j].z, m2, r[8], r[9], r[10], r[11]);
-                        e2m1x8_to_f16x8(cw[j].w, m2, r[12], r[13], r[14], r[15]);
-                        tmem_st16(tmem + lane_addr + aslot[j] * GEMM_A_COLS + tcol, r);
+                        e2m1x8_to_f16x8(cw[b].x, m2, r[0], r[1], r[2], r[3]);
+                        e2m1x8_to_f16x8(cw[b].y, m2, r[4], r[5], r[6], r[7]);
+                        e2m1x8_to_f16x8(cw[b].z, m2, r[8], r[9], r[10], r[11]);
+                        e2m1x8_to_f16x8(cw[b].w, m2, r[12], r[13], r[14], r[15]);
+                        tmem_st16(tmem + lane_addr + aslot[b] * A_COLS + tcol[b], r);
                     }
                 }
                 if (warp_rows) tmem_wait_st();
@@ -333,7 +343,7 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 __syncwarp();
                 if (lane == 0) {
 #pragma unroll
-                    for (int j = 0; j < GEMM_GROUP; ++j)
+                    for (int j = 0; j < SPR; ++j)
                         if (j < g) mbar_arrive(afull_bar(aslot[j]));
                 }
             }

@@ -203,7 +203,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     if (cudaDeviceGetAttribute(&h->nsm, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
         return fail(MOE_ERR_CUDA);
     const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
-    h->KC_gu = (d / 32 + 1) / 2;   // 64-wide chunks of the gate/up GEMM
+    h->KC_gu = (d / 32 + 3) / 4;   // 128-wide chunks of the gate/up GEMM
     h->KC_dn = (f / 32 + 3) / 4;   // 128-wide chunks of the down GEMM
     h->F_gu = (f + 127) / 128;
     h->F_dn = (d + 127) / 128;
@@ -296,7 +296,7 @@ static TiledMatrix tiled(moe_mxfp4* h, int which) {
         M.base = h->w_gu;
         M.N = c.d_ff;
         M.K = c.d_model;
-        M.BPC = 2;
+        M.BPC = 4;
         M.NM = 2;
         M.sub = which;
     } else {
