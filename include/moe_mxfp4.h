@@ -173,6 +173,38 @@ int64_t moe_mxfp4_expert_param_count(const moe_mxfp4_config_t* cfg);
 /* MXFP4 bytes of one expert: codes + scales = 17/32 byte per parameter. */
 int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg);
 
+/* Routing without any device allocation.  No counterpart on the pages: this
+ * is an interface convenience, not part of the method.  Some callers cannot
+ * call cudaMalloc -- code that must not synchronise the device (cudaMalloc
+ * may), hosts whose device memory is owned by another allocator, or a
+ * process that has no handle (moe_mxfp4_create allocates).  This call runs
+ * the same router kernel as moe_mxfp4_forward (scores, top-k with ties to the
+ * lower index, softmax over the selected scores, per-expert counts) with its
+ * scratch in one fixed static device array inside the library
+ * (MOE_ROUTE_NOALLOC_SCRATCH_BYTES on every device that loads the library,
+ * held until exit).  Inputs and outputs are caller-owned device memory:
+ *   x:             [T][d_model], act_dtype (MOE_DTYPE_F32 or MOE_DTYPE_BF16)
+ *   w_router:      [E][d_model], act_dtype
+ *   router_bias:   fp32 [E] or NULL
+ *   topk_idx:      int32 [T][top_k]; topk_w: fp32 [T][top_k]
+ *   expert_counts: int32 [E] or NULL
+ * Limits: 1 <= T <= MOE_ROUTE_NOALLOC_MAX_TOKENS, E <= MOE_ROUTE_NOALLOC_MAX_EXPERTS,
+ * 1 <= top_k <= min(8, E), d_model a positive multiple of 32 up to 16384;
+ * anything larger returns MOE_ERR_UNSUPPORTED (nothing is launched).  The
+ * first call on a device looks up the array's device address (with that
+ * device current) and sets the kernel's shared-memory limit: make that first
+ * call before any stream capture.  Every call resets the counters it needs and
+ * otherwise reuses the array, so calls that overlap on the GPU (different
+ * streams without ordering, or several host threads) race on it.
+ * Asynchronous on `stream`. */
+#define MOE_ROUTE_NOALLOC_MAX_TOKENS 256
+#define MOE_ROUTE_NOALLOC_MAX_EXPERTS 128
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (2304 * 1024)
+moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_router, const float* router_bias,
+                                     int32_t T, int32_t d_model, int32_t n_experts, int32_t top_k,
+                                     int32_t act_dtype, int32_t* topk_idx, float* topk_w,
+                                     int32_t* expert_counts, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,6 +53,7 @@ SIGNATURES = {
     "moe_mxfp4_launch_count": (ctypes.c_uint64, [_VP]),
     "moe_mxfp4_expert_param_count": (ctypes.c_int64, [ctypes.POINTER(moe_mxfp4_config_t)]),
     "moe_mxfp4_expert_weight_bytes": (ctypes.c_int64, [ctypes.POINTER(moe_mxfp4_config_t)]),
+    "moe_mxfp4_route_noalloc": (_ST, [_VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
 }
 
 _lib = None
@@ -82,6 +83,21 @@ def __getattr__(name):
     if name in SIGNATURES:
         return getattr(load(), name)
     raise AttributeError(name)
+
+
+MOE_ROUTE_NOALLOC_MAX_TOKENS = 256
+MOE_ROUTE_NOALLOC_MAX_EXPERTS = 128
+
+
+def route_noalloc(x, w_router, router_bias, top_k, topk_idx, topk_w, expert_counts=None, stream=None):
+    """Router + top-k + softmax with no device allocation (see moe_mxfp4_route_noalloc)."""
+    import torch
+    dt = MOE_DTYPE_BF16 if x.dtype == torch.bfloat16 else MOE_DTYPE_F32
+    T, d = int(x.shape[0]), int(x.shape[1])
+    E = int(w_router.shape[0])
+    check(load().moe_mxfp4_route_noalloc(_p(x), _p(w_router), _p(router_bias), T, d, E, int(top_k), dt,
+                                         _p(topk_idx), _p(topk_w), _p(expert_counts), _stream(stream)),
+          "route_noalloc")
 
 
 class MoeError(RuntimeError):

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -626,3 +627,127 @@ moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Routing with no device allocation (moe_mxfp4_route_noalloc).
+//
+// The router kernel's scratch -- partial scores, tile and global arrival
+// counters, per-tile histograms and ranks, offsets and schedule slots -- lives
+// in one file-scope static device array.  Host code must not pass the array's
+// name to a kernel (on the host it is only a stand-in symbol); the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+namespace {
+
+constexpr int NOALLOC_MAX_SPLITS = 8;
+constexpr size_t NOALLOC_PART_BYTES = sizeof(double) * NOALLOC_MAX_SPLITS * MOE_ROUTE_NOALLOC_MAX_TOKENS *
+                                      MOE_ROUTE_NOALLOC_MAX_EXPERTS;
+constexpr int NOALLOC_MAX_TILES = (MOE_ROUTE_NOALLOC_MAX_TOKENS + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+// byte offsets inside the array (each 256-byte aligned)
+constexpr size_t NA_OFF_PART = 0;
+constexpr size_t NA_OFF_HIST = NA_OFF_PART + NOALLOC_PART_BYTES;
+constexpr size_t NA_OFF_RANK = NA_OFF_HIST + 4096 * 4;
+constexpr size_t NA_OFF_CNT = NA_OFF_RANK + sizeof(int32_t) * MOE_ROUTE_NOALLOC_MAX_TOKENS * MAX_TOPK;
+constexpr size_t NA_OFF_OFFS = NA_OFF_CNT + 256;
+constexpr size_t NA_OFF_SCHED = NA_OFF_OFFS + 4096;
+constexpr size_t NA_END = NA_OFF_SCHED + 256;
+static_assert(NOALLOC_MAX_TILES * MOE_ROUTE_NOALLOC_MAX_EXPERTS * 4 <= 4096 * 4, "histogram region too small");
+static_assert(NOALLOC_MAX_TILES + 1 <= 64, "counter region too small");
+static_assert(NA_END <= MOE_ROUTE_NOALLOC_SCRATCH_BYTES, "scratch array too small");
+
+__device__ __align__(256) unsigned char g_route_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocDevice {
+    bool ready = false;
+    unsigned char* scratch = nullptr;  // device address of g_route_scratch on this device
+    int nsm = 0;
+};
+constexpr int NOALLOC_MAX_DEVICES = 64;
+NoallocDevice g_noalloc[NOALLOC_MAX_DEVICES];
+std::mutex g_noalloc_mutex;
+
+moe_status_t noalloc_setup(int dev, NoallocDevice** out) {
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return MOE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    NoallocDevice& nd = g_noalloc[dev];
+    if (!nd.ready) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+        int nsm = 0;
+        if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+        const int smem = static_cast<int>(router_smem_bytes(MOE_ROUTE_NOALLOC_MAX_EXPERTS));
+        if (cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
+        nd.scratch = static_cast<unsigned char*>(ptr);
+        nd.nsm = nsm;
+        nd.ready = true;
+    }
+    *out = &nd;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_router, const float* router_bias,
+                                                int32_t T, int32_t d_model, int32_t n_experts, int32_t top_k,
+                                                int32_t act_dtype, int32_t* topk_idx, float* topk_w,
+                                                int32_t* expert_counts, cudaStream_t stream) {
+    if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (T <= 0 || d_model <= 0 || n_experts <= 0 || top_k <= 0) return MOE_ERR_INVALID_ARG;
+    if (act_dtype != MOE_DTYPE_F32 && act_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (T > MOE_ROUTE_NOALLOC_MAX_TOKENS || n_experts > MOE_ROUTE_NOALLOC_MAX_EXPERTS ||
+        top_k > std::min(MAX_TOPK, static_cast<int>(n_experts)) || d_model % 32 || d_model > 16384)
+        return MOE_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    NoallocDevice* nd = nullptr;
+    moe_status_t st = noalloc_setup(dev, &nd);
+    if (st != MOE_OK) return st;
+    unsigned char* sc = nd->scratch;
+    const int tiles = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
+    int* counters = reinterpret_cast<int*>(sc + NA_OFF_CNT);
+    // the arrival counters must start at zero (a previous call may have been cut short)
+    if (cudaMemsetAsync(counters, 0, sizeof(int) * (tiles + 1), stream) != cudaSuccess) return MOE_ERR_CUDA;
+    RouterArgs ra;
+    ra.x = x;
+    ra.wr = w_router;
+    ra.bias = router_bias;
+    ra.T = T;
+    ra.d = d_model;
+    ra.E = n_experts;
+    ra.k = top_k;
+    ra.S = std::min(NOALLOC_MAX_SPLITS, router_splits(T, d_model, nd->nsm));
+    ra.part = reinterpret_cast<double*>(sc + NA_OFF_PART);
+    ra.tile_cnt = counters;
+    ra.glob_cnt = counters + tiles;
+    ra.idx_out = topk_idx;
+    ra.w_out = topk_w;
+    ra.local_rank = reinterpret_cast<int32_t*>(sc + NA_OFF_RANK);
+    ra.hist = reinterpret_cast<int32_t*>(sc + NA_OFF_HIST);
+    ra.zero_rows = nullptr;
+    ra.zero_ld = 0;
+    // no expert GEMMs follow: zero feature tiles, so the schedule step only
+    // totals the histogram (expert_counts) and emits no units
+    ra.BN = 16;
+    ra.F_gu = 0;
+    ra.F_dn = 0;
+    ra.KC_gu = 1;
+    ra.KC_dn = 1;
+    ra.nsm = nd->nsm;
+    ra.split_rows_cap = 0;
+    ra.max_units = 0;
+    ra.offsets = reinterpret_cast<int32_t*>(sc + NA_OFF_OFFS);
+    ra.counts_out = expert_counts;
+    ra.units_gu = nullptr;
+    ra.units_dn = nullptr;
+    ra.sched = reinterpret_cast<int32_t*>(sc + NA_OFF_SCHED);
+    const dim3 grid(tiles, ra.S);
+    const size_t smem = router_smem_bytes(n_experts);
+    if (act_dtype == MOE_DTYPE_BF16)
+        router_kernel<__nv_bfloat16><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    else
+        router_kernel<float><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    return cuda_status(cudaGetLastError());
+}
