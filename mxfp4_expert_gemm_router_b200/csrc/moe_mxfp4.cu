@@ -141,6 +141,24 @@ static int router_splits(int T, int d, int nsm) {
     return std::max(1, std::min(kch, want));
 }
 
+// Router launch for the expert count: EPT = experts per lane, 1/2/4/8.
+template <typename TA>
+static void launch_router(const RouterArgs& ra, dim3 grid, size_t smem, cudaStream_t stream) {
+    const int ept = (ra.E + 31) / 32;
+    if (ept <= 1) router_kernel<TA, 1><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    else if (ept <= 2) router_kernel<TA, 2><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    else if (ept <= 4) router_kernel<TA, 4><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    else router_kernel<TA, 8><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+}
+template <typename TA>
+static cudaError_t set_router_smem(int bytes) {
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(router_kernel<TA, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
+    if ((e = cudaFuncSetAttribute(router_kernel<TA, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
+    if ((e = cudaFuncSetAttribute(router_kernel<TA, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
+    return cudaFuncSetAttribute(router_kernel<TA, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 static int stages_for(int mode, int BN) {
     const size_t budget = 227 * 1024 - 1024 - 512;
     int s = static_cast<int>(budget / gemm_stage_bytes(mode, BN));
@@ -270,10 +288,8 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
                 cudaSuccess ||
             cudaFuncSetAttribute(expert_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess ||
-            cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess)
+            set_router_smem<float>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess ||
+            set_router_smem<__nv_bfloat16>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess)
             return fail(MOE_ERR_CUDA);
         g_attrs_set = true;
     }
@@ -474,9 +490,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     const size_t rsm = router_smem_bytes(E);
     const dim3 rgrid(nblk, ra.S);
     if (bf16)
-        router_kernel<__nv_bfloat16><<<rgrid, ROUTER_THREADS, rsm, stream>>>(ra);
+        launch_router<__nv_bfloat16>(ra, rgrid, rsm, stream);
     else
-        router_kernel<float><<<rgrid, ROUTER_THREADS, rsm, stream>>>(ra);
+        launch_router<float>(ra, rgrid, rsm, stream);
     h->stage_ran[0] = true;
     // 1: gather into grouped rows
     mark(1);
@@ -675,10 +691,7 @@ moe_status_t noalloc_setup(int dev, NoallocDevice** out) {
         int nsm = 0;
         if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
         const int smem = static_cast<int>(router_smem_bytes(MOE_ROUTE_NOALLOC_MAX_EXPERTS));
-        if (cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess)
+        if (set_router_smem<float>(smem) != cudaSuccess || set_router_smem<__nv_bfloat16>(smem) != cudaSuccess)
             return MOE_ERR_CUDA;
         nd.scratch = static_cast<unsigned char*>(ptr);
         nd.nsm = nsm;
@@ -746,8 +759,8 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     const dim3 grid(tiles, ra.S);
     const size_t smem = router_smem_bytes(n_experts);
     if (act_dtype == MOE_DTYPE_BF16)
-        router_kernel<__nv_bfloat16><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+        launch_router<__nv_bfloat16>(ra, grid, smem, stream);
     else
-        router_kernel<float><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+        launch_router<float>(ra, grid, smem, stream);
     return cuda_status(cudaGetLastError());
 }

@@ -180,7 +180,9 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
 // slot) pairs within their expert, writes the tile histogram and zeroes the
 // output accumulator rows of its tokens.  The last tile to finish builds the
 // schedule (schedule_block).
-template <typename TA>
+// EPT = experts per lane (ceil(E / 32) rounded up to 1, 2, 4 or 8): the
+// register tile scales with the expert count.
+template <typename TA, int EPT>
 __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
     extern __shared__ float rsm[];
     float* xs = rsm;                                      // [32][65]
@@ -201,32 +203,32 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     const int ntiles = gridDim.x;
     const int t0 = tile * ROUTER_TOKENS;
     const int ntok = min(ROUTER_TOKENS, a.T - t0);
-    const int EPT = (E + 31) / 32;  // experts per lane
     const int KCH = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
     const int kc0 = split * KCH / a.S, kc1 = (split + 1) * KCH / a.S;
 
-    double tot[MAX_EXPERTS / 32][4];
+    double tot[EPT][4];
 #pragma unroll
-    for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+    for (int i = 0; i < EPT; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
 
-    // Each thread owns one 8-element group of the x chunk (token tid/8) and up to
-    // EPT groups of the router chunk (expert (tid + 256 i)/8); the next chunk is
-    // loaded into registers while the current one is multiplied.
+    // Each thread owns one 8-element group of the x chunk (token tid/8) and EPT
+    // groups of the router chunk (group idx = tid + 256 i: expert idx % 32*EPT,
+    // K offset 8 * (idx / 32*EPT), so the transposed shared-memory stores of
+    // consecutive threads hit consecutive banks); the next chunk is loaded into
+    // registers while the current one is multiplied.
+    constexpr int EP = 32 * EPT;              // expert slots covered by the register tile
     const int xt = tid >> 3, xv8 = (tid & 7) * 8;
-    Raw8<TA> xr, wrr[MAX_EXPERTS / 32];
+    Raw8<TA> xr, wrr[EPT];
     auto load_chunk = [&](int kc) {
         if (xt < ntok && kc + xv8 < d) xr.load(x + static_cast<size_t>(t0 + xt) * d + kc + xv8);
         else xr.zero();
 #pragma unroll
-        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-            if (i < EPT) {
-                const int idx = tid + ROUTER_THREADS * i;
-                const int e = idx >> 3, k8 = (idx & 7) * 8;
-                if (e < E && kc + k8 < d) wrr[i].load(wr + static_cast<size_t>(e) * d + kc + k8);
-                else wrr[i].zero();
-            }
+        for (int i = 0; i < EPT; ++i) {
+            const int idx = tid + ROUTER_THREADS * i;
+            const int e = idx % EP, k8 = (idx / EP) * 8;
+            if (e < E && k8 < ROUTER_KCHUNK && kc + k8 < d) wrr[i].load(wr + static_cast<size_t>(e) * d + kc + k8);
+            else wrr[i].zero();
         }
     };
     if (kc0 < kc1) load_chunk(kc0 * ROUTER_KCHUNK);
@@ -236,48 +238,44 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
 #pragma unroll
         for (int j = 0; j < 8; ++j) xs[xt * (ROUTER_KCHUNK + 1) + xv8 + j] = xr.get(j);
 #pragma unroll
-        for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-            if (i < EPT) {
-                const int idx = tid + ROUTER_THREADS * i;
-                const int e = idx >> 3, k8 = (idx & 7) * 8;
-                if (e < E) {
+        for (int i = 0; i < EPT; ++i) {
+            const int idx = tid + ROUTER_THREADS * i;
+            const int e = idx % EP, k8 = (idx / EP) * 8;
+            if (e < E && k8 < ROUTER_KCHUNK) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) ws[(k8 + j) * E + e] = wrr[i].get(j);
-                }
+                for (int j = 0; j < 8; ++j) ws[(k8 + j) * E + e] = wrr[i].get(j);
             }
         }
         __syncthreads();
         if (c + 1 < kc1) load_chunk(kc + ROUTER_KCHUNK);
-        float acc[MAX_EXPERTS / 32][4];
+        float acc[EPT][4];
 #pragma unroll
-        for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+        for (int i = 0; i < EPT; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
         for (int kk = 0; kk < ROUTER_KCHUNK; ++kk) {
             float xv[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) xv[j] = xs[(warp * 4 + j) * (ROUTER_KCHUNK + 1) + kk];
 #pragma unroll
-            for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
-                if (i < EPT) {
-                    const int e = lane + 32 * i;
-                    const float wv = (e < E) ? ws[kk * E + e] : 0.f;
+            for (int i = 0; i < EPT; ++i) {
+                const int e = lane + 32 * i;
+                const float wv = (e < E) ? ws[kk * E + e] : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(wv, xv[j], acc[i][j]);
-                }
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(wv, xv[j], acc[i][j]);
             }
         }
 #pragma unroll
-        for (int i = 0; i < MAX_EXPERTS / 32; ++i)
+        for (int i = 0; i < EPT; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) tot[i][j] += static_cast<double>(acc[i][j]);
     }
     // partial scores of this split
 #pragma unroll
-    for (int i = 0; i < MAX_EXPERTS / 32; ++i) {
+    for (int i = 0; i < EPT; ++i) {
         const int e = lane + 32 * i;
-        if (i < EPT && e < E) {
+        if (e < E) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int tl = warp * 4 + j;
