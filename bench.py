@@ -134,6 +134,24 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (replicas report the slowest one)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_step: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s: every replica processes tokens_per_step each step."""
+    return tokens_per_step * steps * world / (max_total_ms / 1e3)
+
+
 # ---------------------------------------------------------------- our arm
 
 def build_layer(cfg: mi.MoeConfig, max_tokens: int):
@@ -222,11 +240,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if rank == 0 and not args.no_clocks else None
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev, world)
 
     # per-stage breakdown: a separate pass with events between the kernels
     stage_ms = []
@@ -252,11 +266,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             layer.forward_host(xh, yh, stream=stream)
             e_e[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
-    t2 = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t2.item())
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev, world)
     touched = int((counts.cpu().numpy() > 0).sum())
     del graph
     return {"total_ms": total_ms, "e2e_ms": e2e_ms, "stage_ms": stage_ms,
@@ -370,9 +380,8 @@ def main():
     if rank != 0:
         return 0
 
-    tokens = cfg.T * args.steps * world
-    value = tokens / (r["total_ms"] / 1e3)
-    e2e_value = tokens / (r["e2e_ms"] / 1e3)
+    value = job_throughput(cfg.T, args.steps, world, r["total_ms"])
+    e2e_value = job_throughput(cfg.T, args.steps, world, r["e2e_ms"])
     stages = {}
     for name in r["stage_ms"][0]:
         vals = [s[name] for s in r["stage_ms"]]

@@ -1,0 +1,52 @@
+"""The replica (N > 1) host path of bench.py on CPU: two gloo ranks.
+
+The layer has no exchange step, so N GPUs run N independent replicas; the only
+collective is the max over ranks of the per-rank device time.  This checks that
+reduction and the whole-job throughput formula with world_size 2."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as tmp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    import sys
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        per_rank_ms = [12.5, 40.0][rank]
+        m = bench.max_over_ranks(per_rank_ms, torch.device("cpu"), world)
+        out[rank] = (m, bench.job_throughput(64, 10, world, m))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_replica_timing():
+    port = _free_port()
+    with tmp.Manager() as mgr:
+        out = mgr.dict()
+        tmp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 40.0
+    # 2 replicas x 10 steps x 64 tokens in 40 ms
+    assert res[0][1] == pytest.approx(2 * 10 * 64 / 0.040)
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+    assert bench.max_over_ranks(3.0, None, 1) == 3.0
+    assert bench.job_throughput(1, 5, 1, 10.0) == pytest.approx(500.0)
