@@ -324,6 +324,20 @@ expert_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams 
                 if (MODE == 0) aslot[1] = aslot[0];
                 tc_fence_after();
                 // -- decode and store to tensor memory
+                if (MODE == 0 && mine[0] && mine[1]) {
+                    // the thread's two blocks are adjacent columns of one slot: one x32 store
+                    uint32_t r[32];
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) {
+                        const uint32_t m1 = f16_pow2_bits(sc[b] - rs_mine);
+                        const uint32_t m2 = m1 | (m1 << 16);
+                        e2m1x8_to_f16x8(cw[b].x, m2, r[16 * b + 0], r[16 * b + 1], r[16 * b + 2], r[16 * b + 3]);
+                        e2m1x8_to_f16x8(cw[b].y, m2, r[16 * b + 4], r[16 * b + 5], r[16 * b + 6], r[16 * b + 7]);
+                        e2m1x8_to_f16x8(cw[b].z, m2, r[16 * b + 8], r[16 * b + 9], r[16 * b + 10], r[16 * b + 11]);
+                        e2m1x8_to_f16x8(cw[b].w, m2, r[16 * b + 12], r[16 * b + 13], r[16 * b + 14], r[16 * b + 15]);
+                    }
+                    tmem_st32(tmem + lane_addr + aslot[0] * A_COLS + tcol[0], r);
+                } else
 #pragma unroll
                 for (int b = 0; b < 2; ++b) {
                     if (MODE == 1 && b >= g) break;
