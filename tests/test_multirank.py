@@ -50,3 +50,24 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.0, None, 1) == 3.0
     assert bench.job_throughput(1, 5, 1, 10.0) == pytest.approx(500.0)
+
+
+def test_roofline_bound_follows_machine_balance():
+    """Decode-sized expert GEMMs are HBM-bound (each weight byte feeds a few
+    FLOPs), prefill-sized ones with hundreds of rows per expert tensor-bound."""
+    import bench
+    import moe_inputs as mi
+
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    dec = mi.CONFIGS["dec64"]
+    w = bench.algorithmic_work(dec, dec.T, dec.n_experts)["gate_up_swiglu"]
+    r = bench.roofline(w, 1e-4, peaks, "gate_up_swiglu", "f16")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - w["bytes"] / 1e-4 / 1e9) < 1e-6 * r["achieved"]
+    pre = mi.CONFIGS["zipf"]
+    w = bench.algorithmic_work(pre, pre.T, pre.n_experts)["gate_up_swiglu"]
+    r = bench.roofline(w, 1e-3, peaks, "gate_up_swiglu", "f16")
+    assert r["bound"] == "tensor" and r["peak"] == 1600.0
+    # FP4 operands run at 4x the bf16 rate, which moves the balance point up
+    r4 = bench.roofline(w, 1e-3, peaks, "gate_up_swiglu", "mxf4")
+    assert r4["peak"] == 6400.0
