@@ -54,6 +54,12 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
  * MOE_ERR_TIMEOUT through moe_mxfp4_get_status. */
 #define MOE_FLAG_TEST_SKIP_FIRST_COPY (1u << 30)
 
+/* Token rows per expert-GEMM tile (BN).  0 (default): chosen per forward from
+ * T, top_k and n_experts; 1..4 force BN = 16, 32, 48 or 64.  Every choice
+ * computes the same layer; the tile only changes how work is cut. */
+#define MOE_FLAG_TOKEN_TILE_SHIFT 8
+#define MOE_FLAG_TOKEN_TILE_MASK (0xFu << MOE_FLAG_TOKEN_TILE_SHIFT)
+
 typedef struct {
     int32_t d_model;        /* model width; multiple of 32                    */
     int32_t d_ff;           /* expert hidden width; multiple of 32            */

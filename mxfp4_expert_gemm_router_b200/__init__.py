@@ -21,6 +21,15 @@ LIB_PATH = os.path.join(HERE, "libmoe_mxfp4.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_NOT_QUANTIZED, MOE_ERR_TIMEOUT = range(6)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_FLAG_TEST_SKIP_FIRST_COPY = 1 << 30
+MOE_FLAG_TOKEN_TILE_SHIFT = 8
+MOE_FLAG_TOKEN_TILE_MASK = 0xF << MOE_FLAG_TOKEN_TILE_SHIFT
+
+
+def token_tile_flag(bn: int) -> int:
+    """Config flag that forces BN token rows per expert-GEMM tile (16, 32, 48 or 64)."""
+    if bn not in (16, 32, 48, 64):
+        raise ValueError("token tile must be 16, 32, 48 or 64")
+    return (bn // 16) << MOE_FLAG_TOKEN_TILE_SHIFT
 MOE_NUM_STAGES = 6
 
 

@@ -1,0 +1,318 @@
+// expert_mxf4.cuh -- grouped expert GEMMs on block-scaled MXFP4 tensor cores.
+//
+// Method (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card", §3.2 Les
+// Experts): each expert is (Swish(x . W_gate) (.) (x . W_up)) . W_down with
+// Swish(z) = z sigma(z); §2.1: the k expert outputs of a token are summed with
+// the router weights; §4: the expert weights are MXFP4.
+//
+// The MMA is tcgen05.mma kind::mxf4 with 32-element block scaling: both
+// operands are packed E2M1 in shared memory and every row carries one E8M0
+// scale per 32 elements of K, held in tensor memory.  Orientation:
+// D[feature, n] = W[feature, :] . B[n, :]^T with M = 128 weight rows (output
+// features) as the A operand and N = 3 * BN operand rows, the three MXFP4 terms
+// of BN grouped token rows (mxq.cuh), as B.  The weights reach the tensor core
+// exactly as stored, with no decode step: one bulk copy per K = 128 stage
+// brings codes and scale atoms, a 4-D TMA box {16 B, BN rows, 3 terms, 4
+// blocks} brings the activation codes and a bulk copy their scale atoms.
+// tcgen05.cp moves the scale atoms into a ring of tensor-memory slots; fp32
+// accumulators stay in tensor memory (two buffers when they fit, so the
+// epilogue of one unit overlaps the main loop of the next).
+//
+//   MODE 0 (gate/up): per stage gate and up chunks (17408 bytes), two
+//     accumulators for the same 128 features; epilogue: g and u are the sums
+//     of the three term columns, H = Swish(g) * u is encoded as three MXFP4
+//     terms straight into the down GEMM's B operand (lanes of a warp = 32
+//     consecutive features = one MXFP4 block of H); with a K split, fp32
+//     partials are added into GU instead and a finish kernel does the rest.
+//   MODE 1 (down): per stage the down chunk (8704 bytes), one accumulator;
+//     epilogue: y[token, f] += w_row * d, red.add into the fp32 output
+//     accumulator (the weighted scatter-combine).
+//
+// Persistent kernel: one CTA per SM, units (expert | token tile, first row,
+// valid rows, feature tile | K split) taken round-robin from a device-built
+// list.  Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer
+// (warp-uniform loops, elect.sync issues), warps 2..9 epilogue (warp w reads
+// TMEM lanes 32*(w%4).. and every other group of 8 token columns).  Every
+// mbarrier wait is bounded; on a timeout the CTA raises an abort flag, all
+// roles leave their loops, in-flight copies and MMAs are drained, TMEM is
+// freed and the status word reports the timeout.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+
+#include "mxq.cuh"
+#include "quantize.cuh"
+#include "routing.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int MXG_EPI_WARPS = 8;
+constexpr int MXG_THREADS = (2 + MXG_EPI_WARPS) * 32;
+constexpr int MXG_MAX_STAGES = 16;
+constexpr int MXG_TMEM_COLS = 512;
+constexpr int MXG_SF_COL0 = 448;      // scale-factor ring: MXG_SF_SLOTS slots of 16 columns
+constexpr int MXG_SF_SLOTS = 4;       //   [A (gate) 4 | A (up) 4 | B atom 0 4 | B atom 1 4]
+constexpr int MXG_SF_SLOT_COLS = 16;
+constexpr int MXG_MAX_ACC = 2;
+constexpr int MXG_MAX_BN = 64;
+constexpr int MXG_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+
+struct MxgParams {
+    const uint8_t* wpack;     // tiled MXFP4 weights (quantize.cuh layout)
+    const int4* units;        // {expert | token tile << 8, first grouped row, valid rows, feature tile | split << 16}
+    const int32_t* sched;
+    TiledMatrix M;            // geometry of the (first) matrix streamed
+    int N;                    // output features
+    int K;                    // contraction length
+    int BN;                   // token rows per tile (16, 32, 48 or 64)
+    int stages;
+    int nacc;                 // accumulator buffers (1 or 2)
+    const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][natb][512]
+    int natb;
+    uint32_t idesc;           // M = 128, N = 3 * BN, without scale-factor ids
+    GroupedOperand Hd;        // MODE 0: H as the down GEMM's B operand
+    float* GU;                // MODE 0 split partials [rows][2N]
+    float* yacc;              // MODE 1 output accumulator [T][N]
+    const int32_t* row_token; // MODE 1
+    const float* row_weight;  // MODE 1
+    int* status;
+    uint64_t timeout_ns;
+    uint32_t skip_first_copy; // test hook: producer skips its first copy
+};
+
+// Weight bytes per stage (codes of 128 rows x 4 blocks + one scale atom, per
+// matrix), B bytes per stage (4 blocks x 3 terms x BN rows x 16 B), B scale
+// atoms per stage, accumulator columns (rounded to 32).
+__host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
+__host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
+__host__ __device__ constexpr int mxg_natb(int BN) { return (MXQ_TERMS * BN + 127) / 128; }
+__host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
+    return mxg_w_stage(mode) + mxg_b_bytes(BN) + 512u * mxg_natb(BN);
+}
+__host__ __device__ constexpr int mxg_mat_cols(int BN) { return ((MXQ_TERMS * BN + 31) / 32) * 32; }
+__host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
+__host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
+__host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
+    const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN) +
+                     (2 * stages + 2 * MXG_MAX_ACC + 1) * 8 + 64;
+    return b < static_cast<size_t>(MXG_MIN_SMEM) ? static_cast<size_t>(MXG_MIN_SMEM) : b;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(MXG_THREADS, 1)
+expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t W_STAGE = mxg_w_stage(MODE);
+
+    const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
+    const uint32_t b_bytes = mxg_b_bytes(BN);
+    const uint32_t sf_bytes = 512u * static_cast<uint32_t>(p.natb);
+    const uint32_t stage_bytes = W_STAGE + b_bytes + sf_bytes;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const uint32_t bar0 = base + S * stage_bytes;                 // barriers (8-byte aligned)
+    auto w_sm = [&](int s) { return base + s * stage_bytes; };    // stage: weights | B codes | B scale atoms
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto accf_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto acce_bar = [&](int b) { return bar0 + 8u * (2 * S + MXG_MAX_ACC + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * MXG_MAX_ACC);
+    uint8_t* ctl = smem_raw + (drain_bar + 8u - raw);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
+    const int mat_cols = mxg_mat_cols(BN);
+    const int acc_cols = (MODE == 0 ? 2 : 1) * mat_cols;
+    const int NACC = p.nacc;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);   // the MMA commit of the stage
+        }
+        for (int b = 0; b < MXG_MAX_ACC; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), MXG_EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), MXG_TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_b);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int num_units = p.sched[MODE == 0 ? SCHED_UNITS_GU : SCHED_UNITS_DN];
+    const int nsplit = p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN];
+    const int KC = p.M.chunks();
+    const size_t expert_bytes = p.M.expert_bytes();
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        // Warp-uniform loop; one elected lane issues each copy.
+        int s = 0;
+        uint32_t ph = 0;
+        int pend_ph[MXG_MAX_STAGES];
+        for (int i = 0; i < MXG_MAX_STAGES; ++i) pend_ph[i] = -1;
+        bool skip = p.skip_first_copy != 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int e = U.x & 0xFF, tile = U.x >> 8;
+            const int ft = U.w & 0xFFFF, sp = U.w >> 16;
+            const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
+            const int rf = min(128, p.N - ft * 128);
+            const uint8_t* we = p.wpack + static_cast<size_t>(e) * expert_bytes;
+            for (int c = c0; c < c1; ++c) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
+                if (skip) {
+                    skip = false;  // test hook: this stage is never filled
+                } else {
+                    const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
+                    const uint32_t st = w_sm(s);
+                    mbar_arrive_expect_tx_warp(full_bar(s), wb + b_bytes + sf_bytes);
+                    bulk_g2s_warp(st, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
+                    tma_load_4d_warp(st + W_STAGE, &tmap_b, 0, U.y, 0, 4 * c, full_bar(s));
+                    bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * sf_bytes,
+                                  sf_bytes, full_bar(s));
+                    pend_ph[s] = static_cast<int>(ph);
+                }
+                if (++s == S) { s = 0; ph ^= 1u; }
+            }
+        }
+        // copies still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int i = 0; i < S; ++i)
+                if (pend_ph[i] >= 0) mbar_wait_drain(full_bar(i), static_cast<uint32_t>(pend_ph[i]), 200000000ull);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        // Per stage: scale atoms to the next tensor-memory slot, then one MMA
+        // per matrix for each pair of 32-blocks (K = 64), scale-factor id 0 or 2.
+        int s = 0, sfs = 0, buf = 0;
+        uint32_t ph = 0;
+        uint32_t eph[MXG_MAX_ACC] = {0u, 0u};
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int ft = U.w & 0xFFFF, sp = U.w >> 16;
+            const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
+            const int rf = min(128, p.N - ft * 128);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(acce_bar(buf), eph[buf] ^ 1u, abort_flag, p.status, p.timeout_ns));
+            if (!ok) break;
+            eph[buf] ^= 1u;
+            tc_fence_after();
+            const uint32_t d0 = tmem + static_cast<uint32_t>(buf * acc_cols);
+            for (int c = c0; c < c1; ++c) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const int nbc = p.M.blocks_in_chunk(c);
+                const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16);
+                const uint32_t mat_b = codes_b + 512u;
+                const uint32_t ws = w_sm(s), bs = ws + W_STAGE, ss = bs + b_bytes;
+                const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
+                tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
+                if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
+                tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
+                if (p.natb > 1) tc_cp_sf_warp(sfc + 12, desc_noswz(ss + 512, 0, 128));
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (2 * i < nbc) {
+                        const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
+                        const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
+                        const uint64_t ad = desc_noswz(ws + 2 * i * rf * 16, rf * 16, 128);
+                        const uint64_t bd = desc_noswz(bs + 2 * i * NB3 * 16, NB3 * 16, 128);
+                        mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8, acc);
+                        if (MODE == 0) mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8, acc);
+                    }
+                }
+                tc_commit_warp(empty_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
+                if (++sfs == MXG_SF_SLOTS) sfs = 0;
+            }
+            if (!ok) break;
+            tc_commit_warp(accf_bar(buf));
+            if (++buf == NACC) buf = 0;
+        }
+        tc_commit_warp(drain_bar);
+        if (lane == 0) mbar_wait_drain(drain_bar, 0, 200000000ull);
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;               // TMEM lane quarter (hardware rule: warp % 4)
+        const int hh = (warp - 2) >> 2;       // which groups of 8 token columns
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        int buf = 0;
+        uint32_t fph[MXG_MAX_ACC] = {0u, 0u};
+        bool ok = true;
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const int4 U = p.units[u];
+            const int tile = U.x >> 8, row0 = U.y, nvalid = U.z;
+            const int ft = U.w & 0xFFFF;
+            const int rf = min(128, p.N - ft * 128);
+            const bool warp_rows = 32 * q < rf;
+            const int n = ft * 128 + 32 * q + lane;
+            {
+                const bool w_ok = mbar_wait_bounded(accf_bar(buf), fph[buf], abort_flag, p.status, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+            }
+            fph[buf] ^= 1u;
+            tc_fence_after();
+            if (warp_rows) {
+                const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
+                for (int r0 = 8 * hh; r0 < nvalid; r0 += 16) {
+                    uint32_t g[MXQ_TERMS][8], v[MXQ_TERMS][8];
+#pragma unroll
+                    for (int t = 0; t < MXQ_TERMS; ++t) {
+                        tmem_ld8(d0 + t * BN + r0, g[t]);
+                        if (MODE == 0) tmem_ld8(d0 + mat_cols + t * BN + r0, v[t]);
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = r0 + j;
+                        if (r < nvalid) {
+                            const float gg = __uint_as_float(g[0][j]) + __uint_as_float(g[1][j]) + __uint_as_float(g[2][j]);
+                            if (MODE == 0) {
+                                const float uu =
+                                    __uint_as_float(v[0][j]) + __uint_as_float(v[1][j]) + __uint_as_float(v[2][j]);
+                                if (nsplit == 1) {
+                                    store_h_block(p.Hd, swish_f(gg) * uu, lane, 4 * ft + q, row0 + r, tile, r, BN);
+                                } else {
+                                    float* gu = p.GU + static_cast<size_t>(row0 + r) * 2 * p.N;
+                                    atomicAdd(gu + n, gg);
+                                    atomicAdd(gu + p.N + n, uu);
+                                }
+                            } else {
+                                const int rr = row0 + r;
+                                atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n, gg * p.row_weight[rr]);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar(buf));
+            if (++buf == NACC) buf = 0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, MXG_TMEM_COLS);
+    }
+}
+
+}  // namespace moe

@@ -7,10 +7,12 @@
 //                        selected scores, per-tile histogram and ranks, zeroing
 //                        of the output rows; its last CTA builds the schedule
 //                        (expert offsets, K splits, unit lists)
-//   gather_kernel        grouped rows (token, weight) and f16 activation gather
-//   expert_gemm<0>       gate/up GEMM, SwiGLU epilogue
+//   gather_kernel        grouped rows (token, weight, tile slot); activations
+//                        encoded as three MXFP4 terms (the B operand)
+//   expert_mxf4<0>       gate/up GEMM on block-scaled MXFP4 tensor cores,
+//                        SwiGLU epilogue encoding H for the down GEMM
 //   swiglu_finish_kernel only when the gate/up GEMM may split K
-//   expert_gemm<1>       down GEMM, routing-weighted scatter-combine epilogue
+//   expert_mxf4<1>       down GEMM, routing-weighted scatter-combine epilogue
 //   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -25,7 +27,7 @@
 #include <new>
 
 #include "../../include/moe_mxfp4.h"
-#include "expert_gemm.cuh"
+#include "expert_mxf4.cuh"
 #include "quantize.cuh"
 #include "routing.cuh"
 
@@ -33,7 +35,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int BN_OPTIONS = 8;  // BN = 16 * (i + 1)
+constexpr int BN_OPTIONS = 4;  // BN = 16 * (i + 1): 16, 32, 48, 64
 constexpr int SPLIT_ROWS_CAP = 2048;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -64,8 +66,6 @@ struct moe_mxfp4 {
     // weights
     uint8_t* w_gu = nullptr;   // tiled gate+up
     uint8_t* w_dn = nullptr;   // tiled down
-    uint8_t* rs_gu = nullptr;  // [E][2][d_ff]
-    uint8_t* rs_dn = nullptr;  // [E][d_model]
     void* w_router = nullptr;
     float* bias = nullptr;
     bool has_bias = false, router_set = false;
@@ -79,13 +79,18 @@ struct moe_mxfp4 {
     int* counters = nullptr;   // [nblk_max] tile counters + [1] global counter
     int32_t* local_rank = nullptr;
     int32_t* offsets = nullptr;
+    int32_t* tile_base = nullptr;
     int32_t* sched = nullptr;
     int4* units_gu = nullptr;
     int4* units_dn = nullptr;
     int32_t* row_token = nullptr;
     float* row_weight = nullptr;
-    __half* Xp = nullptr;
-    __half* H = nullptr;
+    int32_t* row_slot = nullptr;
+    uint8_t* Xq = nullptr;     // x as three MXFP4 terms [d/32][3][TK][16]
+    uint8_t* Hq = nullptr;     // H as three MXFP4 terms [d_ff/32][3][TK][16]
+    uint8_t* sfx = nullptr;    // scale atoms of Xq per (token tile, K chunk)
+    uint8_t* sfh = nullptr;    // scale atoms of Hq per (token tile, K chunk)
+    size_t sfx_bytes = 0, sfh_bytes = 0, xq_bytes = 0, hq_bytes = 0;
     float* GU = nullptr;
     float* yacc = nullptr;
     int* status = nullptr;
@@ -116,9 +121,9 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
     } while (0)
 
 static void free_all(moe_mxfp4* h) {
-    void* ptrs[] = {h->w_gu, h->w_dn, h->rs_gu, h->rs_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
-                    h->part, h->counters, h->local_rank,
-                    h->offsets, h->sched, h->units_gu, h->units_dn, h->row_token, h->row_weight, h->Xp, h->H,
+    void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
+                    h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
+                    h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
     for (void* p : ptrs)
         if (p) cudaFree(p);
@@ -127,11 +132,46 @@ static void free_all(moe_mxfp4* h) {
     delete[] h->expert_done;
 }
 
-static int choose_bn(int T, int k, int E) {
-    long per_expert = (static_cast<long>(T) * k + E - 1) / E;
-    long want = std::min<long>(T, std::max<long>(1, 4 * per_expert));
-    int bn = static_cast<int>((want + 15) / 16) * 16;
-    return std::max(16, std::min(128, bn));
+// Token rows per tile: about three times the mean rows per expert, so that
+// most experts need one tile (each tile streams the expert's weights once),
+// rounded up to 16 and capped at 64 (N = 3 * BN <= 192).  Flags may force it.
+static int choose_bn(int T, int k, int E, uint32_t flags) {
+    const uint32_t forced = (flags & MOE_FLAG_TOKEN_TILE_MASK) >> MOE_FLAG_TOKEN_TILE_SHIFT;
+    if (forced >= 1 && forced <= BN_OPTIONS) return 16 * static_cast<int>(forced);
+    const long per_expert = (static_cast<long>(T) * k + E - 1) / E;
+    const long want = std::min<long>(T, std::max<long>(1, 3 * per_expert));
+    const int bn = static_cast<int>((want + 15) / 16) * 16;
+    return std::max(16, std::min(MXG_MAX_BN, bn));
+}
+
+// Largest (token tiles x scale atoms per chunk) over the tile sizes: tiles of
+// an expert with n rows = ceil(n / BN), so at most TK / BN + E tiles.
+static size_t max_tile_atoms(size_t TK, int E) {
+    size_t m = 0;
+    for (int i = 0; i < BN_OPTIONS; ++i) {
+        const int BN = 16 * (i + 1);
+        m = std::max(m, (TK / BN + E) * static_cast<size_t>(mxg_natb(BN)));
+    }
+    return m;
+}
+
+static TiledMatrix tiled(moe_mxfp4* h, int which) {
+    const auto& c = h->cfg;
+    TiledMatrix M;
+    if (which < 2) {
+        M.base = h->w_gu;
+        M.N = c.d_ff;
+        M.K = c.d_model;
+        M.NM = 2;
+        M.sub = which;
+    } else {
+        M.base = h->w_dn;
+        M.N = c.d_model;
+        M.K = c.d_ff;
+        M.NM = 1;
+        M.sub = 0;
+    }
+    return M;
 }
 
 static int router_splits(int T, int d, int nsm) {
@@ -161,8 +201,8 @@ static cudaError_t set_router_smem(int bytes) {
 
 static int stages_for(int mode, int BN) {
     const size_t budget = 227 * 1024 - 1024 - 512;
-    int s = static_cast<int>(budget / gemm_stage_bytes(mode, BN));
-    return std::max(2, std::min(GEMM_MAX_STAGES, s));
+    int s = static_cast<int>(budget / mxg_stage_bytes(mode, BN));
+    return std::max(2, std::min(MXG_MAX_STAGES, s));
 }
 
 extern "C" {
@@ -229,25 +269,29 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     h->TK = c.max_tokens * k;
     h->nblk_max = (c.max_tokens + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
     {
-        const long tiles_big = static_cast<long>(h->TK) / 128 + E + 2;
-        const long tiles_small = 512 / 16 + E + 2;
+        // every unit of the unsplit schedule fits: at most TK / 16 + E token
+        // tiles (the smallest tile) times the feature tiles; K splits are only
+        // chosen while the split list still fits
+        const long tiles = static_cast<long>(h->TK) / 16 + E + 2;
         const long F = std::max(h->F_gu, h->F_dn);
-        h->max_units = static_cast<int>(std::max(tiles_big, tiles_small) * F + 8L * h->nsm + 64);
+        h->max_units = static_cast<int>(tiles * F + 8L * h->nsm + 64);
     }
     h->gu_rows = std::min(h->TK, SPLIT_ROWS_CAP);
     h->part_elems = static_cast<size_t>(64 * h->nsm + ROUTER_TOKENS * h->nblk_max + ROUTER_TOKENS) * E;
     h->expert_done = new (std::nothrow) bool[E]();
     if (!h->expert_done) return fail(MOE_ERR_CUDA);
 
-    const size_t gu_bytes = static_cast<size_t>(E) * f * (d / 32) * 17 * 2;
-    const size_t dn_bytes = static_cast<size_t>(E) * d * (f / 32) * 17;
     const size_t TK = h->TK;
+    h->xq_bytes = static_cast<size_t>(d / 32) * MXQ_TERMS * TK * 16;
+    h->hq_bytes = static_cast<size_t>(f / 32) * MXQ_TERMS * TK * 16;
+    h->sfx_bytes = max_tile_atoms(TK, E) * h->KC_gu * 512;
+    h->sfh_bytes = max_tile_atoms(TK, E) * h->KC_dn * 512;
+    const size_t gu_bytes = static_cast<size_t>(E) * tiled(h, 0).expert_bytes();
+    const size_t dn_bytes = static_cast<size_t>(E) * tiled(h, 2).expert_bytes();
     struct A { void** p; size_t bytes; };
     A allocs[] = {
         {reinterpret_cast<void**>(&h->w_gu), gu_bytes},
         {reinterpret_cast<void**>(&h->w_dn), dn_bytes},
-        {reinterpret_cast<void**>(&h->rs_gu), static_cast<size_t>(E) * 2 * f},
-        {reinterpret_cast<void**>(&h->rs_dn), static_cast<size_t>(E) * d},
         {&h->w_router, static_cast<size_t>(E) * d * h->act_bytes},
         {reinterpret_cast<void**>(&h->bias), sizeof(float) * E},
         {reinterpret_cast<void**>(&h->idx_ws), sizeof(int32_t) * TK},
@@ -257,13 +301,17 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->counters), sizeof(int) * (h->nblk_max + 1)},
         {reinterpret_cast<void**>(&h->local_rank), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->offsets), sizeof(int32_t) * (E + 1)},
+        {reinterpret_cast<void**>(&h->tile_base), sizeof(int32_t) * E},
         {reinterpret_cast<void**>(&h->sched), sizeof(int32_t) * SCHED_SLOTS},
         {reinterpret_cast<void**>(&h->units_gu), sizeof(int4) * h->max_units},
         {reinterpret_cast<void**>(&h->units_dn), sizeof(int4) * h->max_units},
         {reinterpret_cast<void**>(&h->row_token), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->row_weight), sizeof(float) * TK},
-        {reinterpret_cast<void**>(&h->Xp), sizeof(__half) * TK * d},
-        {reinterpret_cast<void**>(&h->H), sizeof(__half) * TK * f},
+        {reinterpret_cast<void**>(&h->row_slot), sizeof(int32_t) * TK},
+        {reinterpret_cast<void**>(&h->Xq), h->xq_bytes},
+        {reinterpret_cast<void**>(&h->Hq), h->hq_bytes},
+        {reinterpret_cast<void**>(&h->sfx), h->sfx_bytes},
+        {reinterpret_cast<void**>(&h->sfh), h->sfh_bytes},
         {reinterpret_cast<void**>(&h->GU), sizeof(float) * h->gu_rows * 2 * f},
         {reinterpret_cast<void**>(&h->yacc), sizeof(float) * static_cast<size_t>(c.max_tokens) * d},
         {reinterpret_cast<void**>(&h->status), sizeof(int) * 4},
@@ -274,19 +322,23 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     };
     for (auto& a : allocs)
         if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
-    // Grouped activation / hidden buffers start as zeros so rows a tile reads past
-    // its expert's segment are finite; the status word starts clear.
-    if (cudaMemset(h->Xp, 0, sizeof(__half) * TK * d) != cudaSuccess ||
-        cudaMemset(h->H, 0, sizeof(__half) * TK * f) != cudaSuccess ||
+    // Operand buffers start as zeros: codes, scale atoms and the weights' padding
+    // are then always finite (an E2M1 code is never NaN; scale bytes written by
+    // the kernels are at most 253, never the E8M0 NaN 0xFF), so operand rows a
+    // tile reads past its expert's rows only feed accumulator columns that the
+    // epilogue drops.  The status word starts clear.
+    if (cudaMemset(h->Xq, 0, h->xq_bytes) != cudaSuccess || cudaMemset(h->Hq, 0, h->hq_bytes) != cudaSuccess ||
+        cudaMemset(h->sfx, 0, h->sfx_bytes) != cudaSuccess || cudaMemset(h->sfh, 0, h->sfh_bytes) != cudaSuccess ||
+        cudaMemset(h->w_gu, 0, gu_bytes) != cudaSuccess || cudaMemset(h->w_dn, 0, dn_bytes) != cudaSuccess ||
         cudaMemset(h->status, 0, sizeof(int) * 4) != cudaSuccess ||
         cudaMemset(h->counters, 0, sizeof(int) * (h->nblk_max + 1)) != cudaSuccess ||
         cudaMemset(h->bias, 0, sizeof(float) * E) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return fail(MOE_ERR_CUDA);
 
     if (!g_attrs_set) {
-        if (cudaFuncSetAttribute(expert_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+        if (cudaFuncSetAttribute(expert_mxf4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(expert_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaFuncSetAttribute(expert_mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
                 cudaSuccess ||
             set_router_smem<float>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess ||
             set_router_smem<__nv_bfloat16>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess)
@@ -306,26 +358,6 @@ void moe_mxfp4_destroy(moe_mxfp4_t* h) {
     delete h;
 }
 
-static TiledMatrix tiled(moe_mxfp4* h, int which) {
-    const auto& c = h->cfg;
-    TiledMatrix M;
-    if (which < 2) {
-        M.base = h->w_gu;
-        M.N = c.d_ff;
-        M.K = c.d_model;
-        M.BPC = 4;
-        M.NM = 2;
-        M.sub = which;
-    } else {
-        M.base = h->w_dn;
-        M.N = c.d_model;
-        M.K = c.d_ff;
-        M.BPC = 4;
-        M.NM = 1;
-        M.sub = 0;
-    }
-    return M;
-}
 
 // Quantise experts [e0, e0+ne) of one matrix from fp32 [ne][K][N].
 static moe_status_t quantize_matrix(moe_mxfp4* h, int which, const float* W, int e0, int ne, cudaStream_t s) {
@@ -334,17 +366,6 @@ static moe_status_t quantize_matrix(moe_mxfp4* h, int which, const float* W, int
     const dim3 blk(128);
     const dim3 grid((M.N + 127) / 128, M.nb(), ne);
     quantize_kernel<<<grid, blk, 0, s>>>(W, static_cast<size_t>(M.K) * M.N, M);
-    h->launches++;
-    uint8_t* rs;
-    size_t rs_stride;
-    if (which < 2) {
-        rs = h->rs_gu + (static_cast<size_t>(e0) * 2 + which) * M.N;
-        rs_stride = 2 * static_cast<size_t>(M.N);
-    } else {
-        rs = h->rs_dn + static_cast<size_t>(e0) * M.N;
-        rs_stride = M.N;
-    }
-    rowscale_kernel<<<dim3((M.N + 127) / 128, 1, ne), blk, 0, s>>>(M, rs, rs_stride);
     h->launches++;
     return cuda_status(cudaGetLastError());
 }
@@ -407,21 +428,26 @@ moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* hc, int32_t which, uint
     return cuda_status(cudaGetLastError());
 }
 
+// 4-D maps over the three-term operands [K/32 blocks][3 terms][TK rows][16 B]:
+// box {16 B, BN rows, 3 terms, 4 blocks} lands in shared memory as
+// [4 blocks][3 terms][BN rows][16 B], the unswizzled K-major layout of an
+// N = 3 * BN operand.  Rows past TK and blocks past K/32 read as zeros.
 static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
     const int i = BN / 16 - 1;
     if (h->tm_ok[i]) return MOE_OK;
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return MOE_ERR_CUDA;
     const auto& c = h->cfg;
+    const cuuint64_t R = static_cast<cuuint64_t>(h->TK);
     for (int which = 0; which < 2; ++which) {
-        const cuuint64_t cols = which == 0 ? c.d_model : c.d_ff;
-        cuuint64_t dims[2] = {cols, static_cast<cuuint64_t>(h->TK)};
-        cuuint64_t strides[1] = {cols * sizeof(__half)};
-        cuuint32_t box[2] = {64, static_cast<cuuint32_t>(BN)};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                         which == 0 ? static_cast<void*>(h->Xp) : static_cast<void*>(h->H), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        const cuuint64_t nb = (which == 0 ? c.d_model : c.d_ff) / 32;
+        cuuint64_t dims[4] = {16, R, MXQ_TERMS, nb};
+        cuuint64_t strides[3] = {16, R * 16, R * 16 * MXQ_TERMS};
+        cuuint32_t box[4] = {16, static_cast<cuuint32_t>(BN), MXQ_TERMS, 4};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+                         which == 0 ? static_cast<void*>(h->Xq) : static_cast<void*>(h->Hq), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
     }
@@ -440,7 +466,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     h->last_stream = stream;
     if (T == 0) return MOE_OK;
     const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
-    const int BN = choose_bn(T, k, E);
+    const int BN = choose_bn(T, k, E, c.flags);
     moe_status_t st = ensure_tmaps(h, BN);
     if (st != MOE_OK) return st;
     const int nblk = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
@@ -456,7 +482,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
 
     // 0: router + top-k + softmax + schedule
     mark(0);
-    RouterArgs ra;
+    RouterArgs ra{};
     ra.x = x;
     ra.wr = h->w_router;
     ra.bias = h->has_bias ? h->bias : nullptr;
@@ -483,6 +509,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.split_rows_cap = h->gu_rows;
     ra.max_units = h->max_units;
     ra.offsets = h->offsets;
+    ra.tile_base = h->tile_base;
     ra.counts_out = expert_counts;
     ra.units_gu = h->units_gu;
     ra.units_dn = h->units_dn;
@@ -497,21 +524,23 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 1: gather into grouped rows
     mark(1);
     const int gblocks = (T * k + GATHER_WARPS - 1) / GATHER_WARPS;
+    const int natb = mxg_natb(BN);
+    GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, natb};
+    GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, natb};
     if (bf16)
         gather_kernel<__nv_bfloat16><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, T, d, E, k,
-            h->row_token, h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+            static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E,
+            k, BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, h->sched);
     else
         gather_kernel<float><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
-            static_cast<const float*>(x), idx, wts, h->local_rank, h->hist, h->offsets, T, d, E, k, h->row_token,
-            h->row_weight, h->Xp, h->GU, 2 * f, h->sched);
+            static_cast<const float*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E, k, BN,
+            h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, h->sched);
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);
     const uint64_t tmo = static_cast<uint64_t>(c.wait_timeout_ms > 0 ? c.wait_timeout_ms : 2000) * 1000000ull;
-    GemmParams gp;
+    MxgParams gp{};
     gp.wpack = h->w_gu;
-    gp.rowscale = h->rs_gu;
     gp.units = h->units_gu;
     gp.sched = h->sched;
     gp.M = tiled(h, 0);
@@ -519,9 +548,11 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.K = d;
     gp.BN = BN;
     gp.stages = stages_for(0, BN);
-    gp.a_slots = gemm_a_slots(0, BN);
-    gp.idesc = idesc_f16_f32(128, BN);
-    gp.H = h->H;
+    gp.nacc = mxg_nacc(0, BN);
+    gp.sfb = h->sfx;
+    gp.natb = natb;
+    gp.idesc = idesc_mxf4(128, MXQ_TERMS * BN);
+    gp.Hd = Hop;
     gp.GU = h->GU;
     gp.yacc = nullptr;
     gp.row_token = h->row_token;
@@ -530,32 +561,32 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.timeout_ns = tmo;
     gp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
     const int grid = h->nsm;
-    expert_gemm_kernel<0><<<grid, GEMM_THREADS, gemm_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
+    expert_mxf4_kernel<0><<<grid, MXG_THREADS, mxg_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
     h->stage_ran[2] = true;
     // 3: split-K finish (no-op unless the schedule split K)
     mark(3);
     const bool may_split = static_cast<long>(T) * k <= h->gu_rows;
     if (may_split) {
-        const int blocks = std::min<long>(4L * h->nsm, (static_cast<long>(T) * k * f + 255) / 256);
-        swiglu_finish_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->GU, h->H, f, h->sched);
+        const long items = static_cast<long>(T) * k * (f / 32);
+        const int blocks = static_cast<int>(std::min<long>(4L * h->nsm, (items + 7) / 8));
+        swiglu_finish_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->GU, Hop, f, BN, h->row_slot, h->sched);
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine
     mark(4);
-    GemmParams dp = gp;
+    MxgParams dp = gp;
     dp.wpack = h->w_dn;
-    dp.rowscale = h->rs_dn;
     dp.units = h->units_dn;
     dp.M = tiled(h, 2);
     dp.N = d;
     dp.K = f;
     dp.stages = stages_for(1, BN);
-    dp.a_slots = gemm_a_slots(1, BN);
-    dp.H = nullptr;
+    dp.nacc = mxg_nacc(1, BN);
+    dp.sfb = h->sfh;
     dp.GU = nullptr;
     dp.yacc = acc;
     dp.skip_first_copy = 0;
-    expert_gemm_kernel<1><<<grid, GEMM_THREADS, gemm_smem_bytes(1, BN, dp.stages), stream>>>(h->tm_h[BN / 16 - 1], dp);
+    expert_mxf4_kernel<1><<<grid, MXG_THREADS, mxg_smem_bytes(1, BN, dp.stages), stream>>>(h->tm_h[BN / 16 - 1], dp);
     h->stage_ran[4] = true;
     // 5: output cast
     mark(5);
@@ -723,7 +754,7 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     int* counters = reinterpret_cast<int*>(sc + NA_OFF_CNT);
     // the arrival counters must start at zero (a previous call may have been cut short)
     if (cudaMemsetAsync(counters, 0, sizeof(int) * (tiles + 1), stream) != cudaSuccess) return MOE_ERR_CUDA;
-    RouterArgs ra;
+    RouterArgs ra{};
     ra.x = x;
     ra.wr = w_router;
     ra.bias = router_bias;
@@ -752,6 +783,7 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     ra.split_rows_cap = 0;
     ra.max_units = 0;
     ra.offsets = reinterpret_cast<int32_t*>(sc + NA_OFF_OFFS);
+    ra.tile_base = nullptr;
     ra.counts_out = expert_counts;
     ra.units_gu = nullptr;
     ra.units_dn = nullptr;

@@ -1,0 +1,117 @@
+// mxq.cuh -- activations as sums of three MXFP4 terms, the operand format the
+// block-scaled expert GEMMs read.
+//
+// The expert weights are MXFP4 (page "GPT-OSS-20B : Architecture MoE & Résumé
+// du Model Card", §4 Quantification MXFP4: E2M1 values in blocks of 32 with
+// one shared E8M0 scale).  The tensor cores' block-scaled MMA multiplies two
+// MXFP4 operands, so the activations (x for gate/up, the SwiGLU output H for
+// down) are encoded in the same format.  One MXFP4 term keeps about two
+// significant bits, far too coarse for the layer's accuracy, so a block v of
+// 32 values is written as v ~= q1 + q2 + q3: q1 encodes v, q2 encodes the
+// residual v - q1, q3 the residual v - q1 - q2, each with its own scale.  The
+// MMA takes the three terms as three groups of N rows; the epilogue adds the
+// three accumulator columns.  Measured on the oracle's weights (double
+// precision emulation), the layer error of the 3-term encoding is about 0.25 %
+// of max|y| (2 terms: about 3 %).
+//
+// Scale rule of a term: the smallest power of two 2^e with max|v| <= 6 * 2^e,
+// so no element saturates; elements round to the nearest E2M1 value with ties
+// to the even code (the hardware conversion).
+//
+// Operand layouts in global memory (R = row capacity, NB = K / 32 blocks):
+//   codes   [NB][3 terms][R rows][16 B]   (element 2i of the block in the low nibble of byte i)
+//   scales  per (token tile, K chunk of 128): natb atoms of 512 B; operand row
+//           n = term * BN + row-in-tile, block q (0..3) of the chunk at byte
+//           sf_atom_offset(n, q).
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int MXQ_TERMS = 3;
+
+// Byte of the scale of operand row n (n < 256) and block q (0..3) within the
+// scale atoms of one K chunk: atom n / 128, then 16 * (n % 32) + 4 * ((n / 32) % 4) + q.
+// tcgen05.cp 32x128b.warpx4 copies an atom into 4 tensor-memory columns of lanes
+// 0..31 (replicated over the lane quarters); the MMA reads row n's scales at
+// column n / 32, byte q (+ the sf id).
+__host__ __device__ constexpr uint32_t sf_atom_offset(int n, int q) {
+    return static_cast<uint32_t>((n >> 7) * 512 + 16 * (n & 31) + 4 * ((n >> 5) & 3) + q);
+}
+
+// Exponent e of the scale 2^e of a term whose largest magnitude has bits
+// `amax_bits`: the smallest e with amax <= 6 * 2^e.  amax = m 2^E0 with m in
+// [1, 2): e = E0 - 2 when m <= 1.5, else E0 - 1.  -127 for zero or subnormal
+// amax (the E8M0 minimum).
+__device__ __forceinline__ int mxq_exp(uint32_t amax_bits) {
+    const int ex = static_cast<int>(amax_bits >> 23);
+    if (ex == 0) return -127;
+    const int e = ex - 129 + ((amax_bits & 0x7FFFFFu) > 0x400000u ? 1 : 0);
+    return e < -127 ? -127 : e;
+}
+// 2^-e for e in [-127, 126] and 2^e for e in [-127, 127], exact.
+__device__ __forceinline__ float mxq_inv(int e) { return __int_as_float((127 - e) << 23); }
+__device__ __forceinline__ float mxq_scale(int e) {
+    return e > -127 ? __int_as_float((127 + e) << 23) : __int_as_float(0x00400000);
+}
+
+// One thread encodes one block of 32 values (v is overwritten with the final
+// residual).  codes[t] = the 16 code bytes of term t, sbyte[t] = its E8M0 byte.
+__device__ __forceinline__ void mxq_block_thread(float (&v)[32], uint4 (&codes)[MXQ_TERMS],
+                                                 uint32_t (&sbyte)[MXQ_TERMS]) {
+#pragma unroll
+    for (int t = 0; t < MXQ_TERMS; ++t) {
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+        const int e = mxq_exp(__float_as_uint(am));
+        sbyte[t] = static_cast<uint32_t>(e + 127);
+        const float inv = mxq_inv(e), sc = mxq_scale(e);
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t byte = e2m1x2_from_f32(v[2 * i] * inv, v[2 * i + 1] * inv);
+            w[i >> 2] |= byte << (8 * (i & 3));
+            if (t + 1 < MXQ_TERMS) {
+                const uint32_t h2 = e2m1x2_to_f16x2(byte);
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+                v[2 * i] -= f.x * sc;
+                v[2 * i + 1] -= f.y * sc;
+            }
+        }
+        codes[t] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// A full warp encodes one block: lane l holds element l.  On return, lanes 0,
+// 8, 16 and 24 hold word l / 8 of each term's 16 code bytes in word[t]; every
+// lane holds the scale bytes.
+__device__ __forceinline__ void mxq_block_warp(float v, int lane, uint32_t (&word)[MXQ_TERMS],
+                                               uint32_t (&sbyte)[MXQ_TERMS]) {
+    const bool odd = (lane & 1) != 0;
+    float r = v;
+#pragma unroll
+    for (int t = 0; t < MXQ_TERMS; ++t) {
+        // |r| compares as an unsigned integer: the warp maximum in one reduction
+        const uint32_t amb = __reduce_max_sync(0xffffffffu, __float_as_uint(r) & 0x7FFFFFFFu);
+        const int e = mxq_exp(amb);
+        sbyte[t] = static_cast<uint32_t>(e + 127);
+        const float a = r * mxq_inv(e);
+        const float o = __shfl_xor_sync(0xffffffffu, a, 1);
+        const uint32_t byte = e2m1x2_from_f32(odd ? o : a, odd ? a : o);
+        if (t + 1 < MXQ_TERMS) {
+            const uint32_t h2 = e2m1x2_to_f16x2(byte);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+            r -= (odd ? f.y : f.x) * mxq_scale(e);
+        }
+        uint32_t w = byte;
+        w |= __shfl_down_sync(0xffffffffu, w, 2) << 8;
+        w |= __shfl_down_sync(0xffffffffu, w, 4) << 16;
+        word[t] = w;
+    }
+}
+
+}  // namespace moe

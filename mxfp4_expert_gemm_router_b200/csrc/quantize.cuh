@@ -10,18 +10,20 @@
 // even code, magnitudes above 6 saturate, the sign bit is kept; an all-zero
 // block gets scale byte 127.
 //
-// Streamed layout ("tiled"): rows (output features) are cut into 128-row
-// feature tiles (the last one holds the remainder rf) and each row's nb = K/32
-// blocks into chunks of BPC blocks (the last chunk may hold fewer, nb_c).  For
-// each (tile, chunk) the bytes of the NM interleaved matrices (gate and up, or
-// down alone) are contiguous, matrix after matrix:
-//     codes  [nb_c blocks][rf rows][16 B]   (even element in the low nibble)
-//     scales [nb_c blocks][rf rows]          (E8M0 bytes)
-// i.e. 17 bytes per row per block, exactly 4.25 bits per parameter with no
-// padding.  One further byte per row, the largest scale over the row's
-// non-zero blocks ("row scale", 127 if none), lets the GEMM decode each block
-// as f16 relative to its row and apply 2^(row scale - 127) in fp32 after
-// accumulation.
+// Streamed layout ("tiled"), the A operand of the block-scaled MMA: rows
+// (output features) are cut into 128-row feature tiles (the last one holds the
+// remainder rf) and each row's nb = K/32 blocks into chunks of 4 blocks (K =
+// 128; the last chunk may hold fewer, nbc).  For each (tile, chunk) the NM
+// interleaved matrices (gate and up, or down alone) follow one another, each as
+//     codes  [nbc blocks][rf rows][16 B]   (even element in the low nibble)
+//     scales one 512-byte atom: row r, block h at 16*(r%32) + 4*(r/32) + h
+// so that one bulk copy brings a chunk into shared memory where the codes are
+// a K-major, unswizzled canonical operand (8-row core matrices of 128 B) and
+// the atom is what tcgen05.cp moves into tensor memory.  Codes take exactly
+// 4 bits per parameter; the scale atoms add 8 bits per 32 parameters, plus
+// padding where a tile has fewer than 128 rows or a chunk fewer than 4 blocks
+// (0.26 % for the 2880 x 2880 experts).  Padding bytes stay zero (a finite
+// scale, 2^-127).
 #pragma once
 #include <cstdint>
 
@@ -30,19 +32,28 @@ namespace moe {
 struct TiledMatrix {
     uint8_t* base;   // expert 0 of the packed array
     int N, K;        // rows, contraction length (K % 32 == 0)
-    int BPC;         // 32-blocks per chunk
     int NM;          // matrices interleaved per chunk (2: gate+up, 1: down)
     int sub;         // which matrix of the chunk this one is (0 or 1)
+    static constexpr int BPC = 4;   // 32-blocks per chunk
     __host__ __device__ int nb() const { return K / 32; }
     __host__ __device__ int chunks() const { return (nb() + BPC - 1) / BPC; }
-    __host__ __device__ size_t expert_bytes() const { return static_cast<size_t>(N) * nb() * 17 * NM; }
+    __host__ __device__ int tiles() const { return (N + 127) / 128; }
     __host__ __device__ int blocks_in_chunk(int c) const { return min(BPC, nb() - c * BPC); }
+    // bytes of one matrix's part of a chunk: codes + one scale atom
+    __host__ __device__ size_t mat_bytes(int c, int rf) const {
+        return static_cast<size_t>(blocks_in_chunk(c)) * rf * 16 + 512;
+    }
+    __host__ __device__ size_t chunk_bytes(int c, int rf) const { return NM * mat_bytes(c, rf); }
+    __host__ __device__ size_t tile_offset(int ft) const {
+        return static_cast<size_t>(ft) * NM * (static_cast<size_t>(128) * 16 * nb() + 512 * static_cast<size_t>(chunks()));
+    }
     // byte offset, within one expert, of feature tile ft's chunk c (all NM matrices)
     __host__ __device__ size_t chunk_offset(int ft, int c, int rf) const {
-        return static_cast<size_t>(ft) * 128 * nb() * 17 * NM + static_cast<size_t>(c) * BPC * 17 * NM * rf;
+        return tile_offset(ft) + static_cast<size_t>(c) * NM * (static_cast<size_t>(BPC) * rf * 16 + 512);
     }
-    __host__ __device__ size_t chunk_bytes(int c, int rf) const {
-        return static_cast<size_t>(blocks_in_chunk(c)) * 17 * NM * rf;
+    __host__ __device__ size_t expert_bytes() const {
+        return static_cast<size_t>(NM) *
+               (static_cast<size_t>(N) * 16 * nb() + 512 * static_cast<size_t>(chunks()) * tiles());
     }
     // byte offsets (within one expert) of block b of row n of this matrix
     __host__ __device__ void locate(int n, int b, size_t& code_off, size_t& scale_off) const {
@@ -50,9 +61,9 @@ struct TiledMatrix {
         const int rf = min(128, N - (ft << 7));
         const int c = b / BPC, h = b % BPC;
         const int nbc = blocks_in_chunk(c);
-        const size_t base_m = chunk_offset(ft, c, rf) + static_cast<size_t>(sub) * 17 * nbc * rf;
+        const size_t base_m = chunk_offset(ft, c, rf) + static_cast<size_t>(sub) * mat_bytes(c, rf);
         code_off = base_m + static_cast<size_t>(h * rf + r) * 16;
-        scale_off = base_m + 16 * static_cast<size_t>(nbc) * rf + h * rf + r;
+        scale_off = base_m + static_cast<size_t>(nbc) * rf * 16 + 16 * (r & 31) + 4 * (r >> 5) + h;
     }
 };
 
@@ -107,24 +118,6 @@ __global__ void quantize_kernel(const float* __restrict__ W, size_t w_expert_str
     }
     *reinterpret_cast<uint4*>(dst + co) = out;
     dst[so] = static_cast<uint8_t>(scale);
-}
-
-// Row scale = largest scale byte over the row's blocks that hold a non-zero
-// code (127 when the row is all zero).
-__global__ void rowscale_kernel(TiledMatrix M, uint8_t* __restrict__ rowscale, size_t rs_expert_stride) {
-    const int n = blockIdx.x * blockDim.x + threadIdx.x;
-    const int e = blockIdx.z;
-    if (n >= M.N) return;
-    const uint8_t* src = M.base + static_cast<size_t>(e) * M.expert_bytes();
-    int best = -1;
-    for (int b = 0; b < M.nb(); ++b) {
-        size_t co, so;
-        M.locate(n, b, co, so);
-        const uint4 c = *reinterpret_cast<const uint4*>(src + co);
-        const uint32_t nz = (c.x | c.y | c.z | c.w) & 0x77777777u;
-        if (nz) best = max(best, static_cast<int>(src[so]));
-    }
-    rowscale[static_cast<size_t>(e) * rs_expert_stride + n] = static_cast<uint8_t>(best < 0 ? 127 : best);
 }
 
 // Tiled -> canonical: codes [E][N][K/2], scales [E][N][K/32].

@@ -12,6 +12,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "mxq.cuh"
+
 namespace moe {
 
 constexpr int ROUTER_TOKENS = 32;   // tokens per router tile
@@ -80,6 +82,7 @@ struct RouterArgs {
     // schedule
     int BN, F_gu, F_dn, KC_gu, KC_dn, nsm, split_rows_cap, max_units;
     int32_t* offsets;      // [E+1]
+    int32_t* tile_base;    // [E] first token tile of each expert (tiles numbered over all experts), or null
     int32_t* counts_out;   // [E] or null
     int4* units_gu;
     int4* units_dn;
@@ -147,25 +150,34 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
     }
     __syncthreads();
     for (int e = tid; e <= a.E; e += blockDim.x) a.offsets[e] = off[e];
+    if (a.tile_base && tid == 0) {
+        int tb = 0;
+        for (int e = 0; e < a.E; ++e) {
+            a.tile_base[e] = tb;
+            tb += (cnt[e] + a.BN - 1) / a.BN;
+        }
+    }
     if (a.counts_out)
         for (int e = tid; e < a.E; e += blockDim.x) a.counts_out[e] = cnt[e];
     for (int g = 0; g < 2; ++g) {
         const int F = g ? a.F_dn : a.F_gu;
         const int S = split_s[g];
         int4* units = g ? a.units_dn : a.units_gu;
-        int ubase = 0;
+        int ubase = 0, tb = 0;
         for (int e = 0; e < a.E; ++e) {
             const int n = cnt[e];
-            const int nu = ((n + a.BN - 1) / a.BN) * F * S;
+            const int mt = (n + a.BN - 1) / a.BN;
+            const int nu = mt * F * S;
             for (int i = tid; i < nu; i += blockDim.x) {
                 const int u = ubase + i;
                 if (u >= a.max_units) break;
                 const int m = i / (F * S);
                 const int rem = i - m * F * S;
                 const int ft = rem / S, sp = rem - ft * S;
-                units[u] = make_int4(e, off[e] + m * a.BN, min(a.BN, n - m * a.BN), ft | (sp << 16));
+                units[u] = make_int4(e | ((tb + m) << 8), off[e] + m * a.BN, min(a.BN, n - m * a.BN), ft | (sp << 16));
             }
             ubase += nu;
+            tb += mt;
         }
     }
 }
@@ -384,70 +396,96 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     schedule_block(a, ntiles, cnt_s, off_s, split_s);
 }
 
-__device__ __forceinline__ __half to_half_sat(float v) {
-    v = fminf(fmaxf(v, -65504.f), 65504.f);
-    return __float2half_rn(v);
-}
-
-template <typename TA> struct RowLoader;
-template <> struct RowLoader<__nv_bfloat16> {
-    // 8 consecutive elements -> 8 f16 (one 16-byte store)
-    static __device__ __forceinline__ uint4 load8(const __nv_bfloat16* p) {
-        const uint4 v = *reinterpret_cast<const uint4*>(p);
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
-        uint4 o;
-        __half2* h = reinterpret_cast<__half2*>(&o);
+// One 32-element block of a token's activations as floats.
+template <typename TA> struct BlockLoader;
+template <> struct BlockLoader<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[32]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(b[i]);
-            h[i] = __halves2half2(to_half_sat(f.x), to_half_sat(f.y));
+            const uint4 q = reinterpret_cast<const uint4*>(p)[i];
+            const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(b[j]);
+                v[8 * i + 2 * j] = f.x;
+                v[8 * i + 2 * j + 1] = f.y;
+            }
         }
-        return o;
     }
 };
-template <> struct RowLoader<float> {
-    static __device__ __forceinline__ uint4 load8(const float* p) {
-        const float4 a = *reinterpret_cast<const float4*>(p);
-        const float4 b = *reinterpret_cast<const float4*>(p + 4);
-        uint4 o;
-        __half2* h = reinterpret_cast<__half2*>(&o);
-        h[0] = __halves2half2(to_half_sat(a.x), to_half_sat(a.y));
-        h[1] = __halves2half2(to_half_sat(a.z), to_half_sat(a.w));
-        h[2] = __halves2half2(to_half_sat(b.x), to_half_sat(b.y));
-        h[3] = __halves2half2(to_half_sat(b.z), to_half_sat(b.w));
-        return o;
+template <> struct BlockLoader<float> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[32]) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 q = reinterpret_cast<const float4*>(p)[i];
+            v[4 * i] = q.x;
+            v[4 * i + 1] = q.y;
+            v[4 * i + 2] = q.z;
+            v[4 * i + 3] = q.w;
+        }
     }
 };
 
 constexpr int GATHER_WARPS = 8;
 
+// Where the grouped operands live.
+struct GroupedOperand {
+    uint8_t* codes;   // [K/32][3][R][16]
+    uint8_t* scales;  // [tiles][KC][natb][512]
+    int R;            // row capacity
+    int KC;           // chunks of 128 along K
+    int natb;         // scale atoms per chunk (3 * BN rows / 128, rounded up)
+};
+
+__device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int tile, int chunk) {
+    return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * g.natb * 512;
+}
+
 // One warp per (token, slot) pair p = t*k + j: its grouped row is
 // offsets[e] + (rows of e in earlier tiles) + (its rank within its tile), so the
-// rows of an expert are in (token, slot) order.  The warp records the row's
-// token and routing weight and copies the token's activations into the grouped
-// matrix as f16 (16-byte vectors); when the gate/up GEMM splits K it also
-// zeroes the row of the fp32 partial-sum buffer.
+// rows of an expert are in (token, slot) order; the row's place in the expert's
+// token tiles is (tile_base[e] + (row - offsets[e]) / BN, (row - offsets[e]) % BN).
+// The warp records the row's token, routing weight and tile slot, and encodes
+// the token's activations as three MXFP4 terms into the grouped operand: lane
+// l takes blocks l, l + 32, ... (one 16-byte store per term and block, one
+// scale byte into the block's scale atom).  When the gate/up GEMM splits K it
+// also zeroes the row of the fp32 partial-sum buffer.
 template <typename TA>
 __global__ void __launch_bounds__(GATHER_WARPS * 32)
 gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
               const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
-              const int32_t* __restrict__ offsets, int T, int d, int E, int k, int32_t* __restrict__ row_token,
-              float* __restrict__ row_weight, __half* __restrict__ Xp, float* __restrict__ GU, int gu_ld,
-              const int32_t* __restrict__ sched) {
+              const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
+              int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
+              GroupedOperand X, float* __restrict__ GU, int gu_ld, const int32_t* __restrict__ sched) {
     const int lane = threadIdx.x & 31;
     const int p = blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
     if (p >= T * k) return;
     const int t = p / k;
     const int e = idx[p];
-    const int pos = offsets[e] + tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+    const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+    const int pos = offsets[e] + loc;
+    const int tile = tile_base[e] + loc / BN, rloc = loc % BN;
     if (lane == 0) {
         row_token[pos] = t;
         row_weight[pos] = w[p];
+        row_slot[pos] = tile * BN + rloc;
     }
     const TA* src = x + static_cast<size_t>(t) * d;
-    uint4* dst = reinterpret_cast<uint4*>(Xp + static_cast<size_t>(pos) * d);
-    const int nvec = d / 8;
-    for (int v = lane; v < nvec; v += 32) dst[v] = RowLoader<TA>::load8(src + v * 8);
+    const int nb = d / 32;
+    for (int b = lane; b < nb; b += 32) {
+        float v[32];
+        BlockLoader<TA>::load(src + b * 32, v);
+        uint4 codes[MXQ_TERMS];
+        uint32_t sb[MXQ_TERMS];
+        mxq_block_thread(v, codes, sb);
+        uint8_t* atoms = scale_atom_base(X, tile, b >> 2);
+#pragma unroll
+        for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+            *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) =
+                codes[tt];
+            atoms[sf_atom_offset(tt * BN + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
+        }
+    }
     if (sched[SCHED_SPLIT_GU] > 1) {
         float4* g = reinterpret_cast<float4*>(GU + static_cast<size_t>(pos) * gu_ld);
         for (int v = lane; v < gu_ld / 4; v += 32) g[v] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -456,18 +494,41 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
 
 __device__ __forceinline__ float swish_f(float z) { return z / (1.0f + __expf(-z)); }
 
-// Split-K finish of the gate/up GEMM: H = Swish(G) * U from the fp32 partial
-// sums (only when the schedule split K).
-__global__ void swiglu_finish_kernel(const float* __restrict__ GU, __half* __restrict__ H, int d_ff,
-                                     const int32_t* __restrict__ sched) {
+// A full warp stores H = Swish(g) * u for 32 consecutive features (one block,
+// lane = feature) of grouped row `row` as three MXFP4 terms: lanes 0, 8, 16, 24
+// write one 4-byte word each per term, lane 0 the scale bytes.
+__device__ __forceinline__ void store_h_block(const GroupedOperand& Hd, float h, int lane, int blk, int row,
+                                              int tile, int rloc, int BN) {
+    uint32_t word[MXQ_TERMS], sb[MXQ_TERMS];
+    mxq_block_warp(h, lane, word, sb);
+    uint8_t* atoms = scale_atom_base(Hd, tile, blk >> 2);
+#pragma unroll
+    for (int t = 0; t < MXQ_TERMS; ++t) {
+        if ((lane & 7) == 0)
+            *reinterpret_cast<uint32_t*>(Hd.codes + ((static_cast<size_t>(blk) * MXQ_TERMS + t) * Hd.R + row) * 16 +
+                                         4 * (lane >> 3)) = word[t];
+        if (lane == 0) atoms[sf_atom_offset(t * BN + rloc, blk & 3)] = static_cast<uint8_t>(sb[t]);
+    }
+}
+
+// Split-K finish of the gate/up GEMM (only when the schedule split K): one
+// warp per (grouped row, 32-feature block) applies SwiGLU to the fp32 partial
+// sums and encodes H for the down GEMM.
+__global__ void swiglu_finish_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
+                                     const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
     if (sched[SCHED_SPLIT_GU] <= 1) return;
     const int rows = sched[SCHED_ROWS];
-    const size_t n = static_cast<size_t>(rows) * d_ff;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const size_t r = i / d_ff, f = i % d_ff;
-        const float g = GU[r * 2 * d_ff + f], u = GU[r * 2 * d_ff + d_ff + f];
-        H[i] = to_half_sat(swish_f(g) * u);
+    const int nbf = d_ff / 32;
+    const int lane = threadIdx.x & 31;
+    const long items = static_cast<long>(rows) * nbf;
+    const long nwarps = static_cast<long>(gridDim.x) * (blockDim.x >> 5);
+    for (long it = blockIdx.x * static_cast<long>(blockDim.x >> 5) + (threadIdx.x >> 5); it < items; it += nwarps) {
+        const int row = static_cast<int>(it / nbf), blk = static_cast<int>(it % nbf);
+        const int f = blk * 32 + lane;
+        const float* gu = GU + static_cast<size_t>(row) * 2 * d_ff;
+        const float h = swish_f(gu[f]) * gu[d_ff + f];
+        const int slot = row_slot[row];
+        store_h_block(Hd, h, lane, blk, row, slot / BN, slot % BN, BN);
     }
 }
 

@@ -133,6 +133,17 @@ __device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
+// 4-D tiled tensor copy global -> shared (no multicast); c0 is the innermost
+// coordinate and must be a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_4d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                                 uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+        : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -191,6 +202,32 @@ __device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
         : "memory");
 }
+// D[tmem] (+)= (A . diag) * (B . diag)^T with kind::mxf4 block scaling: A and B
+// packed E2M1 in shared memory (descriptors), one E8M0 scale per 32 elements of
+// K for every row of A and B, read from tensor memory at `sfa` / `sfb`; the
+// instruction consumes K = 64 (two scale bytes per row, chosen by the sf ids in
+// the instruction descriptor).  Warp-collective: elect.sync picks the issuer.
+__device__ __forceinline__ void mma_mxf4_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+// Copy one 512-byte scale-factor atom (32 rows x 16 B) from shared memory to 4
+// tensor-memory columns of lanes 0..31, replicated to the four lane quarters.
+// Warp-collective; ordered with the tcgen05.mma instructions the same thread issues.
+__device__ __forceinline__ void tc_cp_sf_warp(uint32_t taddr, uint64_t sdesc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+        "l"(sdesc)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -234,6 +271,22 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
            (static_cast<uint64_t>(2) << 61);
 }
 
+// Shared-memory matrix descriptor, no swizzle, K-major: core matrices of 8 rows
+// x 16 B stored as 128 contiguous bytes; `sbo` = bytes between 8-row groups,
+// `lbo` = bytes between K-adjacent core matrices; descriptor version 1.
+__host__ __device__ constexpr uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46);
+}
+// Instruction descriptor, kind::mxf4 block-scaled: E2M1 A and B (format 1),
+// E8M0 scales (bit 23), f32 accumulator, both K-major.  The scale-factor ids
+// (bits 4-5 for B, 29-30 for A) are or-ed in per instruction.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t sf_id) { return (sf_id << 29) | (sf_id << 4); }
+
 // Instruction descriptor, kind::f16: f16 A and B (format 0), f32 accumulator
 // (format 1), both K-major, M in bits 24.., N in bits 17...
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
@@ -260,6 +313,28 @@ __device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t mult2, uint
         "mul.rn.f16x2 %3, t3, %5;\n\t}"
         : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
         : "r"(w), "r"(mult2));
+}
+
+// Two floats -> one byte of two E2M1 codes (lo in the low nibble), rounded to
+// nearest with ties to the even code, saturating at +-6.
+__device__ __forceinline__ uint32_t e2m1x2_from_f32(float lo, float hi) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(d)
+        : "f"(hi), "f"(lo));
+    return d;
+}
+// One byte of two E2M1 codes -> f16x2 (low nibble in the low half), exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t d;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
+        : "=r"(d)
+        : "r"(byte));
+    return d;
 }
 
 // f16 bit pattern of 2^rel for rel <= 0 (normal down to 2^-14, subnormal down to

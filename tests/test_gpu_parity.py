@@ -124,6 +124,21 @@ def test_e128_layer_parity():
     check_layer(cfg, x, L.wr, L.bias, y, idx, w, counts, ox, n_sample=12)
 
 
+@pytest.mark.parametrize("d,f_", [(192, 320), (96, 160)])
+@pytest.mark.parametrize("bn", [16, 32, 48, 64])
+def test_every_token_tile_on_ragged_shapes(d, f_, bn):
+    """Each token tile (N = 3 * BN operand rows: one or two scale atoms, one or
+    two accumulator buffers) on shapes with a short last feature tile (64 or 32
+    rows), a short last K chunk, and K a multiple of 32 but not of 64."""
+    import mxfp4_expert_gemm_router_b200 as mx
+    cfg = mi.MoeConfig("ragged", 40, d, f_, 4, 2, "f32")
+    L = GpuLayer(cfg, cfg.T, flags=mx.token_tile_flag(bn))
+    ox = OracleExperts(cfg)
+    x = filtered_x(cfg, L.wr, L.bias)
+    y, idx, w, counts = L.forward(x)
+    check_layer(cfg, x, L.wr, L.bias, y, idx, w, counts, ox, n_sample=cfg.T)
+
+
 def test_ragged_token_counts(layer20b, ox20b):
     """Token counts that are not multiples of the router block (32) or of the tile."""
     for T in (3, 37, 130):
