@@ -156,12 +156,12 @@ def job_throughput(tokens_per_step: int, steps: int, world: int, max_total_ms: f
 
 # ---------------------------------------------------------------- our arm
 
-def build_layer(cfg: mi.MoeConfig, max_tokens: int):
+def build_layer(cfg: mi.MoeConfig, max_tokens: int, flags: int = 0):
     import torch
     import mxfp4_expert_gemm_router_b200 as mx
     from mxfp4_expert_gemm_router_b200 import build as mxbuild
     mxbuild.build()
-    layer = mx.MoeMxfp4(cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k, max_tokens, cfg.act_dtype)
+    layer = mx.MoeMxfp4(cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k, max_tokens, cfg.act_dtype, flags)
     for e in range(cfg.n_experts):
         wg, wu, wd = mi.draw_expert(cfg, e)
         layer.quantize_expert(e, torch.from_numpy(wg).cuda(), torch.from_numpy(wu).cuda(),
@@ -191,7 +191,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     T = cfg.T
-    layer, _ = build_layer(cfg, T)
+    import mxfp4_expert_gemm_router_b200 as mx
+    layer, _ = build_layer(cfg, T, mx.token_tile_flag(args.token_tile) if args.token_tile else 0)
     x = act_tensor(cfg, mi.draw_x(cfg), dev)
     y = torch.empty_like(x)
     counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
@@ -337,7 +338,8 @@ def config_dict(cfg, args):
             "T": cfg.T, "d_model": cfg.d_model, "d_ff": cfg.d_ff, "n_experts": cfg.n_experts, "top_k": cfg.top_k,
             "seed": cfg.seed, "parallelism": f"replicas x{args.gpus}",
             "l2": "256 MB flush written between timed steps (outside each step's event span)",
-            "launch": "forward captured once as a CUDA graph, replayed per timed step"}
+            "launch": "forward captured once as a CUDA graph, replayed per timed step",
+            "token_tile": getattr(args, "token_tile", 0) or "auto"}
 
 
 # Dense tensor-core rate of the experts' MMA operand type relative to bf16
@@ -385,6 +387,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--token-tile", type=int, default=0, choices=[0, 16, 32, 48, 64, 80, 96, 112, 128],
+                    help="token rows per expert-GEMM tile (0: chosen per forward)")
     args = ap.parse_args()
     cfg = mi.CONFIGS[args.config]
 

@@ -55,7 +55,7 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 #define MOE_FLAG_TEST_SKIP_FIRST_COPY (1u << 30)
 
 /* Token rows per expert-GEMM tile (BN).  0 (default): chosen per forward from
- * T, top_k and n_experts; 1..4 force BN = 16, 32, 48 or 64.  Every choice
+ * T, top_k and n_experts; v = 1..8 forces BN = 16 v (16 .. 128).  Every choice
  * computes the same layer; the tile only changes how work is cut. */
 #define MOE_FLAG_TOKEN_TILE_SHIFT 8
 #define MOE_FLAG_TOKEN_TILE_MASK (0xFu << MOE_FLAG_TOKEN_TILE_SHIFT)
@@ -163,7 +163,7 @@ moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */
 #define MOE_NUM_STAGES 6
 /* 0 router + top-k + softmax + grouping schedule, 1 gather into grouped rows,
- * 2 gate/up + SwiGLU, 3 split-K SwiGLU finish, 4 down + weighted combine,
+ * 2 gate/up + SwiGLU, 3 H encoding (three MXFP4 terms), 4 down + weighted combine,
  * 5 output cast.  Synchronises;
  * writes the last profiled forward's durations in ms (0 for stages that did
  * not run) into ms[0..min(n, MOE_NUM_STAGES)). */

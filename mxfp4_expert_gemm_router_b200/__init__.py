@@ -25,10 +25,13 @@ MOE_FLAG_TOKEN_TILE_SHIFT = 8
 MOE_FLAG_TOKEN_TILE_MASK = 0xF << MOE_FLAG_TOKEN_TILE_SHIFT
 
 
+TOKEN_TILES = tuple(range(16, 129, 16))
+
+
 def token_tile_flag(bn: int) -> int:
-    """Config flag that forces BN token rows per expert-GEMM tile (16, 32, 48 or 64)."""
-    if bn not in (16, 32, 48, 64):
-        raise ValueError("token tile must be 16, 32, 48 or 64")
+    """Config flag that forces BN token rows per expert-GEMM tile (16, 32, ..., 128)."""
+    if bn not in TOKEN_TILES:
+        raise ValueError("token tile must be a multiple of 16 from 16 to 128")
     return (bn // 16) << MOE_FLAG_TOKEN_TILE_SHIFT
 MOE_NUM_STAGES = 6
 

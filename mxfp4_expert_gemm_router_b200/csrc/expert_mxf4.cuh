@@ -8,22 +8,22 @@
 // The MMA is tcgen05.mma kind::mxf4 with 32-element block scaling: both
 // operands are packed E2M1 in shared memory and every row carries one E8M0
 // scale per 32 elements of K, held in tensor memory.  Orientation:
-// D[feature, n] = W[feature, :] . B[n, :]^T with M = 128 weight rows (output
-// features) as the A operand and N = 3 * BN operand rows, the three MXFP4 terms
-// of BN grouped token rows (mxq.cuh), as B.  The weights reach the tensor core
-// exactly as stored, with no decode step: one bulk copy per K = 128 stage
-// brings codes and scale atoms, a 4-D TMA box {16 B, BN rows, 3 terms, 4
-// blocks} brings the activation codes and a bulk copy their scale atoms.
+// D[feature, token] = W[feature, :] . X[token, :]^T with M = 128 weight rows
+// (output features) as the A operand and N = BN grouped token rows as B.  The
+// activations are three MXFP4 terms (mxq.cuh); one MMA per term accumulates
+// into the same D, so the tensor core sums the terms.  The weights reach the
+// tensor core exactly as stored, with no decode step: one bulk copy per K =
+// 128 stage brings codes and scale atoms, a 3-D TMA box {BN rows x 16 B, 3
+// terms, 4 blocks} brings the activation codes and a bulk copy their scale
+// atoms (one per term).
 // tcgen05.cp moves the scale atoms into a ring of tensor-memory slots; fp32
 // accumulators stay in tensor memory (two buffers when they fit, so the
 // epilogue of one unit overlaps the main loop of the next).
 //
 //   MODE 0 (gate/up): per stage gate and up chunks (17408 bytes), two
-//     accumulators for the same 128 features; epilogue: g and u are the sums
-//     of the three term columns, H = Swish(g) * u is encoded as three MXFP4
-//     terms straight into the down GEMM's B operand (lanes of a warp = 32
-//     consecutive features = one MXFP4 block of H); with a K split, fp32
-//     partials are added into GU instead and a finish kernel does the rest.
+//     accumulators for the same 128 features; epilogue: H = Swish(g) * u,
+//     stored as f16 (h_encode_kernel then encodes it for the down GEMM); with
+//     a K split, fp32 partials are added into GU instead.
 //   MODE 1 (down): per stage the down chunk (8704 bytes), one accumulator;
 //     epilogue: y[token, f] += w_row * d, red.add into the fp32 output
 //     accumulator (the weighted scatter-combine).
@@ -51,11 +51,11 @@ constexpr int MXG_EPI_WARPS = 8;
 constexpr int MXG_THREADS = (2 + MXG_EPI_WARPS) * 32;
 constexpr int MXG_MAX_STAGES = 16;
 constexpr int MXG_TMEM_COLS = 512;
-constexpr int MXG_SF_COL0 = 448;      // scale-factor ring: MXG_SF_SLOTS slots of 16 columns
-constexpr int MXG_SF_SLOTS = 4;       //   [A (gate) 4 | A (up) 4 | B atom 0 4 | B atom 1 4]
-constexpr int MXG_SF_SLOT_COLS = 16;
+constexpr int MXG_SF_COL0 = 448;      // scale-factor ring: MXG_SF_SLOTS slots of 32 columns
+constexpr int MXG_SF_SLOTS = 2;       //   [A (gate) 4 | A (up) 4 | B term 0 4 | B term 1 4 | B term 2 4]
+constexpr int MXG_SF_SLOT_COLS = 32;
 constexpr int MXG_MAX_ACC = 2;
-constexpr int MXG_MAX_BN = 64;
+constexpr int MXG_MAX_BN = 128;
 constexpr int MXG_MIN_SMEM = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
 struct MxgParams {
@@ -65,13 +65,12 @@ struct MxgParams {
     TiledMatrix M;            // geometry of the (first) matrix streamed
     int N;                    // output features
     int K;                    // contraction length
-    int BN;                   // token rows per tile (16, 32, 48 or 64)
+    int BN;                   // token rows per tile (multiple of 16, at most 128)
     int stages;
     int nacc;                 // accumulator buffers (1 or 2)
-    const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][natb][512]
-    int natb;
-    uint32_t idesc;           // M = 128, N = 3 * BN, without scale-factor ids
-    GroupedOperand Hd;        // MODE 0: H as the down GEMM's B operand
+    const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][3 terms][512]
+    uint32_t idesc;           // M = 128, N = BN, without scale-factor ids
+    __half* H16;              // MODE 0 output H = Swish(g) * u, f16 [rows][N]
     float* GU;                // MODE 0 split partials [rows][2N]
     float* yacc;              // MODE 1 output accumulator [T][N]
     const int32_t* row_token; // MODE 1
@@ -83,14 +82,14 @@ struct MxgParams {
 
 // Weight bytes per stage (codes of 128 rows x 4 blocks + one scale atom, per
 // matrix), B bytes per stage (4 blocks x 3 terms x BN rows x 16 B), B scale
-// atoms per stage, accumulator columns (rounded to 32).
+// atoms per stage (one per term), accumulator columns (rounded to 32).
 __host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
 __host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
-__host__ __device__ constexpr int mxg_natb(int BN) { return (MXQ_TERMS * BN + 127) / 128; }
+constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
 __host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
-    return mxg_w_stage(mode) + mxg_b_bytes(BN) + 512u * mxg_natb(BN);
+    return mxg_w_stage(mode) + mxg_b_bytes(BN) + MXG_SFB_BYTES;
 }
-__host__ __device__ constexpr int mxg_mat_cols(int BN) { return ((MXQ_TERMS * BN + 31) / 32) * 32; }
+__host__ __device__ constexpr int mxg_mat_cols(int BN) { return ((BN + 31) / 32) * 32; }
 __host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
 __host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
 __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
@@ -108,7 +107,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
 
     const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
     const uint32_t b_bytes = mxg_b_bytes(BN);
-    const uint32_t sf_bytes = 512u * static_cast<uint32_t>(p.natb);
+    const uint32_t sf_bytes = MXG_SFB_BYTES;
     const uint32_t stage_bytes = W_STAGE + b_bytes + sf_bytes;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -180,7 +179,8 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                     const uint32_t st = w_sm(s);
                     mbar_arrive_expect_tx_warp(full_bar(s), wb + b_bytes + sf_bytes);
                     bulk_g2s_warp(st, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
-                    tma_load_4d_warp(st + W_STAGE, &tmap_b, 0, U.y, 0, 4 * c, full_bar(s));
+                    // rows U.y .. U.y + BN - 1 of every (block, term): 8-byte elements 2 * U.y ..
+                    tma_load_3d_warp(st + W_STAGE, &tmap_b, 2 * U.y, 0, 4 * c, full_bar(s));
                     bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * sf_bytes,
                                   sf_bytes, full_bar(s));
                     pend_ph[s] = static_cast<int>(ph);
@@ -222,17 +222,22 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
                 tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
                 if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
-                tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
-                if (p.natb > 1) tc_cp_sf_warp(sfc + 12, desc_noswz(ss + 512, 0, 128));
+#pragma unroll
+                for (int t = 0; t < MXQ_TERMS; ++t) tc_cp_sf_warp(sfc + 8 + 4 * t, desc_noswz(ss + 512 * t, 0, 128));
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     if (2 * i < nbc) {
-                        const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
                         const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
                         const uint64_t ad = desc_noswz(ws + 2 * i * rf * 16, rf * 16, 128);
-                        const uint64_t bd = desc_noswz(bs + 2 * i * NB3 * 16, NB3 * 16, 128);
-                        mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8, acc);
-                        if (MODE == 0) mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8, acc);
+#pragma unroll
+                        for (int t = 0; t < MXQ_TERMS; ++t) {
+                            // B of term t, blocks 2i and 2i+1: smem [block][term][row][16 B]
+                            const uint32_t acc = (c > c0 || i > 0 || t > 0) ? 1u : 0u;
+                            const uint64_t bd = desc_noswz(bs + (2 * i * MXQ_TERMS + t) * BN * 16, NB3 * 16, 128);
+                            mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8 + 4 * t, acc);
+                            if (MODE == 0)
+                                mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8 + 4 * t, acc);
+                        }
                     }
                 }
                 tc_commit_warp(empty_bar(s));
@@ -256,7 +261,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         bool ok = true;
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const int4 U = p.units[u];
-            const int tile = U.x >> 8, row0 = U.y, nvalid = U.z;
+            const int row0 = U.y, nvalid = U.z;
             const int ft = U.w & 0xFFFF;
             const int rf = min(128, p.N - ft * 128);
             const bool warp_rows = 32 * q < rf;
@@ -270,31 +275,40 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
             if (warp_rows) {
                 const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
                 for (int r0 = 8 * hh; r0 < nvalid; r0 += 16) {
-                    uint32_t g[MXQ_TERMS][8], v[MXQ_TERMS][8];
-#pragma unroll
-                    for (int t = 0; t < MXQ_TERMS; ++t) {
-                        tmem_ld8(d0 + t * BN + r0, g[t]);
-                        if (MODE == 0) tmem_ld8(d0 + mat_cols + t * BN + r0, v[t]);
-                    }
+                    uint32_t g[8], v[8];
+                    tmem_ld8(d0 + r0, g);
+                    if (MODE == 0) tmem_ld8(d0 + mat_cols + r0, v);
                     tmem_wait_ld();
+                    float gs[8], us[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const int r = r0 + j;
-                        if (r < nvalid) {
-                            const float gg = __uint_as_float(g[0][j]) + __uint_as_float(g[1][j]) + __uint_as_float(g[2][j]);
-                            if (MODE == 0) {
-                                const float uu =
-                                    __uint_as_float(v[0][j]) + __uint_as_float(v[1][j]) + __uint_as_float(v[2][j]);
-                                if (nsplit == 1) {
-                                    store_h_block(p.Hd, swish_f(gg) * uu, lane, 4 * ft + q, row0 + r, tile, r, BN);
-                                } else {
-                                    float* gu = p.GU + static_cast<size_t>(row0 + r) * 2 * p.N;
-                                    atomicAdd(gu + n, gg);
-                                    atomicAdd(gu + p.N + n, uu);
+                        gs[j] = __uint_as_float(g[j]);
+                        us[j] = MODE == 0 ? __uint_as_float(v[j]) : 0.f;
+                    }
+                    const int nv = min(8, nvalid - r0);   // valid token columns in this group (warp-uniform)
+                    if (MODE == 0) {
+                        if (nsplit == 1) {
+                            // H = Swish(g) * u as f16 (32 lanes = 64 contiguous bytes per row)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                if (j < nv)
+                                    p.H16[static_cast<size_t>(row0 + r0 + j) * p.N + n] = to_half_sat(swish_f(gs[j]) * us[j]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                if (j < nv) {
+                                    float* gu = p.GU + static_cast<size_t>(row0 + r0 + j) * 2 * p.N;
+                                    atomicAdd(gu + n, gs[j]);
+                                    atomicAdd(gu + p.N + n, us[j]);
                                 }
-                            } else {
-                                const int rr = row0 + r;
-                                atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n, gg * p.row_weight[rr]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (j < nv) {
+                                const int rr = row0 + r0 + j;
+                                atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n, gs[j] * p.row_weight[rr]);
                             }
                         }
                     }

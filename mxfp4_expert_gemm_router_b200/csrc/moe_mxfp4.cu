@@ -10,8 +10,8 @@
 //   gather_kernel        grouped rows (token, weight, tile slot); activations
 //                        encoded as three MXFP4 terms (the B operand)
 //   expert_mxf4<0>       gate/up GEMM on block-scaled MXFP4 tensor cores,
-//                        SwiGLU epilogue encoding H for the down GEMM
-//   swiglu_finish_kernel only when the gate/up GEMM may split K
+//                        SwiGLU epilogue (H as f16, or fp32 partials when K is split)
+//   h_encode_kernel      H encoded as three MXFP4 terms for the down GEMM
 //   expert_mxf4<1>       down GEMM, routing-weighted scatter-combine epilogue
 //   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
 #include <cuda.h>
@@ -35,7 +35,7 @@ using namespace moe;
 
 namespace {
 
-constexpr int BN_OPTIONS = 4;  // BN = 16 * (i + 1): 16, 32, 48, 64
+constexpr int BN_OPTIONS = 8;  // BN = 16 * (i + 1): 16 .. 128
 constexpr int SPLIT_ROWS_CAP = 2048;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -88,6 +88,7 @@ struct moe_mxfp4 {
     int32_t* row_slot = nullptr;
     uint8_t* Xq = nullptr;     // x as three MXFP4 terms [d/32][3][TK][16]
     uint8_t* Hq = nullptr;     // H as three MXFP4 terms [d_ff/32][3][TK][16]
+    __half* H16 = nullptr;     // H = Swish(g) * u, f16 [TK][d_ff]
     uint8_t* sfx = nullptr;    // scale atoms of Xq per (token tile, K chunk)
     uint8_t* sfh = nullptr;    // scale atoms of Hq per (token tile, K chunk)
     size_t sfx_bytes = 0, sfh_bytes = 0, xq_bytes = 0, hq_bytes = 0;
@@ -123,7 +124,7 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 static void free_all(moe_mxfp4* h) {
     void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
-                    h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
+                    h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->H16, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
     for (void* p : ptrs)
         if (p) cudaFree(p);
@@ -134,7 +135,7 @@ static void free_all(moe_mxfp4* h) {
 
 // Token rows per tile: about three times the mean rows per expert, so that
 // most experts need one tile (each tile streams the expert's weights once),
-// rounded up to 16 and capped at 64 (N = 3 * BN <= 192).  Flags may force it.
+// rounded up to 16 and capped at 128.  Flags may force it.
 static int choose_bn(int T, int k, int E, uint32_t flags) {
     const uint32_t forced = (flags & MOE_FLAG_TOKEN_TILE_MASK) >> MOE_FLAG_TOKEN_TILE_SHIFT;
     if (forced >= 1 && forced <= BN_OPTIONS) return 16 * static_cast<int>(forced);
@@ -144,16 +145,10 @@ static int choose_bn(int T, int k, int E, uint32_t flags) {
     return std::max(16, std::min(MXG_MAX_BN, bn));
 }
 
-// Largest (token tiles x scale atoms per chunk) over the tile sizes: tiles of
-// an expert with n rows = ceil(n / BN), so at most TK / BN + E tiles.
-static size_t max_tile_atoms(size_t TK, int E) {
-    size_t m = 0;
-    for (int i = 0; i < BN_OPTIONS; ++i) {
-        const int BN = 16 * (i + 1);
-        m = std::max(m, (TK / BN + E) * static_cast<size_t>(mxg_natb(BN)));
-    }
-    return m;
-}
+// Scale atoms per K chunk over all token tiles: an expert with n rows has
+// ceil(n / BN) tiles, so at most TK / 16 + E tiles (the smallest tile), each
+// with one atom per term.
+static size_t max_tile_atoms(size_t TK, int E) { return (TK / 16 + E) * MXQ_TERMS; }
 
 static TiledMatrix tiled(moe_mxfp4* h, int which) {
     const auto& c = h->cfg;
@@ -221,7 +216,7 @@ const char* moe_mxfp4_status_string(moe_status_t s) {
 
 const char* moe_mxfp4_stage_name(int32_t stage) {
     static const char* names[MOE_NUM_STAGES] = {"router_topk_schedule", "gather", "gate_up_swiglu",
-                                                 "swiglu_finish", "down_combine", "cast_out"};
+                                                 "h_encode", "down_combine", "cast_out"};
     return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "unknown";
 }
 
@@ -310,6 +305,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->row_slot), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->Xq), h->xq_bytes},
         {reinterpret_cast<void**>(&h->Hq), h->hq_bytes},
+        {reinterpret_cast<void**>(&h->H16), sizeof(__half) * TK * f},
         {reinterpret_cast<void**>(&h->sfx), h->sfx_bytes},
         {reinterpret_cast<void**>(&h->sfh), h->sfh_bytes},
         {reinterpret_cast<void**>(&h->GU), sizeof(float) * h->gu_rows * 2 * f},
@@ -428,10 +424,12 @@ moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* hc, int32_t which, uint
     return cuda_status(cudaGetLastError());
 }
 
-// 4-D maps over the three-term operands [K/32 blocks][3 terms][TK rows][16 B]:
-// box {16 B, BN rows, 3 terms, 4 blocks} lands in shared memory as
-// [4 blocks][3 terms][BN rows][16 B], the unswizzled K-major layout of an
-// N = 3 * BN operand.  Rows past TK and blocks past K/32 read as zeros.
+// 3-D maps over the three-term operands [K/32 blocks][3 terms][TK rows x 16 B],
+// read as 8-byte elements so that the innermost box dimension is one
+// contiguous run of BN rows (BN * 16 bytes): box {2 BN, 3 terms, 4 blocks}
+// lands in shared memory as [4 blocks][3 terms][BN rows][16 B], the
+// unswizzled K-major layout of each term's operand.  Rows past TK and blocks
+// past K/32 read as zeros.
 static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
     const int i = BN / 16 - 1;
     if (h->tm_ok[i]) return MOE_OK;
@@ -441,11 +439,11 @@ static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
     const cuuint64_t R = static_cast<cuuint64_t>(h->TK);
     for (int which = 0; which < 2; ++which) {
         const cuuint64_t nb = (which == 0 ? c.d_model : c.d_ff) / 32;
-        cuuint64_t dims[4] = {16, R, MXQ_TERMS, nb};
-        cuuint64_t strides[3] = {16, R * 16, R * 16 * MXQ_TERMS};
-        cuuint32_t box[4] = {16, static_cast<cuuint32_t>(BN), MXQ_TERMS, 4};
-        cuuint32_t estr[4] = {1, 1, 1, 1};
-        CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+        cuuint64_t dims[3] = {2 * R, MXQ_TERMS, nb};
+        cuuint64_t strides[2] = {R * 16, R * 16 * MXQ_TERMS};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(2 * BN), MXQ_TERMS, 4};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_UINT64, 3,
                          which == 0 ? static_cast<void*>(h->Xq) : static_cast<void*>(h->Hq), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -524,9 +522,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 1: gather into grouped rows
     mark(1);
     const int gblocks = (T * k + GATHER_WARPS - 1) / GATHER_WARPS;
-    const int natb = mxg_natb(BN);
-    GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, natb};
-    GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, natb};
+    GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu};
+    GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn};
     if (bf16)
         gather_kernel<__nv_bfloat16><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E,
@@ -550,9 +547,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.stages = stages_for(0, BN);
     gp.nacc = mxg_nacc(0, BN);
     gp.sfb = h->sfx;
-    gp.natb = natb;
-    gp.idesc = idesc_mxf4(128, MXQ_TERMS * BN);
-    gp.Hd = Hop;
+    gp.idesc = idesc_mxf4(128, BN);
+    gp.H16 = h->H16;
     gp.GU = h->GU;
     gp.yacc = nullptr;
     gp.row_token = h->row_token;
@@ -563,13 +559,11 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     const int grid = h->nsm;
     expert_mxf4_kernel<0><<<grid, MXG_THREADS, mxg_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
     h->stage_ran[2] = true;
-    // 3: split-K finish (no-op unless the schedule split K)
+    // 3: H (f16, or split-K partials) -> three MXFP4 terms for the down GEMM
     mark(3);
-    const bool may_split = static_cast<long>(T) * k <= h->gu_rows;
-    if (may_split) {
-        const long items = static_cast<long>(T) * k * (f / 32);
-        const int blocks = static_cast<int>(std::min<long>(4L * h->nsm, (items + 7) / 8));
-        swiglu_finish_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->GU, Hop, f, BN, h->row_slot, h->sched);
+    {
+        const int blocks = (T * k + HENC_WARPS - 1) / HENC_WARPS;
+        h_encode_kernel<<<blocks, HENC_WARPS * 32, 0, stream>>>(h->H16, h->GU, Hop, f, BN, h->row_slot, h->sched);
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine

@@ -9,8 +9,8 @@
 // significant bits, far too coarse for the layer's accuracy, so a block v of
 // 32 values is written as v ~= q1 + q2 + q3: q1 encodes v, q2 encodes the
 // residual v - q1, q3 the residual v - q1 - q2, each with its own scale.  The
-// MMA takes the three terms as three groups of N rows; the epilogue adds the
-// three accumulator columns.  Measured on the oracle's weights (double
+// GEMM issues one MMA per term into the same accumulator, so the tensor core
+// adds the three products.  Measured on the oracle's weights (double
 // precision emulation), the layer error of the 3-term encoding is about 0.25 %
 // of max|y| (2 terms: about 3 %).
 //
@@ -20,9 +20,9 @@
 //
 // Operand layouts in global memory (R = row capacity, NB = K / 32 blocks):
 //   codes   [NB][3 terms][R rows][16 B]   (element 2i of the block in the low nibble of byte i)
-//   scales  per (token tile, K chunk of 128): natb atoms of 512 B; operand row
-//           n = term * BN + row-in-tile, block q (0..3) of the chunk at byte
-//           sf_atom_offset(n, q).
+//   scales  per (token tile, K chunk of 128): one 512-byte atom per term; row r
+//           of the tile (r < 128), term t, block q (0..3) of the chunk at byte
+//           sf_atom_offset(t * 128 + r, q).
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -83,34 +83,6 @@ __device__ __forceinline__ void mxq_block_thread(float (&v)[32], uint4 (&codes)[
             }
         }
         codes[t] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-// A full warp encodes one block: lane l holds element l.  On return, lanes 0,
-// 8, 16 and 24 hold word l / 8 of each term's 16 code bytes in word[t]; every
-// lane holds the scale bytes.
-__device__ __forceinline__ void mxq_block_warp(float v, int lane, uint32_t (&word)[MXQ_TERMS],
-                                               uint32_t (&sbyte)[MXQ_TERMS]) {
-    const bool odd = (lane & 1) != 0;
-    float r = v;
-#pragma unroll
-    for (int t = 0; t < MXQ_TERMS; ++t) {
-        // |r| compares as an unsigned integer: the warp maximum in one reduction
-        const uint32_t amb = __reduce_max_sync(0xffffffffu, __float_as_uint(r) & 0x7FFFFFFFu);
-        const int e = mxq_exp(amb);
-        sbyte[t] = static_cast<uint32_t>(e + 127);
-        const float a = r * mxq_inv(e);
-        const float o = __shfl_xor_sync(0xffffffffu, a, 1);
-        const uint32_t byte = e2m1x2_from_f32(odd ? o : a, odd ? a : o);
-        if (t + 1 < MXQ_TERMS) {
-            const uint32_t h2 = e2m1x2_to_f16x2(byte);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-            r -= (odd ? f.y : f.x) * mxq_scale(e);
-        }
-        uint32_t w = byte;
-        w |= __shfl_down_sync(0xffffffffu, w, 2) << 8;
-        w |= __shfl_down_sync(0xffffffffu, w, 4) << 16;
-        word[t] = w;
     }
 }
 

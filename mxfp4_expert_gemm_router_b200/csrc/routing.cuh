@@ -431,14 +431,13 @@ constexpr int GATHER_WARPS = 8;
 // Where the grouped operands live.
 struct GroupedOperand {
     uint8_t* codes;   // [K/32][3][R][16]
-    uint8_t* scales;  // [tiles][KC][natb][512]
+    uint8_t* scales;  // [tiles][KC][3 terms][512]
     int R;            // row capacity
     int KC;           // chunks of 128 along K
-    int natb;         // scale atoms per chunk (3 * BN rows / 128, rounded up)
 };
 
 __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int tile, int chunk) {
-    return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * g.natb * 512;
+    return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * MXQ_TERMS * 512;
 }
 
 // One warp per (token, slot) pair p = t*k + j: its grouped row is
@@ -483,7 +482,7 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
         for (int tt = 0; tt < MXQ_TERMS; ++tt) {
             *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) =
                 codes[tt];
-            atoms[sf_atom_offset(tt * BN + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
+            atoms[sf_atom_offset(tt * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
         }
     }
     if (sched[SCHED_SPLIT_GU] > 1) {
@@ -492,43 +491,69 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
     }
 }
 
-__device__ __forceinline__ float swish_f(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float swish_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-// A full warp stores H = Swish(g) * u for 32 consecutive features (one block,
-// lane = feature) of grouped row `row` as three MXFP4 terms: lanes 0, 8, 16, 24
-// write one 4-byte word each per term, lane 0 the scale bytes.
-__device__ __forceinline__ void store_h_block(const GroupedOperand& Hd, float h, int lane, int blk, int row,
-                                              int tile, int rloc, int BN) {
-    uint32_t word[MXQ_TERMS], sb[MXQ_TERMS];
-    mxq_block_warp(h, lane, word, sb);
-    uint8_t* atoms = scale_atom_base(Hd, tile, blk >> 2);
-#pragma unroll
-    for (int t = 0; t < MXQ_TERMS; ++t) {
-        if ((lane & 7) == 0)
-            *reinterpret_cast<uint32_t*>(Hd.codes + ((static_cast<size_t>(blk) * MXQ_TERMS + t) * Hd.R + row) * 16 +
-                                         4 * (lane >> 3)) = word[t];
-        if (lane == 0) atoms[sf_atom_offset(t * BN + rloc, blk & 3)] = static_cast<uint8_t>(sb[t]);
-    }
+__device__ __forceinline__ __half to_half_sat(float v) {
+    v = fminf(fmaxf(v, -65504.f), 65504.f);
+    return __float2half_rn(v);
 }
 
-// Split-K finish of the gate/up GEMM (only when the schedule split K): one
-// warp per (grouped row, 32-feature block) applies SwiGLU to the fp32 partial
-// sums and encodes H for the down GEMM.
-__global__ void swiglu_finish_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
-                                     const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
-    if (sched[SCHED_SPLIT_GU] <= 1) return;
+constexpr int HENC_WARPS = 8;
+
+// Encodes H for the down GEMM: one warp per grouped row, lane l takes the
+// 32-feature blocks l, l + 32, ... of the row.  H comes from the gate/up
+// epilogue as f16 (Swish(g) * u already applied), or, when the gate/up GEMM
+// split K, from the fp32 partial sums of g and u (Swish applied here).  Each
+// block is encoded as three MXFP4 terms (mxq_block_thread) into the down
+// GEMM's B operand: 16 code bytes per term, one scale byte per term into the
+// scale atom of the row's token tile.
+__global__ void __launch_bounds__(HENC_WARPS * 32)
+h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
+                const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
     const int rows = sched[SCHED_ROWS];
-    const int nbf = d_ff / 32;
+    const bool split = sched[SCHED_SPLIT_GU] > 1;
+    const int row = blockIdx.x * HENC_WARPS + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    const long items = static_cast<long>(rows) * nbf;
-    const long nwarps = static_cast<long>(gridDim.x) * (blockDim.x >> 5);
-    for (long it = blockIdx.x * static_cast<long>(blockDim.x >> 5) + (threadIdx.x >> 5); it < items; it += nwarps) {
-        const int row = static_cast<int>(it / nbf), blk = static_cast<int>(it % nbf);
-        const int f = blk * 32 + lane;
-        const float* gu = GU + static_cast<size_t>(row) * 2 * d_ff;
-        const float h = swish_f(gu[f]) * gu[d_ff + f];
-        const int slot = row_slot[row];
-        store_h_block(Hd, h, lane, blk, row, slot / BN, slot % BN, BN);
+    if (row >= rows) return;
+    const int slot = row_slot[row];
+    const int tile = slot / BN, rloc = slot % BN;
+    const int nb = d_ff / 32;
+    for (int b = lane; b < nb; b += 32) {
+        float v[32];
+        if (split) {
+            const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
+            const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 gg = g[i], uu = u[i];
+                v[4 * i] = swish_f(gg.x) * uu.x;
+                v[4 * i + 1] = swish_f(gg.y) * uu.y;
+                v[4 * i + 2] = swish_f(gg.z) * uu.z;
+                v[4 * i + 3] = swish_f(gg.w) * uu.w;
+            }
+        } else {
+            const uint4* hp = reinterpret_cast<const uint4*>(H16 + static_cast<size_t>(row) * d_ff + 32 * b);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 q = hp[i];
+                const __half2* h2 = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __half22float2(h2[j]);
+                    v[8 * i + 2 * j] = f.x;
+                    v[8 * i + 2 * j + 1] = f.y;
+                }
+            }
+        }
+        uint4 codes[MXQ_TERMS];
+        uint32_t sb[MXQ_TERMS];
+        mxq_block_thread(v, codes, sb);
+        uint8_t* atoms = scale_atom_base(Hd, tile, b >> 2);
+#pragma unroll
+        for (int t = 0; t < MXQ_TERMS; ++t) {
+            *reinterpret_cast<uint4*>(Hd.codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * Hd.R + row) * 16) = codes[t];
+            atoms[sf_atom_offset(t * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
+        }
     }
 }
 

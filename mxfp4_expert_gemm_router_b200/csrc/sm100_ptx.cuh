@@ -133,6 +133,17 @@ __device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
+// 3-D tiled tensor copy global -> shared (no multicast); c0 is the innermost
+// coordinate and must be a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                                 uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
 // 4-D tiled tensor copy global -> shared (no multicast); c0 is the innermost
 // coordinate and must be a multiple of 16 bytes' worth of elements.
 __device__ __forceinline__ void tma_load_4d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,

@@ -125,11 +125,11 @@ def test_e128_layer_parity():
 
 
 @pytest.mark.parametrize("d,f_", [(192, 320), (96, 160)])
-@pytest.mark.parametrize("bn", [16, 32, 48, 64])
+@pytest.mark.parametrize("bn", [16, 48, 112, 128])
 def test_every_token_tile_on_ragged_shapes(d, f_, bn):
-    """Each token tile (N = 3 * BN operand rows: one or two scale atoms, one or
-    two accumulator buffers) on shapes with a short last feature tile (64 or 32
-    rows), a short last K chunk, and K a multiple of 32 but not of 64."""
+    """Token tiles from 16 to 128 rows (one or two accumulator buffers) on
+    shapes with a short last feature tile (64 or 32 rows), a short last K
+    chunk, and K a multiple of 32 but not of 64."""
     import mxfp4_expert_gemm_router_b200 as mx
     cfg = mi.MoeConfig("ragged", 40, d, f_, 4, 2, "f32")
     L = GpuLayer(cfg, cfg.T, flags=mx.token_tile_flag(bn))
