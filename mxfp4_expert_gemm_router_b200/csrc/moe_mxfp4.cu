@@ -169,11 +169,13 @@ static TiledMatrix tiled(moe_mxfp4* h, int which) {
     return M;
 }
 
+// K splits of the router: enough CTAs to cover the SMs once, at most
+// ROUTER_MAX_SPLITS (the last CTA of a token tile sums the splits' partials).
 static int router_splits(int T, int d, int nsm) {
     const int tiles = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
     const int kch = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
-    const int want = (2 * nsm + tiles - 1) / tiles;
-    return std::max(1, std::min(kch, want));
+    const int want = (nsm + tiles - 1) / tiles;
+    return std::max(1, std::min(std::min(kch, ROUTER_MAX_SPLITS), want));
 }
 
 // Router launch for the expert count: EPT = experts per lane, 1/2/4/8.
@@ -496,8 +498,6 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.w_out = wts;
     ra.local_rank = h->local_rank;
     ra.hist = h->hist;
-    ra.zero_rows = acc;
-    ra.zero_ld = d;
     ra.BN = BN;
     ra.F_gu = h->F_gu;
     ra.F_dn = h->F_dn;
@@ -521,17 +521,18 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     h->stage_ran[0] = true;
     // 1: gather into grouped rows
     mark(1);
-    const int gblocks = (T * k + GATHER_WARPS - 1) / GATHER_WARPS;
+    const long gitems = static_cast<long>(T) * k * (d / 32);
+    const int gblocks = static_cast<int>((gitems + GATHER_THREADS - 1) / GATHER_THREADS);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu};
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn};
     if (bf16)
-        gather_kernel<__nv_bfloat16><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
+        gather_kernel<__nv_bfloat16><<<gblocks, GATHER_THREADS, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E,
-            k, BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, h->sched);
+            k, BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc, h->sched);
     else
-        gather_kernel<float><<<gblocks, GATHER_WARPS * 32, 0, stream>>>(
+        gather_kernel<float><<<gblocks, GATHER_THREADS, 0, stream>>>(
             static_cast<const float*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E, k, BN,
-            h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, h->sched);
+            h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc, h->sched);
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);
@@ -562,8 +563,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 3: H (f16, or split-K partials) -> three MXFP4 terms for the down GEMM
     mark(3);
     {
-        const int blocks = (T * k + HENC_WARPS - 1) / HENC_WARPS;
-        h_encode_kernel<<<blocks, HENC_WARPS * 32, 0, stream>>>(h->H16, h->GU, Hop, f, BN, h->row_slot, h->sched);
+        const long items = static_cast<long>(T) * k * (f / 32);
+        const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
+        h_encode_kernel<<<blocks, HENC_THREADS, 0, stream>>>(h->H16, h->GU, Hop, f, BN, h->row_slot, h->sched);
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine
@@ -679,7 +681,7 @@ moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n) {
 // address comes from cudaGetSymbolAddress, looked up once per device.
 namespace {
 
-constexpr int NOALLOC_MAX_SPLITS = 8;
+constexpr int NOALLOC_MAX_SPLITS = ROUTER_MAX_SPLITS;
 constexpr size_t NOALLOC_PART_BYTES = sizeof(double) * NOALLOC_MAX_SPLITS * MOE_ROUTE_NOALLOC_MAX_TOKENS *
                                       MOE_ROUTE_NOALLOC_MAX_EXPERTS;
 constexpr int NOALLOC_MAX_TILES = (MOE_ROUTE_NOALLOC_MAX_TOKENS + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
@@ -764,8 +766,6 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     ra.w_out = topk_w;
     ra.local_rank = reinterpret_cast<int32_t*>(sc + NA_OFF_RANK);
     ra.hist = reinterpret_cast<int32_t*>(sc + NA_OFF_HIST);
-    ra.zero_rows = nullptr;
-    ra.zero_ld = 0;
     // no expert GEMMs follow: zero feature tiles, so the schedule step only
     // totals the histogram (expert_counts) and emits no units
     ra.BN = 16;

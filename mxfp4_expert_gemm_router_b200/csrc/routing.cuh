@@ -49,10 +49,15 @@ template <> struct Raw8<float> {
 
 // Dynamic shared memory of router_kernel (floats): x chunk [32][65], router
 // chunk [64][E], scores [32][E+1].
+constexpr int ROUTER_MAX_SPLITS = 8;
 __host__ __device__ inline size_t router_smem_bytes(int E) {
-    return sizeof(float) * (static_cast<size_t>(ROUTER_TOKENS) * (ROUTER_KCHUNK + 1) +
+    return sizeof(float) * (static_cast<size_t>(ROUTER_TOKENS) * ROUTER_KCHUNK +
                             static_cast<size_t>(ROUTER_KCHUNK) * E + static_cast<size_t>(ROUTER_TOKENS) * (E + 1));
 }
+// Column of token t in row kk of the transposed x chunk: an XOR swizzle that
+// keeps each group of 4 tokens contiguous (one 16-byte read) and spreads the
+// rows a warp writes over all 32 banks.
+__device__ __forceinline__ int xs_col(int kk, int t) { return t ^ (4 * ((kk >> 3) & 7)); }
 
 // Schedule slots.
 enum : int {
@@ -77,8 +82,6 @@ struct RouterArgs {
     float* w_out;          // [T][k]
     int32_t* local_rank;   // [T][k] rank of the pair among earlier pairs of its tile with the same expert
     int32_t* hist;         // [tiles][E] per-tile counts, turned into per-tile prefixes by the schedule
-    float* zero_rows;      // output accumulator rows to clear, [T][zero_ld], or null
-    int zero_ld;
     // schedule
     int BN, F_gu, F_dn, KC_gu, KC_dn, nsm, split_rows_cap, max_units;
     int32_t* offsets;      // [E+1]
@@ -104,10 +107,13 @@ __device__ inline int pick_split(int base, int nsm, int KC) {
 }
 
 // Run by the last router CTA to finish: per-expert totals and per-tile
-// prefixes of the histogram (warp scans over tiles), group offsets, K splits,
-// and the unit lists of both expert GEMMs, ordered (expert, token tile, feature
-// tile, split).
-__device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt, int* off, int* split_s) {
+// prefixes of the histogram (warp scans over tiles), group offsets and token
+// tile bases (one warp-wide scan over experts), K splits, and the unit lists of
+// both expert GEMMs.  Units are ordered (expert, token tile, feature tile,
+// split); token tiles are numbered consecutively over the experts, so unit u
+// is token tile u / (F S), feature tile (u / S) % F, split u % S, and its
+// expert is found by binary search over the tile bases.
+__device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt, int* off, int* tb, int* split_s) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     for (int e = warp; e < a.E; e += nwarps) {
         int carry = 0;
@@ -126,58 +132,76 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
         if (lane == 0) cnt[e] = carry;
     }
     __syncthreads();
-    if (tid == 0) {
-        int s = 0, base_gu = 0, base_dn = 0;
-        for (int e = 0; e < a.E; ++e) {
-            off[e] = s;
-            s += cnt[e];
-            const int mt = (cnt[e] + a.BN - 1) / a.BN;
-            base_gu += mt * a.F_gu;
-            base_dn += mt * a.F_dn;
+    if (warp == 0) {
+        // lane l owns experts [l*epl, (l+1)*epl): exclusive scans of rows and tiles
+        const int epl = (a.E + 31) / 32;
+        int rows = 0, tiles = 0;
+        for (int i = 0; i < epl; ++i) {
+            const int e = lane * epl + i;
+            if (e < a.E) {
+                rows += cnt[e];
+                tiles += (cnt[e] + a.BN - 1) / a.BN;
+            }
         }
-        off[a.E] = s;
-        int sg = (s <= a.split_rows_cap) ? pick_split(base_gu, a.nsm, a.KC_gu) : 1;
-        int sd = pick_split(base_dn, a.nsm, a.KC_dn);
-        while (sg > 1 && base_gu * sg > a.max_units) --sg;
-        while (sd > 1 && base_dn * sd > a.max_units) --sd;
-        split_s[0] = sg;
-        split_s[1] = sd;
-        a.sched[SCHED_UNITS_GU] = min(base_gu * sg, a.max_units);
-        a.sched[SCHED_UNITS_DN] = min(base_dn * sd, a.max_units);
-        a.sched[SCHED_SPLIT_GU] = sg;
-        a.sched[SCHED_SPLIT_DN] = sd;
-        a.sched[SCHED_ROWS] = s;
+        int rinc = rows, tinc = tiles;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int rn = __shfl_up_sync(0xffffffffu, rinc, o), tn = __shfl_up_sync(0xffffffffu, tinc, o);
+            if (lane >= o) { rinc += rn; tinc += tn; }
+        }
+        int r = rinc - rows, tt = tinc - tiles;
+        for (int i = 0; i < epl; ++i) {
+            const int e = lane * epl + i;
+            if (e < a.E) {
+                off[e] = r;
+                tb[e] = tt;
+                r += cnt[e];
+                tt += (cnt[e] + a.BN - 1) / a.BN;
+            }
+        }
+        const int total_rows = __shfl_sync(0xffffffffu, rinc, 31), total_tiles = __shfl_sync(0xffffffffu, tinc, 31);
+        if (lane == 0) {
+            off[a.E] = total_rows;
+            tb[a.E] = total_tiles;
+            const int base_gu = total_tiles * a.F_gu, base_dn = total_tiles * a.F_dn;
+            int sg = (total_rows <= a.split_rows_cap) ? pick_split(base_gu, a.nsm, a.KC_gu) : 1;
+            int sd = pick_split(base_dn, a.nsm, a.KC_dn);
+            while (sg > 1 && base_gu * sg > a.max_units) --sg;
+            while (sd > 1 && base_dn * sd > a.max_units) --sd;
+            split_s[0] = sg;
+            split_s[1] = sd;
+            a.sched[SCHED_UNITS_GU] = min(base_gu * sg, a.max_units);
+            a.sched[SCHED_UNITS_DN] = min(base_dn * sd, a.max_units);
+            a.sched[SCHED_SPLIT_GU] = sg;
+            a.sched[SCHED_SPLIT_DN] = sd;
+            a.sched[SCHED_ROWS] = total_rows;
+        }
     }
     __syncthreads();
     for (int e = tid; e <= a.E; e += blockDim.x) a.offsets[e] = off[e];
-    if (a.tile_base && tid == 0) {
-        int tb = 0;
-        for (int e = 0; e < a.E; ++e) {
-            a.tile_base[e] = tb;
-            tb += (cnt[e] + a.BN - 1) / a.BN;
-        }
-    }
     if (a.counts_out)
         for (int e = tid; e < a.E; e += blockDim.x) a.counts_out[e] = cnt[e];
+    if (a.tile_base)
+        for (int e = tid; e < a.E; e += blockDim.x) a.tile_base[e] = tb[e];
+    const int total_tiles = tb[a.E];
     for (int g = 0; g < 2; ++g) {
         const int F = g ? a.F_dn : a.F_gu;
         const int S = split_s[g];
         int4* units = g ? a.units_dn : a.units_gu;
-        int ubase = 0, tb = 0;
-        for (int e = 0; e < a.E; ++e) {
-            const int n = cnt[e];
-            const int mt = (n + a.BN - 1) / a.BN;
-            const int nu = mt * F * S;
-            for (int i = tid; i < nu; i += blockDim.x) {
-                const int u = ubase + i;
-                if (u >= a.max_units) break;
-                const int m = i / (F * S);
-                const int rem = i - m * F * S;
-                const int ft = rem / S, sp = rem - ft * S;
-                units[u] = make_int4(e | ((tb + m) << 8), off[e] + m * a.BN, min(a.BN, n - m * a.BN), ft | (sp << 16));
+        const int nu = min(total_tiles * F * S, a.max_units);
+        for (int u = tid; u < nu; u += blockDim.x) {
+            const int tile = u / (F * S);
+            const int rem = u - tile * F * S;
+            const int ft = rem / S, sp = rem - ft * S;
+            // the last e with tb[e] <= tile: an expert with no tiles shares its base
+            // with the next one, so this e owns the tile
+            int lo = 0, hi = a.E - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (tb[mid] <= tile) lo = mid; else hi = mid - 1;
             }
-            ubase += nu;
-            tb += mt;
+            const int m = tile - tb[lo];
+            units[u] = make_int4(lo | (tile << 8), off[lo] + m * a.BN, min(a.BN, cnt[lo] - m * a.BN), ft | (sp << 16));
         }
     }
 }
@@ -189,21 +213,21 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
 // order (deterministic), adds the bias, and with one warp per token selects
 // the top-k by k rounds of warp arg-max (ties to the lower index) and applies
 // the softmax over the k selected scores; it also ranks the tile's (token,
-// slot) pairs within their expert, writes the tile histogram and zeroes the
-// output accumulator rows of its tokens.  The last tile to finish builds the
-// schedule (schedule_block).
+// slot) pairs within their expert and writes the tile histogram.  The last
+// tile to finish builds the schedule (schedule_block).
 // EPT = experts per lane (ceil(E / 32) rounded up to 1, 2, 4 or 8): the
 // register tile scales with the expert count.
 template <typename TA, int EPT>
 __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
-    extern __shared__ float rsm[];
-    float* xs = rsm;                                      // [32][65]
-    float* ws = xs + ROUTER_TOKENS * (ROUTER_KCHUNK + 1);  // [64][E]
+    extern __shared__ __align__(16) float rsm[];
+    float* xs = rsm;                                      // [64 k][32 tokens], swizzled (xs_col)
+    float* ws = xs + ROUTER_TOKENS * ROUTER_KCHUNK;        // [64 k][E]
     float* lg = ws + ROUTER_KCHUNK * a.E;                  // [32][E+1]
     __shared__ int hist_s[MAX_EXPERTS];
     __shared__ int es[ROUTER_TOKENS * MAX_TOPK];
     __shared__ int cnt_s[MAX_EXPERTS];
     __shared__ int off_s[MAX_EXPERTS + 1];
+    __shared__ int tb_s[MAX_EXPERTS + 1];
     __shared__ int split_s[2];
     __shared__ int last_s;
 
@@ -248,7 +272,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
         const int kc = c * ROUTER_KCHUNK;
         __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[xt * (ROUTER_KCHUNK + 1) + xv8 + j] = xr.get(j);
+        for (int j = 0; j < 8; ++j) xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = xr.get(j);
 #pragma unroll
         for (int i = 0; i < EPT; ++i) {
             const int idx = tid + ROUTER_THREADS * i;
@@ -267,9 +291,9 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
             for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 8
         for (int kk = 0; kk < ROUTER_KCHUNK; ++kk) {
-            float xv[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) xv[j] = xs[(warp * 4 + j) * (ROUTER_KCHUNK + 1) + kk];
+            // x of the warp's 4 tokens at kk: one broadcast 16-byte read
+            const float4 x4 = *reinterpret_cast<const float4*>(xs + kk * ROUTER_TOKENS + xs_col(kk, warp * 4));
+            const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
             for (int i = 0; i < EPT; ++i) {
                 const int e = lane + 32 * i;
@@ -304,24 +328,33 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
 
     for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
-    for (int i = tid; i < ntok * E; i += ROUTER_THREADS) {
-        const int tl = i / E, e = i % E;
-        // partials summed in split order (deterministic), four loads in flight
-        double s = 0.0;
-        const double* pp = a.part + static_cast<size_t>(t0 + tl) * E + e;
+    {
+        // logits = partials summed in split order (deterministic) + bias; each
+        // thread takes 2 outputs with all their partial loads in flight
         const size_t pstride = static_cast<size_t>(a.T) * E;
-        int sp = 0;
-        for (; sp + 4 <= a.S; sp += 4) {
-            const double p0 = __ldcg(pp + (sp + 0) * pstride), p1 = __ldcg(pp + (sp + 1) * pstride);
-            const double p2 = __ldcg(pp + (sp + 2) * pstride), p3 = __ldcg(pp + (sp + 3) * pstride);
-            s += p0;
-            s += p1;
-            s += p2;
-            s += p3;
+        for (int i0 = tid; i0 < ntok * E; i0 += 2 * ROUTER_THREADS) {
+            double pv[2][ROUTER_MAX_SPLITS];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                const double* pp = a.part + static_cast<size_t>(t0 + i / E) * E + i % E;
+#pragma unroll
+                for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
+                    pv[m][sp] = (i < ntok * E && sp < a.S) ? __ldcg(pp + sp * pstride) : 0.0;
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                if (i < ntok * E) {
+                    double s = 0.0;
+#pragma unroll
+                    for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) s += pv[m][sp];
+                    const int tl = i / E, e = i % E;
+                    if (a.bias) s += a.bias[e];
+                    lg[tl * (E + 1) + e] = static_cast<float>(s);
+                }
+            }
         }
-        for (; sp < a.S; ++sp) s += __ldcg(pp + sp * pstride);
-        if (a.bias) s += a.bias[e];
-        lg[tl * (E + 1) + e] = static_cast<float>(s);
     }
     __syncthreads();
 
@@ -363,27 +396,28 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
                 a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
                 a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
                 es[tl * k + r] = sel_e[r];
-                atomicAdd(&hist_s[sel_e[r]], 1);
             }
         }
     }
     __syncthreads();
-    // stable rank of each pair among the tile's earlier pairs with the same expert
-    for (int p = tid; p < ntok * k; p += ROUTER_THREADS) {
-        const int e = es[p];
-        int rank = 0;
-        for (int q = 0; q < p; ++q) rank += (es[q] == e);
-        a.local_rank[static_cast<size_t>(t0) * k + p] = rank;
-    }
-    for (int e = tid; e < E; e += ROUTER_THREADS) a.hist[static_cast<size_t>(tile) * E + e] = hist_s[e];
-    if (a.zero_rows) {
-        const int nvec = a.zero_ld / 4;
-        for (int i = tid; i < ntok * nvec; i += ROUTER_THREADS) {
-            const int t = i / nvec, v = i % nvec;
-            reinterpret_cast<float4*>(a.zero_rows + static_cast<size_t>(t0 + t) * a.zero_ld)[v] =
-                make_float4(0.f, 0.f, 0.f, 0.f);
+    // stable rank of each pair among the tile's earlier pairs with the same
+    // expert, and the tile histogram: warp 0 walks the pairs in order, 32 at a
+    // time; lanes with the same expert find one another with match_any.
+    if (warp == 0) {
+        for (int p0 = 0; p0 < ntok * k; p0 += 32) {
+            const int p = p0 + lane;
+            const bool valid = p < ntok * k;
+            const int e = valid ? es[p] : -1 - lane;   // idle lanes form groups of their own
+            const unsigned grp = __match_any_sync(0xffffffffu, e);
+            const int before = __popc(grp & ((1u << lane) - 1u));
+            if (valid) a.local_rank[static_cast<size_t>(t0) * k + p] = hist_s[e] + before;
+            __syncwarp();
+            if (valid && before == 0) hist_s[e] += __popc(grp);
+            __syncwarp();
         }
     }
+    __syncthreads();
+    for (int e = tid; e < E; e += ROUTER_THREADS) a.hist[static_cast<size_t>(tile) * E + e] = hist_s[e];
 
     // the last tile builds the schedule
     __threadfence();
@@ -393,7 +427,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     if (!last_s) return;
     __threadfence();
     if (tid == 0) *a.glob_cnt = 0;
-    schedule_block(a, ntiles, cnt_s, off_s, split_s);
+    schedule_block(a, ntiles, cnt_s, off_s, tb_s, split_s);
 }
 
 // One 32-element block of a token's activations as floats.
@@ -426,7 +460,7 @@ template <> struct BlockLoader<float> {
     }
 };
 
-constexpr int GATHER_WARPS = 8;
+constexpr int GATHER_THREADS = 128;
 
 // Where the grouped operands live.
 struct GroupedOperand {
@@ -440,54 +474,61 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
     return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * MXQ_TERMS * 512;
 }
 
-// One warp per (token, slot) pair p = t*k + j: its grouped row is
-// offsets[e] + (rows of e in earlier tiles) + (its rank within its tile), so the
-// rows of an expert are in (token, slot) order; the row's place in the expert's
-// token tiles is (tile_base[e] + (row - offsets[e]) / BN, (row - offsets[e]) % BN).
-// The warp records the row's token, routing weight and tile slot, and encodes
-// the token's activations as three MXFP4 terms into the grouped operand: lane
-// l takes blocks l, l + 32, ... (one 16-byte store per term and block, one
-// scale byte into the block's scale atom).  When the gate/up GEMM splits K it
-// also zeroes the row of the fp32 partial-sum buffer.
+// One thread per (token, slot) pair p = t*k + j and 32-block b of d_model
+// (consecutive threads take consecutive blocks of a pair: coalesced reads).
+// The pair's grouped row is offsets[e] + (rows of e in earlier tiles) + (its
+// rank within its tile), so the rows of an expert are in (token, slot) order;
+// the row's place in the expert's token tiles is (tile_base[e] + (row -
+// offsets[e]) / BN, (row - offsets[e]) % BN).  The thread encodes its block of
+// the token's activations as three MXFP4 terms into the grouped operand (16
+// bytes per term, one scale byte per term into the block's scale atom); the
+// block-0 thread records the row's token, routing weight and tile slot.  The
+// slot-0 pair of each token clears the token's row of the fp32 output
+// accumulator (block by block) for the down GEMM's scatter-add.  When the
+// gate/up GEMM splits K it also zeroes its part of the row of the fp32
+// partial-sum buffer.
 template <typename TA>
-__global__ void __launch_bounds__(GATHER_WARPS * 32)
+__global__ void __launch_bounds__(GATHER_THREADS)
 gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
               const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
               const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
               int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
-              GroupedOperand X, float* __restrict__ GU, int gu_ld, const int32_t* __restrict__ sched) {
-    const int lane = threadIdx.x & 31;
-    const int p = blockIdx.x * GATHER_WARPS + (threadIdx.x >> 5);
-    if (p >= T * k) return;
+              GroupedOperand X, float* __restrict__ GU, int gu_ld, float* __restrict__ yacc,
+              const int32_t* __restrict__ sched) {
+    const int nb = d / 32;
+    const long item = static_cast<long>(blockIdx.x) * GATHER_THREADS + threadIdx.x;
+    if (item >= static_cast<long>(T) * k * nb) return;
+    const int p = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
     const int t = p / k;
     const int e = idx[p];
     const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
     const int pos = offsets[e] + loc;
     const int tile = tile_base[e] + loc / BN, rloc = loc % BN;
-    if (lane == 0) {
+    if (b == 0) {
         row_token[pos] = t;
         row_weight[pos] = w[p];
         row_slot[pos] = tile * BN + rloc;
     }
-    const TA* src = x + static_cast<size_t>(t) * d;
-    const int nb = d / 32;
-    for (int b = lane; b < nb; b += 32) {
-        float v[32];
-        BlockLoader<TA>::load(src + b * 32, v);
-        uint4 codes[MXQ_TERMS];
-        uint32_t sb[MXQ_TERMS];
-        mxq_block_thread(v, codes, sb);
-        uint8_t* atoms = scale_atom_base(X, tile, b >> 2);
+    if (p % k == 0) {
+        float4* yz = reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d + b * 32);
 #pragma unroll
-        for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-            *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) =
-                codes[tt];
-            atoms[sf_atom_offset(tt * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
-        }
+        for (int i = 0; i < 8; ++i) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float v[32];
+    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+    uint4 codes[MXQ_TERMS];
+    uint32_t sb[MXQ_TERMS];
+    mxq_block_thread(v, codes, sb);
+    uint8_t* atoms = scale_atom_base(X, tile, b >> 2);
+#pragma unroll
+    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+        *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) = codes[tt];
+        atoms[sf_atom_offset(tt * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
     }
     if (sched[SCHED_SPLIT_GU] > 1) {
-        float4* g = reinterpret_cast<float4*>(GU + static_cast<size_t>(pos) * gu_ld);
-        for (int v = lane; v < gu_ld / 4; v += 32) g[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // the pair's nb threads zero the row together (consecutive floats per step)
+        float* g = GU + static_cast<size_t>(pos) * gu_ld;
+        for (int i = b; i < gu_ld; i += nb) g[i] = 0.f;
     }
 }
 
@@ -498,62 +539,59 @@ __device__ __forceinline__ __half to_half_sat(float v) {
     return __float2half_rn(v);
 }
 
-constexpr int HENC_WARPS = 8;
+constexpr int HENC_THREADS = 128;
 
-// Encodes H for the down GEMM: one warp per grouped row, lane l takes the
-// 32-feature blocks l, l + 32, ... of the row.  H comes from the gate/up
-// epilogue as f16 (Swish(g) * u already applied), or, when the gate/up GEMM
-// split K, from the fp32 partial sums of g and u (Swish applied here).  Each
-// block is encoded as three MXFP4 terms (mxq_block_thread) into the down
+// Encodes H for the down GEMM: one thread per (grouped row, 32-feature block),
+// consecutive threads taking consecutive blocks of a row.  H comes from the
+// gate/up epilogue as f16 (Swish(g) * u already applied), or, when the gate/up
+// GEMM split K, from the fp32 partial sums of g and u (Swish applied here).
+// Each block is encoded as three MXFP4 terms (mxq_block_thread) into the down
 // GEMM's B operand: 16 code bytes per term, one scale byte per term into the
 // scale atom of the row's token tile.
-__global__ void __launch_bounds__(HENC_WARPS * 32)
+__global__ void __launch_bounds__(HENC_THREADS)
 h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
                 const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
-    const int rows = sched[SCHED_ROWS];
+    const int nb = d_ff / 32;
+    const long item = static_cast<long>(blockIdx.x) * HENC_THREADS + threadIdx.x;
+    if (item >= static_cast<long>(sched[SCHED_ROWS]) * nb) return;
+    const int row = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
     const bool split = sched[SCHED_SPLIT_GU] > 1;
-    const int row = blockIdx.x * HENC_WARPS + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
     const int slot = row_slot[row];
     const int tile = slot / BN, rloc = slot % BN;
-    const int nb = d_ff / 32;
-    for (int b = lane; b < nb; b += 32) {
-        float v[32];
-        if (split) {
-            const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
-            const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);
+    float v[32];
+    if (split) {
+        const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
+        const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 gg = g[i], uu = u[i];
-                v[4 * i] = swish_f(gg.x) * uu.x;
-                v[4 * i + 1] = swish_f(gg.y) * uu.y;
-                v[4 * i + 2] = swish_f(gg.z) * uu.z;
-                v[4 * i + 3] = swish_f(gg.w) * uu.w;
-            }
-        } else {
-            const uint4* hp = reinterpret_cast<const uint4*>(H16 + static_cast<size_t>(row) * d_ff + 32 * b);
+        for (int i = 0; i < 8; ++i) {
+            const float4 gg = g[i], uu = u[i];
+            v[4 * i] = swish_f(gg.x) * uu.x;
+            v[4 * i + 1] = swish_f(gg.y) * uu.y;
+            v[4 * i + 2] = swish_f(gg.z) * uu.z;
+            v[4 * i + 3] = swish_f(gg.w) * uu.w;
+        }
+    } else {
+        const uint4* hp = reinterpret_cast<const uint4*>(H16 + static_cast<size_t>(row) * d_ff + 32 * b);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 q = hp[i];
-                const __half2* h2 = reinterpret_cast<const __half2*>(&q);
+        for (int i = 0; i < 4; ++i) {
+            const uint4 q = hp[i];
+            const __half2* h2 = reinterpret_cast<const __half2*>(&q);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = __half22float2(h2[j]);
-                    v[8 * i + 2 * j] = f.x;
-                    v[8 * i + 2 * j + 1] = f.y;
-                }
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(h2[j]);
+                v[8 * i + 2 * j] = f.x;
+                v[8 * i + 2 * j + 1] = f.y;
             }
         }
-        uint4 codes[MXQ_TERMS];
-        uint32_t sb[MXQ_TERMS];
-        mxq_block_thread(v, codes, sb);
-        uint8_t* atoms = scale_atom_base(Hd, tile, b >> 2);
+    }
+    uint4 codes[MXQ_TERMS];
+    uint32_t sb[MXQ_TERMS];
+    mxq_block_thread(v, codes, sb);
+    uint8_t* atoms = scale_atom_base(Hd, tile, b >> 2);
 #pragma unroll
-        for (int t = 0; t < MXQ_TERMS; ++t) {
-            *reinterpret_cast<uint4*>(Hd.codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * Hd.R + row) * 16) = codes[t];
-            atoms[sf_atom_offset(t * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
-        }
+    for (int t = 0; t < MXQ_TERMS; ++t) {
+        *reinterpret_cast<uint4*>(Hd.codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * Hd.R + row) * 16) = codes[t];
+        atoms[sf_atom_offset(t * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
     }
 }
 
