@@ -68,8 +68,9 @@ struct MxgParams {
     int BN;                   // token rows per tile (multiple of 16, at most 128)
     int stages;
     int nacc;                 // accumulator buffers (1 or 2)
-    const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][3 terms][512]
-    uint32_t idesc;           // M = 128, N = BN, without scale-factor ids
+    const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][3][512]
+    int stacked;              // 1: the three terms are N = 3 * BN rows of one MMA (3 * BN <= 128)
+    uint32_t idesc;           // M = 128, N = BN (or 3 * BN stacked), without scale-factor ids
     __half* H16;              // MODE 0 output H = Swish(g) * u, f16 [rows][N]
     float* GU;                // MODE 0 split partials [rows][2N]
     float* yacc;              // MODE 1 output accumulator [T][N]
@@ -89,7 +90,12 @@ constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
 __host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
     return mxg_w_stage(mode) + mxg_b_bytes(BN) + MXG_SFB_BYTES;
 }
-__host__ __device__ constexpr int mxg_mat_cols(int BN) { return ((BN + 31) / 32) * 32; }
+// Stacked terms for small tiles: one MMA per K step reads the weight tile once
+// (separate per-term MMAs would read it three times); needs 3 * BN <= 128.
+__host__ __device__ constexpr bool mxg_stacked(int BN) { return MXQ_TERMS * BN <= 128; }
+__host__ __device__ constexpr int mxg_mat_cols(int BN) {
+    return (((mxg_stacked(BN) ? MXQ_TERMS : 1) * BN + 31) / 32) * 32;
+}
 __host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
 __host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
 __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
@@ -107,7 +113,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
 
     const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
     const uint32_t b_bytes = mxg_b_bytes(BN);
-    const uint32_t sf_bytes = MXG_SFB_BYTES;
+    const uint32_t sf_bytes = p.stacked ? 512u : MXG_SFB_BYTES;   // atoms used per stage
     const uint32_t stage_bytes = W_STAGE + b_bytes + sf_bytes;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -181,7 +187,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                     bulk_g2s_warp(st, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
                     // rows U.y .. U.y + BN - 1 of every (block, term): 8-byte elements 2 * U.y ..
                     tma_load_3d_warp(st + W_STAGE, &tmap_b, 2 * U.y, 0, 4 * c, full_bar(s));
-                    bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * sf_bytes,
+                    bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * MXG_SFB_BYTES,
                                   sf_bytes, full_bar(s));
                     pend_ph[s] = static_cast<int>(ph);
                 }
@@ -222,21 +228,37 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
                 tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
                 if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
+                if (p.stacked) {
+                    // one MMA per K step and matrix: N = 3 * BN rows (term-major), one B scale atom
+                    tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
 #pragma unroll
-                for (int t = 0; t < MXQ_TERMS; ++t) tc_cp_sf_warp(sfc + 8 + 4 * t, desc_noswz(ss + 512 * t, 0, 128));
+                    for (int i = 0; i < 2; ++i) {
+                        if (2 * i < nbc) {
+                            const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
+                            const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
+                            const uint64_t ad = desc_noswz(ws + 2 * i * rf * 16, rf * 16, 128);
+                            const uint64_t bd = desc_noswz(bs + 2 * i * NB3 * 16, NB3 * 16, 128);
+                            mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8, acc);
+                            if (MODE == 0) mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8, acc);
+                        }
+                    }
+                } else {
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (2 * i < nbc) {
-                        const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
-                        const uint64_t ad = desc_noswz(ws + 2 * i * rf * 16, rf * 16, 128);
+                    for (int t = 0; t < MXQ_TERMS; ++t) tc_cp_sf_warp(sfc + 8 + 4 * t, desc_noswz(ss + 512 * t, 0, 128));
 #pragma unroll
-                        for (int t = 0; t < MXQ_TERMS; ++t) {
-                            // B of term t, blocks 2i and 2i+1: smem [block][term][row][16 B]
-                            const uint32_t acc = (c > c0 || i > 0 || t > 0) ? 1u : 0u;
-                            const uint64_t bd = desc_noswz(bs + (2 * i * MXQ_TERMS + t) * BN * 16, NB3 * 16, 128);
-                            mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8 + 4 * t, acc);
-                            if (MODE == 0)
-                                mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8 + 4 * t, acc);
+                    for (int i = 0; i < 2; ++i) {
+                        if (2 * i < nbc) {
+                            const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
+                            const uint64_t ad = desc_noswz(ws + 2 * i * rf * 16, rf * 16, 128);
+#pragma unroll
+                            for (int t = 0; t < MXQ_TERMS; ++t) {
+                                // B of term t, blocks 2i and 2i+1: smem [block][term][row][16 B]
+                                const uint32_t acc = (c > c0 || i > 0 || t > 0) ? 1u : 0u;
+                                const uint64_t bd = desc_noswz(bs + (2 * i * MXQ_TERMS + t) * BN * 16, NB3 * 16, 128);
+                                mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8 + 4 * t, acc);
+                                if (MODE == 0)
+                                    mma_mxf4_warp(d0 + mat_cols, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8 + 4 * t, acc);
+                            }
                         }
                     }
                 }
@@ -275,15 +297,32 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
             if (warp_rows) {
                 const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
                 for (int r0 = 8 * hh; r0 < nvalid; r0 += 16) {
-                    uint32_t g[8], v[8];
-                    tmem_ld8(d0 + r0, g);
-                    if (MODE == 0) tmem_ld8(d0 + mat_cols + r0, v);
-                    tmem_wait_ld();
                     float gs[8], us[8];
+                    if (p.stacked) {
+                        // the three term columns of each token are BN apart: add them
+                        uint32_t g[MXQ_TERMS][8], v[MXQ_TERMS][8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        gs[j] = __uint_as_float(g[j]);
-                        us[j] = MODE == 0 ? __uint_as_float(v[j]) : 0.f;
+                        for (int t = 0; t < MXQ_TERMS; ++t) {
+                            tmem_ld8(d0 + t * BN + r0, g[t]);
+                            if (MODE == 0) tmem_ld8(d0 + mat_cols + t * BN + r0, v[t]);
+                        }
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            gs[j] = __uint_as_float(g[0][j]) + __uint_as_float(g[1][j]) + __uint_as_float(g[2][j]);
+                            us[j] = MODE == 0 ? __uint_as_float(v[0][j]) + __uint_as_float(v[1][j]) + __uint_as_float(v[2][j])
+                                              : 0.f;
+                        }
+                    } else {
+                        uint32_t g[8], v[8];
+                        tmem_ld8(d0 + r0, g);
+                        if (MODE == 0) tmem_ld8(d0 + mat_cols + r0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            gs[j] = __uint_as_float(g[j]);
+                            us[j] = MODE == 0 ? __uint_as_float(v[j]) : 0.f;
+                        }
                     }
                     const int nv = min(8, nvalid - r0);   // valid token columns in this group (warp-uniform)
                     if (MODE == 0) {

@@ -523,8 +523,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     mark(1);
     const long gitems = static_cast<long>(T) * k * (d / 32);
     const int gblocks = static_cast<int>((gitems + GATHER_THREADS - 1) / GATHER_THREADS);
-    GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu};
-    GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn};
+    const bool stacked = mxg_stacked(BN);
+    GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
+    GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
     if (bf16)
         gather_kernel<__nv_bfloat16><<<gblocks, GATHER_THREADS, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E,
@@ -548,7 +549,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.stages = stages_for(0, BN);
     gp.nacc = mxg_nacc(0, BN);
     gp.sfb = h->sfx;
-    gp.idesc = idesc_mxf4(128, BN);
+    gp.stacked = stacked ? 1 : 0;
+    gp.idesc = idesc_mxf4(128, (stacked ? MXQ_TERMS : 1) * BN);
     gp.H16 = h->H16;
     gp.GU = h->GU;
     gp.yacc = nullptr;

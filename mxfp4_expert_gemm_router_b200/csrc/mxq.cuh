@@ -9,8 +9,9 @@
 // significant bits, far too coarse for the layer's accuracy, so a block v of
 // 32 values is written as v ~= q1 + q2 + q3: q1 encodes v, q2 encodes the
 // residual v - q1, q3 the residual v - q1 - q2, each with its own scale.  The
-// GEMM issues one MMA per term into the same accumulator, so the tensor core
-// adds the three products.  Measured on the oracle's weights (double
+// GEMM either issues one MMA per term into the same accumulator (the tensor
+// core adds the three products) or, for small token tiles, stacks the terms
+// as 3 * BN rows of one MMA and adds the three accumulator columns itself.  Measured on the oracle's weights (double
 // precision emulation), the layer error of the 3-term encoding is about 0.25 %
 // of max|y| (2 terms: about 3 %).
 //
@@ -20,9 +21,10 @@
 //
 // Operand layouts in global memory (R = row capacity, NB = K / 32 blocks):
 //   codes   [NB][3 terms][R rows][16 B]   (element 2i of the block in the low nibble of byte i)
-//   scales  per (token tile, K chunk of 128): one 512-byte atom per term; row r
-//           of the tile (r < 128), term t, block q (0..3) of the chunk at byte
-//           sf_atom_offset(t * 128 + r, q).
+//   scales  per (token tile, K chunk of 128): three 512-byte atoms; row r of
+//           the tile, term t, block q (0..3) of the chunk at byte
+//           sf_atom_offset(t * R_t + r, q), R_t = 128 (terms as separate MMAs,
+//           atom t) or BN (terms stacked, 3 * BN <= 128 rows in atom 0).
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>

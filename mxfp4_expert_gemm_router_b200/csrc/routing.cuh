@@ -465,9 +465,11 @@ constexpr int GATHER_THREADS = 128;
 // Where the grouped operands live.
 struct GroupedOperand {
     uint8_t* codes;   // [K/32][3][R][16]
-    uint8_t* scales;  // [tiles][KC][3 terms][512]
+    uint8_t* scales;  // [tiles][KC][3 atoms][512]
     int R;            // row capacity
     int KC;           // chunks of 128 along K
+    int term_rows;    // operand row of (term t, tile row r) = t * term_rows + r: 128 when each term
+                      // is its own MMA (atom t), BN when the terms are stacked into one MMA
 };
 
 __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int tile, int chunk) {
@@ -523,7 +525,7 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
 #pragma unroll
     for (int tt = 0; tt < MXQ_TERMS; ++tt) {
         *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) = codes[tt];
-        atoms[sf_atom_offset(tt * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
+        atoms[sf_atom_offset(tt * X.term_rows + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
     }
     if (sched[SCHED_SPLIT_GU] > 1) {
         // the pair's nb threads zero the row together (consecutive floats per step)
@@ -591,7 +593,7 @@ h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, Gr
 #pragma unroll
     for (int t = 0; t < MXQ_TERMS; ++t) {
         *reinterpret_cast<uint4*>(Hd.codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * Hd.R + row) * 16) = codes[t];
-        atoms[sf_atom_offset(t * 128 + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
+        atoms[sf_atom_offset(t * Hd.term_rows + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
     }
 }
 
