@@ -149,10 +149,14 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) prefetch_tmap(&tmap_b);
+    pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // everything above is local set-up; the unit list and the B operand come
+    // from the preceding kernels
+    pdl_wait();
 
     const int num_units = p.sched[MODE == 0 ? SCHED_UNITS_GU : SCHED_UNITS_DN];
     const int nsplit = p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN];

@@ -113,6 +113,28 @@ struct moe_mxfp4 {
 
 static bool g_attrs_set = false;
 
+// Launch with programmatic stream serialization when `pdl` is set: the kernel
+// may start while the previous kernel in the stream finishes (it runs its
+// local set-up, then waits in pdl_wait for the previous kernel's results).
+// Used for decode-sized forwards, where launch latency and kernel ramp-up are
+// a large share of the step; with large grids, dependents launched early only
+// take residency from the running kernel.
+template <typename... KArgs, typename... Args>
+static void launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 #define MOE_TRY(expr)                                   \
@@ -521,19 +543,26 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     h->stage_ran[0] = true;
     // 1: gather into grouped rows
     mark(1);
+    const bool pdl = static_cast<long>(T) * k <= h->gu_rows;
     const long gitems = static_cast<long>(T) * k * (d / 32);
     const int gblocks = static_cast<int>((gitems + GATHER_THREADS - 1) / GATHER_THREADS);
     const bool stacked = mxg_stacked(BN);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
     if (bf16)
-        gather_kernel<__nv_bfloat16><<<gblocks, GATHER_THREADS, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E,
-            k, BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc, h->sched);
+        launch_pdl(pdl, gather_kernel<__nv_bfloat16>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
+                   static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(idx),
+                   static_cast<const float*>(wts), static_cast<const int32_t*>(h->local_rank),
+                   static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
+                   static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
+                   h->row_slot, Xop, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched));
     else
-        gather_kernel<float><<<gblocks, GATHER_THREADS, 0, stream>>>(
-            static_cast<const float*>(x), idx, wts, h->local_rank, h->hist, h->offsets, h->tile_base, T, d, E, k, BN,
-            h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc, h->sched);
+        launch_pdl(pdl, gather_kernel<float>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
+                   static_cast<const float*>(x), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
+                   static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
+                   static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
+                   BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc,
+                   static_cast<const int32_t*>(h->sched));
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);
@@ -560,14 +589,17 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.timeout_ns = tmo;
     gp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
     const int grid = h->nsm;
-    expert_mxf4_kernel<0><<<grid, MXG_THREADS, mxg_smem_bytes(0, BN, gp.stages), stream>>>(h->tm_x[BN / 16 - 1], gp);
+    launch_pdl(pdl, expert_mxf4_kernel<0>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(0, BN, gp.stages), stream,
+               h->tm_x[BN / 16 - 1], gp);
     h->stage_ran[2] = true;
     // 3: H (f16, or split-K partials) -> three MXFP4 terms for the down GEMM
     mark(3);
     {
         const long items = static_cast<long>(T) * k * (f / 32);
         const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
-        h_encode_kernel<<<blocks, HENC_THREADS, 0, stream>>>(h->H16, h->GU, Hop, f, BN, h->row_slot, h->sched);
+        launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const __half*>(h->H16),
+                   static_cast<const float*>(h->GU), Hop, f, BN, static_cast<const int32_t*>(h->row_slot),
+                   static_cast<const int32_t*>(h->sched));
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine
@@ -584,14 +616,16 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.GU = nullptr;
     dp.yacc = acc;
     dp.skip_first_copy = 0;
-    expert_mxf4_kernel<1><<<grid, MXG_THREADS, mxg_smem_bytes(1, BN, dp.stages), stream>>>(h->tm_h[BN / 16 - 1], dp);
+    launch_pdl(pdl, expert_mxf4_kernel<1>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages), stream,
+               h->tm_h[BN / 16 - 1], dp);
     h->stage_ran[4] = true;
     // 5: output cast
     mark(5);
     if (bf16) {
         const size_t n4 = static_cast<size_t>(T) * d / 4;
         const int blocks = static_cast<int>(std::min<size_t>(4 * static_cast<size_t>(h->nsm), (n4 + 255) / 256));
-        cast_out_kernel<<<std::max(1, blocks), 256, 0, stream>>>(h->yacc, static_cast<__nv_bfloat16*>(y), n4);
+        launch_pdl(pdl, cast_out_kernel, dim3(std::max(1, blocks)), dim3(256), 0, stream, static_cast<const float*>(h->yacc),
+                   static_cast<__nv_bfloat16*>(y), n4);
         h->stage_ran[5] = true;
     }
     mark(6);

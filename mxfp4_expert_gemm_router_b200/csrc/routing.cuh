@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     __shared__ int split_s[2];
     __shared__ int last_s;
 
+    pdl_launch_dependents();
     const TA* x = static_cast<const TA*>(a.x);
     const TA* wr = static_cast<const TA*>(a.wr);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -497,6 +498,8 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
               int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
               GroupedOperand X, float* __restrict__ GU, int gu_ld, float* __restrict__ yacc,
               const int32_t* __restrict__ sched) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int nb = d / 32;
     const long item = static_cast<long>(blockIdx.x) * GATHER_THREADS + threadIdx.x;
     if (item >= static_cast<long>(T) * k * nb) return;
@@ -553,6 +556,8 @@ constexpr int HENC_THREADS = 128;
 __global__ void __launch_bounds__(HENC_THREADS)
 h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
                 const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int nb = d_ff / 32;
     const long item = static_cast<long>(blockIdx.x) * HENC_THREADS + threadIdx.x;
     if (item >= static_cast<long>(sched[SCHED_ROWS]) * nb) return;
@@ -599,6 +604,7 @@ h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, Gr
 
 // fp32 accumulator -> bf16 output, 4 elements per thread-iteration.
 __global__ void cast_out_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y, size_t n4) {
+    pdl_wait();
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const float4 v = reinterpret_cast<const float4*>(acc)[i];

@@ -58,6 +58,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
     return ok != 0;
 }
 
+// ------------------------------------------------------------------ dependent launches
+// The next kernel in the stream may launch (it blocks in pdl_wait until this
+// grid has finished and its memory operations are visible).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until the preceding kernel in the stream has completed and its writes
+// are visible; a no-op for a kernel launched without programmatic serialization.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Device-side status words shared with the host.
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 
