@@ -21,9 +21,12 @@
 // epilogue of one unit overlaps the main loop of the next).
 //
 //   MODE 0 (gate/up): per stage gate and up chunks (17408 bytes), two
-//     accumulators for the same 128 features; epilogue: H = Swish(g) * u,
-//     stored as f16 (h_encode_kernel then encodes it for the down GEMM); with
-//     a K split, fp32 partials are added into GU instead.
+//     accumulators for the same 128 features; epilogue: H = Swish(g) * u for
+//     32 tokens x 32 features per warp goes through a small shared-memory tile
+//     (f16, transposed) so that each lane then holds one token's 32-feature
+//     block and encodes it as three MXFP4 terms straight into the down GEMM's
+//     B operand; with a K split, fp32 partials are added into GU instead (and
+//     h_encode_kernel encodes H).
 //   MODE 1 (down): per stage the down chunk (8704 bytes), one accumulator;
 //     epilogue: y[token, f] += w_row * d, red.add into the fp32 output
 //     accumulator (the weighted scatter-combine).
@@ -71,7 +74,7 @@ struct MxgParams {
     const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][3][512]
     int stacked;              // 1: the three terms are N = 3 * BN rows of one MMA (3 * BN <= 128)
     uint32_t idesc;           // M = 128, N = BN (or 3 * BN stacked), without scale-factor ids
-    __half* H16;              // MODE 0 output H = Swish(g) * u, f16 [rows][N]
+    GroupedOperand Hd;        // MODE 0 output: H as the down GEMM's B operand
     float* GU;                // MODE 0 split partials [rows][2N]
     float* yacc;              // MODE 1 output accumulator [T][N]
     const int32_t* row_token; // MODE 1
@@ -98,9 +101,14 @@ __host__ __device__ constexpr int mxg_mat_cols(int BN) {
 }
 __host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
 __host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
+// MODE 0 epilogue tiles: per epilogue warp 32 tokens x 32 features of f16, rows
+// padded to 33 so both the row writes and the column reads are conflict-free.
+constexpr int MXG_HT_STRIDE = 33;
+constexpr uint32_t MXG_HT_BYTES = MXG_EPI_WARPS * 32 * MXG_HT_STRIDE * 2;
+__host__ __device__ constexpr uint32_t mxg_extra_smem(int mode) { return mode == 0 ? MXG_HT_BYTES : 0u; }
 __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
     const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN) +
-                     (2 * stages + 2 * MXG_MAX_ACC + 1) * 8 + 64;
+                     (2 * stages + 2 * MXG_MAX_ACC + 1) * 8 + 64 + mxg_extra_smem(mode);
     return b < static_cast<size_t>(MXG_MIN_SMEM) ? static_cast<size_t>(MXG_MIN_SMEM) : b;
 }
 
@@ -127,6 +135,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
     uint8_t* ctl = smem_raw + (drain_bar + 8u - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
+    __half* htile_all = reinterpret_cast<__half*>(ctl + 64);   // MODE 0 epilogue tiles
     const int mat_cols = mxg_mat_cols(BN);
     const int acc_cols = (MODE == 0 ? 2 : 1) * mat_cols;
     const int NACC = p.nacc;
@@ -287,7 +296,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         bool ok = true;
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const int4 U = p.units[u];
-            const int row0 = U.y, nvalid = U.z;
+            const int tile = U.x >> 8, row0 = U.y, nvalid = U.z;
             const int ft = U.w & 0xFFFF;
             const int rf = min(128, p.N - ft * 128);
             const bool warp_rows = 32 * q < rf;
@@ -300,8 +309,8 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
             tc_fence_after();
             if (warp_rows) {
                 const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
-                for (int r0 = 8 * hh; r0 < nvalid; r0 += 16) {
-                    float gs[8], us[8];
+                // accumulators of token columns r0 .. r0 + 7 for this lane's feature
+                auto load8 = [&](int r0, float (&gs)[8], float (&us)[8]) {
                     if (p.stacked) {
                         // the three term columns of each token are BN apart: add them
                         uint32_t g[MXQ_TERMS][8], v[MXQ_TERMS][8];
@@ -328,30 +337,56 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                             us[j] = MODE == 0 ? __uint_as_float(v[j]) : 0.f;
                         }
                     }
-                    const int nv = min(8, nvalid - r0);   // valid token columns in this group (warp-uniform)
-                    if (MODE == 0) {
-                        if (nsplit == 1) {
-                            // H = Swish(g) * u as f16 (32 lanes = 64 contiguous bytes per row)
+                };
+                if (MODE == 0 && nsplit == 1) {
+                    // groups of 32 tokens alternate between the quarter's two warps
+                    __half* ht = htile_all + (warp - 2) * 32 * MXG_HT_STRIDE;
+                    const int blk = 4 * ft + q;
+                    uint8_t* atoms = scale_atom_base(p.Hd, tile, ft);
+                    for (int g0 = 32 * hh; g0 < nvalid; g0 += 64) {
+                        for (int s8 = 0; s8 < 32 && g0 + s8 < nvalid; s8 += 8) {
+                            float gs[8], us[8];
+                            load8(g0 + s8, gs, us);
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
-                                if (j < nv)
-                                    p.H16[static_cast<size_t>(row0 + r0 + j) * p.N + n] = to_half_sat(swish_f(gs[j]) * us[j]);
-                        } else {
+                                ht[(s8 + j) * MXG_HT_STRIDE + lane] = to_half_sat(swish_f(gs[j]) * us[j]);
+                        }
+                        __syncwarp();
+                        const int r = g0 + lane;   // this lane's token: one 32-feature block of H
+                        if (r < nvalid) {
+                            float hv[32];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                if (j < nv) {
-                                    float* gu = p.GU + static_cast<size_t>(row0 + r0 + j) * 2 * p.N;
-                                    atomicAdd(gu + n, gs[j]);
-                                    atomicAdd(gu + p.N + n, us[j]);
-                                }
+                            for (int c = 0; c < 32; ++c) hv[c] = __half2float(ht[lane * MXG_HT_STRIDE + c]);
+                            uint4 codes[MXQ_TERMS];
+                            uint32_t sb[MXQ_TERMS];
+                            mxq_block_thread(hv, codes, sb);
+#pragma unroll
+                            for (int t = 0; t < MXQ_TERMS; ++t) {
+                                *reinterpret_cast<uint4*>(
+                                    p.Hd.codes + ((static_cast<size_t>(blk) * MXQ_TERMS + t) * p.Hd.R + row0 + r) * 16) =
+                                    codes[t];
+                                atoms[sf_atom_offset(t * p.Hd.term_rows + r, q)] = static_cast<uint8_t>(sb[t]);
                             }
                         }
-                    } else {
+                        __syncwarp();
+                    }
+                } else {
+                    for (int r0 = 8 * hh; r0 < nvalid; r0 += 16) {
+                        float gs[8], us[8];
+                        load8(r0, gs, us);
+                        const int nv = min(8, nvalid - r0);   // valid token columns in this group (warp-uniform)
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             if (j < nv) {
                                 const int rr = row0 + r0 + j;
-                                atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n, gs[j] * p.row_weight[rr]);
+                                if (MODE == 0) {
+                                    float* gu = p.GU + static_cast<size_t>(rr) * 2 * p.N;
+                                    atomicAdd(gu + n, gs[j]);
+                                    atomicAdd(gu + p.N + n, us[j]);
+                                } else {
+                                    atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n,
+                                              gs[j] * p.row_weight[rr]);
+                                }
                             }
                         }
                     }

@@ -10,8 +10,9 @@
 //   gather_kernel        grouped rows (token, weight, tile slot); activations
 //                        encoded as three MXFP4 terms (the B operand)
 //   expert_mxf4<0>       gate/up GEMM on block-scaled MXFP4 tensor cores,
-//                        SwiGLU epilogue (H as f16, or fp32 partials when K is split)
-//   h_encode_kernel      H encoded as three MXFP4 terms for the down GEMM
+//                        SwiGLU epilogue encoding H as three MXFP4 terms for the
+//                        down GEMM (fp32 partials instead when K is split)
+//   h_encode_kernel      only when the gate/up GEMM may split K: SwiGLU + encoding
 //   expert_mxf4<1>       down GEMM, routing-weighted scatter-combine epilogue
 //   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
 #include <cuda.h>
@@ -88,7 +89,6 @@ struct moe_mxfp4 {
     int32_t* row_slot = nullptr;
     uint8_t* Xq = nullptr;     // x as three MXFP4 terms [d/32][3][TK][16]
     uint8_t* Hq = nullptr;     // H as three MXFP4 terms [d_ff/32][3][TK][16]
-    __half* H16 = nullptr;     // H = Swish(g) * u, f16 [TK][d_ff]
     uint8_t* sfx = nullptr;    // scale atoms of Xq per (token tile, K chunk)
     uint8_t* sfh = nullptr;    // scale atoms of Hq per (token tile, K chunk)
     size_t sfx_bytes = 0, sfh_bytes = 0, xq_bytes = 0, hq_bytes = 0;
@@ -146,7 +146,7 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 static void free_all(moe_mxfp4* h) {
     void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
-                    h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->H16, h->sfx, h->sfh,
+                    h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
     for (void* p : ptrs)
         if (p) cudaFree(p);
@@ -219,7 +219,7 @@ static cudaError_t set_router_smem(int bytes) {
 }
 
 static int stages_for(int mode, int BN) {
-    const size_t budget = 227 * 1024 - 1024 - 512;
+    const size_t budget = 227 * 1024 - 1024 - 512 - mxg_extra_smem(mode);
     int s = static_cast<int>(budget / mxg_stage_bytes(mode, BN));
     return std::max(2, std::min(MXG_MAX_STAGES, s));
 }
@@ -329,7 +329,6 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->row_slot), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->Xq), h->xq_bytes},
         {reinterpret_cast<void**>(&h->Hq), h->hq_bytes},
-        {reinterpret_cast<void**>(&h->H16), sizeof(__half) * TK * f},
         {reinterpret_cast<void**>(&h->sfx), h->sfx_bytes},
         {reinterpret_cast<void**>(&h->sfh), h->sfh_bytes},
         {reinterpret_cast<void**>(&h->GU), sizeof(float) * h->gu_rows * 2 * f},
@@ -544,7 +543,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 1: gather into grouped rows
     mark(1);
     const bool pdl = static_cast<long>(T) * k <= h->gu_rows;
-    const long gitems = static_cast<long>(T) * k * (d / 32);
+    const long gitems = static_cast<long>(T) * (d / 32);
     const int gblocks = static_cast<int>((gitems + GATHER_THREADS - 1) / GATHER_THREADS);
     const bool stacked = mxg_stacked(BN);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
@@ -580,7 +579,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.sfb = h->sfx;
     gp.stacked = stacked ? 1 : 0;
     gp.idesc = idesc_mxf4(128, (stacked ? MXQ_TERMS : 1) * BN);
-    gp.H16 = h->H16;
+    gp.Hd = Hop;
     gp.GU = h->GU;
     gp.yacc = nullptr;
     gp.row_token = h->row_token;
@@ -592,14 +591,13 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     launch_pdl(pdl, expert_mxf4_kernel<0>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(0, BN, gp.stages), stream,
                h->tm_x[BN / 16 - 1], gp);
     h->stage_ran[2] = true;
-    // 3: H (f16, or split-K partials) -> three MXFP4 terms for the down GEMM
+    // 3: split-K finish (a no-op unless the schedule split K): SwiGLU + H encoding
     mark(3);
-    {
+    if (static_cast<long>(T) * k <= h->gu_rows) {
         const long items = static_cast<long>(T) * k * (f / 32);
         const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
-        launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const __half*>(h->H16),
-                   static_cast<const float*>(h->GU), Hop, f, BN, static_cast<const int32_t*>(h->row_slot),
-                   static_cast<const int32_t*>(h->sched));
+        launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const float*>(h->GU),
+                   Hop, f, BN, static_cast<const int32_t*>(h->row_slot), static_cast<const int32_t*>(h->sched));
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine

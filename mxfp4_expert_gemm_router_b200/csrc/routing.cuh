@@ -477,19 +477,17 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
     return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * MXQ_TERMS * 512;
 }
 
-// One thread per (token, slot) pair p = t*k + j and 32-block b of d_model
-// (consecutive threads take consecutive blocks of a pair: coalesced reads).
-// The pair's grouped row is offsets[e] + (rows of e in earlier tiles) + (its
-// rank within its tile), so the rows of an expert are in (token, slot) order;
-// the row's place in the expert's token tiles is (tile_base[e] + (row -
-// offsets[e]) / BN, (row - offsets[e]) % BN).  The thread encodes its block of
-// the token's activations as three MXFP4 terms into the grouped operand (16
-// bytes per term, one scale byte per term into the block's scale atom); the
-// block-0 thread records the row's token, routing weight and tile slot.  The
-// slot-0 pair of each token clears the token's row of the fp32 output
-// accumulator (block by block) for the down GEMM's scatter-add.  When the
-// gate/up GEMM splits K it also zeroes its part of the row of the fp32
-// partial-sum buffer.
+// One thread per (token t, 32-block b of d_model); consecutive threads take
+// consecutive blocks of a token (coalesced reads).  The thread encodes its
+// block of x once as three MXFP4 terms and stores the codes and scale bytes
+// into each of the token's k grouped rows.  Pair p = t*k + j goes to grouped
+// row offsets[e] + (rows of e in earlier tiles) + (its rank within its tile),
+// so the rows of an expert are in (token, slot) order; the row's place in the
+// expert's token tiles is (tile_base[e] + (row - offsets[e]) / BN,
+// (row - offsets[e]) % BN).  The block-0 thread records each row's token,
+// routing weight and tile slot.  Every thread clears its block of the token's
+// row of the fp32 output accumulator (for the down GEMM's scatter-add) and,
+// when the gate/up GEMM splits K, its share of the fp32 partial-sum rows.
 template <typename TA>
 __global__ void __launch_bounds__(GATHER_THREADS)
 gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
@@ -502,38 +500,53 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
     pdl_wait();
     const int nb = d / 32;
     const long item = static_cast<long>(blockIdx.x) * GATHER_THREADS + threadIdx.x;
-    if (item >= static_cast<long>(T) * k * nb) return;
-    const int p = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
-    const int t = p / k;
-    const int e = idx[p];
-    const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
-    const int pos = offsets[e] + loc;
-    const int tile = tile_base[e] + loc / BN, rloc = loc % BN;
-    if (b == 0) {
-        row_token[pos] = t;
-        row_weight[pos] = w[p];
-        row_slot[pos] = tile * BN + rloc;
-    }
-    if (p % k == 0) {
+    if (item >= static_cast<long>(T) * nb) return;
+    const int t = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
+    {
         float4* yz = reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d + b * 32);
 #pragma unroll
         for (int i = 0; i < 8; ++i) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // the k destinations first (independent load chains in flight together), encoded while they land, then the stores
+    int pos[MAX_TOPK], tile[MAX_TOPK], rloc[MAX_TOPK];
+#pragma unroll
+    for (int j = 0; j < MAX_TOPK; ++j) {
+        if (j < k) {
+            const int p = t * k + j;
+            const int e = idx[p];
+            const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+            pos[j] = offsets[e] + loc;
+            tile[j] = tile_base[e] + loc / BN;
+            rloc[j] = loc % BN;
+        }
     }
     float v[32];
     BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
     uint4 codes[MXQ_TERMS];
     uint32_t sb[MXQ_TERMS];
     mxq_block_thread(v, codes, sb);
-    uint8_t* atoms = scale_atom_base(X, tile, b >> 2);
+    const bool split = sched[SCHED_SPLIT_GU] > 1;
 #pragma unroll
-    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-        *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos) * 16) = codes[tt];
-        atoms[sf_atom_offset(tt * X.term_rows + rloc, b & 3)] = static_cast<uint8_t>(sb[tt]);
-    }
-    if (sched[SCHED_SPLIT_GU] > 1) {
-        // the pair's nb threads zero the row together (consecutive floats per step)
-        float* g = GU + static_cast<size_t>(pos) * gu_ld;
-        for (int i = b; i < gu_ld; i += nb) g[i] = 0.f;
+    for (int j = 0; j < MAX_TOPK; ++j) {
+        if (j < k) {
+            if (b == 0) {
+                row_token[pos[j]] = t;
+                row_weight[pos[j]] = w[t * k + j];
+                row_slot[pos[j]] = tile[j] * BN + rloc[j];
+            }
+            uint8_t* atoms = scale_atom_base(X, tile[j], b >> 2);
+#pragma unroll
+            for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos[j]) * 16) =
+                    codes[tt];
+                atoms[sf_atom_offset(tt * X.term_rows + rloc[j], b & 3)] = static_cast<uint8_t>(sb[tt]);
+            }
+            if (split) {
+                // the token's nb threads zero the row together (consecutive floats per step)
+                float* g = GU + static_cast<size_t>(pos[j]) * gu_ld;
+                for (int i = b; i < gu_ld; i += nb) g[i] = 0.f;
+            }
+        }
     }
 }
 
@@ -546,50 +559,34 @@ __device__ __forceinline__ __half to_half_sat(float v) {
 
 constexpr int HENC_THREADS = 128;
 
-// Encodes H for the down GEMM: one thread per (grouped row, 32-feature block),
-// consecutive threads taking consecutive blocks of a row.  H comes from the
-// gate/up epilogue as f16 (Swish(g) * u already applied), or, when the gate/up
-// GEMM split K, from the fp32 partial sums of g and u (Swish applied here).
-// Each block is encoded as three MXFP4 terms (mxq_block_thread) into the down
-// GEMM's B operand: 16 code bytes per term, one scale byte per term into the
-// scale atom of the row's token tile.
+// Split-K finish of the gate/up GEMM (only when the schedule split K): one
+// thread per (grouped row, 32-feature block), consecutive threads taking
+// consecutive blocks of a row, applies SwiGLU to the fp32 partial sums of g
+// and u and encodes the block of H as three MXFP4 terms into the down GEMM's
+// B operand (16 code bytes per term, one scale byte per term into the scale
+// atom of the row's token tile).
 __global__ void __launch_bounds__(HENC_THREADS)
-h_encode_kernel(const __half* __restrict__ H16, const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
+h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
                 const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
     pdl_launch_dependents();
     pdl_wait();
+    if (sched[SCHED_SPLIT_GU] <= 1) return;
     const int nb = d_ff / 32;
     const long item = static_cast<long>(blockIdx.x) * HENC_THREADS + threadIdx.x;
     if (item >= static_cast<long>(sched[SCHED_ROWS]) * nb) return;
     const int row = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
-    const bool split = sched[SCHED_SPLIT_GU] > 1;
     const int slot = row_slot[row];
     const int tile = slot / BN, rloc = slot % BN;
     float v[32];
-    if (split) {
-        const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
-        const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);
+    const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
+    const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 gg = g[i], uu = u[i];
-            v[4 * i] = swish_f(gg.x) * uu.x;
-            v[4 * i + 1] = swish_f(gg.y) * uu.y;
-            v[4 * i + 2] = swish_f(gg.z) * uu.z;
-            v[4 * i + 3] = swish_f(gg.w) * uu.w;
-        }
-    } else {
-        const uint4* hp = reinterpret_cast<const uint4*>(H16 + static_cast<size_t>(row) * d_ff + 32 * b);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 q = hp[i];
-            const __half2* h2 = reinterpret_cast<const __half2*>(&q);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __half22float2(h2[j]);
-                v[8 * i + 2 * j] = f.x;
-                v[8 * i + 2 * j + 1] = f.y;
-            }
-        }
+    for (int i = 0; i < 8; ++i) {
+        const float4 gg = g[i], uu = u[i];
+        v[4 * i] = swish_f(gg.x) * uu.x;
+        v[4 * i + 1] = swish_f(gg.y) * uu.y;
+        v[4 * i + 2] = swish_f(gg.z) * uu.z;
+        v[4 * i + 3] = swish_f(gg.w) * uu.w;
     }
     uint4 codes[MXQ_TERMS];
     uint32_t sb[MXQ_TERMS];
