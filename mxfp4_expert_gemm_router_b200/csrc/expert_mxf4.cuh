@@ -90,11 +90,8 @@ struct MxgParams {
 __host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
 __host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
 constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
-__host__ __device__ constexpr bool mxg_stacked(int BN);
-// B scale atoms held per stage: one when the terms are stacked, else one per term
-__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN) { return mxg_stacked(BN) ? 512u : MXG_SFB_BYTES; }
 __host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
-    return mxg_w_stage(mode) + mxg_b_bytes(BN) + mxg_sfb_stage(BN);
+    return mxg_w_stage(mode) + mxg_b_bytes(BN) + MXG_SFB_BYTES;
 }
 // Stacked terms for small tiles: one MMA per K step reads the weight tile once
 // (separate per-term MMAs would read it three times); needs 3 * BN <= 128.
@@ -124,7 +121,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
 
     const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
     const uint32_t b_bytes = mxg_b_bytes(BN);
-    const uint32_t sf_bytes = mxg_sfb_stage(BN);   // atoms held per stage
+    const uint32_t sf_bytes = p.stacked ? 512u : MXG_SFB_BYTES;   // atoms used per stage
     const uint32_t stage_bytes = W_STAGE + b_bytes + sf_bytes;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
