@@ -88,3 +88,41 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
             m.load(str(tmp_path / "missing.so"))
     finally:
         m._lib = saved
+
+
+def _header_constants():
+    """#define and enum constants of include/moe_mxfp4.h, evaluated."""
+    src = open(os.path.join(ROOT, "include", "moe_mxfp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    consts = {}
+    for name, val in re.findall(r"#define[ \t]+(MOE_\w+)[ \t]+([^\n]+)", src):
+        consts[name] = val.strip()
+    for name, val in re.findall(r"\b(MOE_\w+)\s*=\s*(\d+)", src):
+        consts[name] = val
+    out = {}
+    for name, expr in consts.items():
+        if not re.fullmatch(r"[\w\s()<>*+u-]+", expr):
+            continue
+        unsuffix = lambda e: re.sub(r"\b(0[xX][0-9A-Fa-f]+|\d+)[uU]\b", r"\1", e)
+        expr = unsuffix(expr)
+        for _ in range(3):
+            expr = unsuffix(re.sub(r"\b(MOE_\w+)\b", lambda m: "(%s)" % consts.get(m.group(1), m.group(1)), expr))
+        out[name] = eval(expr, {"__builtins__": {}})
+    return out
+
+
+def test_binding_constants_match_the_header():
+    hdr = _header_constants()
+    names = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_NOT_QUANTIZED",
+             "MOE_ERR_TIMEOUT", "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_FLAG_TEST_SKIP_FIRST_COPY",
+             "MOE_FLAG_TOKEN_TILE_SHIFT", "MOE_FLAG_TOKEN_TILE_MASK", "MOE_NUM_STAGES",
+             "MOE_ROUTE_NOALLOC_MAX_TOKENS", "MOE_ROUTE_NOALLOC_MAX_EXPERTS"]
+    for n in names:
+        assert getattr(mx, n) == hdr[n], n
+    # the token-tile flag encodes BN / 16 in its field and rejects other sizes
+    for bn in mx.TOKEN_TILES:
+        f = mx.token_tile_flag(bn)
+        assert (f & ~mx.MOE_FLAG_TOKEN_TILE_MASK) == 0 and 16 * (f >> mx.MOE_FLAG_TOKEN_TILE_SHIFT) == bn
+    for bad in (0, 8, 24, 144):
+        with pytest.raises(ValueError):
+            mx.token_tile_flag(bad)
