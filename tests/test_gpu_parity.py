@@ -1,6 +1,6 @@
 """Parity of the CUDA layer (through the C ABI) against the CPU oracle.
 
-Bars (the benchmark spec): quantised codes and scales bit-exact; top-k
+Bars: quantised codes and scales bit-exact; top-k
 indices and per-expert counts bit-exact (inputs redrawn so no selection margin
 is below 1e-4); routing weights within 1e-6; layer output within
 max|gpu - ref| <= 2e-2 * max|ref|.
