@@ -117,9 +117,13 @@ moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router,
  *                  ties to the lower index
  *   topk_w:        device fp32 [T][k] or NULL -- softmax over the selected scores
  *   expert_counts: device int32 [E] or NULL -- rows routed to each expert
- * x and y must not overlap.  Expert matmuls run on f16 operands with fp32
- * accumulation: x converts exactly from bf16 (saturating at +-65504), the
- * SwiGLU output is rounded to f16.  Asynchronous; allocates nothing. */
+ * x and y must not overlap; x must be 16-byte aligned.  The expert matmuls
+ * are block-scaled MXFP4 x MXFP4 products with fp32 accumulation: the weights
+ * enter as quantised, x and the SwiGLU output H enter as sums of three MXFP4
+ * terms (each block of 32 values and its residuals, each term with its own
+ * E8M0 scale); H passes through f16 (|H| must stay below 65504).  The layer
+ * output matches the double-precision definition within about 3e-3 of
+ * max|y| on the 2880-wide workloads.  Asynchronous; allocates nothing. */
 moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y,
                                int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
                                cudaStream_t stream);

@@ -35,7 +35,8 @@
 // valid rows, feature tile | K split) taken round-robin from a device-built
 // list.  Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer
 // (warp-uniform loops, elect.sync issues), warps 2..9 epilogue (warp w reads
-// TMEM lanes 32*(w%4).. and every other group of 8 token columns).  Every
+// TMEM lanes 32*(w%4).. ; the quarter's two warps alternate groups of token
+// columns: 32 for the gate/up encode, 8 otherwise).  Every
 // mbarrier wait is bounded; on a timeout the CTA raises an abort flag, all
 // roles leave their loops, in-flight copies and MMAs are drained, TMEM is
 // freed and the status word reports the timeout.

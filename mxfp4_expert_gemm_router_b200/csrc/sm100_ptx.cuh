@@ -1,6 +1,7 @@
 // sm100_ptx.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the
-// expert GEMMs use: mbarriers, bulk / tensor TMA copies, tcgen05 tensor-memory
-// allocation, loads, stores, MMAs and commits.
+// layer's kernels use: mbarriers, dependent-launch control, bulk / tensor TMA
+// copies, tcgen05 tensor-memory allocation, scale-factor copies, block-scaled
+// MMAs, loads and commits, and the E2M1 conversions.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -76,8 +77,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag, int* status,
                                                   uint64_t limit_ns) {
     // One quick check, then suspend in hardware until the phase completes (or
-    // the hint expires): spinning here would take issue slots from the decoder
-    // warps that share this warp's scheduler.
+    // the hint expires): polling here takes issue slots from the warps that
+    // share this warp's scheduler (measured: every expert GEMM got slower).
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
@@ -109,16 +110,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-// 2-D tiled tensor copy global -> shared (no multicast).  c0 is the innermost
-// coordinate in elements and must be a multiple of 16 bytes' worth.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-        : "memory");
-}
 // Warp-collective forms of the copy-side instructions (one elected lane issues).
 __device__ __forceinline__ void mbar_arrive_expect_tx_warp(uint32_t bar, uint32_t bytes) {
     asm volatile(
@@ -133,14 +124,6 @@ __device__ __forceinline__ void bulk_g2s_warp(uint32_t dst, const void* src, uin
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-__device__ __forceinline__ void tma_load_2d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n\t}" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-        : "memory");
-}
 // 3-D tiled tensor copy global -> shared (no multicast); c0 is the innermost
 // coordinate and must be a multiple of 16 bytes' worth of elements.
 __device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
@@ -150,17 +133,6 @@ __device__ __forceinline__ void tma_load_3d_warp(uint32_t dst, const CUtensorMap
         "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::"r"(
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
-        : "memory");
-}
-// 4-D tiled tensor copy global -> shared (no multicast); c0 is the innermost
-// coordinate and must be a multiple of 16 bytes' worth of elements.
-__device__ __forceinline__ void tma_load_4d_warp(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                                 uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
@@ -188,31 +160,6 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (f16 or bf16 operands, fp32 accumulators).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Warp-collective forms: the whole warp executes the instruction stream (so the
-// operands stay warp-uniform) and elect.sync picks the one lane that issues.
-// Issuing from a warp-uniform, unrolled stream keeps the per-MMA issue cost to a
-// few tens of cycles; operands computed in divergent single-lane code cost
-// several times more per MMA.
-__device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
 }
 __device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
     asm volatile(
@@ -247,29 +194,8 @@ __device__ __forceinline__ void tc_cp_sf_warp(uint32_t taddr, uint64_t sdesc) {
         "l"(sdesc)
         : "memory");
 }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Store 16 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-// Store 32 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
-        "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
 // Load 8 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
 // (x8: the epilogue reads accumulators in groups of 8 token columns.)
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
@@ -278,16 +204,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
         : "r"(taddr)
         : "memory");
-}
-
-// Shared-memory matrix descriptor for a K-major operand tile written by TMA with
-// 128-byte swizzling: rows of 128 B, 8-row groups 1024 B apart (stride byte
-// offset), descriptor version 1, layout type 2 (128B swizzle).  Advancing along
-// K by 16 two-byte elements adds 32 B (2 in the >>4 address field).
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
-    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
-           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
-           (static_cast<uint64_t>(2) << 61);
 }
 
 // Shared-memory matrix descriptor, no swizzle, K-major: core matrices of 8 rows
@@ -305,34 +221,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t sf_id) { return (sf_id << 29) | (sf_id << 4); }
-
-// Instruction descriptor, kind::f16: f16 A and B (format 0), f32 accumulator
-// (format 1), both K-major, M in bits 24.., N in bits 17...
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
-    return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-// ------------------------------------------------------------------ MXFP4 decode
-// Four bytes = eight E2M1 codes (even element in the low nibble) -> four f16x2
-// words, each multiplied by the f16x2 block multiplier `mult2`.  The E2M1 to f16
-// conversion is exact; multiplying by a power of two is exact while the result
-// stays in the f16 range (the multiplier is at most 1).
-__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t mult2, uint32_t& o0, uint32_t& o1,
-                                                uint32_t& o2, uint32_t& o3) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 t0, t1, t2, t3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 t0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 t1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 t2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 t3, b3;\n\t"
-        "mul.rn.f16x2 %0, t0, %5;\n\t"
-        "mul.rn.f16x2 %1, t1, %5;\n\t"
-        "mul.rn.f16x2 %2, t2, %5;\n\t"
-        "mul.rn.f16x2 %3, t3, %5;\n\t}"
-        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
-        : "r"(w), "r"(mult2));
-}
 
 // Two floats -> one byte of two E2M1 codes (lo in the low nibble), rounded to
 // nearest with ties to the even code, saturating at +-6.
@@ -354,21 +242,6 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
         : "=r"(d)
         : "r"(byte));
     return d;
-}
-
-// f16 bit pattern of 2^rel for rel <= 0 (normal down to 2^-14, subnormal down to
-// 2^-24, zero below).
-__device__ __forceinline__ uint32_t f16_pow2_bits(int rel) {
-    rel = rel > 0 ? 0 : rel;
-    if (rel >= -14) return static_cast<uint32_t>(rel + 15) << 10;
-    if (rel >= -24) return 1u << (rel + 24);
-    return 0u;
-}
-
-// 2^e as a float for -149 <= e <= 127.
-__device__ __forceinline__ float pow2f(int e) {
-    if (e >= -126) return __int_as_float((e + 127) << 23);
-    return __int_as_float(1 << (e + 149));
 }
 
 }  // namespace moe
