@@ -591,9 +591,16 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     launch_pdl(pdl, expert_mxf4_kernel<0>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(0, BN, gp.stages), stream,
                h->tm_x[BN / 16 - 1], gp);
     h->stage_ran[2] = true;
-    // 3: split-K finish (a no-op unless the schedule split K): SwiGLU + H encoding
+    // 3: split-K finish (a no-op unless the schedule split K): SwiGLU + H encoding.
+    // The schedule splits the gate/up K only for at most gu_rows grouped rows,
+    // fewer units than SMs and a split limit above 1; the units are at least
+    // ceil(rows / BN) token tiles x F_gu feature tiles, so the launch is left
+    // out whenever that bound already rules a split out.
     mark(3);
-    if (static_cast<long>(T) * k <= h->gu_rows) {
+    const long grows = static_cast<long>(T) * k;
+    const bool may_split = grows <= h->gu_rows && ((grows + BN - 1) / BN) * h->F_gu < h->nsm &&
+                           std::min(8, std::max(1, h->KC_gu / 4)) > 1;
+    if (may_split) {
         const long items = static_cast<long>(T) * k * (f / 32);
         const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
         launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const float*>(h->GU),
