@@ -71,3 +71,25 @@ def test_roofline_bound_follows_machine_balance():
     # FP4 operands run at 4x the bf16 rate, which moves the balance point up
     r4 = bench.roofline(w, 1e-3, peaks, "gate_up_swiglu", "mxf4")
     assert r4["peak"] == 6400.0
+
+
+def test_reference_arm_prints_one_json_line():
+    """`bench.py --impl reference` (the oracle on the host cores) keeps the bench
+    line's contract: one JSON line with the metric, its value and unit, the
+    reference tag, the CPU-baseline description and a zero-copy e2e entry."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "tiny",
+                          "--steps", "1", "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "tokens/s" and rec["value"] > 0
+    assert rec["higher_is_better"] is True and rec["steps"] == 1
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["value"] == rec["value"]
+    assert rec["e2e"] == {"value": rec["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
