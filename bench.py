@@ -2,12 +2,15 @@
 """Benchmark of the MoE-MXFP4 layer (router -> top-k -> softmax -> SwiGLU experts ->
 weighted combine) on B200, through the C ABI.
 
-Default workload: the gpt-oss-20b-shaped decode layer at T=64 tokens
-(d_model = d_ff = 2880, E = 32, top-4, bf16 activations, MXFP4 experts drawn
-N(0, 0.02) and quantised by the library).  One step = one forward of the whole
-layer over one batch of T tokens.
+Default workload: the largest single-GPU configuration, the skewed-routing
+gpt-oss-20b-shaped layer at T=16384 tokens (d_model = d_ff = 2880, E = 32,
+top-4, a router bias that makes expert popularity Zipf-shaped with s = 1.2,
+bf16 activations, MXFP4 experts drawn N(0, 0.02) and quantised by the
+library).  Other workloads (tiny, dec1, dec8, dec64, pre4096, e128) with
+--config.  One step = one forward of the whole layer over one batch of T
+tokens.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config dec64] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config zipf] [--impl ours|reference]
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then K steps,
 each preceded (outside its timed span) by a 256 MB L2 flush and bracketed by
@@ -185,6 +188,14 @@ def act_tensor(cfg, a, device):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
 
 
+def uses_dependent_launches(cfg: mi.MoeConfig, T: int) -> bool:
+    """The library launches a forward's kernels with programmatic (dependent)
+    launches when it has at most 2048 grouped rows; stage events between the
+    kernels would serialise those launches, so such forwards are timed without
+    them and their stage times come from a second captured graph."""
+    return T * cfg.top_k <= 2048
+
+
 def run_ours(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -213,11 +224,22 @@ def run_ours(args, cfg, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     launches_per_step = layer.launch_count() - n0
-    # the forward never synchronises or allocates, so it can be captured once and replayed
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
-    torch.cuda.synchronize()
+
+    def capture(with_stage_events: bool):
+        # the forward never synchronises or allocates, so it can be captured once and replayed
+        layer.set_profiling(with_stage_events)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        torch.cuda.synchronize()
+        layer.set_profiling(False)
+        return g
+
+    # Stage events ride inside the timed graph (event-record nodes between the
+    # kernels) unless the forward uses dependent launches, which the nodes would
+    # serialise; then a second graph with the nodes gives the stage times.
+    stages_in_timed = not uses_dependent_launches(cfg, T)
+    graph = capture(stages_in_timed)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.fill_(1.0)
@@ -226,6 +248,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = []
     clocks = ClockSampler(local_rank)
     if rank == 0 and not args.no_clocks:
         clocks.start()
@@ -239,21 +262,25 @@ def run_ours(args, cfg, rank, world, local_rank):
             starts[i].record(stream)
             graph.replay()
             ends[i].record(stream)
+            if stages_in_timed:
+                # read between steps, outside every step's event span
+                stage_ms.append(layer.kernel_times())
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if rank == 0 and not args.no_clocks else None
     total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dev, world)
+    del graph
 
-    # per-stage breakdown: a separate pass with events between the kernels
-    stage_ms = []
-    layer.set_profiling(True)
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            flush.fill_(float(i))
-            step()
-            stage_ms.append(layer.kernel_times())
-    layer.set_profiling(False)
+    if not stages_in_timed:
+        g2 = capture(True)
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                flush.fill_(float(i))
+                g2.replay()
+                stage_ms.append(layer.kernel_times())
+        torch.cuda.synchronize()
+        del g2
 
     # end-to-end through the public host-buffer entry point
     xh = act_tensor(cfg, mi.draw_x(cfg), "cpu").pin_memory()
@@ -271,8 +298,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev, world)
     touched = int((counts.cpu().numpy() > 0).sum())
-    del graph
     return {"total_ms": total_ms, "e2e_ms": e2e_ms, "stage_ms": stage_ms,
+            "stage_timing": ("event-record nodes inside the timed graph replays" if stages_in_timed else
+                             "a second captured graph with event-record nodes, replayed after the timed region "
+                             "(the timed graph keeps its dependent launches)"),
             "launches": launches_per_step * args.steps, "clocks": clk, "touched": touched,
             "counts": counts.cpu().numpy().tolist(),
             "h2d": xh.numel() * xh.element_size(), "d2h": yh.numel() * yh.element_size()}
@@ -280,52 +309,93 @@ def run_ours(args, cfg, rank, world, local_rank):
 
 # ---------------------------------------------------------------- oracle (CPU) arm
 
-def oracle_sample(cfg: mi.MoeConfig, n_tokens: int, nthreads: int):
-    """Oracle layer on the first n_tokens of the workload (router over the same
-    tokens).  Returns (seconds, tokens).  Weight quantisation by the oracle is set-up,
-    not timed."""
-    import oracle
-    from concurrent.futures import ThreadPoolExecutor
-    x = mi.draw_x(cfg)[:n_tokens]
-    wr = mi.draw_router(cfg)
-    bias = mi.draw_bias(cfg)
-    _, idx, w, _ = oracle.router(x, wr, bias, cfg.top_k)
-    q = oracle.QuantExperts(cfg.d_model, cfg.d_ff, cfg.n_experts)
-    needed = sorted(set(np.unique(idx).tolist()))
-
-    def one(e):
-        q.set_expert(e, *mi.draw_expert(cfg, e))
-
-    with ThreadPoolExecutor(max_workers=nthreads) as ex:
-        list(ex.map(one, needed))
-    t0 = time.perf_counter()
-    _, idx, w, _ = oracle.router(x, wr, bias, cfg.top_k)
-    oracle.moe_forward(x, q, idx, w, nthreads=nthreads)
-    return time.perf_counter() - t0, n_tokens
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
-def cpu_sample_size(cfg):
-    return min(cfg.T, 64 if cfg.d_model >= 1024 else cfg.T)
+def sample_tokens(cfg: mi.MoeConfig, n: int, seed: int = 1):
+    """Seeded sample of n distinct token indices of the workload (all of them when n >= T)."""
+    if n >= cfg.T:
+        return np.arange(cfg.T)
+    return np.sort(np.random.default_rng(seed).choice(cfg.T, size=n, replace=False))
+
+
+class OracleLayer:
+    """The oracle's layer for one workload: router weights, and every expert
+    quantised by the oracle's own code (set-up, not timed)."""
+
+    def __init__(self, cfg: mi.MoeConfig, nthreads: int):
+        import oracle
+        from concurrent.futures import ThreadPoolExecutor
+        self.cfg, self.oracle = cfg, oracle
+        self.wr = mi.draw_router(cfg)
+        self.bias = mi.draw_bias(cfg)
+        self.q = oracle.QuantExperts(cfg.d_model, cfg.d_ff, cfg.n_experts)
+        with ThreadPoolExecutor(max_workers=nthreads) as ex:
+            list(ex.map(lambda e: self.q.set_expert(e, *mi.draw_expert(cfg, e)), range(cfg.n_experts)))
+        self.x = mi.draw_x(cfg)
+
+    def time_tokens(self, tokens, nthreads: int) -> float:
+        """Seconds for the oracle's router + experts over the given tokens."""
+        x = self.x[tokens]
+        t0 = time.perf_counter()
+        _, idx, w, _ = self.oracle.router(x, self.wr, self.bias, self.cfg.top_k)
+        self.oracle.moe_forward(x, self.q, idx, w, nthreads=nthreads)
+        return time.perf_counter() - t0
+
+
+# tokens per sample: all cores (about 10 s of CPU work on 16 host cores at the
+# 2880-wide shape) and one core (about 5 s)
+CPU_SAMPLE_ALL = 2048
+CPU_SAMPLE_ONE = 64
+# tokens per step of the reference arm (each step a bounded sample of the workload)
+REF_STEP_TOKENS = 64
+
+
+def cpu_baseline(cfg: mi.MoeConfig):
+    nthreads = os.cpu_count() or 1
+    ol = OracleLayer(cfg, nthreads)
+    n_all = min(cfg.T, CPU_SAMPLE_ALL if cfg.d_model >= 1024 else cfg.T)
+    n_one = min(cfg.T, CPU_SAMPLE_ONE if cfg.d_model >= 1024 else cfg.T)
+    tok_all = sample_tokens(cfg, n_all)
+    secs_all = ol.time_tokens(tok_all, nthreads)
+    tok_one = sample_tokens(cfg, n_one, seed=2)
+    secs_one = ol.time_tokens(tok_one, 1)
+    return {"value": n_all / secs_all, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": (f"seeded sample of {n_all} of the {cfg.T} tokens (router + experts in double, "
+                       f"{nthreads} threads, {secs_all:.1f} s)"),
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": n_one / secs_one, "unit": "tokens/s", "cores": 1,
+                              "sample": f"seeded sample of {n_one} tokens, {secs_one:.1f} s"}}
 
 
 def run_reference(args, cfg):
     nthreads = os.cpu_count() or 1
-    n = cpu_sample_size(cfg)
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample(cfg, min(n, 8), nthreads)
+    ol = OracleLayer(cfg, nthreads)
+    n = min(cfg.T, REF_STEP_TOKENS if cfg.d_model >= 1024 else cfg.T)
+    for i in range(args.warmup):
+        ol.time_tokens(sample_tokens(cfg, min(n, 8), seed=100 + i), nthreads)
     secs = 0.0
     toks = 0
-    for _ in range(args.steps):
-        s, t = oracle_sample(cfg, n, nthreads)
-        secs += s
-        toks += t
+    for i in range(args.steps):
+        secs += ol.time_tokens(sample_tokens(cfg, n, seed=1000 + i), nthreads)
+        toks += n
     value = toks / secs
-    sample = f"first {n} of {cfg.T} tokens per step (router + experts, double), {args.steps} steps"
+    sample = (f"per step a seeded sample of {n} of the {cfg.T} tokens (router + experts in double, "
+              f"{nthreads} threads), {args.steps} steps")
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(cfg, args), "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                             "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -383,7 +453,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="dec64", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--config", default="zipf", choices=sorted(mi.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -444,17 +514,14 @@ def main():
                       "frac_of_measured": work["layer"]["bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
                       "frac_of_8TBs": work["layer"]["bytes"] / layer_s / 8e12},
         "stage_ms": stages,
+        "stage_timing": r["stage_timing"],
         "experts_touched": r["touched"],
         "gpu_launches": r["launches"],
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "clocks": r["clocks"],
     }
     if world == 1 and not args.no_cpu_baseline:
-        nthreads = os.cpu_count() or 1
-        n = cpu_sample_size(cfg)
-        secs, toks = oracle_sample(cfg, n, nthreads)
-        out["cpu_baseline"] = {"value": toks / secs, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
-                               "sample": f"first {n} of {cfg.T} tokens, router + experts in double, one pass"}
+        out["cpu_baseline"] = cpu_baseline(cfg)
     print(json.dumps(out), flush=True)
     return 0
 

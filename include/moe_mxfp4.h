@@ -73,6 +73,9 @@ typedef struct {
 
 /* Create a handle on the current device.  Allocates every buffer the layer
  * needs for up to cfg->max_tokens tokens, so forward allocates nothing.
+ * Defines: the layer's shape -- d_model (the token width, 2880 for
+ * gpt-oss-20b, §3.1), E experts and top_k selected per token (32 and 4, §2.1),
+ * each expert a SwiGLU FFN of width d_ff (§3.2).
  * Errors: INVALID_ARG (null, non-positive sizes, bad dtype), UNSUPPORTED
  * (d_model or d_ff not a multiple of 32, E > 256, k > min(8, E),
  * d_model or d_ff above 16384), CUDA (allocation failed; nothing leaks). */
@@ -83,6 +86,9 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out);
 void moe_mxfp4_destroy(moe_mxfp4_t* h);
 
 /* Quantise all expert weights to MXFP4 and store the router.
+ * Defines: §4 Quantification MXFP4 (4.25 bits per parameter: blocks of 32 E2M1
+ * codes sharing one E8M0 scale) applied to the three matrices of each §3.2
+ * expert, and the §3.1 router weight W_router.
  *   w_gate, w_up: device fp32 [E][d_model][d_ff]   (expert e maps x -> x . W)
  *   w_down:       device fp32 [E][d_ff][d_model]
  *   w_router:     device [E][d_model] in act_dtype (scores = W_router . h)
@@ -91,44 +97,53 @@ void moe_mxfp4_destroy(moe_mxfp4_t* h);
  * down).  Block rule: scale exponent floor(log2(max|w|)) - 2 clamped to
  * [-127, 127]; elements round to the nearest E2M1 value, ties to the even
  * code, above 6 saturating, sign kept; an all-zero block gets scale 2^0.
- * Inputs must be finite.  May be called again to replace the weights. */
+ * Inputs must be finite; w_gate, w_up, w_down 4-byte aligned (else
+ * INVALID_ARG).  May be called again to replace the weights. */
 moe_status_t moe_mxfp4_quantize_weights(moe_mxfp4_t* h, const float* w_gate,
                                         const float* w_up, const float* w_down,
                                         const void* w_router, const float* router_bias,
                                         cudaStream_t stream);
 
 /* Same quantisation for one expert e (lets callers stream very large expert
- * sets through a small fp32 staging buffer).  w_gate/w_up: device fp32
- * [d_model][d_ff]; w_down: device fp32 [d_ff][d_model]. */
+ * sets through a small fp32 staging buffer).  Defines: §4 on one §3.2 expert.
+ * w_gate/w_up: device fp32 [d_model][d_ff]; w_down: device fp32
+ * [d_ff][d_model]; all 4-byte aligned. */
 moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w_gate,
                                        const float* w_up, const float* w_down,
                                        cudaStream_t stream);
 
 /* Store the router weight (device [E][d_model], act_dtype) and optional bias
- * (device fp32 [E] or NULL).  Copies; the caller may free its buffers after
- * the stream reaches this call. */
+ * (device fp32 [E] or NULL).  Defines: W_router of §3.1 (scores =
+ * W_router . h).  Copies; the caller may free its buffers after the stream
+ * reaches this call. */
 moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router,
                                   const float* router_bias, cudaStream_t stream);
 
 /* The layer for T tokens (0 <= T <= max_tokens; T == 0 launches nothing).
+ * Defines: §3.1 (scores, top-k, softmax over the selected scores), §3.2 (each
+ * selected expert's SwiGLU FFN) and §2.1 step 2 (the k outputs aggregated with
+ * their routing weights).
  *   x:             device [T][d_model], act_dtype
  *   y:             device [T][d_model], act_dtype (written, not accumulated)
  *   topk_idx:      device int32 [T][k] or NULL -- selected experts, score-descending,
  *                  ties to the lower index
  *   topk_w:        device fp32 [T][k] or NULL -- softmax over the selected scores
  *   expert_counts: device int32 [E] or NULL -- rows routed to each expert
- * x and y must not overlap; x must be 16-byte aligned.  The expert matmuls
- * are block-scaled MXFP4 x MXFP4 products with fp32 accumulation: the weights
- * enter as quantised, x and the SwiGLU output H enter as sums of three MXFP4
- * terms (each block of 32 values and its residuals, each term with its own
- * E8M0 scale); H passes through f16 (|H| must stay below 65504).  The layer
- * output matches the double-precision definition within about 3e-3 of
+ * x and y must not overlap.  x and y must be 16-byte aligned and topk_idx,
+ * topk_w, expert_counts 4-byte aligned; the device current at the call must be
+ * the handle's; otherwise INVALID_ARG is returned before anything is
+ * launched.  The expert matmuls are block-scaled MXFP4 x MXFP4 products with
+ * fp32 accumulation: the weights enter as quantised, x and the SwiGLU output
+ * H enter as sums of three MXFP4 terms (each block of 32 values and its
+ * residuals, each term with its own E8M0 scale; H is formed in fp32).  The
+ * layer output matches the double-precision definition within about 3e-3 of
  * max|y| on the 2880-wide workloads.  Asynchronous; allocates nothing. */
 moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y,
                                int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
                                cudaStream_t stream);
 
-/* forward with HOST buffers: copies x (host [T][d_model], act_dtype) in,
+/* forward with HOST buffers (the same layer as moe_mxfp4_forward, §3.1, §3.2,
+ * §2.1): copies x (host [T][d_model], act_dtype) in,
  * runs the layer, copies y (host [T][d_model]) and, if non-NULL, topk_idx
  * (host int32 [T][k]) and topk_w (host fp32 [T][k]) out, and synchronises
  * the stream before returning.  Uses handle-owned device staging buffers. */
@@ -136,7 +151,9 @@ moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t 
                                     void* y_host, int32_t* topk_idx_host,
                                     float* topk_w_host, cudaStream_t stream);
 
-/* Export the quantised weights of one matrix in the canonical MXFP4 layout:
+/* Export the quantised weights of one matrix in the canonical MXFP4 layout
+ * (§4: E2M1 codes in blocks of 32 along the contraction axis, one E8M0 scale
+ * per block); codes must be 16-byte aligned:
  * which = 0 gate, 1 up, 2 down.  For contraction length K and N outputs
  * (gate/up: K = d_model, N = d_ff; down: K = d_ff, N = d_model):
  *   codes:  device uint8 [E][N][K/2]   element k of row n in byte k/2,
@@ -145,7 +162,8 @@ moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t 
 moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* h, int32_t which, uint8_t* codes,
                                       uint8_t* scales, cudaStream_t stream);
 
-/* Grouping produced by the last forward (for inspection and tests):
+/* Grouping produced by the last forward (for inspection and tests; the
+ * tokens each §2.1 expert received):
  *   offsets:    device int32 [E+1]  rows of expert e are [offsets[e], offsets[e+1])
  *   row_token:  device int32 [T*k]  token of each grouped row (or NULL)
  *   row_weight: device fp32  [T*k]  routing weight of each grouped row (or NULL)
@@ -161,7 +179,9 @@ moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h);
 const char* moe_mxfp4_status_string(moe_status_t s);
 
 /* Per-stage timing of later forwards (CUDA events on the forward's stream).
- * enable = 0 turns it off. */
+ * enable = 0 turns it off.  A forward captured into a CUDA graph while
+ * profiling is on records its stage events as event-record nodes of the
+ * graph, so moe_mxfp4_kernel_times then reports the last replay. */
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */
@@ -177,10 +197,13 @@ const char* moe_mxfp4_stage_name(int32_t stage);
 /* Number of kernels this handle has launched since creation. */
 uint64_t moe_mxfp4_launch_count(const moe_mxfp4_t* h);
 
-/* Parameters of one expert: 3 * d_model * d_ff (three matrices, §3.2). */
+/* Parameters of one expert: 3 * d_model * d_ff (three matrices, §3.2; the
+ * page "OpenAI lance gpt-oss-20b" gives 3,145,728 for the GLU variant at
+ * width 1024). */
 int64_t moe_mxfp4_expert_param_count(const moe_mxfp4_config_t* cfg);
 
-/* MXFP4 bytes of one expert: codes + scales = 17/32 byte per parameter. */
+/* MXFP4 bytes of one expert: codes + scales = 17/32 byte per parameter
+ * (4.25 bits, §4). */
 int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg);
 
 /* Routing without any device allocation.  No counterpart on the pages: this
@@ -200,10 +223,13 @@ int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg);
  *   expert_counts: int32 [E] or NULL
  * Limits: 1 <= T <= MOE_ROUTE_NOALLOC_MAX_TOKENS, E <= MOE_ROUTE_NOALLOC_MAX_EXPERTS,
  * 1 <= top_k <= min(8, E), d_model a positive multiple of 32 up to 16384;
- * anything larger returns MOE_ERR_UNSUPPORTED (nothing is launched).  The
- * first call on a device looks up the array's device address (with that
- * device current) and sets the kernel's shared-memory limit: make that first
- * call before any stream capture.  Every call resets the counters it needs and
+ * anything larger returns MOE_ERR_UNSUPPORTED (nothing is launched).  x and
+ * w_router must be 16-byte aligned, router_bias and the outputs 4-byte
+ * aligned (else MOE_ERR_INVALID_ARG, checked before the device is touched).
+ * The first call on a device looks up the array's device address (with that
+ * device current) and sets the router kernel's shared-memory limit to the
+ * value layer handles use (never lower): make that first call before any
+ * stream capture.  Every call resets the counters it needs and
  * otherwise reuses the array, so calls that overlap on the GPU (different
  * streams without ordering, or several host threads) race on it.
  * Asynchronous on `stream`. */

@@ -23,7 +23,7 @@
 //   MODE 0 (gate/up): per stage gate and up chunks (17408 bytes), two
 //     accumulators for the same 128 features; epilogue: H = Swish(g) * u for
 //     32 tokens x 32 features per warp goes through a small shared-memory tile
-//     (f16, transposed) so that each lane then holds one token's 32-feature
+//     (fp32, transposed) so that each lane then holds one token's 32-feature
 //     block and encodes it as three MXFP4 terms straight into the down GEMM's
 //     B operand; with a K split, fp32 partials are added into GU instead (and
 //     h_encode_kernel encodes H).
@@ -91,21 +91,24 @@ struct MxgParams {
 __host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
 __host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
 constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
-__host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
-    return mxg_w_stage(mode) + mxg_b_bytes(BN) + MXG_SFB_BYTES;
-}
 // Stacked terms for small tiles: one MMA per K step reads the weight tile once
 // (separate per-term MMAs would read it three times); needs 3 * BN <= 128.
 __host__ __device__ constexpr bool mxg_stacked(int BN) { return MXQ_TERMS * BN <= 128; }
+// B scale atoms per stage: one (all terms' rows in one atom) when stacked, else one per term.
+__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN) { return mxg_stacked(BN) ? 512u : MXG_SFB_BYTES; }
+__host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
+    return mxg_w_stage(mode) + mxg_b_bytes(BN) + mxg_sfb_stage(BN);
+}
 __host__ __device__ constexpr int mxg_mat_cols(int BN) {
     return (((mxg_stacked(BN) ? MXQ_TERMS : 1) * BN + 31) / 32) * 32;
 }
 __host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
 __host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
-// MODE 0 epilogue tiles: per epilogue warp 32 tokens x 32 features of f16, rows
-// padded to 33 so both the row writes and the column reads are conflict-free.
+// MODE 0 epilogue tiles: per epilogue warp 32 tokens x 32 features of fp32 H,
+// rows padded to 33 so both the row writes and the column reads are
+// conflict-free.  fp32 keeps H's full range and precision into the encoder.
 constexpr int MXG_HT_STRIDE = 33;
-constexpr uint32_t MXG_HT_BYTES = MXG_EPI_WARPS * 32 * MXG_HT_STRIDE * 2;
+constexpr uint32_t MXG_HT_BYTES = MXG_EPI_WARPS * 32 * MXG_HT_STRIDE * 4;
 __host__ __device__ constexpr uint32_t mxg_extra_smem(int mode) { return mode == 0 ? MXG_HT_BYTES : 0u; }
 __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
     const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN) +
@@ -122,8 +125,8 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
 
     const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
     const uint32_t b_bytes = mxg_b_bytes(BN);
-    const uint32_t sf_bytes = p.stacked ? 512u : MXG_SFB_BYTES;   // atoms used per stage
-    const uint32_t stage_bytes = W_STAGE + b_bytes + sf_bytes;
+    const uint32_t sf_bytes = mxg_sfb_stage(BN);                   // atoms used per stage
+    const uint32_t stage_bytes = mxg_stage_bytes(MODE, BN);
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t bar0 = base + S * stage_bytes;                 // barriers (8-byte aligned)
@@ -136,7 +139,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
     uint8_t* ctl = smem_raw + (drain_bar + 8u - raw);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
-    __half* htile_all = reinterpret_cast<__half*>(ctl + 64);   // MODE 0 epilogue tiles
+    float* htile_all = reinterpret_cast<float*>(ctl + 64);     // MODE 0 epilogue tiles
     const int mat_cols = mxg_mat_cols(BN);
     const int acc_cols = (MODE == 0 ? 2 : 1) * mat_cols;
     const int NACC = p.nacc;
@@ -341,7 +344,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 };
                 if (MODE == 0 && nsplit == 1) {
                     // groups of 32 tokens alternate between the quarter's two warps
-                    __half* ht = htile_all + (warp - 2) * 32 * MXG_HT_STRIDE;
+                    float* ht = htile_all + (warp - 2) * 32 * MXG_HT_STRIDE;
                     const int blk = 4 * ft + q;
                     uint8_t* atoms = scale_atom_base(p.Hd, tile, ft);
                     for (int g0 = 32 * hh; g0 < nvalid; g0 += 64) {
@@ -350,14 +353,14 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                             load8(g0 + s8, gs, us);
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
-                                ht[(s8 + j) * MXG_HT_STRIDE + lane] = to_half_sat(swish_f(gs[j]) * us[j]);
+                                ht[(s8 + j) * MXG_HT_STRIDE + lane] = swish_f(gs[j]) * us[j];
                         }
                         __syncwarp();
                         const int r = g0 + lane;   // this lane's token: one 32-feature block of H
                         if (r < nvalid) {
                             float hv[32];
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) hv[c] = __half2float(ht[lane * MXG_HT_STRIDE + c]);
+                            for (int c = 0; c < 32; ++c) hv[c] = ht[lane * MXG_HT_STRIDE + c];
                             uint4 codes[MXQ_TERMS];
                             uint32_t sb[MXQ_TERMS];
                             mxq_block_thread(hv, codes, sb);

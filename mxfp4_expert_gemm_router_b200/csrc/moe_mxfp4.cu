@@ -111,7 +111,15 @@ struct moe_mxfp4 {
     uint64_t launches = 0;
 };
 
-static bool g_attrs_set = false;
+// Kernel attributes belong to the current device's context, so they are set
+// once per device, under a lock (create and the no-allocation router both call
+// this).  The router's shared-memory limit is always the one for the largest
+// expert count, so no caller ever lowers it below what another layer needs.
+constexpr int MOE_MAX_DEVICES = 64;
+static std::mutex g_attr_mutex;
+static bool g_attrs_set[MOE_MAX_DEVICES] = {};
+
+static bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Launch with programmatic stream serialization when `pdl` is set: the kernel
 // may start while the previous kernel in the stream finishes (it runs its
@@ -216,6 +224,30 @@ static cudaError_t set_router_smem(int bytes) {
     if ((e = cudaFuncSetAttribute(router_kernel<TA, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
     if ((e = cudaFuncSetAttribute(router_kernel<TA, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
     return cudaFuncSetAttribute(router_kernel<TA, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// The handle's buffers live on the device that was current at create: calls
+// that launch work require it to be current again.
+static moe_status_t check_device(const moe_mxfp4* h) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
+    return cur == h->dev ? MOE_OK : MOE_ERR_INVALID_ARG;
+}
+
+static cudaError_t ensure_kernel_attrs(int dev) {
+    if (dev < 0 || dev >= MOE_MAX_DEVICES) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    if (g_attrs_set[dev]) return cudaSuccess;
+    const int rsm = static_cast<int>(router_smem_bytes(MAX_EXPERTS));
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
+        return e;
+    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
+        return e;
+    if ((e = set_router_smem<float>(rsm))) return e;
+    if ((e = set_router_smem<__nv_bfloat16>(rsm))) return e;
+    g_attrs_set[dev] = true;
+    return cudaSuccess;
 }
 
 static int stages_for(int mode, int BN) {
@@ -354,16 +386,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         cudaMemset(h->bias, 0, sizeof(float) * E) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return fail(MOE_ERR_CUDA);
 
-    if (!g_attrs_set) {
-        if (cudaFuncSetAttribute(expert_mxf4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(expert_mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-                cudaSuccess ||
-            set_router_smem<float>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess ||
-            set_router_smem<__nv_bfloat16>(static_cast<int>(router_smem_bytes(MAX_EXPERTS))) != cudaSuccess)
-            return fail(MOE_ERR_CUDA);
-        g_attrs_set = true;
-    }
+    if (ensure_kernel_attrs(h->dev) != cudaSuccess) return fail(MOE_ERR_CUDA);
     for (auto& e : h->ev)
         if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
     *out = h;
@@ -410,6 +433,7 @@ moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w
                                        const float* w_down, cudaStream_t stream) {
     if (!h || !w_gate || !w_up || !w_down) return MOE_ERR_INVALID_ARG;
     if (e < 0 || e >= h->cfg.n_experts) return MOE_ERR_INVALID_ARG;
+    if (!aligned_to(w_gate, 4) || !aligned_to(w_up, 4) || !aligned_to(w_down, 4)) return MOE_ERR_INVALID_ARG;
     moe_status_t st;
     if ((st = quantize_matrix(h, 0, w_gate, e, 1, stream)) != MOE_OK) return st;
     if ((st = quantize_matrix(h, 1, w_up, e, 1, stream)) != MOE_OK) return st;
@@ -426,6 +450,7 @@ moe_status_t moe_mxfp4_quantize_weights(moe_mxfp4_t* h, const float* w_gate, con
                                         const float* w_down, const void* w_router, const float* router_bias,
                                         cudaStream_t stream) {
     if (!h || !w_gate || !w_up || !w_down || !w_router) return MOE_ERR_INVALID_ARG;
+    if (!aligned_to(w_gate, 4) || !aligned_to(w_up, 4) || !aligned_to(w_down, 4)) return MOE_ERR_INVALID_ARG;
     const int E = h->cfg.n_experts;
     moe_status_t st;
     if ((st = quantize_matrix(h, 0, w_gate, 0, E, stream)) != MOE_OK) return st;
@@ -439,6 +464,7 @@ moe_status_t moe_mxfp4_quantize_weights(moe_mxfp4_t* h, const float* w_gate, con
 moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* hc, int32_t which, uint8_t* codes, uint8_t* scales,
                                       cudaStream_t stream) {
     if (!hc || !codes || !scales || which < 0 || which > 2) return MOE_ERR_INVALID_ARG;
+    if (!aligned_to(codes, 16)) return MOE_ERR_INVALID_ARG;   // codes are written 16 bytes at a time
     moe_mxfp4* h = const_cast<moe_mxfp4*>(hc);
     TiledMatrix M = tiled(h, which);
     const dim3 grid((M.N + 127) / 128, M.K / 32, h->cfg.n_experts);
@@ -483,7 +509,12 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     if (T < 0) return MOE_ERR_INVALID_ARG;
     if (T > c.max_tokens) return MOE_ERR_UNSUPPORTED;
     if (T > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+    // the kernels read x and write y 16 bytes at a time and the routing outputs 4
+    if (!aligned_to(x, 16) || !aligned_to(y, 16) || !aligned_to(topk_idx, 4) || !aligned_to(topk_w, 4) ||
+        !aligned_to(expert_counts, 4))
+        return MOE_ERR_INVALID_ARG;
     if (!h->router_set || h->experts_quantized < c.n_experts) return MOE_ERR_NOT_QUANTIZED;
+    if (moe_status_t ds = check_device(h)) return ds;
     h->last_stream = stream;
     if (T == 0) return MOE_OK;
     const int E = c.n_experts, d = c.d_model, f = c.d_ff, k = c.top_k;
@@ -497,8 +528,16 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     float* acc = bf16 ? h->yacc : static_cast<float*>(y);
     const bool prof = h->prof;
     for (int i = 0; i < MOE_NUM_STAGES; ++i) h->stage_ran[i] = false;
+    // While the stream is being captured into a CUDA graph, the stage events
+    // become event-record nodes of the graph (recorded at every replay).
+    unsigned ev_flags = cudaEventRecordDefault;
+    if (prof) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+            ev_flags = cudaEventRecordExternal;
+    }
     auto mark = [&](int i) {
-        if (prof) cudaEventRecord(h->ev[i], stream);
+        if (prof) cudaEventRecordWithFlags(h->ev[i], stream, ev_flags);
     };
 
     // 0: router + top-k + softmax + schedule
@@ -646,6 +685,7 @@ moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t 
     if (T < 0) return MOE_ERR_INVALID_ARG;
     if (T > c.max_tokens) return MOE_ERR_UNSUPPORTED;
     if (T > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
+    if (moe_status_t ds = check_device(h)) return ds;
     if (T == 0) return MOE_OK;
     const size_t act = static_cast<size_t>(T) * c.d_model * h->act_bytes;
     MOE_TRY(cudaMemcpyAsync(h->x_stage, x_host, act, cudaMemcpyHostToDevice, stream));
@@ -745,7 +785,7 @@ struct NoallocDevice {
     unsigned char* scratch = nullptr;  // device address of g_route_scratch on this device
     int nsm = 0;
 };
-constexpr int NOALLOC_MAX_DEVICES = 64;
+constexpr int NOALLOC_MAX_DEVICES = MOE_MAX_DEVICES;
 NoallocDevice g_noalloc[NOALLOC_MAX_DEVICES];
 std::mutex g_noalloc_mutex;
 
@@ -758,9 +798,8 @@ moe_status_t noalloc_setup(int dev, NoallocDevice** out) {
         if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
         int nsm = 0;
         if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
-        const int smem = static_cast<int>(router_smem_bytes(MOE_ROUTE_NOALLOC_MAX_EXPERTS));
-        if (set_router_smem<float>(smem) != cudaSuccess || set_router_smem<__nv_bfloat16>(smem) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        // the same per-device attributes as a layer's (never a lower router limit)
+        if (ensure_kernel_attrs(dev) != cudaSuccess) return MOE_ERR_CUDA;
         nd.scratch = static_cast<unsigned char*>(ptr);
         nd.nsm = nsm;
         nd.ready = true;
@@ -781,6 +820,10 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     if (T > MOE_ROUTE_NOALLOC_MAX_TOKENS || n_experts > MOE_ROUTE_NOALLOC_MAX_EXPERTS ||
         top_k > std::min(MAX_TOPK, static_cast<int>(n_experts)) || d_model % 32 || d_model > 16384)
         return MOE_ERR_UNSUPPORTED;
+    // the router reads x and w_router 16 bytes at a time
+    if (!aligned_to(x, 16) || !aligned_to(w_router, 16) || !aligned_to(router_bias, 4) || !aligned_to(topk_idx, 4) ||
+        !aligned_to(topk_w, 4) || !aligned_to(expert_counts, 4))
+        return MOE_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     NoallocDevice* nd = nullptr;

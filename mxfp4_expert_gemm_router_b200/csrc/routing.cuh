@@ -552,11 +552,6 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
 
 __device__ __forceinline__ float swish_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-__device__ __forceinline__ __half to_half_sat(float v) {
-    v = fminf(fmaxf(v, -65504.f), 65504.f);
-    return __float2half_rn(v);
-}
-
 constexpr int HENC_THREADS = 128;
 
 // Split-K finish of the gate/up GEMM (only when the schedule split K): one

@@ -123,14 +123,60 @@ def sample_tokens(idx: np.ndarray, counts_ref: np.ndarray, n: int, seed: int = 0
     return np.array(sorted(picks))
 
 
-def check_layer(cfg, x, wr, bias, y, idx, w, counts, ox: OracleExperts, n_sample=16):
-    """Router bit-exact over all tokens; layer output on a token sample vs the oracle."""
+def library_token_tile(T: int, k: int, E: int) -> int:
+    """Token rows per expert-GEMM tile as the library picks them by default:
+    about three times the mean rows per expert, rounded up to 16, within
+    [16, 128].  Used only to choose which rows to check (tile boundaries)."""
+    per_expert = -(-T * k // E)
+    want = min(T, max(1, 3 * per_expert))
+    return max(16, min(128, -(-want // 16) * 16))
+
+
+def tile_boundary_tokens(idx: np.ndarray, counts_ref: np.ndarray, bn: int, max_full_experts=None, seed=0):
+    """Tokens whose grouped rows lie in the tiles most likely to go wrong:
+    every row of the first and the last token tile of the most-loaded expert,
+    and every row of the last (ragged) tile of every expert.  The rows of an
+    expert are its tokens in ascending order (a token picks an expert at most
+    once), so tile m of expert e holds its tokens [m*bn, (m+1)*bn).  With
+    max_full_experts set, only that many seeded experts (plus the most- and
+    least-loaded) have their whole last tile checked; the others contribute
+    that tile's first and last rows."""
+    E = counts_ref.shape[0]
+    picks = set()
+    loaded = np.nonzero(counts_ref)[0]
+    if loaded.size == 0:
+        return np.array([], np.int64)
+    most = int(loaded[np.argmax(counts_ref[loaded])])
+    least = int(loaded[np.argmin(counts_ref[loaded])])
+    full = set(range(E))
+    if max_full_experts is not None and max_full_experts < loaded.size:
+        rng = np.random.default_rng(seed)
+        full = set(rng.choice(loaded, size=max_full_experts, replace=False).tolist()) | {most, least}
+    for e in loaded.tolist():
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        n = toks.size
+        last0 = ((n - 1) // bn) * bn
+        last = toks[last0:]
+        if e in full:
+            picks.update(last.tolist())
+        else:
+            picks.update([int(last[0]), int(last[-1])])
+        if e == most:
+            picks.update(toks[:bn].tolist())
+    return np.array(sorted(picks), np.int64)
+
+
+def check_layer(cfg, x, wr, bias, y, idx, w, counts, ox: OracleExperts, n_sample=16, extra_tokens=None):
+    """Router bit-exact over all tokens; layer output vs the oracle on a token
+    sample (plus `extra_tokens`, e.g. tile-boundary rows)."""
     _, idx_ref, w_ref, counts_ref = oracle.router(x, wr, bias, cfg.top_k)
     np.testing.assert_array_equal(idx, idx_ref)
     np.testing.assert_array_equal(counts, counts_ref)
     w_err = np.abs(w - w_ref).max()
     assert w_err <= W_ABS_TOL, ("routing weight error", w_err)
     tok = sample_tokens(idx_ref, counts_ref, n_sample)
+    if extra_tokens is not None and len(extra_tokens):
+        tok = np.union1d(tok, np.asarray(extra_tokens, np.int64))
     q = ox.ensure(np.unique(idx_ref[tok]))
     y_ref = oracle.moe_forward(x, q, idx_ref, w_ref, tokens=tok)
     err = np.abs(y[tok] - y_ref).max()

@@ -126,3 +126,27 @@ def test_binding_constants_match_the_header():
     for bad in (0, 8, 24, 144):
         with pytest.raises(ValueError):
             mx.token_tile_flag(bad)
+
+
+def test_route_noalloc_rejects_bad_arguments_before_touching_the_device(lib):
+    """Sizes beyond the static array and misaligned pointers are refused on the
+    host (the pointers here are never dereferenced)."""
+    F32 = mx.MOE_DTYPE_F32
+    ok = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4096 + 8)      # 8 bytes past a 16-byte boundary
+    odd4 = ctypes.c_void_p(4096 + 2)     # not even 4-byte aligned
+    f = lib.moe_mxfp4_route_noalloc
+    assert f(ok, ok, None, mx.MOE_ROUTE_NOALLOC_MAX_TOKENS + 1, 64, 8, 2, F32, ok, ok, None, None) == \
+        mx.MOE_ERR_UNSUPPORTED
+    assert f(ok, ok, None, 4, 64, mx.MOE_ROUTE_NOALLOC_MAX_EXPERTS + 1, 2, F32, ok, ok, None, None) == \
+        mx.MOE_ERR_UNSUPPORTED
+    assert f(ok, ok, None, 4, 60, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_UNSUPPORTED
+    assert f(ok, ok, None, 4, 64, 8, 9, F32, ok, ok, None, None) == mx.MOE_ERR_UNSUPPORTED
+    assert f(odd, ok, None, 4, 64, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, odd, None, 4, 64, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, ok, odd4, 4, 64, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, ok, None, 4, 64, 8, 2, F32, odd4, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, ok, None, 4, 64, 8, 2, F32, ok, odd4, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, ok, None, 4, 64, 8, 2, F32, ok, ok, odd4, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(None, ok, None, 4, 64, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+    assert f(ok, ok, None, 4, 64, 8, 2, 7, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG

@@ -10,7 +10,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from _layer import GpuLayer, OracleExperts, Y_REL_TOL, act_tensor, check_layer, filtered_x, to_f64
+from _layer import (GpuLayer, OracleExperts, W_ABS_TOL, Y_REL_TOL, act_tensor, check_layer, filtered_x,
+                    library_token_tile, tile_boundary_tokens, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -109,7 +110,12 @@ def test_20b_shaped_layer_parity(layer20b, ox20b, name):
     layer20b.set_router(wr, bias)
     x = filtered_x(cfg, wr, bias)
     y, idx, w, counts = layer20b.forward(x)
-    check_layer(cfg, x, wr, bias, y, idx, w, counts, ox20b, n_sample=16)
+    extra = None
+    if cfg.T >= 1024:
+        # every row of the most-loaded expert's first and last token tiles and of
+        # every expert's last (ragged) tile
+        extra = tile_boundary_tokens(idx, counts, library_token_tile(cfg.T, cfg.top_k, cfg.n_experts))
+    check_layer(cfg, x, wr, bias, y, idx, w, counts, ox20b, n_sample=16, extra_tokens=extra)
     if name == "zipf":
         # skewed routing: the most popular expert takes far more than the mean share
         assert counts.max() > 3 * counts.mean()
@@ -121,7 +127,11 @@ def test_e128_layer_parity():
     ox = OracleExperts(cfg)
     x = filtered_x(cfg, L.wr, L.bias)
     y, idx, w, counts = L.forward(x)
-    check_layer(cfg, x, L.wr, L.bias, y, idx, w, counts, ox, n_sample=12)
+    # 128 experts: the whole last tile of 16 seeded experts (and of the most and
+    # least loaded), the first and last rows of every other expert's last tile
+    extra = tile_boundary_tokens(idx, counts, library_token_tile(cfg.T, cfg.top_k, cfg.n_experts),
+                                 max_full_experts=16)
+    check_layer(cfg, x, L.wr, L.bias, y, idx, w, counts, ox, n_sample=12, extra_tokens=extra)
 
 
 @pytest.mark.parametrize("d,f_", [(192, 320), (96, 160)])
@@ -265,3 +275,86 @@ def test_pipeline_timeout_is_reported_not_hung():
     xf = filtered_x(cfg, L2.wr, L2.bias)
     yy, idx, w, counts = L2.forward(xf)
     check_layer(cfg, xf, L2.wr, L2.bias, yy, idx, w, counts, OracleExperts(cfg), n_sample=cfg.T)
+
+
+def test_scaled_activations_stay_within_tolerance(layer20b, ox20b):
+    """x scaled by 16 (exact in bf16): H grows about 256-fold; it is formed and
+    encoded in fp32 (no f16 range limit), so the layer still meets the bar."""
+    cfg = CFG20
+    wr = mi.draw_router(cfg)
+    layer20b.set_router(wr, None)
+    # scaling multiplies every selection margin by 16, so the filter still holds
+    x = filtered_x(cfg, wr, None) * np.float32(16.0)
+    y, idx, w, counts = layer20b.forward(x)
+    check_layer(cfg, x, wr, None, y, idx, w, counts, ox20b, n_sample=16)
+
+
+def test_quantize_weights_entry_point():
+    """The whole-layer loader (all experts, the router and its bias in one
+    call): exported codes and scales byte-for-byte equal to the oracle's
+    quantiser for every expert, and the layer output matches the oracle
+    (the Zipf-biased router at 256 tokens)."""
+    import torch
+    import mxfp4_expert_gemm_router_b200 as mx
+    for cfg in (mi.CONFIGS["tiny"], mi.CONFIGS["zipf"].with_T(256)):
+        E, d, f = cfg.n_experts, cfg.d_model, cfg.d_ff
+        layer = mx.MoeMxfp4(d, f, E, cfg.top_k, cfg.T, cfg.act_dtype)
+        wg = torch.empty((E, d, f), dtype=torch.float32, device="cuda")
+        wu = torch.empty((E, d, f), dtype=torch.float32, device="cuda")
+        wd = torch.empty((E, f, d), dtype=torch.float32, device="cuda")
+        for e in range(E):
+            g_, u_, d_ = mi.draw_expert(cfg, e)
+            wg[e].copy_(torch.from_numpy(g_))
+            wu[e].copy_(torch.from_numpy(u_))
+            wd[e].copy_(torch.from_numpy(d_))
+        wr = mi.draw_router(cfg)
+        bias = mi.draw_bias(cfg)
+        b_t = None if bias is None else torch.from_numpy(bias).cuda()
+        layer.quantize_weights(wg, wu, wd, act_tensor(cfg, wr), b_t)
+        torch.cuda.synchronize()
+        del wg, wu, wd
+        ox = OracleExperts(cfg)
+        q = ox.ensure(range(E))
+        for which, (rc, rs) in enumerate([(q.g_codes, q.g_scales), (q.u_codes, q.u_scales),
+                                          (q.d_codes, q.d_scales)]):
+            c, sc = _export(layer, cfg, which)
+            np.testing.assert_array_equal(c, rc)
+            np.testing.assert_array_equal(sc, rs)
+        x = filtered_x(cfg, wr, bias)
+        xt = act_tensor(cfg, x)
+        y = torch.empty_like(xt)
+        idx = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32, device="cuda")
+        counts = torch.empty((E,), dtype=torch.int32, device="cuda")
+        layer.forward(xt, y, idx, w, counts)
+        torch.cuda.synchronize()
+        assert layer.status() == mx.MOE_OK
+        check_layer(cfg, x, wr, bias, to_f64(y), idx.cpu().numpy(), w.cpu().numpy().astype(np.float64),
+                    counts.cpu().numpy(), ox, n_sample=cfg.T)
+        layer.close()
+
+
+def test_misaligned_pointers_are_rejected_before_any_launch(layer20b):
+    """x and y are read and written 16 bytes at a time: a pointer off that
+    boundary returns INVALID_ARG and launches nothing (no misaligned access)."""
+    import torch
+    import mxfp4_expert_gemm_router_b200 as mx
+    T, d = 8, CFG20.d_model
+    L = mx.load()
+    buf = torch.zeros((T + 1) * d, dtype=torch.bfloat16, device="cuda")
+    good = buf.data_ptr()
+    off = good + 2          # one bf16 element past a 16-byte boundary
+    y = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(T * CFG20.top_k + 1, dtype=torch.int32, device="cuda")
+    n0 = layer20b.layer.launch_count()
+    h = layer20b.layer.h
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.moe_mxfp4_forward(h, off, T, y.data_ptr(), None, None, None, s) == mx.MOE_ERR_INVALID_ARG
+    assert L.moe_mxfp4_forward(h, good, T, off, None, None, None, s) == mx.MOE_ERR_INVALID_ARG
+    assert L.moe_mxfp4_forward(h, good, T, y.data_ptr(), idx.data_ptr() + 2, None, None,
+                               s) == mx.MOE_ERR_INVALID_ARG
+    assert layer20b.layer.launch_count() == n0
+    # the handle still works
+    assert L.moe_mxfp4_forward(h, good, T, y.data_ptr(), None, None, None, s) == mx.MOE_OK
+    torch.cuda.synchronize()
+    assert layer20b.layer.status() == mx.MOE_OK
