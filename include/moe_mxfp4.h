@@ -181,7 +181,9 @@ const char* moe_mxfp4_status_string(moe_status_t s);
 /* Per-stage timing of later forwards (CUDA events on the forward's stream).
  * enable = 0 turns it off.  A forward captured into a CUDA graph while
  * profiling is on records its stage events as event-record nodes of the
- * graph, so moe_mxfp4_kernel_times then reports the last replay. */
+ * graph, so moe_mxfp4_kernel_times then reports the last replay (also after
+ * profiling is turned off again; a forward run eagerly with profiling off
+ * ends the record). */
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */

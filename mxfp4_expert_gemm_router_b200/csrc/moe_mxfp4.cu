@@ -734,7 +734,9 @@ moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h) {
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable) {
     if (!h) return MOE_ERR_INVALID_ARG;
     h->prof = enable != 0;
-    h->prof_valid = false;
+    // turning profiling on starts a new record; turning it off keeps the last
+    // one readable (e.g. the stage events of a graph captured while it was on)
+    if (h->prof) h->prof_valid = false;
     return MOE_OK;
 }
 
