@@ -41,6 +41,11 @@ STREAM_BIAS = 3
 STREAM_WG = 4
 STREAM_WU = 5
 STREAM_WD = 6
+STREAM_GAMMA = 7
+
+# RMSNorm epsilon of the optional pre-norm (the pages give none; a small
+# positive constant keeps an all-zero token finite)
+NORM_EPS = 1e-5
 
 WEIGHT_STD = 0.02
 MARGIN = 1e-4
@@ -132,6 +137,12 @@ def draw_bias(cfg: MoeConfig) -> Optional[np.ndarray]:
     p = ranks.astype(np.float64) ** (-cfg.zipf_s)
     p /= p.sum()
     return np.log(p).astype(np.float32)
+
+
+def draw_gamma(cfg: MoeConfig) -> np.ndarray:
+    """Gain of the optional RMSNorm pre-norm [d_model], 1 + 0.1 N(0,1), float32."""
+    g = _rng(cfg.seed, STREAM_GAMMA).standard_normal(cfg.d_model, dtype=np.float32)
+    return (np.float32(1.0) + np.float32(0.1) * g).astype(np.float32)
 
 
 def draw_expert(cfg: MoeConfig, e: int):

@@ -7,7 +7,8 @@ gcc by oracle/build.py.
 
 Sources (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card"):
 §3.1 Le Routeur, §3.2 Les Experts, §2.1 (weighted aggregation), §4
-Quantification MXFP4.  Parity pins for every function are in
+Quantification MXFP4; page "GPT-OSS vs Qwen3 : comparaison détaillée",
+Adoption de RMSNorm (the optional pre-norm of the block).  Parity pins for every function are in
 tests/test_oracle_pins.py.
 """
 from __future__ import annotations
@@ -43,6 +44,7 @@ def lib():
         L.oracle_expert.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
         L.oracle_moe_forward.argtypes = [vp, i64, i64, i64, i32, vp, vp,
                                          vp, vp, vp, vp, vp, vp, vp, i64, vp, i32]
+        L.oracle_rmsnorm.argtypes = [vp, i64, i64, vp, d, vp]
         _lib = L
     return _lib
 
@@ -174,3 +176,28 @@ def moe_forward(x: np.ndarray, q: QuantExperts, idx: np.ndarray, w: np.ndarray,
                              _ptr(q.u_scales), _ptr(q.d_codes), _ptr(q.d_scales),
                              _ptr(tok), n, _ptr(y), int(max(1, min(nthreads, max(n, 1)))))
     return y
+
+
+def rmsnorm(x: np.ndarray, gamma: Optional[np.ndarray], eps: float) -> np.ndarray:
+    """RMSNorm of each row of x [T, d] in double: x / sqrt(mean(x^2) + eps) * gamma."""
+    x = _c(x, np.float64)
+    T, d = x.shape
+    g = None if gamma is None else _c(gamma, np.float64)
+    out = np.zeros((T, d), np.float64)
+    lib().oracle_rmsnorm(_ptr(x), T, d, _ptr(g), float(eps), _ptr(out))
+    return out
+
+
+def block_forward(x: np.ndarray, q: QuantExperts, wr: np.ndarray, bias: Optional[np.ndarray], k: int,
+                  gamma: Optional[np.ndarray], eps: float, residual: bool,
+                  tokens: Optional[Sequence[int]] = None, nthreads: Optional[int] = None):
+    """The MoE block with its adjacent steps: h = RMSNorm(x) (when gamma is
+    given), routing and experts on h, plus x when `residual`.  Returns
+    (y [len(tokens), d], idx, w, counts) with the routing over all tokens."""
+    x64 = _c(x, np.float64)
+    h = rmsnorm(x64, gamma, eps) if gamma is not None else x64
+    _, idx, w, counts = router(h, wr, bias, k)
+    y = moe_forward(h, q, idx, w, tokens=tokens, nthreads=nthreads)
+    if residual:
+        y = y + (x64 if tokens is None else x64[np.asarray(tokens, np.int64)])
+    return y, idx, w, counts

@@ -9,7 +9,10 @@
  * x sigma(x) and three matrices W_gate, W_up, W_down), §2.1 (weighted
  * aggregation of the k expert outputs), §4 Quantification MXFP4 (4.25 bits
  * per parameter; Microscaling format of Darvish Rouhani et al. 2023: blocks of
- * 32 E2M1 elements sharing one E8M0 scale).
+ * 32 E2M1 elements sharing one E8M0 scale).  Page "GPT-OSS vs Qwen3 :
+ * comparaison détaillée", Adoption de RMSNorm: the normalisation next to the
+ * block divides by the root mean square of the token instead of using the
+ * mean and variance.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - block scale exponent: floor(log2(max|w|)) - 2, clamped to [-127, 127];
@@ -251,4 +254,18 @@ void oracle_moe_forward(const double* x, int64_t d_model, int64_t d_ff, int64_t 
     for (int32_t i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
     free(jobs);
     free(th);
+}
+
+void oracle_rmsnorm(const double* x, int64_t T, int64_t d, const double* gamma,
+                    double eps, double* out) {
+    for (int64_t t = 0; t < T; ++t) {
+        /* root mean square of the token's d values (the mean, not the sum) */
+        double ss = 0.0;
+        for (int64_t i = 0; i < d; ++i) ss += x[t * d + i] * x[t * d + i];
+        const double rms = sqrt(ss / (double)d + eps);
+        for (int64_t i = 0; i < d; ++i) {
+            const double g = gamma ? gamma[i] : 1.0;
+            out[t * d + i] = x[t * d + i] / rms * g;
+        }
+    }
 }

@@ -18,7 +18,9 @@
  *   §4 Quantification MXFP4   4.25 bits per parameter: blocks of 32 FP4
  *                         (E2M1) codes that share one 8-bit power-of-two
  *                         (E8M0) scale -- the Microscaling format of Darvish
- *                         Rouhani et al. 2023, which that page cites.
+ *                         Rouhani et al. 2023, which that page cites;
+ * and, from the page "GPT-OSS vs Qwen3 : comparaison détaillée", Adoption de
+ * RMSNorm: the block's input is normalised by its root mean square.
  *
  * Weight layout used by every function here (the "canonical" layout): for a
  * matrix applied as y = x . W with contraction length K and N outputs, row n
@@ -90,6 +92,14 @@ void oracle_moe_forward(const double* x, int64_t d_model, int64_t d_ff, int64_t 
                         const uint8_t* d_codes, const uint8_t* d_scales,
                         const int64_t* tokens, int64_t n_tok, double* y,
                         int32_t nthreads);
+
+/* RMSNorm of T tokens (page "GPT-OSS vs Qwen3 : comparaison détaillée",
+ * Adoption de RMSNorm: normalise by the root mean square instead of LayerNorm's
+ * mean and variance):
+ *   out[t][i] = x[t][i] / sqrt(mean_j x[t][j]^2 + eps) * gamma[i]
+ * (gamma == NULL means all ones).  x and out may alias only if equal. */
+void oracle_rmsnorm(const double* x, int64_t T, int64_t d, const double* gamma,
+                    double eps, double* out);
 
 #ifdef __cplusplus
 }

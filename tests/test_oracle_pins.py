@@ -361,3 +361,93 @@ def test_expert_weights_dominate_the_20b_footprint():
     total, size = 20.9e9, 12.8e9
     p_exp = (2 * total - size) / (2 - 17 / 32)
     assert 0.90 < p_exp / total < 1.0
+
+
+# ---------------------------------------------------------------- RMSNorm and the residual (N3)
+# Page "GPT-OSS vs Qwen3 : comparaison détaillée", Adoption de RMSNorm: the
+# block input is divided by its root mean square (no mean, no variance).
+
+def test_rmsnorm_hand_worked_cases():
+    for line in _read_table("rmsnorm_cases.txt"):
+        name, xs, gs, eps, want = [p.strip() for p in line.split("|")]
+        x = np.array([[float(v) for v in xs.split()]])
+        g = None if gs == "-" else np.array([float(v) for v in gs.split()])
+        got = oracle.rmsnorm(x, g, float(eps))[0]
+        np.testing.assert_allclose(got, [float(v) for v in want.split()], rtol=1e-15, atol=0, err_msg=name)
+
+
+def test_rmsnorm_is_scale_invariant_and_unit_rms():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 96))
+    base = oracle.rmsnorm(x, None, 0.0)
+    for m in (-3, 1, 7):
+        # powers of two scale the mean square by 4^m exactly: the result is bit-identical
+        np.testing.assert_array_equal(oracle.rmsnorm(x * 2.0 ** m, None, 0.0), base)
+    np.testing.assert_allclose((base ** 2).mean(axis=1), 1.0, rtol=1e-13)
+    # the gain multiplies feature by feature
+    g = rng.standard_normal(96)
+    np.testing.assert_allclose(oracle.rmsnorm(x, g, 0.0), base * g, rtol=1e-14)
+    # eps sits inside the root, added to the mean square
+    e = 0.25
+    np.testing.assert_allclose(oracle.rmsnorm(x, None, e),
+                               x / np.sqrt((x ** 2).mean(axis=1, keepdims=True) + e), rtol=1e-14)
+
+
+def _tiny_block_setup(seed=11, d=64, E=4, k=2, T=12):
+    rng = np.random.default_rng(seed)
+    wr = rng.standard_normal((E, d)) / np.sqrt(d)
+    x = rng.standard_normal((T, d)) * 3.0
+    gamma = 1.0 + 0.1 * rng.standard_normal(d)
+    return rng, wr, x, gamma
+
+
+def test_block_residual_with_zero_down_projection_is_the_input():
+    rng, wr, x, gamma = _tiny_block_setup()
+    d, E = x.shape[1], wr.shape[0]
+    q = oracle.QuantExperts(d, d, E)
+    for e in range(E):
+        q.set_expert(e, rng.standard_normal((d, d)).astype(np.float32) * 0.02,
+                     rng.standard_normal((d, d)).astype(np.float32) * 0.02, np.zeros((d, d), np.float32))
+    y, _, _, _ = oracle.block_forward(x, q, wr, None, 2, gamma, 1e-5, residual=True)
+    np.testing.assert_array_equal(y, x)
+    y0, _, _, _ = oracle.block_forward(x, q, wr, None, 2, gamma, 1e-5, residual=False)
+    np.testing.assert_array_equal(y0, 0.0)
+
+
+def test_block_routes_on_the_normalised_input():
+    """With the pre-norm, routing depends on x only through RMSNorm(x): scaling
+    a token by a power of two (eps = 0) leaves its experts and weights as they
+    were, while the routing of the raw input changes."""
+    rng, wr, x, gamma = _tiny_block_setup()
+    d, E = x.shape[1], wr.shape[0]
+    q = oracle.QuantExperts(d, d, E)
+    for e in range(E):
+        q.set_expert(e, *(rng.standard_normal(s).astype(np.float32) * 0.02 for s in ((d, d), (d, d), (d, d))))
+    _, i1, w1, _ = oracle.block_forward(x, q, wr, None, 2, gamma, 0.0, residual=False)
+    _, i2, w2, _ = oracle.block_forward(x * 8.0, q, wr, None, 2, gamma, 0.0, residual=False)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_allclose(w1, w2, rtol=1e-12)
+    _, _, wraw1, _ = oracle.router(x, wr, None, 2)
+    _, _, wraw2, _ = oracle.router(x * 8.0, wr, None, 2)
+    assert np.abs(wraw1 - wraw2).max() > 1e-3
+
+
+def test_block_identity_experts_closed_form_with_norm_and_residual():
+    """W_gate = a I, W_up = b I, W_down = c I (powers of two, exact in MXFP4):
+    y = x + sum_j w_j c a b h^2 sigma(a h) with h = RMSNorm(x) = x / rms * gamma."""
+    rng, wr, x, gamma = _tiny_block_setup(d=64, E=4, k=2)
+    d, E, k = 64, 4, 2
+    a, b, c = [0.5, 1.0, 2.0, 0.25], [1.0, 2.0, 0.5, 4.0], [2.0, 0.5, 1.0, 0.125]
+    q = oracle.QuantExperts(d, d, E)
+    I = np.eye(d, dtype=np.float32)
+    for e in range(E):
+        q.set_expert(e, I * a[e], I * b[e], I * c[e])
+    eps = 1e-5
+    y, idx, w, _ = oracle.block_forward(x, q, wr, None, k, gamma, eps, residual=True)
+    h = x / np.sqrt((x ** 2).mean(axis=1, keepdims=True) + eps) * gamma
+    ref = x.copy()
+    for j in range(k):
+        e = idx[:, j]
+        A, B, C = (np.array(v)[e][:, None] for v in (a, b, c))
+        ref += w[:, j:j + 1] * C * A * B * h ** 2 / (1 + np.exp(-A * h))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
