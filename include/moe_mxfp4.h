@@ -119,6 +119,19 @@ moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w
 moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router,
                                   const float* router_bias, cudaStream_t stream);
 
+/* Steps adjacent to the MoE block, fused into its kernels (page "GPT-OSS vs
+ * Qwen3 : comparaison détaillée", Adoption de RMSNorm: the block input is
+ * normalised by its root mean square; and the skip connection around the
+ * block).
+ *   gamma:    device fp32 [d_model] (4-byte aligned), or NULL for no pre-norm.
+ *             With it, the router and the experts see
+ *             h = x / sqrt(mean(x^2) + eps) * gamma  (formed in fp32) instead of x.
+ *   eps:      finite, >= 0 (else INVALID_ARG).
+ *   residual: != 0 makes forward write y = x + (the MoE output).
+ * Copies gamma (asynchronously on `stream`); applies to later forwards. */
+moe_status_t moe_mxfp4_set_norm_residual(moe_mxfp4_t* h, const float* gamma, float eps,
+                                         int32_t residual, cudaStream_t stream);
+
 /* The layer for T tokens (0 <= T <= max_tokens; T == 0 launches nothing).
  * Defines: §3.1 (scores, top-k, softmax over the selected scores), §3.2 (each
  * selected expert's SwiGLU FFN) and §2.1 step 2 (the k outputs aggregated with

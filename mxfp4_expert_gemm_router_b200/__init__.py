@@ -53,6 +53,7 @@ SIGNATURES = {
     "moe_mxfp4_quantize_weights": (_ST, [_VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_mxfp4_quantize_expert": (_ST, [_VP, _I32, _VP, _VP, _VP, _VP]),
     "moe_mxfp4_set_router": (_ST, [_VP, _VP, _VP, _VP]),
+    "moe_mxfp4_set_norm_residual": (_ST, [_VP, _VP, ctypes.c_float, _I32, _VP]),
     "moe_mxfp4_forward": (_ST, [_VP, _VP, _I32, _VP, _VP, _VP, _VP, _VP]),
     "moe_mxfp4_forward_host": (_ST, [_VP, _VP, _I32, _VP, _VP, _VP, _VP]),
     "moe_mxfp4_export_weights": (_ST, [_VP, _I32, _VP, _VP, _VP]),
@@ -172,6 +173,10 @@ class MoeMxfp4:
 
     def set_router(self, w_router, router_bias=None, stream=None):
         check(load().moe_mxfp4_set_router(self.h, _p(w_router), _p(router_bias), _stream(stream)), "set_router")
+
+    def set_norm_residual(self, gamma=None, eps=1e-5, residual=False, stream=None):
+        check(load().moe_mxfp4_set_norm_residual(self.h, _p(gamma), float(eps), 1 if residual else 0,
+                                                 _stream(stream)), "set_norm_residual")
 
     def forward(self, x, y, topk_idx=None, topk_w=None, expert_counts=None, stream=None):
         T = int(x.shape[0]) if x is not None else 0

@@ -70,6 +70,10 @@ struct moe_mxfp4 {
     void* w_router = nullptr;
     float* bias = nullptr;
     bool has_bias = false, router_set = false;
+    // optional steps adjacent to the block: pre-norm (gamma) and residual
+    float* gamma = nullptr;    // [d_model]
+    bool use_norm = false, residual = false;
+    float eps = 0.f;
     int experts_quantized = 0;
     bool* expert_done = nullptr;
     // workspace
@@ -77,6 +81,8 @@ struct moe_mxfp4 {
     float* w_ws = nullptr;
     int32_t* hist = nullptr;
     double* part = nullptr;
+    double* part_ss = nullptr;   // router partial sums of x^2 (pre-norm)
+    float* inv_rms = nullptr;    // [max_tokens] 1 / rms(x) (pre-norm)
     int* counters = nullptr;   // [nblk_max] tile counters + [1] global counter
     int32_t* local_rank = nullptr;
     int32_t* offsets = nullptr;
@@ -152,7 +158,8 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
     } while (0)
 
 static void free_all(moe_mxfp4* h) {
-    void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->idx_ws, h->w_ws, h->hist,
+    void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->gamma, h->part_ss, h->inv_rms,
+                    h->idx_ws, h->w_ws, h->hist,
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
@@ -349,6 +356,9 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->w_ws), sizeof(float) * TK},
         {reinterpret_cast<void**>(&h->hist), sizeof(int32_t) * static_cast<size_t>(h->nblk_max) * E},
         {reinterpret_cast<void**>(&h->part), sizeof(double) * h->part_elems},
+        {reinterpret_cast<void**>(&h->part_ss), sizeof(double) * (h->part_elems / E + 64)},
+        {reinterpret_cast<void**>(&h->inv_rms), sizeof(float) * c.max_tokens},
+        {reinterpret_cast<void**>(&h->gamma), sizeof(float) * d},
         {reinterpret_cast<void**>(&h->counters), sizeof(int) * (h->nblk_max + 1)},
         {reinterpret_cast<void**>(&h->local_rank), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->offsets), sizeof(int32_t) * (E + 1)},
@@ -425,6 +435,19 @@ moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router, const fl
     }
     h->has_bias = router_bias != nullptr;
     h->router_set = true;
+    h->last_stream = stream;
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_set_norm_residual(moe_mxfp4_t* h, const float* gamma, float eps, int32_t residual,
+                                        cudaStream_t stream) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1e30f || !aligned_to(gamma, 4)) return MOE_ERR_INVALID_ARG;
+    if (gamma)
+        MOE_TRY(cudaMemcpyAsync(h->gamma, gamma, sizeof(float) * h->cfg.d_model, cudaMemcpyDeviceToDevice, stream));
+    h->use_norm = gamma != nullptr;
+    h->eps = eps;
+    h->residual = residual != 0;
     h->last_stream = stream;
     return MOE_OK;
 }
@@ -552,6 +575,10 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.k = k;
     ra.S = router_splits(T, d, h->nsm);
     ra.part = h->part;
+    ra.gamma = h->use_norm ? h->gamma : nullptr;
+    ra.eps = h->eps;
+    ra.part_ss = h->part_ss;
+    ra.inv_rms = h->inv_rms;
     ra.tile_cnt = h->counters;
     ra.glob_cnt = h->counters + h->nblk_max;
     ra.idx_out = idx;
@@ -587,20 +614,23 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     const bool stacked = mxg_stacked(BN);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
+    const float* gam = h->use_norm ? h->gamma : nullptr;
     if (bf16)
         launch_pdl(pdl, gather_kernel<__nv_bfloat16>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(idx),
                    static_cast<const float*>(wts), static_cast<const int32_t*>(h->local_rank),
                    static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
-                   h->row_slot, Xop, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched));
+                   h->row_slot, Xop, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), gam,
+                   static_cast<const float*>(h->inv_rms), h->residual ? 1 : 0);
     else
         launch_pdl(pdl, gather_kernel<float>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
                    static_cast<const float*>(x), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                    static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
                    BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc,
-                   static_cast<const int32_t*>(h->sched));
+                   static_cast<const int32_t*>(h->sched), gam, static_cast<const float*>(h->inv_rms),
+                   h->residual ? 1 : 0);
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);

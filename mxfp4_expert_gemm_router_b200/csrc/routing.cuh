@@ -76,6 +76,11 @@ struct RouterArgs {
     int T, d, E, k;
     int S;                 // K splits = gridDim.y
     double* part;          // [S][T][E] partial scores
+    // optional pre-norm: scores of h = x * gamma / sqrt(mean(x^2) + eps)
+    const float* gamma;    // [d] or null (no pre-norm)
+    float eps;
+    double* part_ss;       // [S][T] partial sums of x^2 (used with gamma)
+    float* inv_rms;        // [T] 1 / sqrt(mean(x^2) + eps), written with gamma
     int* tile_cnt;         // [tiles] arrival counters (zero between launches)
     int* glob_cnt;         // [1] arrival counter (zero between launches)
     int32_t* idx_out;      // [T][k]
@@ -257,9 +262,18 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     constexpr int EP = 32 * EPT;              // expert slots covered by the register tile
     const int xt = tid >> 3, xv8 = (tid & 7) * 8;
     Raw8<TA> xr, wrr[EPT];
+    // pre-norm: the staged chunk holds x * gamma; the sum of x^2 over the
+    // split's K range is kept per token (the last CTA divides by the RMS)
+    const bool norm = a.gamma != nullptr;
+    float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+    double ss = 0.0;
     auto load_chunk = [&](int kc) {
         if (xt < ntok && kc + xv8 < d) xr.load(x + static_cast<size_t>(t0 + xt) * d + kc + xv8);
         else xr.zero();
+        if (norm && kc + xv8 < d) {
+            g0 = *reinterpret_cast<const float4*>(a.gamma + kc + xv8);
+            g1 = *reinterpret_cast<const float4*>(a.gamma + kc + xv8 + 4);
+        }
 #pragma unroll
         for (int i = 0; i < EPT; ++i) {
             const int idx = tid + ROUTER_THREADS * i;
@@ -272,8 +286,20 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     for (int c = kc0; c < kc1; ++c) {
         const int kc = c * ROUTER_KCHUNK;
         __syncthreads();
+        if (norm) {
+            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            float sq = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = xr.get(j);
+            for (int j = 0; j < 8; ++j) {
+                const float v = xr.get(j);
+                sq = fmaf(v, v, sq);
+                xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = v * gv[j];
+            }
+            ss += static_cast<double>(sq);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = xr.get(j);
+        }
 #pragma unroll
         for (int i = 0; i < EPT; ++i) {
             const int idx = tid + ROUTER_THREADS * i;
@@ -308,6 +334,13 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
 #pragma unroll
             for (int j = 0; j < 4; ++j) tot[i][j] += static_cast<double>(acc[i][j]);
     }
+    if (norm) {
+        // the token's 8 threads are lanes 8m .. 8m+7 of one warp
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+        if ((tid & 7) == 0 && xt < ntok) a.part_ss[static_cast<size_t>(split) * a.T + t0 + xt] = ss;
+    }
     // partial scores of this split
 #pragma unroll
     for (int i = 0; i < EPT; ++i) {
@@ -329,6 +362,15 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
 
     for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
+    __shared__ double inv_s[ROUTER_TOKENS];
+    if (norm && tid < ntok) {
+        double sq = 0.0;
+        for (int sp = 0; sp < a.S; ++sp) sq += __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid);
+        const double inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
+        inv_s[tid] = inv;
+        a.inv_rms[t0 + tid] = static_cast<float>(inv);
+    }
+    __syncthreads();
     {
         // logits = partials summed in split order (deterministic) + bias; each
         // thread takes 2 outputs with all their partial loads in flight
@@ -351,6 +393,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
 #pragma unroll
                     for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) s += pv[m][sp];
                     const int tl = i / E, e = i % E;
+                    if (norm) s *= inv_s[tl];
                     if (a.bias) s += a.bias[e];
                     lg[tl * (E + 1) + e] = static_cast<float>(s);
                 }
@@ -485,9 +528,12 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
 // so the rows of an expert are in (token, slot) order; the row's place in the
 // expert's token tiles is (tile_base[e] + (row - offsets[e]) / BN,
 // (row - offsets[e]) % BN).  The block-0 thread records each row's token,
-// routing weight and tile slot.  Every thread clears its block of the token's
-// row of the fp32 output accumulator (for the down GEMM's scatter-add) and,
-// when the gate/up GEMM splits K, its share of the fp32 partial-sum rows.
+// routing weight and tile slot.  Every thread initialises its block of the
+// token's row of the fp32 output accumulator for the down GEMM's scatter-add
+// (to x itself when the block's residual is fused, else to zero) and, when
+// the gate/up GEMM splits K, clears its share of the fp32 partial-sum rows.
+// With the pre-norm, the block is multiplied by gamma and the token's inverse
+// RMS (computed by the router) before it is encoded.
 template <typename TA>
 __global__ void __launch_bounds__(GATHER_THREADS)
 gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
@@ -495,18 +541,14 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
               const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
               int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
               GroupedOperand X, float* __restrict__ GU, int gu_ld, float* __restrict__ yacc,
-              const int32_t* __restrict__ sched) {
+              const int32_t* __restrict__ sched, const float* __restrict__ gamma,
+              const float* __restrict__ inv_rms, int residual) {
     pdl_launch_dependents();
     pdl_wait();
     const int nb = d / 32;
     const long item = static_cast<long>(blockIdx.x) * GATHER_THREADS + threadIdx.x;
     if (item >= static_cast<long>(T) * nb) return;
     const int t = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
-    {
-        float4* yz = reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d + b * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) yz[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     // the k destinations first (independent load chains in flight together), encoded while they land, then the stores
     int pos[MAX_TOPK], tile[MAX_TOPK], rloc[MAX_TOPK];
 #pragma unroll
@@ -522,6 +564,27 @@ gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const f
     }
     float v[32];
     BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+    {
+        // the output accumulator row starts at x (the block's skip connection) or at zero
+        float4* yz = reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d + b * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            yz[i] = residual ? make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3])
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (gamma) {
+        // pre-norm: the experts see h = x * gamma / rms(x)
+        const float r = inv_rms[t];
+        const float4* g4 = reinterpret_cast<const float4*>(gamma + b * 32);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 g = g4[i];
+            v[4 * i] *= g.x * r;
+            v[4 * i + 1] *= g.y * r;
+            v[4 * i + 2] *= g.z * r;
+            v[4 * i + 3] *= g.w * r;
+        }
+    }
     uint4 codes[MXQ_TERMS];
     uint32_t sb[MXQ_TERMS];
     mxq_block_thread(v, codes, sb);

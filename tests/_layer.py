@@ -183,3 +183,32 @@ def check_layer(cfg, x, wr, bias, y, idx, w, counts, ox: OracleExperts, n_sample
     scale = np.abs(y_ref).max()
     assert err <= Y_REL_TOL * scale, (err, scale, err / scale)
     return err / scale
+
+
+def filtered_x_norm(cfg: mi.MoeConfig, wr, bias, gamma, eps, T=None):
+    """x drawn and margin-filtered on the scores of RMSNorm(x) (what the router sees)."""
+    x = mi.draw_x(cfg, T)
+    x, _ = mi.margin_filter(cfg, x, lambda rows: oracle.router_logits(oracle.rmsnorm(rows, gamma, eps), wr, bias))
+    return x
+
+
+def check_block(cfg, x, wr, bias, gamma, eps, residual, y, idx, w, counts, ox: OracleExperts, n_sample=16,
+                extra_tokens=None):
+    """The block with its adjacent steps: routing of RMSNorm(x) bit-exact over all
+    tokens, output (with the residual) on a token sample vs the oracle."""
+    h = oracle.rmsnorm(x, gamma, eps) if gamma is not None else np.asarray(x, np.float64)
+    _, idx_ref, w_ref, counts_ref = oracle.router(h, wr, bias, cfg.top_k)
+    np.testing.assert_array_equal(idx, idx_ref)
+    np.testing.assert_array_equal(counts, counts_ref)
+    w_err = np.abs(w - w_ref).max()
+    assert w_err <= W_ABS_TOL, ("routing weight error", w_err)
+    tok = sample_tokens(idx_ref, counts_ref, n_sample)
+    if extra_tokens is not None and len(extra_tokens):
+        tok = np.union1d(tok, np.asarray(extra_tokens, np.int64))
+    q = ox.ensure(np.unique(idx_ref[tok]))
+    y_ref, _, _, _ = oracle.block_forward(x, q, wr, bias, cfg.top_k, gamma, eps, residual, tokens=tok)
+    err = np.abs(y[tok] - y_ref).max()
+    # with the residual the bar applies to the MoE part (y - x): the residual is exact
+    scale = np.abs(y_ref - (np.asarray(x, np.float64)[tok] if residual else 0.0)).max()
+    assert err <= Y_REL_TOL * scale, (err, scale, err / scale)
+    return err / scale
