@@ -60,6 +60,18 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 #define MOE_FLAG_TOKEN_TILE_SHIFT 8
 #define MOE_FLAG_TOKEN_TILE_MASK (0xFu << MOE_FLAG_TOKEN_TILE_SHIFT)
 
+/* Forwards of at most 16 tokens run as one cooperative launch (router, both
+ * expert GEMMs and the combine in one persistent grid) when the layer's shape
+ * allows it.  This flag (or a forced token tile) keeps every forward on the
+ * multi-launch path instead; both compute the same layer. */
+#define MOE_FLAG_UNFUSED_DECODE (1u << 12)
+
+/* Test-only: the n-th device allocation of moe_mxfp4_create (n = 1..255 in
+ * this field; 0 = off) fails as if cudaMalloc had, so the failure path can be
+ * exercised; create then returns MOE_ERR_CUDA having freed everything. */
+#define MOE_FLAG_TEST_FAIL_ALLOC_SHIFT 16
+#define MOE_FLAG_TEST_FAIL_ALLOC_MASK (0xFFu << MOE_FLAG_TEST_FAIL_ALLOC_SHIFT)
+
 typedef struct {
     int32_t d_model;        /* model width; multiple of 32                    */
     int32_t d_ff;           /* expert hidden width; multiple of 32            */
@@ -180,7 +192,8 @@ moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* h, int32_t which, uint8
  *   offsets:    device int32 [E+1]  rows of expert e are [offsets[e], offsets[e+1])
  *   row_token:  device int32 [T*k]  token of each grouped row (or NULL)
  *   row_weight: device fp32  [T*k]  routing weight of each grouped row (or NULL)
- * Rows of one expert appear in (token, slot) order. */
+ * Rows of one expert appear in (token, slot) order.  After a forward that ran
+ * the fused decode kernel (no grouping is built) this returns UNSUPPORTED. */
 moe_status_t moe_mxfp4_get_grouping(const moe_mxfp4_t* h, int32_t* offsets, int32_t* row_token,
                                     float* row_weight, cudaStream_t stream);
 
@@ -200,10 +213,10 @@ const char* moe_mxfp4_status_string(moe_status_t s);
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */
-#define MOE_NUM_STAGES 6
+#define MOE_NUM_STAGES 7
 /* 0 router + top-k + softmax + grouping schedule, 1 gather into grouped rows,
  * 2 gate/up + SwiGLU, 3 H encoding (three MXFP4 terms), 4 down + weighted combine,
- * 5 output cast.  Synchronises;
+ * 5 output cast, 6 the fused decode kernel (forwards of at most 16 tokens).  Synchronises;
  * writes the last profiled forward's durations in ms (0 for stages that did
  * not run) into ms[0..min(n, MOE_NUM_STAGES)). */
 moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n);

@@ -23,6 +23,9 @@ MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_FLAG_TEST_SKIP_FIRST_COPY = 1 << 30
 MOE_FLAG_TOKEN_TILE_SHIFT = 8
 MOE_FLAG_TOKEN_TILE_MASK = 0xF << MOE_FLAG_TOKEN_TILE_SHIFT
+MOE_FLAG_UNFUSED_DECODE = 1 << 12
+MOE_FLAG_TEST_FAIL_ALLOC_SHIFT = 16
+MOE_FLAG_TEST_FAIL_ALLOC_MASK = 0xFF << MOE_FLAG_TEST_FAIL_ALLOC_SHIFT
 
 
 TOKEN_TILES = tuple(range(16, 129, 16))
@@ -33,7 +36,7 @@ def token_tile_flag(bn: int) -> int:
     if bn not in TOKEN_TILES:
         raise ValueError("token tile must be a multiple of 16 from 16 to 128")
     return (bn // 16) << MOE_FLAG_TOKEN_TILE_SHIFT
-MOE_NUM_STAGES = 6
+MOE_NUM_STAGES = 7
 
 
 class moe_mxfp4_config_t(ctypes.Structure):

@@ -1,0 +1,829 @@
+// decode_fused.cuh -- the whole layer in one persistent, cooperative launch
+// for small batches (T <= 16 tokens).
+//
+// Method (page "GPT-OSS-20B : Architecture MoE & Résumé du Model Card"):
+// §3.1 Le Routeur (scores = W_router . h, top-k, softmax over the selected
+// scores), §3.2 Les Experts (SwiGLU FFN per selected expert), §2.1 (the k
+// expert outputs summed with the routing weights), §4 (MXFP4 weights); with
+// the optional pre-norm (page "GPT-OSS vs Qwen3 : comparaison détaillée",
+// Adoption de RMSNorm) and the residual around the block.
+//
+// At decode sizes the layer is the weight stream of the touched experts (a
+// few to a few tens of microseconds on B200); a chain of launches spends as
+// long again in launch gaps, ramps and tails.  This kernel runs every step in
+// one grid of one CTA per SM, all resident (cooperative launch):
+//
+//  1. Router, split over the grid: CTA b computes partial scores for
+//     (expert, K split) units -- fp32 within 64-wide K chunks, fp64 across --
+//     and the partial sums of x^2 for the pre-norm.  One grid barrier; then
+//     every CTA sums the partials in split order (identical results in every
+//     CTA), applies the RMS scaling and the bias, takes the top-k (warp
+//     arg-max rounds, ties to the lower index) and the softmax, and lists the
+//     touched experts in ascending order.
+//  2. The B operand is every token of the batch (16 rows per term, the three
+//     MXFP4 terms stacked: N = 48) for every expert.  Columns of tokens not
+//     routed to an expert are computed and dropped: next to the weight stream
+//     the MMA work is negligible, and one B operand for the whole K, encoded
+//     once per CTA into shared memory, replaces the grouping and the gather.
+//  3. Work items: a gate/up item is one 128-wide K chunk of one 128-feature
+//     tile of one touched expert (gate and up: 17,408 bytes); a down item is
+//     two consecutive K chunks of one feature tile of the down matrix (at most
+//     17,408 bytes).  CTA b takes an equal contiguous share of the gate/up
+//     items and of the down items in (expert, tile, chunk) order, so every SM
+//     streams the same number of bytes.  A run of items with the same (expert,
+//     tile) is a piece; it accumulates in one tensor-memory accumulator.
+//  4. Gate/up pieces add fp32 partial sums of g and u into GU (red.add) for
+//     the tokens routed to the expert and then count their chunks in a
+//     per-(expert, feature tile) counter.  A down piece of expert e over d_ff
+//     chunks [c0, c1) needs g and u of features [128 c0, 128 c1): its
+//     epilogue warps wait (bounded) for those counters, form H = Swish(g) u,
+//     encode it as three MXFP4 terms into the shared-memory B operand, and
+//     the MMA warp runs.  Down weight copies never wait: the producer streams
+//     them into the ring while other CTAs finish their gate/up work.
+//  5. Down epilogue: y_acc[t] += w[t, e] D[., t] for the tokens routed to e
+//     (red.add).  The last CTA to finish writes y (cast; + x with the
+//     residual) and resets the counters.
+//
+// State across launches (epoch, grid-barrier arrivals, counters) lives in
+// device memory.  GU and y_acc alternate by the epoch's parity: each launch
+// clears the rows of the other parity that the previous launch used, so the
+// buffers a launch accumulates into are always clear, with no pass of its
+// own.  Every wait (mbarrier phases, the grid barrier, the counters) is
+// bounded; on a timeout the CTA raises its abort flag and the status word,
+// all roles leave their loops, copies and MMAs in flight are drained and the
+// tensor memory is freed.  Every CTA still arrives at the grid barrier and at
+// the finish counter exactly once, so the state stays consistent.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "mxq.cuh"
+#include "quantize.cuh"
+#include "routing.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int DF_MAX_T = 16;                 // token rows per term of the B operand
+constexpr int DF_NB3 = MXQ_TERMS * DF_MAX_T; // 48 operand rows
+constexpr int DF_EPI_WARPS = 8;
+constexpr int DF_THREADS = (2 + DF_EPI_WARPS) * 32;
+constexpr int DF_EPI_THREADS = DF_EPI_WARPS * 32;
+constexpr uint32_t DF_STAGE = 2u * (4u * 128 * 16 + 512);   // 17,408 bytes
+constexpr int DF_MAX_STAGES = 8;
+constexpr int DF_MAT_COLS = 64;              // accumulator columns per matrix (48 used)
+constexpr int DF_ACC_COLS = 2 * DF_MAT_COLS; // gate and up
+constexpr int DF_SF_COL0 = 448;
+constexpr int DF_SF_SLOTS = 2;
+constexpr int DF_SF_SLOT_COLS = 32;
+constexpr uint32_t DF_B_BLOCK = DF_NB3 * 16;  // 768 bytes of B codes per 32-block
+constexpr int DF_MAX_TOUCHED = DF_MAX_T * MAX_TOPK;   // touched experts <= T * k
+
+struct DecodeState {
+    uint32_t bar;      // grid-barrier arrivals: grows by gridDim.x per launch
+    uint32_t epoch;    // launches completed
+    uint32_t finish;   // CTAs finished in the current launch
+    int32_t prev_nt;   // touched experts of the previous launch
+    int32_t prev_T;    // its token count
+    uint32_t pad[3];
+};
+
+struct DecodeParams {
+    const void* x;          // [T][d] act dtype
+    void* y;                // [T][d] act dtype
+    const void* wr;         // [E][d] act dtype
+    const float* bias;      // [E] or null
+    const float* gamma;     // [d] or null (no pre-norm)
+    float eps;
+    int residual;
+    int T, d, f, E, k;
+    TiledMatrix Mgu;        // gate + up (N = f, K = d), expert 0 at base
+    TiledMatrix Mdn;        // down (N = d, K = f)
+    int S;                  // router K splits
+    int stages;             // weight-ring stages
+    int nb_max;             // 32-blocks of the B buffer: max(d, f) / 32
+    int kc_max;             // K chunks of the B buffer: max over both GEMMs
+    int max_touched;        // expert rows of GU per parity
+    DecodeState* st;
+    uint32_t* done;         // [max_touched][F_gu] gate/up chunks finished
+    double* part;           // [S][16][E] partial scores
+    double* part_ss;        // [S][16] partial sums of x^2
+    float* gu;              // [2][max_touched][16][2 f] partial g | u
+    float* yacc;            // [2][16][d]
+    int32_t* topk_idx;      // [T][k] or null
+    float* topk_w;          // [T][k] or null
+    int32_t* counts;        // [E] or null
+    int* status;
+    uint64_t timeout_ns;
+    uint32_t skip_first_copy;   // test hook: each producer skips its first copy
+};
+
+// Shared memory after the 1024-aligned weight ring and B buffer.
+struct DecodeCtl {
+    uint64_t full[DF_MAX_STAGES], empty[DF_MAX_STAGES];
+    uint64_t accf[2], acce[2], xready, bready, drain;
+    int abort_flag;
+    uint32_t tmem;
+    int last;
+    int n_t;
+    double inv_rms[DF_MAX_T];
+    int tok_e[DF_MAX_T][MAX_TOPK];
+    float tok_w[DF_MAX_T][MAX_TOPK];
+    int slot_of[MAX_EXPERTS];
+    int touched[DF_MAX_TOUCHED];
+    float selw[DF_MAX_TOUCHED][DF_MAX_T];   // routing weight of token t for touched slot i (0: not routed)
+};
+
+__host__ __device__ inline uint32_t df_bbuf_bytes(int nb_max, int kc_max) {
+    return static_cast<uint32_t>(nb_max) * DF_B_BLOCK + static_cast<uint32_t>(kc_max) * 512u;
+}
+__host__ inline size_t df_smem_bytes(int stages, int nb_max, int kc_max) {
+    return 1024 + static_cast<size_t>(stages) * DF_STAGE + df_bbuf_bytes(nb_max, kc_max) + sizeof(DecodeCtl) + 16;
+}
+
+// Bytes of the down item j (chunks 2j and 2j+1 of feature tile ft): contiguous in the tiled layout.
+__device__ __forceinline__ uint32_t df_down_item_bytes(const TiledMatrix& M, int j, int rf) {
+    const int c = 2 * j;
+    uint32_t b = static_cast<uint32_t>(M.mat_bytes(c, rf));
+    if (c + 1 < M.chunks()) b += static_cast<uint32_t>(M.mat_bytes(c + 1, rf));
+    return b;
+}
+
+template <typename TA>
+__global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const DecodeParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+    const int T = p.T, d = p.d, f = p.f, E = p.E, k = p.k;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t ring = base;
+    const uint32_t bbuf = base + static_cast<uint32_t>(p.stages) * DF_STAGE;      // B codes
+    const uint32_t bsf = bbuf + static_cast<uint32_t>(p.nb_max) * DF_B_BLOCK;    // B scale atoms
+    uint8_t* bbuf_ptr = base_ptr + static_cast<size_t>(p.stages) * DF_STAGE;
+    uint8_t* bsf_ptr = bbuf_ptr + static_cast<size_t>(p.nb_max) * DF_B_BLOCK;
+    DecodeCtl& C = *reinterpret_cast<DecodeCtl*>(bsf_ptr + static_cast<size_t>(p.kc_max) * 512);
+    volatile int* abort_flag = &C.abort_flag;
+    const int S = p.stages;
+    auto full_bar = [&](int s) { return smem_u32(&C.full[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&C.empty[s]); };
+
+    const int F_gu = p.Mgu.tiles(), KC_gu = p.Mgu.chunks();
+    const int F_dn = p.Mdn.tiles(), KC_dn = p.Mdn.chunks();
+    const int NP = (KC_dn + 1) / 2;   // down items per feature tile
+    const bool norm = p.gamma != nullptr;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&C.accf[b]), 1);
+            mbar_init(smem_u32(&C.acce[b]), DF_EPI_WARPS);
+        }
+        mbar_init(smem_u32(&C.xready), 1);
+        mbar_init(smem_u32(&C.bready), 1);
+        mbar_init(smem_u32(&C.drain), 1);
+        C.abort_flag = 0;
+        C.last = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&C.tmem), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = C.tmem;
+    const uint32_t epoch = ld_acquire_u32(&p.st->epoch);
+    const int par = static_cast<int>(epoch & 1u);
+    const size_t gu_par = static_cast<size_t>(p.max_touched) * DF_MAX_T * 2 * f;
+    float* gu = p.gu + par * gu_par;
+    float* yacc = p.yacc + static_cast<size_t>(par) * DF_MAX_T * d;
+
+    // ---- clear the other parity's rows the previous launch used (nothing in
+    // this launch touches them)
+    {
+        const int pn = p.st->prev_nt, pT = p.st->prev_T;
+        float4* g_other = reinterpret_cast<float4*>(p.gu + (1 - par) * gu_par);
+        const int row4 = 2 * f / 4;
+        const long n4 = static_cast<long>(pn) * pT * row4;
+        for (long i = static_cast<long>(blockIdx.x) * DF_THREADS + tid; i < n4; i += static_cast<long>(G) * DF_THREADS) {
+            const long r = i / row4, c4 = i % row4;
+            const long row = (r / pT) * DF_MAX_T + (r % pT);
+            g_other[row * row4 + c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float4* y_other = reinterpret_cast<float4*>(p.yacc + static_cast<size_t>(1 - par) * DF_MAX_T * d);
+        const long y4 = static_cast<long>(DF_MAX_T) * d / 4;
+        for (long i = static_cast<long>(blockIdx.x) * DF_THREADS + tid; i < y4; i += static_cast<long>(G) * DF_THREADS)
+            y_other[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    // ---- 1. router partials over (expert, K split) units
+    const TA* x = static_cast<const TA*>(p.x);
+    const TA* wr = static_cast<const TA*>(p.wr);
+    const int KCH = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
+    {
+        double* scratch = reinterpret_cast<double*>(base_ptr);   // the ring is free until the producer starts
+        double* scratch_ss = scratch + DF_MAX_T * KCH;
+        for (int u = blockIdx.x; u < E * p.S; u += G) {
+            const int e = u / p.S, sp = u % p.S;
+            const int j0 = sp * KCH / p.S, j1 = (sp + 1) * KCH / p.S, nj = j1 - j0;
+            for (int it = tid; it < T * nj; it += DF_THREADS) {
+                const int t = it / nj, j = j0 + it % nj;
+                float acc = 0.f, sq = 0.f;
+#pragma unroll
+                for (int g8 = 0; g8 < ROUTER_KCHUNK / 8; ++g8) {
+                    const int kk = j * ROUTER_KCHUNK + g8 * 8;
+                    if (kk < d) {
+                        Raw8<TA> xr, wv;
+                        xr.load(x + static_cast<size_t>(t) * d + kk);
+                        wv.load(wr + static_cast<size_t>(e) * d + kk);
+                        if (norm) {
+                            const float4 g0 = *reinterpret_cast<const float4*>(p.gamma + kk);
+                            const float4 g1 = *reinterpret_cast<const float4*>(p.gamma + kk + 4);
+                            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float xv = xr.get(q);
+                                sq = fmaf(xv, xv, sq);
+                                acc = fmaf(xv * gv[q], wv.get(q), acc);
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) acc = fmaf(xr.get(q), wv.get(q), acc);
+                        }
+                    }
+                }
+                scratch[t * nj + (j - j0)] = static_cast<double>(acc);
+                scratch_ss[t * nj + (j - j0)] = static_cast<double>(sq);
+            }
+            __syncthreads();
+            if (tid < T) {
+                double s = 0.0, ss = 0.0;
+                for (int j = 0; j < nj; ++j) {
+                    s += scratch[tid * nj + j];
+                    ss += scratch_ss[tid * nj + j];
+                }
+                p.part[(static_cast<size_t>(sp) * DF_MAX_T + tid) * E + e] = s;
+                if (norm && e == 0) p.part_ss[static_cast<size_t>(sp) * DF_MAX_T + tid] = ss;
+            }
+            __syncthreads();
+        }
+    }
+    // grid barrier: every CTA arrives exactly once per launch
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(&p.st->bar, 1u);
+        const uint32_t target = (epoch + 1u) * static_cast<uint32_t>(G);
+        spin_until_reached(&p.st->bar, target, abort_flag, p.status, p.timeout_ns);
+    }
+    __syncthreads();
+
+    // ---- finish the routing in every CTA (identical order, identical results)
+    {
+        float* lg = reinterpret_cast<float*>(base_ptr);   // [16][E + 1]
+        if (tid < T) {
+            double ss = 0.0;
+            if (norm)
+                for (int sp = 0; sp < p.S; ++sp) ss += __ldcg(p.part_ss + static_cast<size_t>(sp) * DF_MAX_T + tid);
+            C.inv_rms[tid] = norm ? 1.0 / sqrt(ss / static_cast<double>(d) + static_cast<double>(p.eps)) : 1.0;
+        }
+        for (int e = tid; e < E; e += DF_THREADS) {
+            C.slot_of[e] = 0;
+        }
+        __syncthreads();
+        for (int i = tid; i < T * E; i += DF_THREADS) {
+            const int t = i / E, e = i % E;
+            double s = 0.0;
+            for (int sp = 0; sp < p.S; ++sp) s += __ldcg(p.part + (static_cast<size_t>(sp) * DF_MAX_T + t) * E + e);
+            if (norm) s *= C.inv_rms[t];
+            if (p.bias) s += p.bias[e];
+            lg[t * (E + 1) + e] = static_cast<float>(s);
+        }
+        __syncthreads();
+        const int ept = (E + 31) / 32;
+        for (int t = warp; t < T; t += DF_THREADS / 32) {
+            const float* row = lg + t * (E + 1);
+            uint32_t taken = 0;
+            float sel_v[MAX_TOPK];
+            int sel_e[MAX_TOPK];
+            for (int r = 0; r < k; ++r) {
+                float bv = -INFINITY;
+                int be = 0x7FFFFFFF;
+                for (int i = 0; i < ept; ++i) {
+                    const int e = lane + 32 * i;
+                    if (e < E && !((taken >> i) & 1u)) {
+                        const float v = row[e];
+                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+                }
+                be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                sel_v[r] = bv;
+                sel_e[r] = be;
+            }
+            if (lane == 0) {
+                const float m = sel_v[0];
+                float den = 0.f;
+                for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+                const float inv = 1.f / den;
+                for (int r = 0; r < k; ++r) {
+                    C.tok_e[t][r] = sel_e[r];
+                    C.tok_w[t][r] = expf(sel_v[r] - m) * inv;
+                }
+            }
+        }
+        __syncthreads();
+        // touched experts, ascending: mark, then one warp-wide exclusive scan
+        if (tid < T * k) atomicOr(&C.slot_of[C.tok_e[tid / k][tid % k]], 1);
+        __syncthreads();
+        if (warp == 0) {
+            int cnt = 0;
+            for (int i = 0; i < ept; ++i) {
+                const int e = lane * ept + i;
+                if (e < E) cnt += C.slot_of[e];
+            }
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += n;
+            }
+            int pos = inc - cnt;
+            for (int i = 0; i < ept; ++i) {
+                const int e = lane * ept + i;
+                if (e < E) {
+                    if (C.slot_of[e]) {
+                        C.touched[pos] = e;
+                        C.slot_of[e] = pos++;
+                    } else {
+                        C.slot_of[e] = -1;
+                    }
+                }
+            }
+            if (lane == 31) C.n_t = inc;
+        }
+        __syncthreads();
+        for (int i = tid; i < C.n_t * DF_MAX_T; i += DF_THREADS) C.selw[i / DF_MAX_T][i % DF_MAX_T] = 0.f;
+        __syncthreads();
+        if (tid < T * k) {
+            const int t = tid / k, r = tid % k;
+            C.selw[C.slot_of[C.tok_e[t][r]]][t] = C.tok_w[t][r];
+        }
+        if (blockIdx.x == 0) {
+            if (p.topk_idx && tid < T * k) p.topk_idx[tid] = C.tok_e[tid / k][tid % k];
+            if (p.topk_w && tid < T * k) p.topk_w[tid] = C.tok_w[tid / k][tid % k];
+            if (p.counts)
+                for (int e = tid; e < E; e += DF_THREADS) {
+                    int c = 0;
+                    for (int i = 0; i < T * k; ++i) c += (C.tok_e[i / k][i % k] == e);
+                    p.counts[e] = c;
+                }
+        }
+        __syncthreads();
+    }
+    const int n_t = C.n_t;
+    // this CTA's items: equal contiguous shares of the gate/up and the down items
+    const long NG = static_cast<long>(n_t) * F_gu * KC_gu;
+    const long ND = static_cast<long>(n_t) * F_dn * NP;
+    const long g_lo = NG * blockIdx.x / G, g_hi = NG * (blockIdx.x + 1) / G;
+    const long d_lo = ND * blockIdx.x / G, d_hi = ND * (blockIdx.x + 1) / G;
+    const size_t ebytes_gu = p.Mgu.expert_bytes(), ebytes_dn = p.Mdn.expert_bytes();
+    const uint32_t idesc = idesc_mxf4(128, DF_NB3);
+
+    if (warp == 0) {
+        // -------------------------------------------------------------- producer
+        int s = 0;
+        uint32_t ph = 0;
+        int pend_ph[DF_MAX_STAGES];
+        for (int i = 0; i < DF_MAX_STAGES; ++i) pend_ph[i] = -1;
+        bool skip = p.skip_first_copy != 0;
+        bool ok = __all_sync(0xffffffffu, *abort_flag == 0);
+        for (long it = g_lo; it < g_hi + (d_hi - d_lo) && ok; ++it) {
+            const uint8_t* src;
+            uint32_t bytes;
+            if (it < g_hi) {
+                const int i = static_cast<int>(it / (F_gu * KC_gu));
+                const int rem = static_cast<int>(it % (F_gu * KC_gu));
+                const int ft = rem / KC_gu, c = rem % KC_gu;
+                const int rf = min(128, f - ft * 128);
+                src = p.Mgu.base + C.touched[i] * ebytes_gu + p.Mgu.chunk_offset(ft, c, rf);
+                bytes = static_cast<uint32_t>(p.Mgu.chunk_bytes(c, rf));
+            } else {
+                const long jt = d_lo + (it - g_hi);
+                const int i = static_cast<int>(jt / (F_dn * NP));
+                const int rem = static_cast<int>(jt % (F_dn * NP));
+                const int ft = rem / NP, j = rem % NP;
+                const int rf = min(128, d - ft * 128);
+                src = p.Mdn.base + C.touched[i] * ebytes_dn + p.Mdn.chunk_offset(ft, 2 * j, rf);
+                bytes = df_down_item_bytes(p.Mdn, j, rf);
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns));
+            if (!ok) break;
+            if (skip) {
+                skip = false;   // test hook: this stage is never filled
+            } else {
+                mbar_arrive_expect_tx_warp(full_bar(s), bytes);
+                bulk_g2s_warp(ring + s * DF_STAGE, src, bytes, full_bar(s));
+                pend_ph[s] = static_cast<int>(ph);
+            }
+            if (++s == S) { s = 0; ph ^= 1u; }
+        }
+        if (lane == 0)
+            for (int i = 0; i < S; ++i)
+                if (pend_ph[i] >= 0) mbar_wait_drain(full_bar(i), static_cast<uint32_t>(pend_ph[i]), 200000000ull);
+        __syncwarp();
+    } else if (warp == 1) {
+        // -------------------------------------------------------------- MMA issuer
+        int s = 0, sfs = 0, buf = 0;
+        uint32_t ph = 0, bph = 0;
+        uint32_t eph[2] = {0u, 0u};
+        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.xready), 0, abort_flag, p.status, p.timeout_ns));
+        // gate/up pieces
+        long it = g_lo;
+        while (ok && it < g_hi) {
+            const int i = static_cast<int>(it / (F_gu * KC_gu));
+            const int ft = static_cast<int>((it % (F_gu * KC_gu)) / KC_gu);
+            const long piece_end = min(g_hi, static_cast<long>(i) * F_gu * KC_gu + static_cast<long>(ft + 1) * KC_gu);
+            const int rf = min(128, f - ft * 128);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.acce[buf]), eph[buf] ^ 1u, abort_flag, p.status,
+                                                           p.timeout_ns));
+            if (!ok) break;
+            eph[buf] ^= 1u;
+            tc_fence_after();
+            const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
+            bool first = true;   // the piece's first MMA overwrites the accumulator
+            for (; it < piece_end; ++it) {
+                const int c = static_cast<int>(it % KC_gu);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const int nbc = p.Mgu.blocks_in_chunk(c);
+                const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16), mat_b = codes_b + 512u;
+                const uint32_t ws = ring + s * DF_STAGE;
+                const uint32_t sfc = tmem + DF_SF_COL0 + DF_SF_SLOT_COLS * sfs;
+                tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
+                tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
+                tc_cp_sf_warp(sfc + 8, desc_noswz(bsf + c * 512u, 0, 128));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (2 * h < nbc) {
+                        const uint32_t acc = first ? 0u : 1u;
+                        first = false;
+                        const uint32_t id = idesc | idesc_sf_ids(2u * h);
+                        const uint64_t ad = desc_noswz(ws + 2 * h * rf * 16, rf * 16, 128);
+                        const uint64_t bd = desc_noswz(bbuf + (4 * c + 2 * h) * DF_B_BLOCK, DF_B_BLOCK, 128);
+                        mma_mxf4_warp(d0, ad, bd, id, sfc, sfc + 8, acc);
+                        mma_mxf4_warp(d0 + DF_MAT_COLS, ad + (mat_b >> 4), bd, id, sfc + 4, sfc + 8, acc);
+                    }
+                }
+                tc_commit_warp(empty_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
+                if (++sfs == DF_SF_SLOTS) sfs = 0;
+            }
+            if (!ok) break;
+            tc_commit_warp(smem_u32(&C.accf[buf]));
+            buf ^= 1;
+        }
+        // down pieces
+        long jt = d_lo;
+        while (ok && jt < d_hi) {
+            const int i = static_cast<int>(jt / (F_dn * NP));
+            const int ft = static_cast<int>((jt % (F_dn * NP)) / NP);
+            const long piece_end = min(d_hi, static_cast<long>(i) * F_dn * NP + static_cast<long>(ft + 1) * NP);
+            const int rf = min(128, d - ft * 128);
+            const int pc0 = 2 * static_cast<int>(jt % NP);   // first K chunk of the piece
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.bready), bph, abort_flag, p.status, p.timeout_ns));
+            if (!ok) break;
+            bph ^= 1u;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.acce[buf]), eph[buf] ^ 1u, abort_flag, p.status,
+                                                           p.timeout_ns));
+            if (!ok) break;
+            eph[buf] ^= 1u;
+            tc_fence_after();
+            const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
+            bool first = true;
+            for (; jt < piece_end; ++jt) {
+                const int j = static_cast<int>(jt % NP);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ws = ring + s * DF_STAGE;
+                const uint32_t sfc = tmem + DF_SF_COL0 + DF_SF_SLOT_COLS * sfs;
+                uint32_t off = 0;
+                for (int hc = 0; hc < 2; ++hc) {
+                    const int c = 2 * j + hc;
+                    if (c >= KC_dn) break;
+                    const int nbc = p.Mdn.blocks_in_chunk(c);
+                    const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16);
+                    tc_cp_sf_warp(sfc + 4 * hc, desc_noswz(ws + off + codes_b, 0, 128));
+                    tc_cp_sf_warp(sfc + 8 + 4 * hc, desc_noswz(bsf + (c - pc0) * 512u, 0, 128));
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (2 * h < nbc) {
+                            const uint32_t acc = first ? 0u : 1u;
+                            first = false;
+                            const uint32_t id = idesc | idesc_sf_ids(2u * h);
+                            const uint64_t ad = desc_noswz(ws + off + 2 * h * rf * 16, rf * 16, 128);
+                            const uint64_t bd =
+                                desc_noswz(bbuf + (4 * (c - pc0) + 2 * h) * DF_B_BLOCK, DF_B_BLOCK, 128);
+                            mma_mxf4_warp(d0, ad, bd, id, sfc + 4 * hc, sfc + 8 + 4 * hc, acc);
+                        }
+                    }
+                    off += codes_b + 512u;
+                }
+                tc_commit_warp(empty_bar(s));
+                if (++s == S) { s = 0; ph ^= 1u; }
+                if (++sfs == DF_SF_SLOTS) sfs = 0;
+            }
+            if (!ok) break;
+            tc_commit_warp(smem_u32(&C.accf[buf]));
+            buf ^= 1;
+        }
+        tc_commit_warp(smem_u32(&C.drain));
+        if (lane == 0) mbar_wait_drain(smem_u32(&C.drain), 0, 200000000ull);
+        __syncwarp();
+    } else {
+        // -------------------------------------------------------------- epilogue warps
+        const int et = tid - 64;                 // 0 .. 255
+        const int q = warp & 3;                  // TMEM lane quarter (hardware rule: warp % 4)
+        const int hh = (warp - 2) >> 2;          // token columns 8 hh .. 8 hh + 7
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+
+        // x of every token as the B operand: [block][term * 16 + token][16 B]
+        {
+            // scale bytes of blocks past K in a ragged last chunk must be a finite
+            // (zero: 2^-127) E8M0 value, never stale shared memory
+            for (int i = et; i < p.kc_max * 512 / 16; i += DF_EPI_THREADS)
+                reinterpret_cast<uint4*>(bsf_ptr)[i] = make_uint4(0u, 0u, 0u, 0u);
+            named_barrier(1, DF_EPI_THREADS);
+            const int nb = d / 32;
+            for (int itm = et; itm < nb * DF_MAX_T; itm += DF_EPI_THREADS) {
+                const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
+                float v[32];
+                if (t < T) {
+                    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+                    if (norm) {
+                        const float r = static_cast<float>(C.inv_rms[t]);
+                        const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 g = g4[i];
+                            v[4 * i] *= g.x * r;
+                            v[4 * i + 1] *= g.y * r;
+                            v[4 * i + 2] *= g.z * r;
+                            v[4 * i + 3] *= g.w * r;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+                uint4 codes[MXQ_TERMS];
+                uint32_t sb[MXQ_TERMS];
+                mxq_block_thread(v, codes, sb);
+#pragma unroll
+                for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                    *reinterpret_cast<uint4*>(bbuf_ptr + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                        codes[tt];
+                    bsf_ptr[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_barrier(1, DF_EPI_THREADS);
+            if (et == 0) mbar_arrive(smem_u32(&C.xready));
+        }
+        bool ok = named_barrier_and(1, DF_EPI_THREADS, *abort_flag == 0);
+
+        int buf = 0;
+        uint32_t fph[2] = {0u, 0u};
+        // accumulator of token group hh: sum of the three stacked term columns
+        auto load_acc = [&](uint32_t d0, float (&out)[8]) {
+            uint32_t r[MXQ_TERMS][8];
+#pragma unroll
+            for (int tt = 0; tt < MXQ_TERMS; ++tt) tmem_ld8(d0 + lane_addr + tt * DF_MAX_T + 8 * hh, r[tt]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                out[j] = __uint_as_float(r[0][j]) + __uint_as_float(r[1][j]) + __uint_as_float(r[2][j]);
+        };
+
+        // gate/up pieces: partial sums of g and u into GU, then count the chunks
+        long it = g_lo;
+        while (ok && it < g_hi) {
+            const int i = static_cast<int>(it / (F_gu * KC_gu));
+            const int ft = static_cast<int>((it % (F_gu * KC_gu)) / KC_gu);
+            const long piece_end = min(g_hi, static_cast<long>(i) * F_gu * KC_gu + static_cast<long>(ft + 1) * KC_gu);
+            const int rf = min(128, f - ft * 128);
+            const bool w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[buf]), fph[buf], abort_flag,
+                                                                         p.status, p.timeout_ns));
+            fph[buf] ^= 1u;
+            tc_fence_after();
+            if (w_ok && 32 * q < rf && 8 * hh < T) {
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
+                float g[8], u[8];
+                load_acc(d0, g);
+                load_acc(d0 + DF_MAT_COLS, u);
+                const int n = ft * 128 + 32 * q + lane;
+                if (32 * q + lane < rf) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int t = 8 * hh + j;
+                        if (t < T && C.selw[i][t] != 0.f) {
+                            float* row = gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f;
+                            atomicAdd(row + n, g[j]);
+                            atomicAdd(row + f + n, u[j]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (w_ok && lane == 0) mbar_arrive(smem_u32(&C.acce[buf]));
+            buf ^= 1;
+            __threadfence();
+            // every epilogue thread takes the same decision (no thread is left waiting)
+            ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
+            if (!ok) break;
+            if (et == 0) atomicAdd(&p.done[i * F_gu + ft], static_cast<uint32_t>(piece_end - it));
+            it = piece_end;
+        }
+
+        // down pieces: wait for g and u, build the H operand, combine
+        long jt = d_lo;
+        int pend_buf = -1, pend_i = 0, pend_ft = 0, pend_rf = 0;
+        auto drain_pending = [&]() {
+            // the pending piece's MMAs have completed (its accumulator-full phase was waited)
+            if (32 * q < pend_rf && 8 * hh < T) {
+                const uint32_t d0 = tmem + static_cast<uint32_t>(pend_buf * DF_ACC_COLS);
+                float o[8];
+                load_acc(d0, o);
+                const int n = pend_ft * 128 + 32 * q + lane;
+                if (32 * q + lane < pend_rf) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int t = 8 * hh + j;
+                        const float w = t < T ? C.selw[pend_i][t] : 0.f;
+                        if (w != 0.f) atomicAdd(yacc + static_cast<size_t>(t) * d + n, w * o[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&C.acce[pend_buf]));
+            pend_buf = -1;
+        };
+        while (ok && jt < d_hi) {
+            const int i = static_cast<int>(jt / (F_dn * NP));
+            const int ft = static_cast<int>((jt % (F_dn * NP)) / NP);
+            const long piece_end = min(d_hi, static_cast<long>(i) * F_dn * NP + static_cast<long>(ft + 1) * NP);
+            const int rf = min(128, d - ft * 128);
+            const int c0 = 2 * static_cast<int>(jt % NP);
+            const int c1 = min(KC_dn, 2 * static_cast<int>((piece_end - 1) % NP) + 2);
+            // g and u of features [128 c0, 128 c1) complete (gate/up feature tiles c0 .. c1-1)
+            bool w_ok = true;
+            if (et < c1 - c0)
+                w_ok = spin_until_reached(&p.done[i * F_gu + c0 + et], static_cast<uint32_t>(KC_gu), abort_flag,
+                                          p.status, p.timeout_ns);
+            // the previous down piece's MMAs must be done before its operand is overwritten
+            if (pend_buf >= 0) {
+                w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag,
+                                                                 p.status, p.timeout_ns)) && w_ok;
+                fph[pend_buf] ^= 1u;
+                tc_fence_after();
+            }
+            ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
+            if (!ok) break;
+            // H = Swish(g) u of the routed tokens as three MXFP4 terms: [block][term * 16 + t][16 B]
+            {
+                const int nbf = f / 32;
+                const int b0 = 4 * c0, b1 = min(4 * c1, nbf);
+                for (int itm = et; itm < (b1 - b0) * DF_MAX_T; itm += DF_EPI_THREADS) {
+                    const int b = b0 + itm / DF_MAX_T, t = itm % DF_MAX_T;
+                    float v[32];
+                    if (t < T && C.selw[i][t] != 0.f) {
+                        const float4* g4 =
+                            reinterpret_cast<const float4*>(gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f + 32 * b);
+                        const float4* u4 = reinterpret_cast<const float4*>(
+                            gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f + f + 32 * b);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 gg = __ldcg(g4 + q4), uu = __ldcg(u4 + q4);
+                            v[4 * q4] = swish_f(gg.x) * uu.x;
+                            v[4 * q4 + 1] = swish_f(gg.y) * uu.y;
+                            v[4 * q4 + 2] = swish_f(gg.z) * uu.z;
+                            v[4 * q4 + 3] = swish_f(gg.w) * uu.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int q4 = 0; q4 < 32; ++q4) v[q4] = 0.f;
+                    }
+                    uint4 codes[MXQ_TERMS];
+                    uint32_t sb[MXQ_TERMS];
+                    mxq_block_thread(v, codes, sb);
+#pragma unroll
+                    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                        *reinterpret_cast<uint4*>(bbuf_ptr +
+                                                  (static_cast<size_t>(b - b0) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                            codes[tt];
+                        bsf_ptr[((b >> 2) - c0) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] =
+                            static_cast<uint8_t>(sb[tt]);
+                    }
+                }
+                // blocks past d_ff in a ragged last chunk: zero scale bytes (2^-127)
+                for (int itm = et; itm < (4 * c1 - b1) * DF_NB3; itm += DF_EPI_THREADS) {
+                    const int b = b1 + itm / DF_NB3, r = itm % DF_NB3;
+                    bsf_ptr[((b >> 2) - c0) * 512 + sf_atom_offset(r, b & 3)] = 0;
+                }
+                fence_proxy_async_smem();
+                named_barrier(1, DF_EPI_THREADS);
+                if (et == 0) mbar_arrive(smem_u32(&C.bready));
+            }
+            if (pend_buf >= 0) drain_pending();
+            pend_buf = buf;
+            pend_i = i;
+            pend_ft = ft;
+            pend_rf = rf;
+            buf ^= 1;
+            jt = piece_end;
+        }
+        if (ok && pend_buf >= 0) {
+            const bool w_ok =
+                mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag, p.status, p.timeout_ns);
+            if (__all_sync(0xffffffffu, w_ok)) {
+                fph[pend_buf] ^= 1u;
+                tc_fence_after();
+                drain_pending();
+            }
+        }
+        __threadfence();
+    }
+
+    // ---- finish: free tensor memory; the last CTA writes y and resets the state
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (tid == 0) {
+        __threadfence();
+        C.last = (atomicAdd(&p.st->finish, 1u) == static_cast<uint32_t>(G - 1)) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!C.last) return;
+    __threadfence();
+    {
+        const long n4 = static_cast<long>(T) * d / 4;
+        for (long i4 = tid; i4 < n4; i4 += DF_THREADS) {
+            float4 v = __ldcg(reinterpret_cast<const float4*>(yacc) + i4);
+            if (p.residual) {
+                float xv[4];
+                if constexpr (sizeof(TA) == 2) {
+                    const uint2 xr = reinterpret_cast<const uint2*>(p.x)[i4];
+                    xv[0] = __uint_as_float(xr.x << 16);
+                    xv[1] = __uint_as_float(xr.x & 0xFFFF0000u);
+                    xv[2] = __uint_as_float(xr.y << 16);
+                    xv[3] = __uint_as_float(xr.y & 0xFFFF0000u);
+                } else {
+                    const float4 xr = reinterpret_cast<const float4*>(p.x)[i4];
+                    xv[0] = xr.x; xv[1] = xr.y; xv[2] = xr.z; xv[3] = xr.w;
+                }
+                v.x += xv[0]; v.y += xv[1]; v.z += xv[2]; v.w += xv[3];
+            }
+            if constexpr (sizeof(TA) == 2) {
+                __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+                __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+                uint2 o;
+                o.x = *reinterpret_cast<uint32_t*>(&a);
+                o.y = *reinterpret_cast<uint32_t*>(&b);
+                reinterpret_cast<uint2*>(p.y)[i4] = o;
+            } else {
+                reinterpret_cast<float4*>(p.y)[i4] = v;
+            }
+        }
+        for (int i = tid; i < n_t * F_gu; i += DF_THREADS) p.done[i] = 0u;
+        __syncthreads();
+        if (tid == 0) {
+            p.st->prev_nt = n_t;
+            p.st->prev_T = T;
+            p.st->finish = 0u;
+            __threadfence();
+            atomicAdd(&p.st->epoch, 1u);
+        }
+    }
+}
+
+}  // namespace moe

@@ -1,8 +1,10 @@
 // moe_mxfp4.cu -- C ABI of the MoE feed-forward layer with MXFP4 experts
 // (declarations and argument contracts in include/moe_mxfp4.h).
 //
-// One forward = up to six launches on the caller's stream, no host sync and
-// no allocation:
+// A forward of at most 16 tokens is one cooperative launch of
+// decode_fused_kernel (router, both expert GEMMs and the combine in one
+// persistent grid).  Larger forwards are up to six launches on the caller's
+// stream; no host sync and no allocation either way:
 //   router_kernel        scores (K split over the grid), top-k, softmax over the
 //                        selected scores, per-tile histogram and ranks, zeroing
 //                        of the output rows; its last CTA builds the schedule
@@ -28,6 +30,7 @@
 #include <new>
 
 #include "../../include/moe_mxfp4.h"
+#include "decode_fused.cuh"
 #include "expert_mxf4.cuh"
 #include "quantize.cuh"
 #include "routing.cuh"
@@ -109,6 +112,16 @@ struct moe_mxfp4 {
     CUtensorMap tm_x[BN_OPTIONS];
     CUtensorMap tm_h[BN_OPTIONS];
     bool tm_ok[BN_OPTIONS] = {};
+    // fused decode path (forwards of at most DF_MAX_T tokens)
+    bool df_ok = false, last_fused = false;
+    int df_stages = 0, df_S = 0, df_nb_max = 0, df_kc_max = 0, df_max_touched = 0;
+    size_t df_smem = 0;
+    DecodeState* df_state = nullptr;
+    uint32_t* df_done = nullptr;
+    double* df_part = nullptr;
+    double* df_part_ss = nullptr;
+    float* df_gu = nullptr;
+    float* df_yacc = nullptr;
     cudaStream_t last_stream = nullptr;
     // profiling
     bool prof = false, prof_valid = false;
@@ -162,7 +175,8 @@ static void free_all(moe_mxfp4* h) {
                     h->idx_ws, h->w_ws, h->hist,
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
-                    h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage};
+                    h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
+                    h->df_state, h->df_done, h->df_part, h->df_part_ss, h->df_gu, h->df_yacc};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     for (auto& e : h->ev)
@@ -253,6 +267,12 @@ static cudaError_t ensure_kernel_attrs(int dev) {
         return e;
     if ((e = set_router_smem<float>(rsm))) return e;
     if ((e = set_router_smem<__nv_bfloat16>(rsm))) return e;
+    if ((e = cudaFuncSetAttribute(decode_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  227 * 1024)))
+        return e;
+    if ((e = cudaFuncSetAttribute(decode_fused_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  227 * 1024)))
+        return e;
     g_attrs_set[dev] = true;
     return cudaSuccess;
 }
@@ -279,7 +299,7 @@ const char* moe_mxfp4_status_string(moe_status_t s) {
 
 const char* moe_mxfp4_stage_name(int32_t stage) {
     static const char* names[MOE_NUM_STAGES] = {"router_topk_schedule", "gather", "gate_up_swiglu",
-                                                 "h_encode", "down_combine", "cast_out"};
+                                                 "h_encode", "down_combine", "cast_out", "fused_decode"};
     return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "unknown";
 }
 
@@ -381,8 +401,13 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->idx_stage), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->w_stage), sizeof(float) * TK},
     };
-    for (auto& a : allocs)
+    // test hook: the fail_at-th device allocation (1-based) fails as if cudaMalloc had
+    const uint32_t fail_at = (c.flags & MOE_FLAG_TEST_FAIL_ALLOC_MASK) >> MOE_FLAG_TEST_FAIL_ALLOC_SHIFT;
+    uint32_t n_alloc = 0;
+    for (auto& a : allocs) {
+        if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
         if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    }
     // Operand buffers start as zeros: codes, scale atoms and the weights' padding
     // are then always finite (an E2M1 code is never NaN; scale bytes written by
     // the kernels are at most 253, never the E8M0 NaN 0xFF), so operand rows a
@@ -397,6 +422,54 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         return fail(MOE_ERR_CUDA);
 
     if (ensure_kernel_attrs(h->dev) != cudaSuccess) return fail(MOE_ERR_CUDA);
+
+    // fused decode path: one persistent grid for forwards of at most DF_MAX_T
+    // tokens, when its shared-memory plan fits (the whole-K B operand plus at
+    // least two weight stages) and one CTA per SM can be resident
+    {
+        h->df_nb_max = std::max(d, f) / 32;
+        h->df_kc_max = std::max(h->KC_gu, h->KC_dn);
+        const size_t fixed = df_smem_bytes(0, h->df_nb_max, h->df_kc_max);
+        const long st = (227L * 1024 - static_cast<long>(fixed)) / static_cast<long>(DF_STAGE);
+        h->df_stages = static_cast<int>(std::min<long>(st, DF_MAX_STAGES));
+        // the router's scratch (2 x 16 x K chunks doubles) and logits live in the ring
+        const size_t router_scratch = 2 * DF_MAX_T * sizeof(double) * ((d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK);
+        const size_t logits = DF_MAX_T * sizeof(float) * (E + 1);
+        if (h->df_stages >= 2 && std::max(router_scratch, logits) <= static_cast<size_t>(h->df_stages) * DF_STAGE) {
+            h->df_smem = df_smem_bytes(h->df_stages, h->df_nb_max, h->df_kc_max);
+            const int kch = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
+            h->df_S = std::max(1, std::min(h->nsm / E, kch));
+            h->df_max_touched = std::min(E, DF_MAX_T * k);
+            int per_sm = 0;
+            cudaError_t oe =
+                c.act_dtype == MOE_DTYPE_BF16
+                    ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel<__nv_bfloat16>,
+                                                                    DF_THREADS, h->df_smem)
+                    : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_fused_kernel<float>, DF_THREADS,
+                                                                    h->df_smem);
+            if (oe != cudaSuccess) return fail(MOE_ERR_CUDA);
+            if (per_sm >= 1) {
+                const size_t gu_bytes_df = sizeof(float) * 2 * h->df_max_touched * DF_MAX_T * 2 * static_cast<size_t>(f);
+                const size_t ya_bytes_df = sizeof(float) * 2 * DF_MAX_T * static_cast<size_t>(d);
+                const size_t done_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu;
+                A dfa[] = {
+                    {reinterpret_cast<void**>(&h->df_state), sizeof(DecodeState)},
+                    {reinterpret_cast<void**>(&h->df_done), done_bytes},
+                    {reinterpret_cast<void**>(&h->df_part), sizeof(double) * h->df_S * DF_MAX_T * E},
+                    {reinterpret_cast<void**>(&h->df_part_ss), sizeof(double) * h->df_S * DF_MAX_T},
+                    {reinterpret_cast<void**>(&h->df_gu), gu_bytes_df},
+                    {reinterpret_cast<void**>(&h->df_yacc), ya_bytes_df},
+                };
+                for (auto& a : dfa) {
+                    if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
+                    if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+                    if (cudaMemset(*a.p, 0, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+                }
+                if (cudaDeviceSynchronize() != cudaSuccess) return fail(MOE_ERR_CUDA);
+                h->df_ok = true;
+            }
+        }
+    }
     for (auto& e : h->ev)
         if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
     *out = h;
@@ -563,6 +636,65 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         if (prof) cudaEventRecordWithFlags(h->ev[i], stream, ev_flags);
     };
 
+    const uint64_t tmo = static_cast<uint64_t>(c.wait_timeout_ms > 0 ? c.wait_timeout_ms : 2000) * 1000000ull;
+    // at most DF_MAX_T tokens: the whole layer in one cooperative launch
+    if (h->df_ok && T <= DF_MAX_T && !(c.flags & (MOE_FLAG_UNFUSED_DECODE | MOE_FLAG_TOKEN_TILE_MASK))) {
+        DecodeParams dp{};
+        dp.x = x;
+        dp.y = y;
+        dp.wr = h->w_router;
+        dp.bias = h->has_bias ? h->bias : nullptr;
+        dp.gamma = h->use_norm ? h->gamma : nullptr;
+        dp.eps = h->eps;
+        dp.residual = h->residual ? 1 : 0;
+        dp.T = T;
+        dp.d = d;
+        dp.f = f;
+        dp.E = E;
+        dp.k = k;
+        dp.Mgu = tiled(h, 0);
+        dp.Mdn = tiled(h, 2);
+        dp.S = h->df_S;
+        dp.stages = h->df_stages;
+        dp.nb_max = h->df_nb_max;
+        dp.kc_max = h->df_kc_max;
+        dp.max_touched = h->df_max_touched;
+        dp.st = h->df_state;
+        dp.done = h->df_done;
+        dp.part = h->df_part;
+        dp.part_ss = h->df_part_ss;
+        dp.gu = h->df_gu;
+        dp.yacc = h->df_yacc;
+        dp.topk_idx = topk_idx;
+        dp.topk_w = topk_w;
+        dp.counts = expert_counts;
+        dp.status = h->status;
+        dp.timeout_ns = tmo;
+        dp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(h->nsm);
+        lc.blockDim = dim3(DF_THREADS);
+        lc.dynamicSmemBytes = h->df_smem;
+        lc.stream = stream;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: the grid barrier and counters rely on it
+        at[0].val.cooperative = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        mark(6);
+        if (bf16)
+            cudaLaunchKernelEx(&lc, decode_fused_kernel<__nv_bfloat16>, dp);
+        else
+            cudaLaunchKernelEx(&lc, decode_fused_kernel<float>, dp);
+        mark(7);
+        h->stage_ran[6] = true;
+        h->last_fused = true;
+        h->prof_valid = prof;
+        h->launches += 1;
+        return cuda_status(cudaGetLastError());
+    }
+    h->last_fused = false;
+
     // 0: router + top-k + softmax + schedule
     mark(0);
     RouterArgs ra{};
@@ -634,7 +766,6 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);
-    const uint64_t tmo = static_cast<uint64_t>(c.wait_timeout_ms > 0 ? c.wait_timeout_ms : 2000) * 1000000ull;
     MxgParams gp{};
     gp.wpack = h->w_gu;
     gp.units = h->units_gu;
@@ -703,6 +834,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         h->stage_ran[5] = true;
     }
     mark(6);
+    mark(7);   // the record's end event (stage 6, the fused path, did not run)
     h->prof_valid = prof;
     for (int i = 0; i < MOE_NUM_STAGES; ++i) h->launches += h->stage_ran[i] ? 1 : 0;
     return cuda_status(cudaGetLastError());
@@ -735,6 +867,7 @@ moe_status_t moe_mxfp4_get_grouping(const moe_mxfp4_t* hc, int32_t* offsets, int
                                     cudaStream_t stream) {
     if (!hc || !offsets) return MOE_ERR_INVALID_ARG;
     moe_mxfp4* h = const_cast<moe_mxfp4*>(hc);
+    if (h->last_fused) return MOE_ERR_UNSUPPORTED;   // the fused decode path builds no grouping
     const auto& c = h->cfg;
     MOE_TRY(cudaMemcpyAsync(offsets, h->offsets, sizeof(int32_t) * (c.n_experts + 1), cudaMemcpyDeviceToDevice, stream));
     // rows in use = offsets[E]; copy the full capacity bound the caller sized for T*k

@@ -426,6 +426,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
                 const int oe = __shfl_xor_sync(0xffffffffu, be, off);
                 if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
             }
+            be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
             if ((be & 31) == lane) taken |= 1u << (be >> 5);
             sel_v[r] = bv;
             sel_e[r] = be;

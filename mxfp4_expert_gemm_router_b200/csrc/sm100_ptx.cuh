@@ -102,6 +102,58 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
     return true;
 }
 
+// Bounded wait until *p (a counter other CTAs raise with atomics) reaches
+// `target` (compared as a signed difference, so the counter may wrap).  Load
+// with acquire semantics at GPU scope: what the raising CTA wrote before its
+// release is visible afterwards.  Returns false on the abort flag or after
+// `limit_ns` (then it raises the abort flag and the status word).
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ bool spin_until_reached(const uint32_t* p, uint32_t target, volatile int* abort_flag,
+                                                   int* status, uint64_t limit_ns) {
+    if (static_cast<int>(ld_acquire_u32(p) - target) >= 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+    while (true) {
+        __nanosleep(64);
+        if (static_cast<int>(ld_acquire_u32(p) - target) >= 0) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads (tcgen05.mma / tcgen05.cp operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Named barrier over `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also returns the AND of `v` over the participating
+// threads: every participant takes the same decision (e.g. to leave a loop
+// after a bounded wait ran out in one of them).
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 // 1-D bulk copy global -> shared; both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -29,6 +29,13 @@ def ox20b():
     return OracleExperts(CFG20)
 
 
+@pytest.fixture(scope="module")
+def layer20b_unfused():
+    """The same layer with every forward on the multi-launch path."""
+    import mxfp4_expert_gemm_router_b200 as mx
+    return GpuLayer(CFG20, 256, flags=mx.MOE_FLAG_UNFUSED_DECODE)
+
+
 def _export(layer, cfg, which):
     import torch
     K, N = (cfg.d_model, cfg.d_ff) if which < 2 else (cfg.d_ff, cfg.d_model)
@@ -358,3 +365,66 @@ def test_misaligned_pointers_are_rejected_before_any_launch(layer20b):
     assert L.moe_mxfp4_forward(h, good, T, y.data_ptr(), None, None, None, s) == mx.MOE_OK
     torch.cuda.synchronize()
     assert layer20b.layer.status() == mx.MOE_OK
+
+
+# ------------------------------------------------------------------ fused decode path (T <= 16)
+
+@pytest.mark.parametrize("name", ["dec1", "dec8"])
+def test_decode_unfused_path_parity(layer20b_unfused, ox20b, name):
+    """dec1 / dec8 through the multi-launch path (the default is the fused kernel)."""
+    cfg = mi.CONFIGS[name]
+    wr = mi.draw_router(cfg)
+    layer20b_unfused.set_router(wr, None)
+    x = filtered_x(cfg, wr, None)
+    y, idx, w, counts = layer20b_unfused.forward(x)
+    check_layer(cfg, x, wr, None, y, idx, w, counts, ox20b, n_sample=cfg.T)
+
+
+def test_fused_decode_state_across_launches(layer20b, layer20b_unfused, ox20b):
+    """The fused kernel keeps state between launches (epoch, counters, buffers
+    alternating by parity that each launch clears for the next): a run of
+    forwards of varying size must each match the oracle on every token and
+    the multi-launch path."""
+    wr = mi.draw_router(CFG20)
+    layer20b.set_router(wr, None)
+    layer20b_unfused.set_router(wr, None)
+    for i, T in enumerate([8, 1, 16, 3, 16, 16, 2, 8]):
+        cfg = CFG20.with_T(T)
+        x = mi.draw_x(cfg.with_T(64))[8 * i: 8 * i + T] if T <= 8 else mi.draw_x(cfg)
+        x, _ = mi.margin_filter(cfg, x, lambda r: oracle.router_logits(r, wr, None))
+        y, idx, w, counts = layer20b.forward(x)
+        check_layer(cfg, x, wr, None, y, idx, w, counts, ox20b, n_sample=T)
+        y2, idx2, w2, _ = layer20b_unfused.forward(x)
+        np.testing.assert_array_equal(idx, idx2)
+        assert np.abs(w - w2).max() <= W_ABS_TOL
+        assert np.abs(y - y2).max() <= 1e-2 * np.abs(y2).max()
+
+
+@pytest.mark.parametrize("d,f_,E,k", [(192, 320, 4, 2), (96, 160, 5, 3), (64, 64, 256, 4), (2880, 2880, 128, 4)])
+def test_fused_decode_ragged_shapes(d, f_, E, k):
+    """The fused kernel on shapes with a short last feature tile, a short last
+    K chunk (K a multiple of 32 but not of 64), 256 experts (eight per lane in
+    the top-k) and 128 experts at full width, at 16 and 5 tokens."""
+    for T in (16, 5):
+        cfg = mi.MoeConfig("fused_ragged", T, d, f_, E, k, "bf16" if d == 2880 else "f32")
+        L = GpuLayer(cfg, 16)
+        ox = OracleExperts(cfg)
+        x = filtered_x(cfg, L.wr, L.bias)
+        y, idx, w, counts = L.forward(x)
+        check_layer(cfg, x, L.wr, L.bias, y, idx, w, counts, ox, n_sample=cfg.T)
+        L.layer.close()
+
+
+def test_unfused_pipeline_timeout_is_reported_not_hung():
+    """The timeout path of the multi-launch kernels (the fused kernel's is
+    covered by test_pipeline_timeout_is_reported_not_hung at 16 tokens)."""
+    import torch
+    import mxfp4_expert_gemm_router_b200 as mx
+    cfg = mi.CONFIGS["tiny"]
+    L = GpuLayer(cfg, cfg.T, flags=mx.MOE_FLAG_TEST_SKIP_FIRST_COPY | mx.MOE_FLAG_UNFUSED_DECODE,
+                 wait_timeout_ms=100)
+    x = act_tensor(cfg, mi.draw_x(cfg))
+    y = torch.empty((cfg.T, cfg.d_model), device="cuda")
+    L.layer.forward(x, y)
+    assert L.layer.status() == mx.MOE_ERR_TIMEOUT
+    assert L.layer.status() == mx.MOE_OK
