@@ -3,14 +3,16 @@
 //
 // A forward of at most 16 tokens is one cooperative launch of
 // decode_fused_kernel (router, both expert GEMMs and the combine in one
-// persistent grid).  Larger forwards are up to six launches on the caller's
+// persistent grid).  Larger forwards are up to seven launches on the caller's
 // stream; no host sync and no allocation either way:
 //   router_kernel        scores (K split over the grid), top-k, softmax over the
 //                        selected scores, per-tile histogram and ranks, zeroing
 //                        of the output rows; its last CTA builds the schedule
 //                        (expert offsets, K splits, unit lists)
-//   gather_kernel        grouped rows (token, weight, tile slot); activations
-//                        encoded as three MXFP4 terms (the B operand)
+//   rows_kernel          grouped rows (token, weight, tile slot); output
+//                        accumulator initialised (zero, or x for the residual)
+//   encode_rows_kernel   the grouped rows of x encoded as three MXFP4 terms
+//                        (the gate/up GEMM's B operand)
 //   expert_mxf4<0>       gate/up GEMM on block-scaled MXFP4 tensor cores,
 //                        SwiGLU epilogue encoding H as three MXFP4 terms for the
 //                        down GEMM (fp32 partials instead when K is split)
@@ -741,28 +743,36 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 1: gather into grouped rows
     mark(1);
     const bool pdl = static_cast<long>(T) * k <= h->gu_rows;
-    const long gitems = static_cast<long>(T) * (d / 32);
-    const int gblocks = static_cast<int>((gitems + GATHER_THREADS - 1) / GATHER_THREADS);
     const bool stacked = mxg_stacked(BN);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
     const float* gam = h->use_norm ? h->gamma : nullptr;
-    if (bf16)
-        launch_pdl(pdl, gather_kernel<__nv_bfloat16>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
+    const dim3 rgrid_rows((T + ROWS_TOKENS - 1) / ROWS_TOKENS);
+    // token tiles: at most ceil(T k / BN) plus one ragged tile per expert
+    const dim3 egrid(static_cast<unsigned>((static_cast<long>(T) * k + BN - 1) / BN + E), h->KC_gu);
+    if (bf16) {
+        launch_pdl(pdl, rows_kernel<__nv_bfloat16>, rgrid_rows, dim3(ROWS_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(idx),
                    static_cast<const float*>(wts), static_cast<const int32_t*>(h->local_rank),
                    static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
-                   h->row_slot, Xop, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), gam,
-                   static_cast<const float*>(h->inv_rms), h->residual ? 1 : 0);
-    else
-        launch_pdl(pdl, gather_kernel<float>, dim3(gblocks), dim3(GATHER_THREADS), 0, stream,
-                   static_cast<const float*>(x), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
+                   h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0);
+        launch_pdl(pdl, encode_rows_kernel<__nv_bfloat16>, egrid, dim3(ENC_THREADS), 0, stream,
+                   static_cast<const __nv_bfloat16*>(x), gam, static_cast<const float*>(h->inv_rms),
+                   static_cast<const int32_t*>(h->row_token), static_cast<const int4*>(h->units_gu),
+                   static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop);
+    } else {
+        launch_pdl(pdl, rows_kernel<float>, rgrid_rows, dim3(ROWS_THREADS), 0, stream, static_cast<const float*>(x),
+                   static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                    static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
-                   BN, h->row_token, h->row_weight, h->row_slot, Xop, h->GU, 2 * f, acc,
-                   static_cast<const int32_t*>(h->sched), gam, static_cast<const float*>(h->inv_rms),
-                   h->residual ? 1 : 0);
+                   BN, h->row_token, h->row_weight, h->row_slot, h->GU, 2 * f, acc,
+                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0);
+        launch_pdl(pdl, encode_rows_kernel<float>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
+                   gam, static_cast<const float*>(h->inv_rms), static_cast<const int32_t*>(h->row_token),
+                   static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop);
+    }
+    h->launches += 1;   // stage 1 is two launches
     h->stage_ran[1] = true;
     // 2: gate/up GEMM + SwiGLU
     mark(2);

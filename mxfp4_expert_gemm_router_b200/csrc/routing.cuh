@@ -505,8 +505,6 @@ template <> struct BlockLoader<float> {
     }
 };
 
-constexpr int GATHER_THREADS = 128;
-
 // Where the grouped operands live.
 struct GroupedOperand {
     uint8_t* codes;   // [K/32][3][R][16]
@@ -521,97 +519,130 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
     return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * MXQ_TERMS * 512;
 }
 
-// One thread per (token t, 32-block b of d_model); consecutive threads take
-// consecutive blocks of a token (coalesced reads).  The thread encodes its
-// block of x once as three MXFP4 terms and stores the codes and scale bytes
-// into each of the token's k grouped rows.  Pair p = t*k + j goes to grouped
-// row offsets[e] + (rows of e in earlier tiles) + (its rank within its tile),
-// so the rows of an expert are in (token, slot) order; the row's place in the
-// expert's token tiles is (tile_base[e] + (row - offsets[e]) / BN,
-// (row - offsets[e]) % BN).  The block-0 thread records each row's token,
-// routing weight and tile slot.  Every thread initialises its block of the
-// token's row of the fp32 output accumulator for the down GEMM's scatter-add
-// (to x itself when the block's residual is fused, else to zero) and, when
-// the gate/up GEMM splits K, clears its share of the fp32 partial-sum rows.
-// With the pre-norm, the block is multiplied by gamma and the token's inverse
-// RMS (computed by the router) before it is encoded.
+// Grouping, part 1: one CTA per ROWS_TOKENS tokens.  Pair p = t*k + j goes
+// to grouped row offsets[e] + (rows of e in earlier router tiles) + (its rank
+// within its router tile), so the rows of an expert are in (token, slot)
+// order; the row's place in the expert's token tiles is (tile_base[e] +
+// (row - offsets[e]) / BN, (row - offsets[e]) % BN).  One thread per pair
+// records each row's token, routing weight and tile slot.  All threads then
+// initialise the tokens' rows of the fp32 output accumulator for the down
+// GEMM's scatter-add (to x itself when the block's residual is fused, else to
+// zero) and, when the gate/up GEMM splits K, clear the pairs' fp32
+// partial-sum rows.
+constexpr int ROWS_TOKENS = 8;
+constexpr int ROWS_THREADS = 256;
 template <typename TA>
-__global__ void __launch_bounds__(GATHER_THREADS)
-gather_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
-              const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
-              const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
-              int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
-              GroupedOperand X, float* __restrict__ GU, int gu_ld, float* __restrict__ yacc,
-              const int32_t* __restrict__ sched, const float* __restrict__ gamma,
-              const float* __restrict__ inv_rms, int residual) {
+__global__ void __launch_bounds__(ROWS_THREADS)
+rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
+            const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
+            const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
+            int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
+            float* __restrict__ GU, int gu_ld, float* __restrict__ yacc, const int32_t* __restrict__ sched,
+            int residual) {
     pdl_launch_dependents();
     pdl_wait();
-    const int nb = d / 32;
-    const long item = static_cast<long>(blockIdx.x) * GATHER_THREADS + threadIdx.x;
-    if (item >= static_cast<long>(T) * nb) return;
-    const int t = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
-    // the k destinations first (independent load chains in flight together), encoded while they land, then the stores
-    int pos[MAX_TOPK], tile[MAX_TOPK], rloc[MAX_TOPK];
-#pragma unroll
-    for (int j = 0; j < MAX_TOPK; ++j) {
-        if (j < k) {
-            const int p = t * k + j;
-            const int e = idx[p];
-            const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
-            pos[j] = offsets[e] + loc;
-            tile[j] = tile_base[e] + loc / BN;
-            rloc[j] = loc % BN;
-        }
+    __shared__ int pos_s[ROWS_TOKENS * MAX_TOPK];
+    const int t0 = blockIdx.x * ROWS_TOKENS;
+    const int nt = min(ROWS_TOKENS, T - t0);
+    const int tid = threadIdx.x;
+    if (tid < nt * k) {
+        const int p = t0 * k + tid;
+        const int t = p / k;
+        const int e = idx[p];
+        const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+        const int pos = offsets[e] + loc;
+        row_token[pos] = t;
+        row_weight[pos] = w[p];
+        row_slot[pos] = (tile_base[e] + loc / BN) * BN + loc % BN;
+        pos_s[tid] = pos;
     }
-    float v[32];
-    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
-    {
-        // the output accumulator row starts at x (the block's skip connection) or at zero
-        float4* yz = reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d + b * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            yz[i] = residual ? make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3])
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (gamma) {
-        // pre-norm: the experts see h = x * gamma / rms(x)
-        const float r = inv_rms[t];
-        const float4* g4 = reinterpret_cast<const float4*>(gamma + b * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float4 g = g4[i];
-            v[4 * i] *= g.x * r;
-            v[4 * i + 1] *= g.y * r;
-            v[4 * i + 2] *= g.z * r;
-            v[4 * i + 3] *= g.w * r;
-        }
-    }
-    uint4 codes[MXQ_TERMS];
-    uint32_t sb[MXQ_TERMS];
-    mxq_block_thread(v, codes, sb);
-    const bool split = sched[SCHED_SPLIT_GU] > 1;
-#pragma unroll
-    for (int j = 0; j < MAX_TOPK; ++j) {
-        if (j < k) {
-            if (b == 0) {
-                row_token[pos[j]] = t;
-                row_weight[pos[j]] = w[t * k + j];
-                row_slot[pos[j]] = tile[j] * BN + rloc[j];
+    // output accumulator rows: x (residual) or zero
+    const int d4 = d / 4;
+    for (int i = tid; i < nt * d4; i += ROWS_THREADS) {
+        const int t = t0 + i / d4, c4 = i % d4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (residual) {
+            if constexpr (sizeof(TA) == 2) {
+                const uint2 r = reinterpret_cast<const uint2*>(x + static_cast<size_t>(t) * d)[c4];
+                v = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                                __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+            } else {
+                v = reinterpret_cast<const float4*>(x + static_cast<size_t>(t) * d)[c4];
             }
-            uint8_t* atoms = scale_atom_base(X, tile[j], b >> 2);
+        }
+        reinterpret_cast<float4*>(yacc + static_cast<size_t>(t) * d)[c4] = v;
+    }
+    if (sched[SCHED_SPLIT_GU] > 1) {
+        __syncthreads();
+        const int g4 = gu_ld / 4;
+        for (int i = tid; i < nt * k * g4; i += ROWS_THREADS)
+            reinterpret_cast<float4*>(GU + static_cast<size_t>(pos_s[i / g4]) * gu_ld)[i % g4] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// Grouping, part 2: the B operand of the gate/up GEMM.  One CTA per (token
+// tile, K chunk of 128), chunk-major over the grid (blockIdx.x = tile), so the
+// CTAs running together read one 128-wide column slice of x, which stays in
+// L2 while every tile that needs it reads it.  Thread r encodes blocks
+// 4c .. 4c+3 of the tile's row r (x of its token, times gamma / rms(x) with
+// the pre-norm) as three MXFP4 terms: the codes go straight to global memory
+// (consecutive threads, consecutive rows: coalesced), the scale bytes into a
+// shared-memory copy of the tile's scale atoms, which the CTA then writes
+// whole (rows past the tile's valid rows get zero scale bytes).
+constexpr int ENC_THREADS = 128;
+template <typename TA>
+__global__ void __launch_bounds__(ENC_THREADS)
+encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, const float* __restrict__ inv_rms,
+                   const int32_t* __restrict__ row_token, const int4* __restrict__ units_gu,
+                   const int32_t* __restrict__ sched, int F_gu, int d, GroupedOperand X) {
+    pdl_launch_dependents();
+    pdl_wait();
+    __shared__ __align__(16) uint8_t atoms[MXQ_TERMS * 512];
+    const int tile = blockIdx.x, c = blockIdx.y;
+    const int S = sched[SCHED_SPLIT_GU];
+    const long u = static_cast<long>(tile) * F_gu * S;
+    if (u >= sched[SCHED_UNITS_GU]) return;
+    const int4 U = units_gu[u];
+    const int row0 = U.y, nvalid = U.z;
+    const int tid = threadIdx.x;
+    for (int i = tid; i < MXQ_TERMS * 512 / 16; i += ENC_THREADS)
+        reinterpret_cast<uint4*>(atoms)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    if (tid < nvalid) {
+        const int row = row0 + tid;
+        const int t = row_token[row];
+        const int nb = d / 32;
+        const float r = gamma ? inv_rms[t] : 1.f;
+        for (int q = 0; q < 4 && 4 * c + q < nb; ++q) {
+            const int b = 4 * c + q;
+            float v[32];
+            BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+            if (gamma) {
+                const float4* g4 = reinterpret_cast<const float4*>(gamma + b * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 g = g4[i];
+                    v[4 * i] *= g.x * r;
+                    v[4 * i + 1] *= g.y * r;
+                    v[4 * i + 2] *= g.z * r;
+                    v[4 * i + 3] *= g.w * r;
+                }
+            }
+            uint4 codes[MXQ_TERMS];
+            uint32_t sb[MXQ_TERMS];
+            mxq_block_thread(v, codes, sb);
 #pragma unroll
             for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + pos[j]) * 16) =
+                *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + row) * 16) =
                     codes[tt];
-                atoms[sf_atom_offset(tt * X.term_rows + rloc[j], b & 3)] = static_cast<uint8_t>(sb[tt]);
-            }
-            if (split) {
-                // the token's nb threads zero the row together (consecutive floats per step)
-                float* g = GU + static_cast<size_t>(pos[j]) * gu_ld;
-                for (int i = b; i < gu_ld; i += nb) g[i] = 0.f;
+                atoms[sf_atom_offset(tt * X.term_rows + tid, q)] = static_cast<uint8_t>(sb[tt]);
             }
         }
     }
+    __syncthreads();
+    uint4* dst = reinterpret_cast<uint4*>(scale_atom_base(X, tile, c));
+    for (int i = tid; i < MXQ_TERMS * 512 / 16; i += ENC_THREADS) dst[i] = reinterpret_cast<const uint4*>(atoms)[i];
 }
 
 __device__ __forceinline__ float swish_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
