@@ -222,12 +222,15 @@ static TiledMatrix tiled(moe_mxfp4* h, int which) {
     return M;
 }
 
-// K splits of the router: enough CTAs to cover the SMs once, at most
-// ROUTER_MAX_SPLITS (the last CTA of a token tile sums the splits' partials).
-static int router_splits(int T, int d, int nsm) {
+// K splits of the router: enough CTAs (token tiles x expert tiles x splits) to
+// cover the SMs twice, at most ROUTER_MAX_SPLITS and one 64-wide K chunk per
+// split (the last CTA of a token tile sums the splits' partials).
+static int router_etiles(int E) { return (E + ROUTER_ETILE - 1) / ROUTER_ETILE; }
+static int router_splits(int T, int d, int E, int nsm) {
     const int tiles = (T + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
     const int kch = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
-    const int want = (nsm + tiles - 1) / tiles;
+    const int ctas = tiles * router_etiles(E);
+    const int want = (2 * nsm + ctas - 1) / ctas;
     return std::max(1, std::min(std::min(kch, ROUTER_MAX_SPLITS), want));
 }
 
@@ -261,7 +264,7 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     if (dev < 0 || dev >= MOE_MAX_DEVICES) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_attr_mutex);
     if (g_attrs_set[dev]) return cudaSuccess;
-    const int rsm = static_cast<int>(router_smem_bytes(MAX_EXPERTS));
+    const int rsm = static_cast<int>(router_smem_bytes());
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
         return e;
@@ -357,7 +360,8 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         h->max_units = static_cast<int>(tiles * F + 8L * h->nsm + 64);
     }
     h->gu_rows = std::min(h->TK, SPLIT_ROWS_CAP);
-    h->part_elems = static_cast<size_t>(64 * h->nsm + ROUTER_TOKENS * h->nblk_max + ROUTER_TOKENS) * E;
+    // partial scores [S][T][E]: S * T <= ROUTER_TOKENS * (S * tiles) <= ROUTER_TOKENS * (2 nsm + tiles)
+    h->part_elems = static_cast<size_t>(ROUTER_TOKENS) * (2 * h->nsm + h->nblk_max + 1) * E;
     h->expert_done = new (std::nothrow) bool[E]();
     if (!h->expert_done) return fail(MOE_ERR_CUDA);
 
@@ -707,7 +711,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.d = d;
     ra.E = E;
     ra.k = k;
-    ra.S = router_splits(T, d, h->nsm);
+    ra.S = router_splits(T, d, E, h->nsm);
     ra.part = h->part;
     ra.gamma = h->use_norm ? h->gamma : nullptr;
     ra.eps = h->eps;
@@ -733,8 +737,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.units_gu = h->units_gu;
     ra.units_dn = h->units_dn;
     ra.sched = h->sched;
-    const size_t rsm = router_smem_bytes(E);
-    const dim3 rgrid(nblk, ra.S);
+    const size_t rsm = router_smem_bytes();
+    const dim3 rgrid(nblk, ra.S, router_etiles(E));
     if (bf16)
         launch_router<__nv_bfloat16>(ra, rgrid, rsm, stream);
     else
@@ -937,7 +941,7 @@ moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n) {
 // address comes from cudaGetSymbolAddress, looked up once per device.
 namespace {
 
-constexpr int NOALLOC_MAX_SPLITS = ROUTER_MAX_SPLITS;
+constexpr int NOALLOC_MAX_SPLITS = 8;
 constexpr size_t NOALLOC_PART_BYTES = sizeof(double) * NOALLOC_MAX_SPLITS * MOE_ROUTE_NOALLOC_MAX_TOKENS *
                                       MOE_ROUTE_NOALLOC_MAX_EXPERTS;
 constexpr int NOALLOC_MAX_TILES = (MOE_ROUTE_NOALLOC_MAX_TOKENS + ROUTER_TOKENS - 1) / ROUTER_TOKENS;
@@ -1017,7 +1021,7 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     ra.d = d_model;
     ra.E = n_experts;
     ra.k = top_k;
-    ra.S = std::min(NOALLOC_MAX_SPLITS, router_splits(T, d_model, nd->nsm));
+    ra.S = std::min(NOALLOC_MAX_SPLITS, router_splits(T, d_model, n_experts, nd->nsm));
     ra.part = reinterpret_cast<double*>(sc + NA_OFF_PART);
     ra.tile_cnt = counters;
     ra.glob_cnt = counters + tiles;
@@ -1041,8 +1045,8 @@ extern "C" moe_status_t moe_mxfp4_route_noalloc(const void* x, const void* w_rou
     ra.units_gu = nullptr;
     ra.units_dn = nullptr;
     ra.sched = reinterpret_cast<int32_t*>(sc + NA_OFF_SCHED);
-    const dim3 grid(tiles, ra.S);
-    const size_t smem = router_smem_bytes(n_experts);
+    const dim3 grid(tiles, ra.S, router_etiles(n_experts));
+    const size_t smem = router_smem_bytes();
     if (act_dtype == MOE_DTYPE_BF16)
         launch_router<__nv_bfloat16>(ra, grid, smem, stream);
     else

@@ -16,7 +16,7 @@
 
 namespace moe {
 
-constexpr int ROUTER_TOKENS = 32;   // tokens per router tile
+constexpr int ROUTER_TOKENS = 128;  // tokens per router tile
 constexpr int ROUTER_THREADS = 256;
 constexpr int ROUTER_KCHUNK = 64;
 constexpr int MAX_EXPERTS = 256;
@@ -47,17 +47,18 @@ template <> struct Raw8<float> {
     }
 };
 
-// Dynamic shared memory of router_kernel (floats): x chunk [32][65], router
-// chunk [64][E], scores [32][E+1].
-constexpr int ROUTER_MAX_SPLITS = 8;
-__host__ __device__ inline size_t router_smem_bytes(int E) {
-    return sizeof(float) * (static_cast<size_t>(ROUTER_TOKENS) * ROUTER_KCHUNK +
-                            static_cast<size_t>(ROUTER_KCHUNK) * E + static_cast<size_t>(ROUTER_TOKENS) * (E + 1));
+// Router tiles: ROUTER_TOKENS tokens x ROUTER_ETILE experts per CTA (grid.z
+// covers the experts), K split over grid.y.  Dynamic shared memory: the x chunk
+// transposed [64 k][128 tokens] and the router chunk [64 k][32 experts], fp32;
+// the top-k tail reuses it for the scores of 32 tokens [32][E + 1].
+constexpr int ROUTER_ETILE = 32;
+constexpr int ROUTER_MAX_SPLITS = 16;
+constexpr int ROUTER_SUB = 32;   // tokens per pass of the top-k tail
+__host__ __device__ constexpr size_t router_smem_bytes() {
+    return sizeof(float) * (static_cast<size_t>(ROUTER_KCHUNK) * ROUTER_TOKENS +
+                            static_cast<size_t>(ROUTER_KCHUNK) * ROUTER_ETILE);
 }
-// Column of token t in row kk of the transposed x chunk: an XOR swizzle that
-// keeps each group of 4 tokens contiguous (one 16-byte read) and spreads the
-// rows a warp writes over all 32 banks.
-__device__ __forceinline__ int xs_col(int kk, int t) { return t ^ (4 * ((kk >> 3) & 7)); }
+static_assert(sizeof(float) * ROUTER_SUB * (MAX_EXPERTS + 1) <= router_smem_bytes(), "top-k scores must fit");
 
 // Schedule slots.
 enum : int {
@@ -211,23 +212,27 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
     }
 }
 
-// Grid (tiles of 32 tokens, S splits of K).  Each CTA accumulates the scores of
-// its 32 tokens x E experts over its K range: fp32 within a 64-wide chunk
-// staged in shared memory (bf16 x bf16 products are exact in fp32), fp64
-// across chunks.  The last CTA of a tile to finish sums the S partials in split
-// order (deterministic), adds the bias, and with one warp per token selects
-// the top-k by k rounds of warp arg-max (ties to the lower index) and applies
-// the softmax over the k selected scores; it also ranks the tile's (token,
-// slot) pairs within their expert and writes the tile histogram.  The last
-// tile to finish builds the schedule (schedule_block).
-// EPT = experts per lane (ceil(E / 32) rounded up to 1, 2, 4 or 8): the
-// register tile scales with the expert count.
+// Grid (token tiles of 128, S splits of K, expert tiles of 32).  Each CTA
+// accumulates the scores of its 128 tokens x 32 experts over its K range:
+// each thread holds a 4-token x 4-expert register tile, fp32 within a 64-wide
+// K chunk staged in shared memory (bf16 x bf16 products are exact in fp32),
+// fp64 across chunks; the next chunk is loaded into registers while the
+// current one is multiplied.  With the pre-norm the staged router chunk is
+// W_router * gamma (so the scores are of x * gamma) and the sum of x^2 per
+// token is kept (by the expert tile 0 CTAs).  The last CTA of a token tile to
+// finish sums the S partials in split order (deterministic), scales by the
+// inverse RMS, adds the bias, and for 32 tokens at a time selects the top-k
+// with one warp per token by k rounds of warp arg-max (ties to the lower
+// index) and applies the softmax over the k selected scores; it then ranks
+// the tile's (token, slot) pairs within their expert and writes the tile
+// histogram.  The last tile to finish builds the schedule (schedule_block).
+// EPT = experts per lane in the top-k (ceil(E / 32) rounded up to 1, 2, 4, 8).
 template <typename TA, int EPT>
 __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
     extern __shared__ __align__(16) float rsm[];
-    float* xs = rsm;                                      // [64 k][32 tokens], swizzled (xs_col)
-    float* ws = xs + ROUTER_TOKENS * ROUTER_KCHUNK;        // [64 k][E]
-    float* lg = ws + ROUTER_KCHUNK * a.E;                  // [32][E+1]
+    float* xs = rsm;                                        // [64 k][128 tokens]
+    float* ws = xs + ROUTER_KCHUNK * ROUTER_TOKENS;         // [64 k][32 experts]
+    float* lg = rsm;                                        // tail: [32 tokens][E + 1]
     __shared__ int hist_s[MAX_EXPERTS];
     __shared__ int es[ROUTER_TOKENS * MAX_TOPK];
     __shared__ int cnt_s[MAX_EXPERTS];
@@ -235,212 +240,190 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     __shared__ int tb_s[MAX_EXPERTS + 1];
     __shared__ int split_s[2];
     __shared__ int last_s;
+    __shared__ double ss_s[ROUTER_TOKENS];
+    __shared__ double inv_s[ROUTER_TOKENS];
 
     pdl_launch_dependents();
     const TA* x = static_cast<const TA*>(a.x);
     const TA* wr = static_cast<const TA*>(a.wr);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = a.E, d = a.d, k = a.k;
-    const int tile = blockIdx.x, split = blockIdx.y;
+    const int tile = blockIdx.x, split = blockIdx.y, e0 = blockIdx.z * ROUTER_ETILE;
     const int ntiles = gridDim.x;
     const int t0 = tile * ROUTER_TOKENS;
     const int ntok = min(ROUTER_TOKENS, a.T - t0);
     const int KCH = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
     const int kc0 = split * KCH / a.S, kc1 = (split + 1) * KCH / a.S;
-
-    double tot[EPT][4];
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
-
-    // Each thread owns one 8-element group of the x chunk (token tid/8) and EPT
-    // groups of the router chunk (group idx = tid + 256 i: expert idx % 32*EPT,
-    // K offset 8 * (idx / 32*EPT), so the transposed shared-memory stores of
-    // consecutive threads hit consecutive banks); the next chunk is loaded into
-    // registers while the current one is multiplied.
-    constexpr int EP = 32 * EPT;              // expert slots covered by the register tile
-    const int xt = tid >> 3, xv8 = (tid & 7) * 8;
-    Raw8<TA> xr, wrr[EPT];
-    // pre-norm: the staged chunk holds x * gamma; the sum of x^2 over the
-    // split's K range is kept per token (the last CTA divides by the RMS)
     const bool norm = a.gamma != nullptr;
+
+    // staging roles: x -- token tid % 128, K half tid / 128 (32 values);
+    // router -- expert tid % 32, K eighth tid / 32 (8 values)
+    const int xt = tid & (ROUTER_TOKENS - 1), xh = (tid >> 7) * 32;
+    const int we = tid & 31, wk = (tid >> 5) * 8;
+    // compute roles: tokens 4 tq .. 4 tq + 3, experts 4 eq .. 4 eq + 3
+    const int tq = tid >> 3, eq = tid & 7;
+    Raw8<TA> xr[4], wv;
     float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
-    double ss = 0.0;
     auto load_chunk = [&](int kc) {
-        if (xt < ntok && kc + xv8 < d) xr.load(x + static_cast<size_t>(t0 + xt) * d + kc + xv8);
-        else xr.zero();
-        if (norm && kc + xv8 < d) {
-            g0 = *reinterpret_cast<const float4*>(a.gamma + kc + xv8);
-            g1 = *reinterpret_cast<const float4*>(a.gamma + kc + xv8 + 4);
-        }
 #pragma unroll
-        for (int i = 0; i < EPT; ++i) {
-            const int idx = tid + ROUTER_THREADS * i;
-            const int e = idx % EP, k8 = (idx / EP) * 8;
-            if (e < E && k8 < ROUTER_KCHUNK && kc + k8 < d) wrr[i].load(wr + static_cast<size_t>(e) * d + kc + k8);
-            else wrr[i].zero();
+        for (int i = 0; i < 4; ++i) {
+            const int kk = kc + xh + 8 * i;
+            if (xt < ntok && kk < d) xr[i].load(x + static_cast<size_t>(t0 + xt) * d + kk);
+            else xr[i].zero();
+        }
+        const int kk = kc + wk;
+        if (e0 + we < E && kk < d) {
+            wv.load(wr + static_cast<size_t>(e0 + we) * d + kk);
+            if (norm) {
+                g0 = *reinterpret_cast<const float4*>(a.gamma + kk);
+                g1 = *reinterpret_cast<const float4*>(a.gamma + kk + 4);
+            }
+        } else {
+            wv.zero();
         }
     };
+
+    double tot[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
+    double ss = 0.0;
+
     if (kc0 < kc1) load_chunk(kc0 * ROUTER_KCHUNK);
     for (int c = kc0; c < kc1; ++c) {
         const int kc = c * ROUTER_KCHUNK;
         __syncthreads();
-        if (norm) {
-            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            float sq = 0.f;
+        float sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float v = xr.get(j);
+                const float v = xr[i].get(j);
                 sq = fmaf(v, v, sq);
-                xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = v * gv[j];
+                xs[(xh + 8 * i + j) * ROUTER_TOKENS + xt] = v;
             }
-            ss += static_cast<double>(sq);
-        } else {
+        ss += static_cast<double>(sq);
+        {
+            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) xs[(xv8 + j) * ROUTER_TOKENS + xs_col(xv8 + j, xt)] = xr.get(j);
-        }
-#pragma unroll
-        for (int i = 0; i < EPT; ++i) {
-            const int idx = tid + ROUTER_THREADS * i;
-            const int e = idx % EP, k8 = (idx / EP) * 8;
-            if (e < E && k8 < ROUTER_KCHUNK) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) ws[(k8 + j) * E + e] = wrr[i].get(j);
-            }
+            for (int j = 0; j < 8; ++j) ws[(wk + j) * ROUTER_ETILE + we] = norm ? wv.get(j) * gv[j] : wv.get(j);
         }
         __syncthreads();
         if (c + 1 < kc1) load_chunk(kc + ROUTER_KCHUNK);
-        float acc[EPT][4];
+        float acc[4][4];
 #pragma unroll
-        for (int i = 0; i < EPT; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 #pragma unroll 8
         for (int kk = 0; kk < ROUTER_KCHUNK; ++kk) {
-            // x of the warp's 4 tokens at kk: one broadcast 16-byte read
-            const float4 x4 = *reinterpret_cast<const float4*>(xs + kk * ROUTER_TOKENS + xs_col(kk, warp * 4));
-            const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+            const float4 xv = *reinterpret_cast<const float4*>(xs + kk * ROUTER_TOKENS + 4 * tq);
+            const float4 wv4 = *reinterpret_cast<const float4*>(ws + kk * ROUTER_ETILE + 4 * eq);
+            const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+            const float wa[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
 #pragma unroll
-            for (int i = 0; i < EPT; ++i) {
-                const int e = lane + 32 * i;
-                const float wv = (e < E) ? ws[kk * E + e] : 0.f;
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(wv, xv[j], acc[i][j]);
-            }
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
         }
 #pragma unroll
-        for (int i = 0; i < EPT; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) tot[i][j] += static_cast<double>(acc[i][j]);
     }
-    if (norm) {
-        // the token's 8 threads are lanes 8m .. 8m+7 of one warp
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-        if ((tid & 7) == 0 && xt < ntok) a.part_ss[static_cast<size_t>(split) * a.T + t0 + xt] = ss;
-    }
     // partial scores of this split
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E) {
+    for (int i = 0; i < 4; ++i) {
+        const int tl = 4 * tq + i;
+        if (tl < ntok) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int tl = warp * 4 + j;
-                if (tl < ntok) a.part[(static_cast<size_t>(split) * a.T + t0 + tl) * E + e] = tot[i][j];
+                const int e = e0 + 4 * eq + j;
+                if (e < E) a.part[(static_cast<size_t>(split) * a.T + t0 + tl) * E + e] = tot[i][j];
             }
         }
     }
+    if (norm && blockIdx.z == 0) {
+        // the token's two K halves are threads xt and xt + 128
+        if (tid >= ROUTER_TOKENS) ss_s[xt] = ss;
+        __syncthreads();
+        if (tid < ROUTER_TOKENS && xt < ntok) a.part_ss[static_cast<size_t>(split) * a.T + t0 + xt] = ss + ss_s[xt];
+    }
     __threadfence();
     __syncthreads();
-    if (tid == 0) last_s = (atomicAdd(a.tile_cnt + tile, 1) == a.S - 1);
+    if (tid == 0) last_s = (atomicAdd(a.tile_cnt + tile, 1) == a.S * static_cast<int>(gridDim.z) - 1);
     __syncthreads();
     if (!last_s) return;
     __threadfence();
     if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
 
     for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
-    __shared__ double inv_s[ROUTER_TOKENS];
-    if (norm && tid < ntok) {
-        double sq = 0.0;
-        for (int sp = 0; sp < a.S; ++sp) sq += __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid);
-        const double inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
+    if (tid < ntok) {
+        double inv = 1.0;
+        if (norm) {
+            double sq = 0.0;
+            for (int sp = 0; sp < a.S; ++sp) sq += __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid);
+            inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
+            a.inv_rms[t0 + tid] = static_cast<float>(inv);
+        }
         inv_s[tid] = inv;
-        a.inv_rms[t0 + tid] = static_cast<float>(inv);
     }
-    __syncthreads();
-    {
-        // logits = partials summed in split order (deterministic) + bias; each
-        // thread takes 2 outputs with all their partial loads in flight
-        const size_t pstride = static_cast<size_t>(a.T) * E;
-        for (int i0 = tid; i0 < ntok * E; i0 += 2 * ROUTER_THREADS) {
-            double pv[2][ROUTER_MAX_SPLITS];
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int i = i0 + m * ROUTER_THREADS;
-                const double* pp = a.part + static_cast<size_t>(t0 + i / E) * E + i % E;
-#pragma unroll
-                for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
-                    pv[m][sp] = (i < ntok * E && sp < a.S) ? __ldcg(pp + sp * pstride) : 0.0;
-            }
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int i = i0 + m * ROUTER_THREADS;
-                if (i < ntok * E) {
-                    double s = 0.0;
-#pragma unroll
-                    for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) s += pv[m][sp];
-                    const int tl = i / E, e = i % E;
-                    if (norm) s *= inv_s[tl];
-                    if (a.bias) s += a.bias[e];
-                    lg[tl * (E + 1) + e] = static_cast<float>(s);
-                }
-            }
+    const size_t pstride = static_cast<size_t>(a.T) * E;
+    for (int sub = 0; sub < ntok; sub += ROUTER_SUB) {
+        const int nsub = min(ROUTER_SUB, ntok - sub);
+        __syncthreads();
+        // scores = partials summed in split order (deterministic), x inverse RMS, + bias
+        for (int i = tid; i < nsub * E; i += ROUTER_THREADS) {
+            const int tl = i / E, e = i % E;
+            const double* pp = a.part + static_cast<size_t>(t0 + sub + tl) * E + e;
+            double sv = 0.0;
+            for (int sp = 0; sp < a.S; ++sp) sv += __ldcg(pp + sp * pstride);
+            if (norm) sv *= inv_s[sub + tl];
+            if (a.bias) sv += a.bias[e];
+            lg[tl * (E + 1) + e] = static_cast<float>(sv);
         }
-    }
-    __syncthreads();
-
-    // top-k + softmax: warp w handles tokens 4w .. 4w+3
-    for (int j = 0; j < 4; ++j) {
-        const int tl = warp * 4 + j;
-        if (tl >= ntok) break;
-        const float* row = lg + tl * (E + 1);
-        uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-        float sel_v[MAX_TOPK];
-        int sel_e[MAX_TOPK];
-        for (int r = 0; r < k; ++r) {
-            float bv = -INFINITY;
-            int be = 0x7FFFFFFF;
-            for (int i = 0; i < EPT; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E && !((taken >> i) & 1u)) {
-                    const float v = row[e];
-                    if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            sel_v[r] = bv;
-            sel_e[r] = be;
-        }
-        if (lane == 0) {
-            const float m = sel_v[0];
-            float den = 0.f;
-            for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
-            const float inv = 1.f / den;
-            const int t = t0 + tl;
+        __syncthreads();
+        // top-k + softmax: warp w handles tokens sub + 4w .. sub + 4w + 3
+        for (int j = 0; j < 4; ++j) {
+            const int tl = warp * 4 + j;
+            if (tl >= nsub) break;
+            const float* row = lg + tl * (E + 1);
+            uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
+            float sel_v[MAX_TOPK];
+            int sel_e[MAX_TOPK];
             for (int r = 0; r < k; ++r) {
-                a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
-                a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
-                es[tl * k + r] = sel_e[r];
+                float bv = -INFINITY;
+                int be = 0x7FFFFFFF;
+                for (int i = 0; i < EPT; ++i) {
+                    const int e = lane + 32 * i;
+                    if (e < E && !((taken >> i) & 1u)) {
+                        const float v = row[e];
+                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+                }
+                be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                sel_v[r] = bv;
+                sel_e[r] = be;
+            }
+            if (lane == 0) {
+                const float m = sel_v[0];
+                float den = 0.f;
+                for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+                const float inv = 1.f / den;
+                const int t = t0 + sub + tl;
+                for (int r = 0; r < k; ++r) {
+                    a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
+                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
+                    es[(sub + tl) * k + r] = sel_e[r];
+                }
             }
         }
     }
