@@ -44,7 +44,8 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,   /* valid but outside the supported envelope  */
     MOE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
     MOE_ERR_NOT_QUANTIZED = 4, /* forward before quantize_weights            */
-    MOE_ERR_TIMEOUT = 5        /* a device-side pipeline wait ran out        */
+    MOE_ERR_TIMEOUT = 5,       /* a device-side pipeline wait ran out        */
+    MOE_ERR_BOUNDS = 6         /* debug build: an index check failed or a guard region changed */
 } moe_status_t;
 
 typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
@@ -198,8 +199,26 @@ moe_status_t moe_mxfp4_get_grouping(const moe_mxfp4_t* h, int32_t* offsets, int3
                                     float* row_weight, cudaStream_t stream);
 
 /* Synchronise the handle's last stream and return (and clear) the device
- * status: MOE_OK, or MOE_ERR_TIMEOUT if a pipeline wait ran out. */
+ * status: MOE_OK, MOE_ERR_TIMEOUT if a pipeline wait ran out, or (debug
+ * build) MOE_ERR_BOUNDS if an index check failed. */
 moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h);
+
+/* Debug build (the library compiled with MOE_DEBUG_CHECKS,
+ * libmoe_mxfp4_debug.so): every device buffer a handle owns is followed by a
+ * 4096-byte guard region of a fixed pattern, and the kernels check the
+ * indices they scatter and gather through (grouped rows, token tiles, units,
+ * tokens of the combine); a failed check skips the access and makes
+ * moe_mxfp4_get_status return MOE_ERR_BOUNDS.  This call synchronises the
+ * device and returns MOE_ERR_BOUNDS if any guard byte changed, else MOE_OK.
+ * In the release library it returns MOE_ERR_UNSUPPORTED.  No counterpart on
+ * the pages: a debugging aid. */
+moe_status_t moe_mxfp4_check_guards(moe_mxfp4_t* h);
+
+/* Test hook of the debug build: overwrite one byte of the i-th guard region
+ * (from the host), so the detection of moe_mxfp4_check_guards can be tested
+ * without any kernel writing out of bounds.  UNSUPPORTED in the release
+ * library; INVALID_ARG for an i past the handle's guard regions. */
+moe_status_t moe_mxfp4_test_write_guard(moe_mxfp4_t* h, int32_t i);
 
 /* Static description of a status code. */
 const char* moe_mxfp4_status_string(moe_status_t s);

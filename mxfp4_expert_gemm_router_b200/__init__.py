@@ -18,7 +18,8 @@ from typing import Optional
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe_mxfp4.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_NOT_QUANTIZED, MOE_ERR_TIMEOUT = range(6)
+(MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_NOT_QUANTIZED, MOE_ERR_TIMEOUT,
+ MOE_ERR_BOUNDS) = range(7)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 MOE_FLAG_TEST_SKIP_FIRST_COPY = 1 << 30
 MOE_FLAG_TOKEN_TILE_SHIFT = 8
@@ -70,16 +71,17 @@ SIGNATURES = {
     "moe_mxfp4_expert_param_count": (ctypes.c_int64, [ctypes.POINTER(moe_mxfp4_config_t)]),
     "moe_mxfp4_expert_weight_bytes": (ctypes.c_int64, [ctypes.POINTER(moe_mxfp4_config_t)]),
     "moe_mxfp4_route_noalloc": (_ST, [_VP, _VP, _VP, _I32, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP]),
+    "moe_mxfp4_check_guards": (_ST, [_VP]),
+    "moe_mxfp4_test_write_guard": (_ST, [_VP, _I32]),
 }
 
+DEBUG_LIB_PATH = os.path.join(HERE, "libmoe_mxfp4_debug.so")
+
 _lib = None
+_debug_lib = None
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load the C-ABI library (raises RuntimeError if it is missing)."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def _open(path: str) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise RuntimeError(f"{path} not found: build it with mxfp4_expert_gemm_router_b200.build.build()")
     try:
@@ -90,8 +92,24 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
-    _lib = L
     return L
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the C-ABI library (raises RuntimeError if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    _lib = _open(path)
+    return _lib
+
+
+def load_debug(path: str = DEBUG_LIB_PATH) -> ctypes.CDLL:
+    """Load the debug build of the library (index checks, guard regions)."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _open(path)
+    return _debug_lib
 
 
 def __getattr__(name):
@@ -148,16 +166,18 @@ class MoeMxfp4:
     """One layer handle.  Tensors are torch CUDA tensors on the handle's device."""
 
     def __init__(self, d_model, d_ff, n_experts, top_k, max_tokens, act_dtype="bf16", flags=0,
-                 wait_timeout_ms=0):
+                 wait_timeout_ms=0, lib=None):
+        """`lib`: the library to drive (default the release build; load_debug() for the debug build)."""
+        self._L = lib if lib is not None else load()
         self.cfg = make_config(d_model, d_ff, n_experts, top_k, max_tokens, act_dtype, flags, wait_timeout_ms)
         self.act_dtype = act_dtype
         h = ctypes.c_void_p()
-        check(load().moe_mxfp4_create(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_mxfp4_create")
+        check(self._L.moe_mxfp4_create(ctypes.byref(self.cfg), ctypes.byref(h)), "moe_mxfp4_create")
         self.h = h
 
     def close(self):
         if getattr(self, "h", None) is not None and self.h.value:
-            load().moe_mxfp4_destroy(self.h)
+            self._L.moe_mxfp4_destroy(self.h)
             self.h = None
 
     def __del__(self):
@@ -167,48 +187,51 @@ class MoeMxfp4:
             pass
 
     def quantize_weights(self, w_gate, w_up, w_down, w_router, router_bias=None, stream=None):
-        check(load().moe_mxfp4_quantize_weights(self.h, _p(w_gate), _p(w_up), _p(w_down), _p(w_router),
+        check(self._L.moe_mxfp4_quantize_weights(self.h, _p(w_gate), _p(w_up), _p(w_down), _p(w_router),
                                                 _p(router_bias), _stream(stream)), "quantize_weights")
 
     def quantize_expert(self, e, w_gate, w_up, w_down, stream=None):
-        check(load().moe_mxfp4_quantize_expert(self.h, int(e), _p(w_gate), _p(w_up), _p(w_down),
+        check(self._L.moe_mxfp4_quantize_expert(self.h, int(e), _p(w_gate), _p(w_up), _p(w_down),
                                                _stream(stream)), "quantize_expert")
 
     def set_router(self, w_router, router_bias=None, stream=None):
-        check(load().moe_mxfp4_set_router(self.h, _p(w_router), _p(router_bias), _stream(stream)), "set_router")
+        check(self._L.moe_mxfp4_set_router(self.h, _p(w_router), _p(router_bias), _stream(stream)), "set_router")
 
     def set_norm_residual(self, gamma=None, eps=1e-5, residual=False, stream=None):
-        check(load().moe_mxfp4_set_norm_residual(self.h, _p(gamma), float(eps), 1 if residual else 0,
+        check(self._L.moe_mxfp4_set_norm_residual(self.h, _p(gamma), float(eps), 1 if residual else 0,
                                                  _stream(stream)), "set_norm_residual")
 
     def forward(self, x, y, topk_idx=None, topk_w=None, expert_counts=None, stream=None):
         T = int(x.shape[0]) if x is not None else 0
-        check(load().moe_mxfp4_forward(self.h, _p(x), T, _p(y), _p(topk_idx), _p(topk_w), _p(expert_counts),
+        check(self._L.moe_mxfp4_forward(self.h, _p(x), T, _p(y), _p(topk_idx), _p(topk_w), _p(expert_counts),
                                        _stream(stream)), "forward")
 
     def forward_host(self, x_host, y_host, topk_idx_host=None, topk_w_host=None, stream=None):
         T = int(x_host.shape[0])
-        check(load().moe_mxfp4_forward_host(self.h, _p(x_host), T, _p(y_host), _p(topk_idx_host),
+        check(self._L.moe_mxfp4_forward_host(self.h, _p(x_host), T, _p(y_host), _p(topk_idx_host),
                                             _p(topk_w_host), _stream(stream)), "forward_host")
 
     def export_weights(self, which, codes, scales, stream=None):
-        check(load().moe_mxfp4_export_weights(self.h, int(which), _p(codes), _p(scales), _stream(stream)),
+        check(self._L.moe_mxfp4_export_weights(self.h, int(which), _p(codes), _p(scales), _stream(stream)),
               "export_weights")
 
     def get_grouping(self, offsets, row_token=None, row_weight=None, stream=None):
-        check(load().moe_mxfp4_get_grouping(self.h, _p(offsets), _p(row_token), _p(row_weight),
+        check(self._L.moe_mxfp4_get_grouping(self.h, _p(offsets), _p(row_token), _p(row_weight),
                                             _stream(stream)), "get_grouping")
 
     def status(self) -> int:
-        return load().moe_mxfp4_get_status(self.h)
+        return self._L.moe_mxfp4_get_status(self.h)
 
     def set_profiling(self, enable: bool):
-        check(load().moe_mxfp4_set_profiling(self.h, 1 if enable else 0), "set_profiling")
+        check(self._L.moe_mxfp4_set_profiling(self.h, 1 if enable else 0), "set_profiling")
 
     def kernel_times(self):
         buf = (ctypes.c_float * MOE_NUM_STAGES)()
-        check(load().moe_mxfp4_kernel_times(self.h, buf, MOE_NUM_STAGES), "kernel_times")
-        return {load().moe_mxfp4_stage_name(i).decode(): float(buf[i]) for i in range(MOE_NUM_STAGES)}
+        check(self._L.moe_mxfp4_kernel_times(self.h, buf, MOE_NUM_STAGES), "kernel_times")
+        return {self._L.moe_mxfp4_stage_name(i).decode(): float(buf[i]) for i in range(MOE_NUM_STAGES)}
 
     def launch_count(self) -> int:
-        return int(load().moe_mxfp4_launch_count(self.h))
+        return int(self._L.moe_mxfp4_launch_count(self.h))
+
+    def check_guards(self) -> int:
+        return self._L.moe_mxfp4_check_guards(self.h)

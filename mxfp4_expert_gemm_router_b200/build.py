@@ -14,22 +14,35 @@ DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(
     os.path.join(ROOT, "include", "moe_mxfp4.h")]
 
 
+DEBUG_LIB = os.path.join(HERE, "libmoe_mxfp4_debug.so")
+
+
 def nvcc_cmd(out, extra=()):
     return [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
             "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
             "-I", os.path.join(ROOT, "include"), "-o", out, *SOURCES, *extra]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in DEPS)):
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    extra = ("-Xptxas", "-v") if verbose else ()
+def _build_one(lib: str, force: bool, extra) -> str:
+    if (not force and os.path.exists(lib)
+            and os.path.getmtime(lib) >= max(os.path.getmtime(p) for p in DEPS)):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
     subprocess.check_call(nvcc_cmd(tmp, extra))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """The release library (the product path)."""
+    return _build_one(LIB, force, ("-Xptxas", "-v") if verbose else ())
+
+
+def build_debug(force: bool = False) -> str:
+    """The same sources with device index checks and guard regions (MOE_DEBUG_CHECKS)."""
+    return _build_one(DEBUG_LIB, force, ("-DMOE_DEBUG_CHECKS",))
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build_debug(force="--force" in sys.argv))

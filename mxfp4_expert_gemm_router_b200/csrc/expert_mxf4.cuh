@@ -83,7 +83,23 @@ struct MxgParams {
     int* status;
     uint64_t timeout_ns;
     uint32_t skip_first_copy; // test hook: producer skips its first copy
+    int n_experts, T, tiles_cap;   // bounds of the unit fields (checked in the debug build)
 };
+
+// Debug build: a unit whose fields are out of range is skipped by every role
+// (the same decision everywhere, so no wait is left unmatched) and recorded.
+__device__ __forceinline__ bool mxg_unit_ok(const MxgParams& p, const int4& U, int nsplit, bool record) {
+#ifdef MOE_DEBUG_CHECKS
+    const int e = U.x & 0xFF, tile = U.x >> 8, ft = U.w & 0xFFFF, sp = U.w >> 16;
+    const bool ok = e < p.n_experts && tile >= 0 && tile < p.tiles_cap && ft < p.M.tiles() && sp < nsplit &&
+                    U.y >= 0 && U.z > 0 && U.z <= p.BN && U.y + U.z <= p.Hd.R;
+    if (!ok && record) atomicOr(p.status, DEV_BOUNDS);
+    return ok;
+#else
+    (void)p; (void)U; (void)nsplit; (void)record;
+    return true;
+#endif
+}
 
 // Weight bytes per stage (codes of 128 rows x 4 blocks + one scale atom, per
 // matrix), B bytes per stage (4 blocks x 3 terms x BN rows x 16 B), B scale
@@ -187,6 +203,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         bool ok = true;
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const int4 U = p.units[u];
+            if (!mxg_unit_ok(p, U, nsplit, true)) continue;
             const int e = U.x & 0xFF, tile = U.x >> 8;
             const int ft = U.w & 0xFFFF, sp = U.w >> 16;
             const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
@@ -226,6 +243,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         bool ok = true;
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const int4 U = p.units[u];
+            if (!mxg_unit_ok(p, U, nsplit, false)) continue;
             const int ft = U.w & 0xFFFF, sp = U.w >> 16;
             const int c0 = sp * KC / nsplit, c1 = (sp + 1) * KC / nsplit;
             const int rf = min(128, p.N - ft * 128);
@@ -300,6 +318,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         bool ok = true;
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const int4 U = p.units[u];
+            if (!mxg_unit_ok(p, U, nsplit, false)) continue;
             const int tile = U.x >> 8, row0 = U.y, nvalid = U.z;
             const int ft = U.w & 0xFFFF;
             const int rf = min(128, p.N - ft * 128);
@@ -388,8 +407,9 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                                     atomicAdd(gu + n, gs[j]);
                                     atomicAdd(gu + p.N + n, us[j]);
                                 } else {
-                                    atomicAdd(p.yacc + static_cast<size_t>(p.row_token[rr]) * p.N + n,
-                                              gs[j] * p.row_weight[rr]);
+                                    const int tok = p.row_token[rr];
+                                    if (MOE_IN_BOUNDS(tok >= 0 && tok < p.T, p.status))
+                                        atomicAdd(p.yacc + static_cast<size_t>(tok) * p.N + n, gs[j] * p.row_weight[rr]);
                                 }
                             }
                         }

@@ -125,6 +125,9 @@ struct moe_mxfp4 {
     float* df_gu = nullptr;
     float* df_yacc = nullptr;
     cudaStream_t last_stream = nullptr;
+    // debug build: the guard region after each device buffer
+    uint8_t* guard_ptr[48] = {};
+    int n_guards = 0;
     // profiling
     bool prof = false, prof_valid = false;
     cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
@@ -141,6 +144,15 @@ static std::mutex g_attr_mutex;
 static bool g_attrs_set[MOE_MAX_DEVICES] = {};
 
 static bool aligned_to(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Debug build: every device buffer of a handle is followed by MOE_GUARD_BYTES
+// of a known pattern; moe_mxfp4_check_guards reports any that changed.
+#ifdef MOE_DEBUG_CHECKS
+constexpr size_t MOE_GUARD_BYTES = 4096;
+#else
+constexpr size_t MOE_GUARD_BYTES = 0;
+#endif
+constexpr unsigned char MOE_GUARD_BYTE = 0xA5;
 
 // Launch with programmatic stream serialization when `pdl` is set: the kernel
 // may start while the previous kernel in the stream finishes (it runs its
@@ -171,6 +183,19 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
         cudaError_t _e = (expr);                        \
         if (_e != cudaSuccess) return MOE_ERR_CUDA;     \
     } while (0)
+
+// One device allocation of a handle (at least 256 bytes), with the debug
+// build's guard region after it.
+static cudaError_t handle_alloc(moe_mxfp4* h, void** p, size_t bytes) {
+    const size_t n = std::max<size_t>(bytes, 256);
+    cudaError_t e = cudaMalloc(p, n + MOE_GUARD_BYTES);
+    if (e != cudaSuccess || MOE_GUARD_BYTES == 0) return e;
+    uint8_t* g = static_cast<uint8_t*>(*p) + n;
+    if ((e = cudaMemset(g, MOE_GUARD_BYTE, MOE_GUARD_BYTES)) != cudaSuccess) return e;
+    if (h->n_guards < static_cast<int>(sizeof(h->guard_ptr) / sizeof(h->guard_ptr[0])))
+        h->guard_ptr[h->n_guards++] = g;
+    return cudaSuccess;
+}
 
 static void free_all(moe_mxfp4* h) {
     void* ptrs[] = {h->w_gu, h->w_dn, h->w_router, h->bias, h->gamma, h->part_ss, h->inv_rms,
@@ -298,6 +323,7 @@ const char* moe_mxfp4_status_string(moe_status_t s) {
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_NOT_QUANTIZED: return "weights or router not set";
         case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case MOE_ERR_BOUNDS: return "a debug-build bounds check failed or a guard region changed";
     }
     return "unknown status";
 }
@@ -412,7 +438,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     uint32_t n_alloc = 0;
     for (auto& a : allocs) {
         if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
-        if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+        if (handle_alloc(h, a.p, a.bytes) != cudaSuccess) return fail(MOE_ERR_CUDA);
     }
     // Operand buffers start as zeros: codes, scale atoms and the weights' padding
     // are then always finite (an E2M1 code is never NaN; scale bytes written by
@@ -468,7 +494,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
                 };
                 for (auto& a : dfa) {
                     if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
-                    if (cudaMalloc(a.p, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
+                    if (handle_alloc(h, a.p, a.bytes) != cudaSuccess) return fail(MOE_ERR_CUDA);
                     if (cudaMemset(*a.p, 0, std::max<size_t>(a.bytes, 256)) != cudaSuccess) return fail(MOE_ERR_CUDA);
                 }
                 if (cudaDeviceSynchronize() != cudaSuccess) return fail(MOE_ERR_CUDA);
@@ -752,6 +778,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
     const float* gam = h->use_norm ? h->gamma : nullptr;
     const dim3 rgrid_rows((T + ROWS_TOKENS - 1) / ROWS_TOKENS);
+    const int tiles_cap = static_cast<int>(max_tile_atoms(h->TK, E) / MXQ_TERMS);   // token tiles the atoms hold
     // token tiles: at most ceil(T k / BN) plus one ragged tile per expert
     const dim3 egrid(static_cast<unsigned>((static_cast<long>(T) * k + BN - 1) / BN + E), h->KC_gu);
     if (bf16) {
@@ -760,21 +787,23 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const float*>(wts), static_cast<const int32_t*>(h->local_rank),
                    static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
-                   h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0);
+                   h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0,
+                   tiles_cap, h->status);
         launch_pdl(pdl, encode_rows_kernel<__nv_bfloat16>, egrid, dim3(ENC_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), gam, static_cast<const float*>(h->inv_rms),
                    static_cast<const int32_t*>(h->row_token), static_cast<const int4*>(h->units_gu),
-                   static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop);
+                   static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T, h->status);
     } else {
         launch_pdl(pdl, rows_kernel<float>, rgrid_rows, dim3(ROWS_THREADS), 0, stream, static_cast<const float*>(x),
                    static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                    static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
                    BN, h->row_token, h->row_weight, h->row_slot, h->GU, 2 * f, acc,
-                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0);
+                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status);
         launch_pdl(pdl, encode_rows_kernel<float>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
                    gam, static_cast<const float*>(h->inv_rms), static_cast<const int32_t*>(h->row_token),
-                   static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop);
+                   static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T,
+                   h->status);
     }
     h->launches += 1;   // stage 1 is two launches
     h->stage_ran[1] = true;
@@ -801,6 +830,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.status = h->status;
     gp.timeout_ns = tmo;
     gp.skip_first_copy = (c.flags & MOE_FLAG_TEST_SKIP_FIRST_COPY) ? 1u : 0u;
+    gp.n_experts = E;
+    gp.T = T;
+    gp.tiles_cap = tiles_cap;
     const int grid = h->nsm;
     launch_pdl(pdl, expert_mxf4_kernel<0>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(0, BN, gp.stages), stream,
                h->tm_x[BN / 16 - 1], gp);
@@ -818,7 +850,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         const long items = static_cast<long>(T) * k * (f / 32);
         const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
         launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const float*>(h->GU),
-                   Hop, f, BN, static_cast<const int32_t*>(h->row_slot), static_cast<const int32_t*>(h->sched));
+                   Hop, f, BN, static_cast<const int32_t*>(h->row_slot), static_cast<const int32_t*>(h->sched), tiles_cap,
+                   h->status);
         h->stage_ran[3] = true;
     }
     // 4: down GEMM + weighted scatter-combine
@@ -905,7 +938,29 @@ moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h) {
     int s = 0;
     MOE_TRY(cudaMemcpy(&s, h->status, sizeof(int), cudaMemcpyDeviceToHost));
     MOE_TRY(cudaMemset(h->status, 0, sizeof(int)));
-    return s == DEV_OK ? MOE_OK : MOE_ERR_TIMEOUT;
+    return (s & DEV_BOUNDS) ? MOE_ERR_BOUNDS : (s & DEV_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+moe_status_t moe_mxfp4_check_guards(moe_mxfp4_t* h) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (MOE_GUARD_BYTES == 0) return MOE_ERR_UNSUPPORTED;
+    MOE_TRY(cudaDeviceSynchronize());
+    unsigned char buf[MOE_GUARD_BYTES > 0 ? MOE_GUARD_BYTES : 1];
+    for (int i = 0; i < h->n_guards; ++i) {
+        MOE_TRY(cudaMemcpy(buf, h->guard_ptr[i], MOE_GUARD_BYTES, cudaMemcpyDeviceToHost));
+        for (size_t j = 0; j < MOE_GUARD_BYTES; ++j)
+            if (buf[j] != MOE_GUARD_BYTE) return MOE_ERR_BOUNDS;
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_mxfp4_test_write_guard(moe_mxfp4_t* h, int32_t i) {
+    if (!h || i < 0) return MOE_ERR_INVALID_ARG;
+    if (MOE_GUARD_BYTES == 0) return MOE_ERR_UNSUPPORTED;
+    if (i >= h->n_guards) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(cudaDeviceSynchronize());
+    MOE_TRY(cudaMemset(h->guard_ptr[i] + MOE_GUARD_BYTES / 2, 0, 1));
+    return MOE_OK;
 }
 
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable) {

@@ -521,7 +521,7 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
             const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
             int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
             float* __restrict__ GU, int gu_ld, float* __restrict__ yacc, const int32_t* __restrict__ sched,
-            int residual) {
+            int residual, int tiles_cap, int* status) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ int pos_s[ROWS_TOKENS * MAX_TOPK];
@@ -532,12 +532,18 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
         const int p = t0 * k + tid;
         const int t = p / k;
         const int e = idx[p];
-        const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
-        const int pos = offsets[e] + loc;
-        row_token[pos] = t;
-        row_weight[pos] = w[p];
-        row_slot[pos] = (tile_base[e] + loc / BN) * BN + loc % BN;
-        pos_s[tid] = pos;
+        pos_s[tid] = -1;
+        if (MOE_IN_BOUNDS(e >= 0 && e < E, status)) {
+            const int loc = tile_prefix[static_cast<size_t>(t / ROUTER_TOKENS) * E + e] + local_rank[p];
+            const int pos = offsets[e] + loc;
+            const int tl = tile_base[e] + loc / BN;
+            if (MOE_IN_BOUNDS(pos >= 0 && pos < T * k && tl >= 0 && tl < tiles_cap, status)) {
+                row_token[pos] = t;
+                row_weight[pos] = w[p];
+                row_slot[pos] = tl * BN + loc % BN;
+                pos_s[tid] = pos;
+            }
+        }
     }
     // output accumulator rows: x (residual) or zero
     const int d4 = d / 4;
@@ -558,9 +564,11 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
     if (sched[SCHED_SPLIT_GU] > 1) {
         __syncthreads();
         const int g4 = gu_ld / 4;
-        for (int i = tid; i < nt * k * g4; i += ROWS_THREADS)
-            reinterpret_cast<float4*>(GU + static_cast<size_t>(pos_s[i / g4]) * gu_ld)[i % g4] =
-                make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = tid; i < nt * k * g4; i += ROWS_THREADS) {
+            const int pos = pos_s[i / g4];
+            if (pos >= 0)
+                reinterpret_cast<float4*>(GU + static_cast<size_t>(pos) * gu_ld)[i % g4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
 }
 
@@ -578,7 +586,7 @@ template <typename TA>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, const float* __restrict__ inv_rms,
                    const int32_t* __restrict__ row_token, const int4* __restrict__ units_gu,
-                   const int32_t* __restrict__ sched, int F_gu, int d, GroupedOperand X) {
+                   const int32_t* __restrict__ sched, int F_gu, int d, GroupedOperand X, int T, int* status) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ __align__(16) uint8_t atoms[MXQ_TERMS * 512];
@@ -592,9 +600,10 @@ encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, co
     for (int i = tid; i < MXQ_TERMS * 512 / 16; i += ENC_THREADS)
         reinterpret_cast<uint4*>(atoms)[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
-    if (tid < nvalid) {
+    if (tid < nvalid && MOE_IN_BOUNDS(row0 >= 0 && row0 + nvalid <= X.R, status)) {
         const int row = row0 + tid;
-        const int t = row_token[row];
+        int t = row_token[row];
+        if (!MOE_IN_BOUNDS(t >= 0 && t < T, status)) t = 0;
         const int nb = d / 32;
         const float r = gamma ? inv_rms[t] : 1.f;
         for (int q = 0; q < 4 && 4 * c + q < nb; ++q) {
@@ -640,7 +649,7 @@ constexpr int HENC_THREADS = 128;
 // atom of the row's token tile).
 __global__ void __launch_bounds__(HENC_THREADS)
 h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
-                const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched) {
+                const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched, int tiles_cap, int* status) {
     pdl_launch_dependents();
     pdl_wait();
     if (sched[SCHED_SPLIT_GU] <= 1) return;
@@ -650,6 +659,7 @@ h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int B
     const int row = static_cast<int>(item / nb), b = static_cast<int>(item % nb);
     const int slot = row_slot[row];
     const int tile = slot / BN, rloc = slot % BN;
+    if (!MOE_IN_BOUNDS(row < Hd.R && slot >= 0 && tile < tiles_cap, status)) return;
     float v[32];
     const float4* g = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + 32 * b);
     const float4* u = reinterpret_cast<const float4*>(GU + static_cast<size_t>(row) * 2 * d_ff + d_ff + 32 * b);

@@ -67,8 +67,21 @@ __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepc
 // are visible; a no-op for a kernel launched without programmatic serialization.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Device-side status words shared with the host.
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+// Device-side status word shared with the host: a set of bits.
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BOUNDS = 2 };
+
+// Index checks of the debug build (MOE_DEBUG_CHECKS): a failed check records
+// DEV_BOUNDS in the status word and the caller skips the access; it never
+// traps.  In the release build every check is `true` and compiles away.
+#ifdef MOE_DEBUG_CHECKS
+__device__ __forceinline__ bool moe_in_bounds(bool ok, int* status) {
+    if (!ok) atomicOr(status, DEV_BOUNDS);
+    return ok;
+}
+#define MOE_IN_BOUNDS(cond, status) ::moe::moe_in_bounds((cond), (status))
+#else
+#define MOE_IN_BOUNDS(cond, status) true
+#endif
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA's abort
 // flag and the global status word) when `limit_ns` passes, or when another role
@@ -87,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
-            atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+            atomicOr(status, DEV_TIMEOUT);
             return false;
         }
     }
@@ -123,7 +136,7 @@ __device__ __forceinline__ bool spin_until_reached(const uint32_t* p, uint32_t t
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
-            atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+            atomicOr(status, DEV_TIMEOUT);
             return false;
         }
     }

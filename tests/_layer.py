@@ -64,12 +64,12 @@ class GpuLayer:
     """The CUDA layer for one weight set (router + experts drawn from cfg's seed)."""
 
     def __init__(self, cfg: mi.MoeConfig, max_tokens: int, flags: int = 0, wait_timeout_ms: int = 0,
-                 quantize: bool = True):
+                 quantize: bool = True, lib=None):
         import mxfp4_expert_gemm_router_b200 as mx
         torch = torch_mod()
         self.cfg = cfg
         self.layer = mx.MoeMxfp4(cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k, max_tokens, cfg.act_dtype,
-                                 flags, wait_timeout_ms)
+                                 flags, wait_timeout_ms, lib=lib)
         self.wr = mi.draw_router(cfg)
         self.bias = mi.draw_bias(cfg)
         if quantize:

@@ -37,8 +37,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for s in range(6):
-        assert lib.moe_mxfp4_status_string(s)
+    for s in range(7):
+        assert lib.moe_mxfp4_status_string(s) != b"unknown status"
     assert lib.moe_mxfp4_stage_name(2) == b"gate_up_swiglu"
 
 
@@ -114,7 +114,7 @@ def _header_constants():
 def test_binding_constants_match_the_header():
     hdr = _header_constants()
     names = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_NOT_QUANTIZED",
-             "MOE_ERR_TIMEOUT", "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_FLAG_TEST_SKIP_FIRST_COPY",
+             "MOE_ERR_TIMEOUT", "MOE_ERR_BOUNDS", "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_FLAG_TEST_SKIP_FIRST_COPY",
              "MOE_FLAG_TOKEN_TILE_SHIFT", "MOE_FLAG_TOKEN_TILE_MASK", "MOE_NUM_STAGES",
              "MOE_ROUTE_NOALLOC_MAX_TOKENS", "MOE_ROUTE_NOALLOC_MAX_EXPERTS", "MOE_FLAG_UNFUSED_DECODE",
              "MOE_FLAG_TEST_FAIL_ALLOC_SHIFT", "MOE_FLAG_TEST_FAIL_ALLOC_MASK"]
@@ -151,3 +151,11 @@ def test_route_noalloc_rejects_bad_arguments_before_touching_the_device(lib):
     assert f(ok, ok, None, 4, 64, 8, 2, F32, ok, ok, odd4, None) == mx.MOE_ERR_INVALID_ARG
     assert f(None, ok, None, 4, 64, 8, 2, F32, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
     assert f(ok, ok, None, 4, 64, 8, 2, 7, ok, ok, None, None) == mx.MOE_ERR_INVALID_ARG
+
+
+def test_debug_library_exports_the_same_symbols():
+    mxbuild.build_debug()
+    L = mx.load_debug()
+    for n in _declared_functions():
+        assert hasattr(L, n), n
+    assert L.moe_mxfp4_check_guards(None) == mx.MOE_ERR_INVALID_ARG
