@@ -172,7 +172,10 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
  * §2.1): copies x (host [T][d_model], act_dtype) in,
  * runs the layer, copies y (host [T][d_model]) and, if non-NULL, topk_idx
  * (host int32 [T][k]) and topk_w (host fp32 [T][k]) out, and synchronises
- * the stream before returning.  Uses handle-owned device staging buffers. */
+ * the stream before returning.  Uses handle-owned device staging buffers and
+ * two handle-owned copy streams: a batch of T >= 8192 tokens runs as up to 8
+ * chunks whose copies in and out overlap the forwards of their neighbours
+ * (pinned host buffers make the copies asynchronous). */
 moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t T,
                                     void* y_host, int32_t* topk_idx_host,
                                     float* topk_w_host, cudaStream_t stream);

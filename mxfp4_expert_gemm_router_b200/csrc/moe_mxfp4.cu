@@ -125,6 +125,10 @@ struct moe_mxfp4 {
     float* df_gu = nullptr;
     float* df_yacc = nullptr;
     cudaStream_t last_stream = nullptr;
+    // forward_host: copy streams and per-chunk events (copies overlap compute)
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+    cudaEvent_t ev_in[8] = {}, ev_out[8] = {};
     // debug build: the guard region after each device buffer
     uint8_t* guard_ptr[48] = {};
     int n_guards = 0;
@@ -208,6 +212,14 @@ static void free_all(moe_mxfp4* h) {
         if (p) cudaFree(p);
     for (auto& e : h->ev)
         if (e) cudaEventDestroy(e);
+    for (int i = 0; i < 8; ++i) {
+        if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+        if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+    }
+    if (h->ev_start) cudaEventDestroy(h->ev_start);
+    if (h->ev_done) cudaEventDestroy(h->ev_done);
+    if (h->s_in) cudaStreamDestroy(h->s_in);
+    if (h->s_out) cudaStreamDestroy(h->s_out);
     delete[] h->expert_done;
 }
 
@@ -504,6 +516,15 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     }
     for (auto& e : h->ev)
         if (cudaEventCreate(&e) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    if (cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming) != cudaSuccess)
+        return fail(MOE_ERR_CUDA);
+    for (int i = 0; i < 8; ++i)
+        if (cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+            return fail(MOE_ERR_CUDA);
     *out = h;
     return MOE_OK;
 }
@@ -896,16 +917,51 @@ moe_status_t moe_mxfp4_forward_host(moe_mxfp4_t* h, const void* x_host, int32_t 
     if (T > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
     if (moe_status_t ds = check_device(h)) return ds;
     if (T == 0) return MOE_OK;
-    const size_t act = static_cast<size_t>(T) * c.d_model * h->act_bytes;
-    MOE_TRY(cudaMemcpyAsync(h->x_stage, x_host, act, cudaMemcpyHostToDevice, stream));
-    moe_status_t st = moe_mxfp4_forward(h, h->x_stage, T, h->y_stage, h->idx_stage, h->w_stage, nullptr, stream);
-    if (st != MOE_OK) return st;
-    MOE_TRY(cudaMemcpyAsync(y_host, h->y_stage, act, cudaMemcpyDeviceToHost, stream));
-    const size_t tk = static_cast<size_t>(T) * c.top_k;
-    if (topk_idx_host)
-        MOE_TRY(cudaMemcpyAsync(topk_idx_host, h->idx_stage, tk * sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
-    if (topk_w_host)
-        MOE_TRY(cudaMemcpyAsync(topk_w_host, h->w_stage, tk * sizeof(float), cudaMemcpyDeviceToHost, stream));
+    const size_t row_bytes = static_cast<size_t>(c.d_model) * h->act_bytes;
+    // Large batches run as up to 8 chunks of at least FH_MIN_CHUNK tokens: the
+    // copy of chunk i+1 in and of chunk i-1 out overlap the forward of chunk i
+    // (the rows of a forward are independent, so chunking changes nothing in
+    // the result beyond fp32 summation order).  The forwards themselves run in
+    // order on `stream`; the copies on the handle's two copy streams.
+    constexpr int FH_MIN_CHUNK = 4096;
+    const int nch = std::max(1, std::min(8, T / FH_MIN_CHUNK));
+    const int chunk = (T + nch - 1) / nch;
+    auto* xs = static_cast<uint8_t*>(h->x_stage);
+    auto* ys = static_cast<uint8_t*>(h->y_stage);
+    const uint8_t* xh = static_cast<const uint8_t*>(x_host);
+    uint8_t* yh = static_cast<uint8_t*>(y_host);
+    const int k = c.top_k;
+    // the copy streams start after the work already queued on `stream`
+    MOE_TRY(cudaEventRecord(h->ev_start, stream));
+    MOE_TRY(cudaStreamWaitEvent(h->s_in, h->ev_start, 0));
+    MOE_TRY(cudaStreamWaitEvent(h->s_out, h->ev_start, 0));
+    for (int i = 0; i < nch; ++i) {
+        const int t0 = i * chunk, n = std::min(chunk, T - t0);
+        if (n <= 0) break;
+        const size_t off = static_cast<size_t>(t0) * row_bytes, bytes = static_cast<size_t>(n) * row_bytes;
+        MOE_TRY(cudaMemcpyAsync(xs + off, xh + off, bytes, cudaMemcpyHostToDevice, h->s_in));
+        MOE_TRY(cudaEventRecord(h->ev_in[i], h->s_in));
+        MOE_TRY(cudaStreamWaitEvent(stream, h->ev_in[i], 0));
+        moe_status_t st = moe_mxfp4_forward(h, xs + off, n, ys + off, h->idx_stage + static_cast<size_t>(t0) * k,
+                                            h->w_stage + static_cast<size_t>(t0) * k, nullptr, stream);
+        if (st != MOE_OK) {
+            cudaStreamSynchronize(h->s_in);
+            return st;
+        }
+        MOE_TRY(cudaEventRecord(h->ev_out[i], stream));
+        MOE_TRY(cudaStreamWaitEvent(h->s_out, h->ev_out[i], 0));
+        MOE_TRY(cudaMemcpyAsync(yh + off, ys + off, bytes, cudaMemcpyDeviceToHost, h->s_out));
+        const size_t tk = static_cast<size_t>(n) * k, tk0 = static_cast<size_t>(t0) * k;
+        if (topk_idx_host)
+            MOE_TRY(cudaMemcpyAsync(topk_idx_host + tk0, h->idx_stage + tk0, tk * sizeof(int32_t),
+                                    cudaMemcpyDeviceToHost, h->s_out));
+        if (topk_w_host)
+            MOE_TRY(cudaMemcpyAsync(topk_w_host + tk0, h->w_stage + tk0, tk * sizeof(float), cudaMemcpyDeviceToHost,
+                                    h->s_out));
+    }
+    // `stream` ends after the last copy out
+    MOE_TRY(cudaEventRecord(h->ev_done, h->s_out));
+    MOE_TRY(cudaStreamWaitEvent(stream, h->ev_done, 0));
     MOE_TRY(cudaStreamSynchronize(stream));
     return MOE_OK;
 }

@@ -428,3 +428,22 @@ def test_unfused_pipeline_timeout_is_reported_not_hung():
     L.layer.forward(x, y)
     assert L.layer.status() == mx.MOE_ERR_TIMEOUT
     assert L.layer.status() == mx.MOE_OK
+
+
+def test_forward_host_chunked_matches_device(layer20b):
+    """At 12288 tokens the host-buffer entry point runs three chunks whose copies
+    overlap the neighbouring forwards: same routing and output as one device
+    forward of the whole batch."""
+    import torch
+    cfg = CFG20.with_T(12288)
+    layer20b.set_router(mi.draw_router(cfg), None)
+    x = mi.draw_x(cfg)
+    y_dev, idx_dev, w_dev, _ = layer20b.forward(x)
+    xh = act_tensor(cfg, x, device="cpu").pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    ih = torch.empty((cfg.T, cfg.top_k), dtype=torch.int32).pin_memory()
+    wh = torch.empty((cfg.T, cfg.top_k), dtype=torch.float32).pin_memory()
+    layer20b.layer.forward_host(xh, yh, ih, wh)
+    np.testing.assert_array_equal(ih.numpy(), idx_dev)
+    np.testing.assert_allclose(wh.numpy(), w_dev, atol=1e-7)
+    assert np.abs(to_f64(yh) - y_dev).max() <= 1e-2 * np.abs(y_dev).max()
