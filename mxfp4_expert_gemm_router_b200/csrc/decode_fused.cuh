@@ -23,8 +23,10 @@
 //  2. The B operand is every token of the batch (16 rows per term, the three
 //     MXFP4 terms stacked: N = 48) for every expert.  Columns of tokens not
 //     routed to an expert are computed and dropped: next to the weight stream
-//     the MMA work is negligible, and one B operand for the whole K, encoded
-//     once per CTA into shared memory, replaces the grouping and the gather.
+//     the MMA work is negligible, and one B operand for the whole K replaces
+//     the grouping and the gather.  The grid encodes it once (each CTA a
+//     share of the (block, token) items, into global memory); each CTA then
+//     bulk-copies it into shared memory when every share is written.
 //  3. Work items: a gate/up item is one 128-wide K chunk of one 128-feature
 //     tile of one touched expert (gate and up: 17,408 bytes); a down item is
 //     two consecutive K chunks of one feature tile of the down matrix (at most
@@ -34,12 +36,14 @@
 //     tile) is a piece; it accumulates in one tensor-memory accumulator.
 //  4. Gate/up pieces add fp32 partial sums of g and u into GU (red.add) for
 //     the tokens routed to the expert and then count their chunks in a
-//     per-(expert, feature tile) counter.  A down piece of expert e over d_ff
-//     chunks [c0, c1) needs g and u of features [128 c0, 128 c1): its
-//     epilogue warps wait (bounded) for those counters, form H = Swish(g) u,
-//     encode it as three MXFP4 terms into the shared-memory B operand, and
-//     the MMA warp runs.  Down weight copies never wait: the producer streams
-//     them into the ring while other CTAs finish their gate/up work.
+//     per-(expert, feature tile) counter.  The CTA whose count completes a
+//     tile forms H = Swish(g) u for it, encodes it as three MXFP4 terms into
+//     the expert's H operand in global memory and stamps the tile with the
+//     epoch.  A down piece of expert e over d_ff chunks [c0, c1) waits
+//     (bounded) for the stamps of gate/up feature tiles c0 .. c1-1, bulk-copies
+//     that range of the H operand into shared memory, and the MMA warp runs.
+//     Down weight copies never wait: the producer streams them into the ring
+//     while other CTAs finish their gate/up work.
 //  5. Down epilogue: y_acc[t] += w[t, e] D[., t] for the tokens routed to e
 //     (red.add).  The last CTA to finish writes y (cast; + x with the
 //     residual) and resets the counters.
@@ -86,7 +90,8 @@ struct DecodeState {
     uint32_t finish;   // CTAs finished in the current launch
     int32_t prev_nt;   // touched experts of the previous launch
     int32_t prev_T;    // its token count
-    uint32_t pad[3];
+    uint32_t xdone;    // CTAs that wrote their share of x's operand: grows by gridDim.x per launch
+    uint32_t pad[2];
 };
 
 struct DecodeParams {
@@ -111,6 +116,10 @@ struct DecodeParams {
     double* part_ss;        // [S][16] partial sums of x^2
     float* gu;              // [2][max_touched][16][2 f] partial g | u
     float* yacc;            // [2][16][d]
+    uint8_t* xq;            // x as the B operand: codes [d/32][48][16 B], then scale atoms [KC_gu][512]
+    uint8_t* hq;            // H per touched slot (stride hq_stride): codes [f/32][48][16 B], atoms [KC_dn][512]
+    size_t hq_stride;
+    uint32_t* hdone;        // [max_touched][F_gu] epoch + 1 once H of (slot, feature tile) is in hq
     int32_t* topk_idx;      // [T][k] or null
     float* topk_w;          // [T][k] or null
     int32_t* counts;        // [E] or null
@@ -127,6 +136,7 @@ struct DecodeCtl {
     uint32_t tmem;
     int last;
     int n_t;
+    int tile_done;     // this CTA completed a gate/up feature tile: it writes that tile's H
     double inv_rms[DF_MAX_T];
     int tok_e[DF_MAX_T][MAX_TOPK];
     float tok_w[DF_MAX_T][MAX_TOPK];
@@ -395,6 +405,50 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         __syncthreads();
     }
     const int n_t = C.n_t;
+    const int nb_d = d / 32, nb_f = f / 32;
+    // ---- this CTA's share of x's B operand (every token row, 16 per term; rows
+    // past T are zero), written to global memory; the count tells the grid
+    {
+        uint8_t* xcodes = p.xq;
+        uint8_t* xatoms = p.xq + static_cast<size_t>(nb_d) * DF_B_BLOCK;
+        const int items = nb_d * DF_MAX_T;
+        const int i0 = static_cast<int>(static_cast<long>(items) * blockIdx.x / G);
+        const int i1 = static_cast<int>(static_cast<long>(items) * (blockIdx.x + 1) / G);
+        for (int itm = i0 + tid; itm < i1; itm += DF_THREADS) {
+            const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
+            uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                                      make_uint4(0u, 0u, 0u, 0u)};
+            uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
+            if (t < T) {
+                float v[32];
+                BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+                if (norm) {
+                    const float r = static_cast<float>(C.inv_rms[t]);
+                    const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 g = g4[i];
+                        v[4 * i] *= g.x * r;
+                        v[4 * i + 1] *= g.y * r;
+                        v[4 * i + 2] *= g.z * r;
+                        v[4 * i + 3] *= g.w * r;
+                    }
+                }
+                mxq_block_thread(v, codes, sb);
+            }
+#pragma unroll
+            for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                *reinterpret_cast<uint4*>(xcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                    codes[tt];
+                xatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&p.st->xdone, 1u);
+        }
+    }
     // this CTA's items: equal contiguous shares of the gate/up and the down items
     const long NG = static_cast<long>(n_t) * F_gu * KC_gu;
     const long ND = static_cast<long>(n_t) * F_dn * NP;
@@ -562,48 +616,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         const int hh = (warp - 2) >> 2;          // token columns 8 hh .. 8 hh + 7
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
-        // x of every token as the B operand: [block][term * 16 + token][16 B]
-        {
-            // scale bytes of blocks past K in a ragged last chunk must be a finite
-            // (zero: 2^-127) E8M0 value, never stale shared memory
-            for (int i = et; i < p.kc_max * 512 / 16; i += DF_EPI_THREADS)
-                reinterpret_cast<uint4*>(bsf_ptr)[i] = make_uint4(0u, 0u, 0u, 0u);
-            named_barrier(1, DF_EPI_THREADS);
-            const int nb = d / 32;
-            for (int itm = et; itm < nb * DF_MAX_T; itm += DF_EPI_THREADS) {
-                const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
-                float v[32];
-                if (t < T) {
-                    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
-                    if (norm) {
-                        const float r = static_cast<float>(C.inv_rms[t]);
-                        const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 g = g4[i];
-                            v[4 * i] *= g.x * r;
-                            v[4 * i + 1] *= g.y * r;
-                            v[4 * i + 2] *= g.z * r;
-                            v[4 * i + 3] *= g.w * r;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                }
-                uint4 codes[MXQ_TERMS];
-                uint32_t sb[MXQ_TERMS];
-                mxq_block_thread(v, codes, sb);
-#pragma unroll
-                for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                    *reinterpret_cast<uint4*>(bbuf_ptr + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
-                        codes[tt];
-                    bsf_ptr[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
-                }
+        // x's B operand: once every CTA has written its share, one thread copies
+        // it (codes and scale atoms) into shared memory; xready completes on
+        // the bytes
+        if (et == 0) {
+            const uint32_t target = (epoch + 1u) * static_cast<uint32_t>(G);
+            if (spin_until_reached(&p.st->xdone, target, abort_flag, p.status, p.timeout_ns)) {
+                const uint32_t cb = static_cast<uint32_t>(nb_d) * DF_B_BLOCK, ab = static_cast<uint32_t>(KC_gu) * 512u;
+                mbar_arrive_expect_tx(smem_u32(&C.xready), cb + ab);
+                bulk_g2s(bbuf, p.xq, cb, smem_u32(&C.xready));
+                bulk_g2s(bsf, p.xq + cb, ab, smem_u32(&C.xready));
             }
-            fence_proxy_async_smem();
-            named_barrier(1, DF_EPI_THREADS);
-            if (et == 0) mbar_arrive(smem_u32(&C.xready));
         }
         bool ok = named_barrier_and(1, DF_EPI_THREADS, *abort_flag == 0);
 
@@ -657,7 +680,50 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             // every epilogue thread takes the same decision (no thread is left waiting)
             ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
             if (!ok) break;
-            if (et == 0) atomicAdd(&p.done[i * F_gu + ft], static_cast<uint32_t>(piece_end - it));
+            if (et == 0) {
+                const uint32_t n = static_cast<uint32_t>(piece_end - it);
+                const uint32_t old = atomicAdd(&p.done[i * F_gu + ft], n);
+                __threadfence();   // acquire: the other contributors' partial sums are visible
+                C.tile_done = (old + n == static_cast<uint32_t>(KC_gu)) ? 1 : 0;
+            }
+            named_barrier(1, DF_EPI_THREADS);
+            if (C.tile_done) {
+                // H of feature tile ft (blocks 4 ft .. 4 ft + 3) for every token row of
+                // the slot: Swish(g) u of the routed tokens, zero rows for the rest
+                uint8_t* hcodes = p.hq + i * p.hq_stride;
+                uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
+                for (int itm = et; itm < 4 * DF_MAX_T; itm += DF_EPI_THREADS) {
+                    const int b = 4 * ft + itm / DF_MAX_T, t = itm % DF_MAX_T;
+                    if (b >= nb_f) continue;
+                    uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                                              make_uint4(0u, 0u, 0u, 0u)};
+                    uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
+                    if (t < T && C.selw[i][t] != 0.f) {
+                        const float* row = gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f;
+                        const float4* g4 = reinterpret_cast<const float4*>(row + 32 * b);
+                        const float4* u4 = reinterpret_cast<const float4*>(row + f + 32 * b);
+                        float v[32];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 gg = __ldcg(g4 + q4), uu = __ldcg(u4 + q4);
+                            v[4 * q4] = swish_f(gg.x) * uu.x;
+                            v[4 * q4 + 1] = swish_f(gg.y) * uu.y;
+                            v[4 * q4 + 2] = swish_f(gg.z) * uu.z;
+                            v[4 * q4 + 3] = swish_f(gg.w) * uu.w;
+                        }
+                        mxq_block_thread(v, codes, sb);
+                    }
+#pragma unroll
+                    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                        *reinterpret_cast<uint4*>(hcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                            codes[tt];
+                        hatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
+                    }
+                }
+                __threadfence();
+                named_barrier(1, DF_EPI_THREADS);
+                if (et == 0) atomicExch(&p.hdone[i * F_gu + ft], epoch + 1u);
+            }
             it = piece_end;
         }
 
@@ -692,11 +758,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             const int rf = min(128, d - ft * 128);
             const int c0 = 2 * static_cast<int>(jt % NP);
             const int c1 = min(KC_dn, 2 * static_cast<int>((piece_end - 1) % NP) + 2);
-            // g and u of features [128 c0, 128 c1) complete (gate/up feature tiles c0 .. c1-1)
+            // H of features [128 c0, 128 c1) written (gate/up feature tiles c0 .. c1-1 stamped)
             bool w_ok = true;
             if (et < c1 - c0)
-                w_ok = spin_until_reached(&p.done[i * F_gu + c0 + et], static_cast<uint32_t>(KC_gu), abort_flag,
-                                          p.status, p.timeout_ns);
+                w_ok = spin_until_reached(&p.hdone[i * F_gu + c0 + et], epoch + 1u, abort_flag, p.status,
+                                          p.timeout_ns);
             // the previous down piece's MMAs must be done before its operand is overwritten
             if (pend_buf >= 0) {
                 w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag,
@@ -706,50 +772,16 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             }
             ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
             if (!ok) break;
-            // H = Swish(g) u of the routed tokens as three MXFP4 terms: [block][term * 16 + t][16 B]
-            {
-                const int nbf = f / 32;
-                const int b0 = 4 * c0, b1 = min(4 * c1, nbf);
-                for (int itm = et; itm < (b1 - b0) * DF_MAX_T; itm += DF_EPI_THREADS) {
-                    const int b = b0 + itm / DF_MAX_T, t = itm % DF_MAX_T;
-                    float v[32];
-                    if (t < T && C.selw[i][t] != 0.f) {
-                        const float4* g4 =
-                            reinterpret_cast<const float4*>(gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f + 32 * b);
-                        const float4* u4 = reinterpret_cast<const float4*>(
-                            gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f + f + 32 * b);
-#pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 gg = __ldcg(g4 + q4), uu = __ldcg(u4 + q4);
-                            v[4 * q4] = swish_f(gg.x) * uu.x;
-                            v[4 * q4 + 1] = swish_f(gg.y) * uu.y;
-                            v[4 * q4 + 2] = swish_f(gg.z) * uu.z;
-                            v[4 * q4 + 3] = swish_f(gg.w) * uu.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int q4 = 0; q4 < 32; ++q4) v[q4] = 0.f;
-                    }
-                    uint4 codes[MXQ_TERMS];
-                    uint32_t sb[MXQ_TERMS];
-                    mxq_block_thread(v, codes, sb);
-#pragma unroll
-                    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                        *reinterpret_cast<uint4*>(bbuf_ptr +
-                                                  (static_cast<size_t>(b - b0) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
-                            codes[tt];
-                        bsf_ptr[((b >> 2) - c0) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] =
-                            static_cast<uint8_t>(sb[tt]);
-                    }
-                }
-                // blocks past d_ff in a ragged last chunk: zero scale bytes (2^-127)
-                for (int itm = et; itm < (4 * c1 - b1) * DF_NB3; itm += DF_EPI_THREADS) {
-                    const int b = b1 + itm / DF_NB3, r = itm % DF_NB3;
-                    bsf_ptr[((b >> 2) - c0) * 512 + sf_atom_offset(r, b & 3)] = 0;
-                }
-                fence_proxy_async_smem();
-                named_barrier(1, DF_EPI_THREADS);
-                if (et == 0) mbar_arrive(smem_u32(&C.bready));
+            // the piece's range of the expert's H operand into shared memory (bready
+            // completes on the bytes)
+            if (et == 0) {
+                const uint8_t* hcodes = p.hq + i * p.hq_stride;
+                const uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
+                const int b0 = 4 * c0, b1 = min(4 * c1, nb_f);
+                const uint32_t cb = static_cast<uint32_t>(b1 - b0) * DF_B_BLOCK, ab = static_cast<uint32_t>(c1 - c0) * 512u;
+                mbar_arrive_expect_tx(smem_u32(&C.bready), cb + ab);
+                bulk_g2s(bbuf, hcodes + static_cast<size_t>(b0) * DF_B_BLOCK, cb, smem_u32(&C.bready));
+                bulk_g2s(bsf, hatoms + static_cast<size_t>(c0) * 512, ab, smem_u32(&C.bready));
             }
             if (pend_buf >= 0) drain_pending();
             pend_buf = buf;

@@ -124,6 +124,10 @@ struct moe_mxfp4 {
     double* df_part_ss = nullptr;
     float* df_gu = nullptr;
     float* df_yacc = nullptr;
+    uint8_t* df_xq = nullptr;
+    uint8_t* df_hq = nullptr;
+    size_t df_hq_stride = 0;
+    uint32_t* df_hdone = nullptr;
     cudaStream_t last_stream = nullptr;
     // forward_host: copy streams and per-chunk events (copies overlap compute)
     cudaStream_t s_in = nullptr, s_out = nullptr;
@@ -207,7 +211,8 @@ static void free_all(moe_mxfp4* h) {
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
-                    h->df_state, h->df_done, h->df_part, h->df_part_ss, h->df_gu, h->df_yacc};
+                    h->df_state, h->df_done, h->df_part, h->df_part_ss, h->df_gu, h->df_yacc,
+                    h->df_xq, h->df_hq, h->df_hdone};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     for (auto& e : h->ev)
@@ -496,6 +501,8 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
                 const size_t gu_bytes_df = sizeof(float) * 2 * h->df_max_touched * DF_MAX_T * 2 * static_cast<size_t>(f);
                 const size_t ya_bytes_df = sizeof(float) * 2 * DF_MAX_T * static_cast<size_t>(d);
                 const size_t done_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu;
+                const size_t xq_bytes = static_cast<size_t>(d / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_gu) * 512;
+                h->df_hq_stride = static_cast<size_t>(f / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_dn) * 512;
                 A dfa[] = {
                     {reinterpret_cast<void**>(&h->df_state), sizeof(DecodeState)},
                     {reinterpret_cast<void**>(&h->df_done), done_bytes},
@@ -503,6 +510,9 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
                     {reinterpret_cast<void**>(&h->df_part_ss), sizeof(double) * h->df_S * DF_MAX_T},
                     {reinterpret_cast<void**>(&h->df_gu), gu_bytes_df},
                     {reinterpret_cast<void**>(&h->df_yacc), ya_bytes_df},
+                    {reinterpret_cast<void**>(&h->df_xq), xq_bytes},
+                    {reinterpret_cast<void**>(&h->df_hq), h->df_hq_stride * h->df_max_touched},
+                    {reinterpret_cast<void**>(&h->df_hdone), done_bytes},
                 };
                 for (auto& a : dfa) {
                     if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
@@ -718,6 +728,10 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         dp.part_ss = h->df_part_ss;
         dp.gu = h->df_gu;
         dp.yacc = h->df_yacc;
+        dp.xq = h->df_xq;
+        dp.hq = h->df_hq;
+        dp.hq_stride = h->df_hq_stride;
+        dp.hdone = h->df_hdone;
         dp.topk_idx = topk_idx;
         dp.topk_w = topk_w;
         dp.counts = expert_counts;
@@ -999,24 +1013,30 @@ moe_status_t moe_mxfp4_get_status(moe_mxfp4_t* h) {
 
 moe_status_t moe_mxfp4_check_guards(moe_mxfp4_t* h) {
     if (!h) return MOE_ERR_INVALID_ARG;
-    if (MOE_GUARD_BYTES == 0) return MOE_ERR_UNSUPPORTED;
+#ifndef MOE_DEBUG_CHECKS
+    return MOE_ERR_UNSUPPORTED;
+#else
     MOE_TRY(cudaDeviceSynchronize());
-    unsigned char buf[MOE_GUARD_BYTES > 0 ? MOE_GUARD_BYTES : 1];
+    unsigned char buf[MOE_GUARD_BYTES];
     for (int i = 0; i < h->n_guards; ++i) {
         MOE_TRY(cudaMemcpy(buf, h->guard_ptr[i], MOE_GUARD_BYTES, cudaMemcpyDeviceToHost));
         for (size_t j = 0; j < MOE_GUARD_BYTES; ++j)
             if (buf[j] != MOE_GUARD_BYTE) return MOE_ERR_BOUNDS;
     }
     return MOE_OK;
+#endif
 }
 
 moe_status_t moe_mxfp4_test_write_guard(moe_mxfp4_t* h, int32_t i) {
     if (!h || i < 0) return MOE_ERR_INVALID_ARG;
-    if (MOE_GUARD_BYTES == 0) return MOE_ERR_UNSUPPORTED;
+#ifndef MOE_DEBUG_CHECKS
+    return MOE_ERR_UNSUPPORTED;
+#else
     if (i >= h->n_guards) return MOE_ERR_INVALID_ARG;
     MOE_TRY(cudaDeviceSynchronize());
     MOE_TRY(cudaMemset(h->guard_ptr[i] + MOE_GUARD_BYTES / 2, 0, 1));
     return MOE_OK;
+#endif
 }
 
 moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable) {
