@@ -27,36 +27,36 @@
 //     the grouping and the gather.  The grid encodes it once (each CTA a
 //     share of the (block, token) items, into global memory); each CTA then
 //     bulk-copies it into shared memory when every share is written.
-//  3. Work items: a gate/up item is one 128-wide K chunk of one 128-feature
-//     tile of one touched expert (gate and up: 17,408 bytes); a down item is
-//     two consecutive K chunks of one feature tile of the down matrix (at most
-//     17,408 bytes).  CTA b takes an equal contiguous share of the gate/up
-//     items and of the down items in (expert, tile, chunk) order, so every SM
-//     streams the same number of bytes.  A run of items with the same (expert,
-//     tile) is a piece; it accumulates in one tensor-memory accumulator.
-//  4. Gate/up pieces add fp32 partial sums of g and u into GU (red.add) for
-//     the tokens routed to the expert and then count their chunks in a
-//     per-(expert, feature tile) counter.  The CTA whose count completes a
-//     tile forms H = Swish(g) u for it, encodes it as three MXFP4 terms into
-//     the expert's H operand in global memory and stamps the tile with the
-//     epoch.  A down piece of expert e over d_ff chunks [c0, c1) waits
-//     (bounded) for the stamps of gate/up feature tiles c0 .. c1-1, bulk-copies
-//     that range of the H operand into shared memory, and the MMA warp runs.
-//     Down weight copies never wait: the producer streams them into the ring
-//     while other CTAs finish their gate/up work.
+//  3. Gate/up work comes in whole feature tiles (128 features of one touched
+//     expert over all of K, gate and up: 23 chunks of 17,408 bytes at the
+//     2880-wide shape), dealt round-robin over the CTAs; a CTA accumulates a
+//     tile in tensor memory and its epilogue forms H = Swish(g) u for the
+//     tokens routed to the expert straight from the accumulator, encodes it
+//     as three MXFP4 terms (one 32-feature block per warp, one element per
+//     lane) into the expert's H operand in global memory, and stamps the tile
+//     with the launch's epoch.  Down work comes in items of two consecutive K
+//     chunks of one feature tile of the down matrix (at most 17,408 bytes),
+//     dealt in contiguous ranges sized so that every CTA streams the same
+//     total number of bytes; a run of down items of the same (expert, tile) is
+//     a piece.
+//  4. A down piece over d_ff chunks [c0, c1) waits (bounded) for the stamps
+//     of gate/up feature tiles c0 .. c1-1, bulk-copies that range of the
+//     expert's H operand into shared memory, and the MMA warp runs.  Down
+//     weight copies never wait: the producer streams them into the ring while
+//     other CTAs finish their gate/up tiles.
 //  5. Down epilogue: y_acc[t] += w[t, e] D[., t] for the tokens routed to e
 //     (red.add).  The last CTA to finish writes y (cast; + x with the
-//     residual) and resets the counters.
+//     residual).
 //
-// State across launches (epoch, grid-barrier arrivals, counters) lives in
-// device memory.  GU and y_acc alternate by the epoch's parity: each launch
-// clears the rows of the other parity that the previous launch used, so the
-// buffers a launch accumulates into are always clear, with no pass of its
-// own.  Every wait (mbarrier phases, the grid barrier, the counters) is
+// State across launches (epoch, grid-barrier and x-operand arrival counts)
+// lives in device memory; every CTA arrives at each count exactly once per
+// launch, so targets are (epoch + 1) * gridDim.x and nothing is reset.  The
+// output accumulator alternates by the epoch's parity: each launch clears the
+// other parity, so the buffer a launch accumulates into is always clear.
+// Every wait (mbarrier phases, the grid barrier, the counts, the stamps) is
 // bounded; on a timeout the CTA raises its abort flag and the status word,
 // all roles leave their loops, copies and MMAs in flight are drained and the
-// tensor memory is freed.  Every CTA still arrives at the grid barrier and at
-// the finish counter exactly once, so the state stays consistent.
+// tensor memory is freed.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -88,10 +88,8 @@ struct DecodeState {
     uint32_t bar;      // grid-barrier arrivals: grows by gridDim.x per launch
     uint32_t epoch;    // launches completed
     uint32_t finish;   // CTAs finished in the current launch
-    int32_t prev_nt;   // touched experts of the previous launch
-    int32_t prev_T;    // its token count
     uint32_t xdone;    // CTAs that wrote their share of x's operand: grows by gridDim.x per launch
-    uint32_t pad[2];
+    uint32_t pad[4];
 };
 
 struct DecodeParams {
@@ -109,12 +107,9 @@ struct DecodeParams {
     int stages;             // weight-ring stages
     int nb_max;             // 32-blocks of the B buffer: max(d, f) / 32
     int kc_max;             // K chunks of the B buffer: max over both GEMMs
-    int max_touched;        // expert rows of GU per parity
     DecodeState* st;
-    uint32_t* done;         // [max_touched][F_gu] gate/up chunks finished
     double* part;           // [S][16][E] partial scores
     double* part_ss;        // [S][16] partial sums of x^2
-    float* gu;              // [2][max_touched][16][2 f] partial g | u
     float* yacc;            // [2][16][d]
     uint8_t* xq;            // x as the B operand: codes [d/32][48][16 B], then scale atoms [KC_gu][512]
     uint8_t* hq;            // H per touched slot (stride hq_stride): codes [f/32][48][16 B], atoms [KC_dn][512]
@@ -136,7 +131,6 @@ struct DecodeCtl {
     uint32_t tmem;
     int last;
     int n_t;
-    int tile_done;     // this CTA completed a gate/up feature tile: it writes that tile's H
     double inv_rms[DF_MAX_T];
     int tok_e[DF_MAX_T][MAX_TOPK];
     float tok_w[DF_MAX_T][MAX_TOPK];
@@ -211,22 +205,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
     const uint32_t tmem = C.tmem;
     const uint32_t epoch = ld_acquire_u32(&p.st->epoch);
     const int par = static_cast<int>(epoch & 1u);
-    const size_t gu_par = static_cast<size_t>(p.max_touched) * DF_MAX_T * 2 * f;
-    float* gu = p.gu + par * gu_par;
     float* yacc = p.yacc + static_cast<size_t>(par) * DF_MAX_T * d;
 
-    // ---- clear the other parity's rows the previous launch used (nothing in
-    // this launch touches them)
+    // ---- clear the other parity's output accumulator (nothing in this launch
+    // touches it; the next launch accumulates into it)
     {
-        const int pn = p.st->prev_nt, pT = p.st->prev_T;
-        float4* g_other = reinterpret_cast<float4*>(p.gu + (1 - par) * gu_par);
-        const int row4 = 2 * f / 4;
-        const long n4 = static_cast<long>(pn) * pT * row4;
-        for (long i = static_cast<long>(blockIdx.x) * DF_THREADS + tid; i < n4; i += static_cast<long>(G) * DF_THREADS) {
-            const long r = i / row4, c4 = i % row4;
-            const long row = (r / pT) * DF_MAX_T + (r % pT);
-            g_other[row * row4 + c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
         float4* y_other = reinterpret_cast<float4*>(p.yacc + static_cast<size_t>(1 - par) * DF_MAX_T * d);
         const long y4 = static_cast<long>(DF_MAX_T) * d / 4;
         for (long i = static_cast<long>(blockIdx.x) * DF_THREADS + tid; i < y4; i += static_cast<long>(G) * DF_THREADS)
@@ -406,54 +389,27 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
     }
     const int n_t = C.n_t;
     const int nb_d = d / 32, nb_f = f / 32;
-    // ---- this CTA's share of x's B operand (every token row, 16 per term; rows
-    // past T are zero), written to global memory; the count tells the grid
-    {
-        uint8_t* xcodes = p.xq;
-        uint8_t* xatoms = p.xq + static_cast<size_t>(nb_d) * DF_B_BLOCK;
-        const int items = nb_d * DF_MAX_T;
-        const int i0 = static_cast<int>(static_cast<long>(items) * blockIdx.x / G);
-        const int i1 = static_cast<int>(static_cast<long>(items) * (blockIdx.x + 1) / G);
-        for (int itm = i0 + tid; itm < i1; itm += DF_THREADS) {
-            const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
-            uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                                      make_uint4(0u, 0u, 0u, 0u)};
-            uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
-            if (t < T) {
-                float v[32];
-                BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
-                if (norm) {
-                    const float r = static_cast<float>(C.inv_rms[t]);
-                    const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 g = g4[i];
-                        v[4 * i] *= g.x * r;
-                        v[4 * i + 1] *= g.y * r;
-                        v[4 * i + 2] *= g.z * r;
-                        v[4 * i + 3] *= g.w * r;
-                    }
-                }
-                mxq_block_thread(v, codes, sb);
-            }
-#pragma unroll
-            for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                *reinterpret_cast<uint4*>(xcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
-                    codes[tt];
-                xatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
-            }
-        }
-        __syncthreads();
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(&p.st->xdone, 1u);
-        }
-    }
-    // this CTA's items: equal contiguous shares of the gate/up and the down items
-    const long NG = static_cast<long>(n_t) * F_gu * KC_gu;
+    // gate/up: whole tiles u = b, b + G, ...; down: a contiguous range of items
+    // sized so that every CTA streams about the same number of bytes (a gate/up
+    // chunk and a down item are both at most 17,408 bytes)
+    const int NT = n_t * F_gu;
     const long ND = static_cast<long>(n_t) * F_dn * NP;
-    const long g_lo = NG * blockIdx.x / G, g_hi = NG * (blockIdx.x + 1) / G;
-    const long d_lo = ND * blockIdx.x / G, d_hi = ND * (blockIdx.x + 1) / G;
+    long d_lo, d_hi;
+    {
+        const long q = NT / G, r = NT % G;
+        const long W = static_cast<long>(NT) * KC_gu + ND;             // items of the whole launch
+        const long defA = max(0L, W - static_cast<long>(G) * (q + 1) * KC_gu);   // CTAs b < r (one tile more)
+        const long defB = max(0L, W - static_cast<long>(G) * q * KC_gu);
+        const long tot = r * defA + (G - r) * defB;
+        auto D = [&](long b) -> long {
+            if (b <= 0 || tot == 0) return 0;
+            if (b >= G) return ND;
+            const long pre = b < r ? b * defA : r * defA + (b - r) * defB;
+            return ND * pre / tot;
+        };
+        d_lo = D(blockIdx.x);
+        d_hi = D(blockIdx.x + 1);
+    }
     const size_t ebytes_gu = p.Mgu.expert_bytes(), ebytes_dn = p.Mdn.expert_bytes();
     const uint32_t idesc = idesc_mxf4(128, DF_NB3);
 
@@ -465,27 +421,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         for (int i = 0; i < DF_MAX_STAGES; ++i) pend_ph[i] = -1;
         bool skip = p.skip_first_copy != 0;
         bool ok = __all_sync(0xffffffffu, *abort_flag == 0);
-        for (long it = g_lo; it < g_hi + (d_hi - d_lo) && ok; ++it) {
-            const uint8_t* src;
-            uint32_t bytes;
-            if (it < g_hi) {
-                const int i = static_cast<int>(it / (F_gu * KC_gu));
-                const int rem = static_cast<int>(it % (F_gu * KC_gu));
-                const int ft = rem / KC_gu, c = rem % KC_gu;
-                const int rf = min(128, f - ft * 128);
-                src = p.Mgu.base + C.touched[i] * ebytes_gu + p.Mgu.chunk_offset(ft, c, rf);
-                bytes = static_cast<uint32_t>(p.Mgu.chunk_bytes(c, rf));
-            } else {
-                const long jt = d_lo + (it - g_hi);
-                const int i = static_cast<int>(jt / (F_dn * NP));
-                const int rem = static_cast<int>(jt % (F_dn * NP));
-                const int ft = rem / NP, j = rem % NP;
-                const int rf = min(128, d - ft * 128);
-                src = p.Mdn.base + C.touched[i] * ebytes_dn + p.Mdn.chunk_offset(ft, 2 * j, rf);
-                bytes = df_down_item_bytes(p.Mdn, j, rf);
-            }
+        auto issue = [&](const uint8_t* src, uint32_t bytes) {
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, p.status, p.timeout_ns));
-            if (!ok) break;
+            if (!ok) return;
             if (skip) {
                 skip = false;   // test hook: this stage is never filled
             } else {
@@ -494,6 +432,21 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                 pend_ph[s] = static_cast<int>(ph);
             }
             if (++s == S) { s = 0; ph ^= 1u; }
+        };
+        for (int u = blockIdx.x; u < NT && ok; u += G) {
+            const int i = u / F_gu, ft = u % F_gu;
+            const int rf = min(128, f - ft * 128);
+            const uint8_t* we = p.Mgu.base + C.touched[i] * ebytes_gu;
+            for (int c = 0; c < KC_gu && ok; ++c)
+                issue(we + p.Mgu.chunk_offset(ft, c, rf), static_cast<uint32_t>(p.Mgu.chunk_bytes(c, rf)));
+        }
+        for (long jt = d_lo; jt < d_hi && ok; ++jt) {
+            const int i = static_cast<int>(jt / (F_dn * NP));
+            const int rem = static_cast<int>(jt % (F_dn * NP));
+            const int ft = rem / NP, j = rem % NP;
+            const int rf = min(128, d - ft * 128);
+            issue(p.Mdn.base + C.touched[i] * ebytes_dn + p.Mdn.chunk_offset(ft, 2 * j, rf),
+                  df_down_item_bytes(p.Mdn, j, rf));
         }
         if (lane == 0)
             for (int i = 0; i < S; ++i)
@@ -505,12 +458,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         uint32_t ph = 0, bph = 0;
         uint32_t eph[2] = {0u, 0u};
         bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.xready), 0, abort_flag, p.status, p.timeout_ns));
-        // gate/up pieces
-        long it = g_lo;
-        while (ok && it < g_hi) {
-            const int i = static_cast<int>(it / (F_gu * KC_gu));
-            const int ft = static_cast<int>((it % (F_gu * KC_gu)) / KC_gu);
-            const long piece_end = min(g_hi, static_cast<long>(i) * F_gu * KC_gu + static_cast<long>(ft + 1) * KC_gu);
+        // gate/up tiles
+        for (int u = blockIdx.x; u < NT && ok; u += G) {
+            const int ft = u % F_gu;
             const int rf = min(128, f - ft * 128);
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.acce[buf]), eph[buf] ^ 1u, abort_flag, p.status,
                                                            p.timeout_ns));
@@ -518,9 +468,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             eph[buf] ^= 1u;
             tc_fence_after();
             const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
-            bool first = true;   // the piece's first MMA overwrites the accumulator
-            for (; it < piece_end; ++it) {
-                const int c = static_cast<int>(it % KC_gu);
+            for (int c = 0; c < KC_gu; ++c) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
@@ -534,8 +482,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     if (2 * h < nbc) {
-                        const uint32_t acc = first ? 0u : 1u;
-                        first = false;
+                        const uint32_t acc = (c > 0 || h > 0) ? 1u : 0u;
                         const uint32_t id = idesc | idesc_sf_ids(2u * h);
                         const uint64_t ad = desc_noswz(ws + 2 * h * rf * 16, rf * 16, 128);
                         const uint64_t bd = desc_noswz(bbuf + (4 * c + 2 * h) * DF_B_BLOCK, DF_B_BLOCK, 128);
@@ -616,16 +563,58 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         const int hh = (warp - 2) >> 2;          // token columns 8 hh .. 8 hh + 7
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
-        // x's B operand: once every CTA has written its share, one thread copies
-        // it (codes and scale atoms) into shared memory; xready completes on
-        // the bytes
-        if (et == 0) {
-            const uint32_t target = (epoch + 1u) * static_cast<uint32_t>(G);
-            if (spin_until_reached(&p.st->xdone, target, abort_flag, p.status, p.timeout_ns)) {
-                const uint32_t cb = static_cast<uint32_t>(nb_d) * DF_B_BLOCK, ab = static_cast<uint32_t>(KC_gu) * 512u;
-                mbar_arrive_expect_tx(smem_u32(&C.xready), cb + ab);
-                bulk_g2s(bbuf, p.xq, cb, smem_u32(&C.xready));
-                bulk_g2s(bsf, p.xq + cb, ab, smem_u32(&C.xready));
+        // this CTA's share of x's B operand (every token row, 16 per term; rows
+        // past T are zero), written to global memory; the count tells the grid
+        {
+            uint8_t* xcodes = p.xq;
+            uint8_t* xatoms = p.xq + static_cast<size_t>(nb_d) * DF_B_BLOCK;
+            const int items = nb_d * DF_MAX_T;
+            const int i0 = static_cast<int>(static_cast<long>(items) * blockIdx.x / G);
+            const int i1 = static_cast<int>(static_cast<long>(items) * (blockIdx.x + 1) / G);
+            for (int itm = i0 + et; itm < i1; itm += DF_EPI_THREADS) {
+                const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
+                uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                                          make_uint4(0u, 0u, 0u, 0u)};
+                uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
+                if (t < T) {
+                    float v[32];
+                    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
+                    if (norm) {
+                        const float r = static_cast<float>(C.inv_rms[t]);
+                        const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 g = g4[i];
+                            v[4 * i] *= g.x * r;
+                            v[4 * i + 1] *= g.y * r;
+                            v[4 * i + 2] *= g.z * r;
+                            v[4 * i + 3] *= g.w * r;
+                        }
+                    }
+                    mxq_block_thread(v, codes, sb);
+                }
+#pragma unroll
+                for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                    *reinterpret_cast<uint4*>(xcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                        codes[tt];
+                    xatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
+                }
+            }
+            named_barrier(1, DF_EPI_THREADS);
+            if (et == 0) {
+                __threadfence();
+                atomicAdd(&p.st->xdone, 1u);
+                // when every share is written, copy the operand (codes and scale
+                // atoms) into shared memory; xready completes on the bytes
+                const uint32_t target = (epoch + 1u) * static_cast<uint32_t>(G);
+                if (spin_until_reached(&p.st->xdone, target, abort_flag, p.status, p.timeout_ns)) {
+                    fence_proxy_async_global();
+                    const uint32_t cb = static_cast<uint32_t>(nb_d) * DF_B_BLOCK,
+                                   ab = static_cast<uint32_t>(KC_gu) * 512u;
+                    mbar_arrive_expect_tx(smem_u32(&C.xready), cb + ab);
+                    bulk_g2s(bbuf, p.xq, cb, smem_u32(&C.xready));
+                    bulk_g2s(bsf, p.xq + cb, ab, smem_u32(&C.xready));
+                }
             }
         }
         bool ok = named_barrier_and(1, DF_EPI_THREADS, *abort_flag == 0);
@@ -643,32 +632,40 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                 out[j] = __uint_as_float(r[0][j]) + __uint_as_float(r[1][j]) + __uint_as_float(r[2][j]);
         };
 
-        // gate/up pieces: partial sums of g and u into GU, then count the chunks
-        long it = g_lo;
-        while (ok && it < g_hi) {
-            const int i = static_cast<int>(it / (F_gu * KC_gu));
-            const int ft = static_cast<int>((it % (F_gu * KC_gu)) / KC_gu);
-            const long piece_end = min(g_hi, static_cast<long>(i) * F_gu * KC_gu + static_cast<long>(ft + 1) * KC_gu);
+        // gate/up tiles: H of the tile's 128 features for every token row (zero
+        // rows for tokens not routed to the expert) into the expert's H operand,
+        // then the tile's stamp
+        for (int u = blockIdx.x; u < NT && ok; u += G) {
+            const int i = u / F_gu, ft = u % F_gu;
             const int rf = min(128, f - ft * 128);
             const bool w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[buf]), fph[buf], abort_flag,
                                                                          p.status, p.timeout_ns));
             fph[buf] ^= 1u;
             tc_fence_after();
-            if (w_ok && 32 * q < rf && 8 * hh < T) {
+            if (w_ok && 32 * q < rf) {
                 const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
-                float g[8], u[8];
+                float g[8], uu[8];
                 load_acc(d0, g);
-                load_acc(d0 + DF_MAT_COLS, u);
-                const int n = ft * 128 + 32 * q + lane;
-                if (32 * q + lane < rf) {
+                load_acc(d0 + DF_MAT_COLS, uu);
+                const int b = 4 * ft + q;   // the warp's 32-feature block of H
+                uint8_t* hcodes = p.hq + i * p.hq_stride;
+                uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j) {
+                    const int t = 8 * hh + j;
+                    uint32_t w[MXQ_TERMS] = {0u, 0u, 0u}, sb[MXQ_TERMS] = {0u, 0u, 0u};
+                    if (t < T && C.selw[i][t] != 0.f) mxq_block_warp(swish_f(g[j]) * uu[j], w, sb);
+                    if (lane < 4) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int t = 8 * hh + j;
-                        if (t < T && C.selw[i][t] != 0.f) {
-                            float* row = gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f;
-                            atomicAdd(row + n, g[j]);
-                            atomicAdd(row + f + n, u[j]);
-                        }
+                        for (int tt = 0; tt < MXQ_TERMS; ++tt)
+                            reinterpret_cast<uint32_t*>(hcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) *
+                                                                     16)[lane] = w[tt];
+                    }
+                    if (lane == 0) {
+#pragma unroll
+                        for (int tt = 0; tt < MXQ_TERMS; ++tt)
+                            hatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] =
+                                static_cast<uint8_t>(sb[tt]);
                     }
                 }
             }
@@ -676,58 +673,16 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             __syncwarp();
             if (w_ok && lane == 0) mbar_arrive(smem_u32(&C.acce[buf]));
             buf ^= 1;
-            __threadfence();
             // every epilogue thread takes the same decision (no thread is left waiting)
             ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
             if (!ok) break;
             if (et == 0) {
-                const uint32_t n = static_cast<uint32_t>(piece_end - it);
-                const uint32_t old = atomicAdd(&p.done[i * F_gu + ft], n);
-                __threadfence();   // acquire: the other contributors' partial sums are visible
-                C.tile_done = (old + n == static_cast<uint32_t>(KC_gu)) ? 1 : 0;
-            }
-            named_barrier(1, DF_EPI_THREADS);
-            if (C.tile_done) {
-                // H of feature tile ft (blocks 4 ft .. 4 ft + 3) for every token row of
-                // the slot: Swish(g) u of the routed tokens, zero rows for the rest
-                uint8_t* hcodes = p.hq + i * p.hq_stride;
-                uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
-                for (int itm = et; itm < 4 * DF_MAX_T; itm += DF_EPI_THREADS) {
-                    const int b = 4 * ft + itm / DF_MAX_T, t = itm % DF_MAX_T;
-                    if (b >= nb_f) continue;
-                    uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                                              make_uint4(0u, 0u, 0u, 0u)};
-                    uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
-                    if (t < T && C.selw[i][t] != 0.f) {
-                        const float* row = gu + (static_cast<size_t>(i) * DF_MAX_T + t) * 2 * f;
-                        const float4* g4 = reinterpret_cast<const float4*>(row + 32 * b);
-                        const float4* u4 = reinterpret_cast<const float4*>(row + f + 32 * b);
-                        float v[32];
-#pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 gg = __ldcg(g4 + q4), uu = __ldcg(u4 + q4);
-                            v[4 * q4] = swish_f(gg.x) * uu.x;
-                            v[4 * q4 + 1] = swish_f(gg.y) * uu.y;
-                            v[4 * q4 + 2] = swish_f(gg.z) * uu.z;
-                            v[4 * q4 + 3] = swish_f(gg.w) * uu.w;
-                        }
-                        mxq_block_thread(v, codes, sb);
-                    }
-#pragma unroll
-                    for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                        *reinterpret_cast<uint4*>(hcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
-                            codes[tt];
-                        hatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
-                    }
-                }
                 __threadfence();
-                named_barrier(1, DF_EPI_THREADS);
-                if (et == 0) atomicExch(&p.hdone[i * F_gu + ft], epoch + 1u);
+                atomicExch(&p.hdone[i * F_gu + ft], epoch + 1u);
             }
-            it = piece_end;
         }
 
-        // down pieces: wait for g and u, build the H operand, combine
+        // down pieces: wait for H, copy it in, combine
         long jt = d_lo;
         int pend_buf = -1, pend_i = 0, pend_ft = 0, pend_rf = 0;
         auto drain_pending = [&]() {
@@ -775,6 +730,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             // the piece's range of the expert's H operand into shared memory (bready
             // completes on the bytes)
             if (et == 0) {
+                __threadfence();   // acquire side of the stamps the other threads read
+                fence_proxy_async_global();
                 const uint8_t* hcodes = p.hq + i * p.hq_stride;
                 const uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
                 const int b0 = 4 * c0, b1 = min(4 * c1, nb_f);
@@ -800,10 +757,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                 drain_pending();
             }
         }
-        __threadfence();
     }
 
-    // ---- finish: free tensor memory; the last CTA writes y and resets the state
+    // ---- finish: free tensor memory; the last CTA writes y
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -846,11 +802,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                 reinterpret_cast<float4*>(p.y)[i4] = v;
             }
         }
-        for (int i = tid; i < n_t * F_gu; i += DF_THREADS) p.done[i] = 0u;
         __syncthreads();
         if (tid == 0) {
-            p.st->prev_nt = n_t;
-            p.st->prev_T = T;
             p.st->finish = 0u;
             __threadfence();
             atomicAdd(&p.st->epoch, 1u);

@@ -119,10 +119,8 @@ struct moe_mxfp4 {
     int df_stages = 0, df_S = 0, df_nb_max = 0, df_kc_max = 0, df_max_touched = 0;
     size_t df_smem = 0;
     DecodeState* df_state = nullptr;
-    uint32_t* df_done = nullptr;
     double* df_part = nullptr;
     double* df_part_ss = nullptr;
-    float* df_gu = nullptr;
     float* df_yacc = nullptr;
     uint8_t* df_xq = nullptr;
     uint8_t* df_hq = nullptr;
@@ -211,8 +209,7 @@ static void free_all(moe_mxfp4* h) {
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
-                    h->df_state, h->df_done, h->df_part, h->df_part_ss, h->df_gu, h->df_yacc,
-                    h->df_xq, h->df_hq, h->df_hdone};
+                    h->df_state, h->df_part, h->df_part_ss, h->df_yacc, h->df_xq, h->df_hq, h->df_hdone};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     for (auto& e : h->ev)
@@ -498,21 +495,18 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
                                                                     h->df_smem);
             if (oe != cudaSuccess) return fail(MOE_ERR_CUDA);
             if (per_sm >= 1) {
-                const size_t gu_bytes_df = sizeof(float) * 2 * h->df_max_touched * DF_MAX_T * 2 * static_cast<size_t>(f);
                 const size_t ya_bytes_df = sizeof(float) * 2 * DF_MAX_T * static_cast<size_t>(d);
-                const size_t done_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu;
+                const size_t stamp_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu;
                 const size_t xq_bytes = static_cast<size_t>(d / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_gu) * 512;
                 h->df_hq_stride = static_cast<size_t>(f / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_dn) * 512;
                 A dfa[] = {
                     {reinterpret_cast<void**>(&h->df_state), sizeof(DecodeState)},
-                    {reinterpret_cast<void**>(&h->df_done), done_bytes},
                     {reinterpret_cast<void**>(&h->df_part), sizeof(double) * h->df_S * DF_MAX_T * E},
                     {reinterpret_cast<void**>(&h->df_part_ss), sizeof(double) * h->df_S * DF_MAX_T},
-                    {reinterpret_cast<void**>(&h->df_gu), gu_bytes_df},
                     {reinterpret_cast<void**>(&h->df_yacc), ya_bytes_df},
                     {reinterpret_cast<void**>(&h->df_xq), xq_bytes},
                     {reinterpret_cast<void**>(&h->df_hq), h->df_hq_stride * h->df_max_touched},
-                    {reinterpret_cast<void**>(&h->df_hdone), done_bytes},
+                    {reinterpret_cast<void**>(&h->df_hdone), stamp_bytes},
                 };
                 for (auto& a : dfa) {
                     if (++n_alloc == fail_at) return fail(MOE_ERR_CUDA);
@@ -721,12 +715,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         dp.stages = h->df_stages;
         dp.nb_max = h->df_nb_max;
         dp.kc_max = h->df_kc_max;
-        dp.max_touched = h->df_max_touched;
         dp.st = h->df_state;
-        dp.done = h->df_done;
         dp.part = h->df_part;
         dp.part_ss = h->df_part_ss;
-        dp.gu = h->df_gu;
         dp.yacc = h->df_yacc;
         dp.xq = h->df_xq;
         dp.hq = h->df_hq;

@@ -88,4 +88,36 @@ __device__ __forceinline__ void mxq_block_thread(float (&v)[32], uint4 (&codes)[
     }
 }
 
+// One block of 32 values held one per lane (lane = element) encoded as three
+// MXFP4 terms by the whole warp, with the same rule and rounding as
+// mxq_block_thread.  Lanes 0..3 return word `lane` of each term's 16 code
+// bytes in w[t]; every lane returns the E8M0 bytes in sbyte[t].
+__device__ __forceinline__ void mxq_block_warp(float v, uint32_t (&w)[MXQ_TERMS], uint32_t (&sbyte)[MXQ_TERMS]) {
+    const int lane = threadIdx.x & 31;
+    const bool even = (lane & 1) == 0;
+#pragma unroll
+    for (int t = 0; t < MXQ_TERMS; ++t) {
+        float am = fabsf(v);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        const int e = mxq_exp(__float_as_uint(am));
+        sbyte[t] = static_cast<uint32_t>(e + 127);
+        const float q = v * mxq_inv(e);
+        const float qn = __shfl_xor_sync(0xffffffffu, q, 1);
+        // both lanes of a pair form the byte of elements (2i, 2i+1)
+        const uint32_t byte = even ? e2m1x2_from_f32(q, qn) : e2m1x2_from_f32(qn, q);
+        if (t + 1 < MXQ_TERMS) {
+            const uint32_t h2 = e2m1x2_to_f16x2(byte);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+            v -= (even ? f.x : f.y) * mxq_scale(e);
+        }
+        // word m holds bytes 4m .. 4m+3, i.e. the bytes of lanes 8m, 8m+2, 8m+4, 8m+6
+        const int m = lane & 3;
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) word |= (__shfl_sync(0xffffffffu, byte, 8 * m + 2 * j) & 0xFFu) << (8 * j);
+        w[t] = word;
+    }
+}
+
 }  // namespace moe

@@ -147,6 +147,12 @@ __device__ __forceinline__ bool spin_until_reached(const uint32_t* p, uint32_t t
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Order global-memory accesses of the generic proxy (what this thread has
+// acquired: data other CTAs wrote with ordinary stores) before this thread's
+// later async-proxy accesses (bulk copies reading that data).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 // Named barrier over `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
