@@ -216,6 +216,57 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             y_other[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
+    // ---- this CTA's share of x's B operand (every token row, 16 per term; rows
+    // past T are zero), written to global memory; xdone tells the grid.  x does
+    // not depend on the routing: without the pre-norm the share is written
+    // first, so the operand is complete by the time the routing is; with it
+    // the share waits for the RMS of each token.
+    const int nb_d = d / 32, nb_f = f / 32;
+    auto x_share = [&](int first, int stride) {
+        uint8_t* xcodes = p.xq;
+        uint8_t* xatoms = p.xq + static_cast<size_t>(nb_d) * DF_B_BLOCK;
+        const int items = nb_d * DF_MAX_T;
+        const int i0 = static_cast<int>(static_cast<long>(items) * blockIdx.x / G);
+        const int i1 = static_cast<int>(static_cast<long>(items) * (blockIdx.x + 1) / G);
+        for (int itm = i0 + first; itm < i1; itm += stride) {
+            const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
+            uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                                      make_uint4(0u, 0u, 0u, 0u)};
+            uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
+            if (t < T) {
+                float v[32];
+                BlockLoader<TA>::load(static_cast<const TA*>(p.x) + static_cast<size_t>(t) * d + b * 32, v);
+                if (norm) {
+                    const float r = static_cast<float>(C.inv_rms[t]);
+                    const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 g = g4[i];
+                        v[4 * i] *= g.x * r;
+                        v[4 * i + 1] *= g.y * r;
+                        v[4 * i + 2] *= g.z * r;
+                        v[4 * i + 3] *= g.w * r;
+                    }
+                }
+                mxq_block_thread(v, codes, sb);
+            }
+#pragma unroll
+            for (int tt = 0; tt < MXQ_TERMS; ++tt) {
+                *reinterpret_cast<uint4*>(xcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
+                    codes[tt];
+                xatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
+            }
+        }
+    };
+    if (!norm) {
+        x_share(tid, DF_THREADS);
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(&p.st->xdone, 1u);
+        }
+    }
+
     // ---- 1. router partials over (expert, K split) units
     const TA* x = static_cast<const TA*>(p.x);
     const TA* wr = static_cast<const TA*>(p.wr);
@@ -388,7 +439,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         __syncthreads();
     }
     const int n_t = C.n_t;
-    const int nb_d = d / 32, nb_f = f / 32;
     // gate/up: whole tiles u = b, b + G, ...; down: a contiguous range of items
     // sized so that every CTA streams about the same number of bytes (a gate/up
     // chunk and a down item are both at most 17,408 bytes)
@@ -563,47 +613,15 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         const int hh = (warp - 2) >> 2;          // token columns 8 hh .. 8 hh + 7
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
 
-        // this CTA's share of x's B operand (every token row, 16 per term; rows
-        // past T are zero), written to global memory; the count tells the grid
+        // with the pre-norm, this CTA's share of x's operand now (see above)
         {
-            uint8_t* xcodes = p.xq;
-            uint8_t* xatoms = p.xq + static_cast<size_t>(nb_d) * DF_B_BLOCK;
-            const int items = nb_d * DF_MAX_T;
-            const int i0 = static_cast<int>(static_cast<long>(items) * blockIdx.x / G);
-            const int i1 = static_cast<int>(static_cast<long>(items) * (blockIdx.x + 1) / G);
-            for (int itm = i0 + et; itm < i1; itm += DF_EPI_THREADS) {
-                const int b = itm / DF_MAX_T, t = itm % DF_MAX_T;
-                uint4 codes[MXQ_TERMS] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                                          make_uint4(0u, 0u, 0u, 0u)};
-                uint32_t sb[MXQ_TERMS] = {0u, 0u, 0u};
-                if (t < T) {
-                    float v[32];
-                    BlockLoader<TA>::load(x + static_cast<size_t>(t) * d + b * 32, v);
-                    if (norm) {
-                        const float r = static_cast<float>(C.inv_rms[t]);
-                        const float4* g4 = reinterpret_cast<const float4*>(p.gamma + b * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 g = g4[i];
-                            v[4 * i] *= g.x * r;
-                            v[4 * i + 1] *= g.y * r;
-                            v[4 * i + 2] *= g.z * r;
-                            v[4 * i + 3] *= g.w * r;
-                        }
-                    }
-                    mxq_block_thread(v, codes, sb);
-                }
-#pragma unroll
-                for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                    *reinterpret_cast<uint4*>(xcodes + (static_cast<size_t>(b) * DF_NB3 + tt * DF_MAX_T + t) * 16) =
-                        codes[tt];
-                    xatoms[(b >> 2) * 512 + sf_atom_offset(tt * DF_MAX_T + t, b & 3)] = static_cast<uint8_t>(sb[tt]);
-                }
-            }
+            if (norm) x_share(et, DF_EPI_THREADS);
             named_barrier(1, DF_EPI_THREADS);
             if (et == 0) {
-                __threadfence();
-                atomicAdd(&p.st->xdone, 1u);
+                if (norm) {
+                    __threadfence();
+                    atomicAdd(&p.st->xdone, 1u);
+                }
                 // when every share is written, copy the operand (codes and scale
                 // atoms) into shared memory; xready completes on the bytes
                 const uint32_t target = (epoch + 1u) * static_cast<uint32_t>(G);
@@ -713,11 +731,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             const int rf = min(128, d - ft * 128);
             const int c0 = 2 * static_cast<int>(jt % NP);
             const int c1 = min(KC_dn, 2 * static_cast<int>((piece_end - 1) % NP) + 2);
-            // H of features [128 c0, 128 c1) written (gate/up feature tiles c0 .. c1-1 stamped)
+            // H of features [128 c0, 128 c1) written (gate/up feature tiles c0 .. c1-1
+            // stamped): one thread polls the stamps in turn (they share a line or two)
             bool w_ok = true;
-            if (et < c1 - c0)
-                w_ok = spin_until_reached(&p.hdone[i * F_gu + c0 + et], epoch + 1u, abort_flag, p.status,
-                                          p.timeout_ns);
+            if (et == 0)
+                for (int ft_g = c0; ft_g < c1 && w_ok; ++ft_g)
+                    w_ok = spin_until_reached(&p.hdone[i * F_gu + ft_g], epoch + 1u, abort_flag, p.status,
+                                              p.timeout_ns);
             // the previous down piece's MMAs must be done before its operand is overwritten
             if (pend_buf >= 0) {
                 w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag,

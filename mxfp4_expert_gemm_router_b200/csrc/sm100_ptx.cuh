@@ -125,13 +125,18 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// The polling interval backs off from 32 ns to 512 ns: many CTAs polling one
+// line of L2 at a high rate slow down the slice that holds it, and with it
+// every stream that passes through that slice.
 __device__ __forceinline__ bool spin_until_reached(const uint32_t* p, uint32_t target, volatile int* abort_flag,
                                                    int* status, uint64_t limit_ns) {
     if (static_cast<int>(ld_acquire_u32(p) - target) >= 0) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint32_t pause = 32;
 #pragma unroll 1
     while (true) {
-        __nanosleep(64);
+        __nanosleep(pause);
+        if (pause < 512) pause <<= 1;
         if (static_cast<int>(ld_acquire_u32(p) - target) >= 0) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
