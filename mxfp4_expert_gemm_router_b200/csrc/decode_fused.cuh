@@ -72,7 +72,9 @@ namespace moe {
 constexpr int DF_MAX_T = 16;                 // token rows per term of the B operand
 constexpr int DF_NB3 = MXQ_TERMS * DF_MAX_T; // 48 operand rows
 constexpr int DF_EPI_WARPS = 8;
-constexpr int DF_THREADS = (2 + DF_EPI_WARPS) * 32;
+// warps: 0 weight producer, 1 MMA issuer, 2..9 epilogue, 10 H-operand issuer
+constexpr int DF_HWARP = 2 + DF_EPI_WARPS;
+constexpr int DF_THREADS = (3 + DF_EPI_WARPS) * 32;
 constexpr int DF_EPI_THREADS = DF_EPI_WARPS * 32;
 constexpr uint32_t DF_STAGE = 2u * (4u * 128 * 16 + 512);   // 17,408 bytes
 constexpr int DF_MAX_STAGES = 8;
@@ -83,6 +85,9 @@ constexpr int DF_SF_SLOTS = 2;
 constexpr int DF_SF_SLOT_COLS = 32;
 constexpr uint32_t DF_B_BLOCK = DF_NB3 * 16;  // 768 bytes of B codes per 32-block
 constexpr int DF_MAX_TOUCHED = DF_MAX_T * MAX_TOPK;   // touched experts <= T * k
+// H ring slot of one down item (two K chunks): codes [2][4 blocks][48][16 B], then two scale atoms
+constexpr uint32_t DF_HSLOT_CODES = 2u * 4u * DF_B_BLOCK;   // 6144
+constexpr uint32_t DF_HSLOT = DF_HSLOT_CODES + 2u * 512u;   // 7168
 
 struct DecodeState {
     uint32_t bar;      // grid-barrier arrivals: grows by gridDim.x per launch
@@ -114,7 +119,7 @@ struct DecodeParams {
     uint8_t* xq;            // x as the B operand: codes [d/32][48][16 B], then scale atoms [KC_gu][512]
     uint8_t* hq;            // H per touched slot (stride hq_stride): codes [f/32][48][16 B], atoms [KC_dn][512]
     size_t hq_stride;
-    uint32_t* hdone;        // [max_touched][F_gu] epoch + 1 once H of (slot, feature tile) is in hq
+    uint32_t* hdone;        // [max_touched][F_gu][8] epoch + 1 once epilogue warp w wrote its part of the tile's H
     int32_t* topk_idx;      // [T][k] or null
     float* topk_w;          // [T][k] or null
     int32_t* counts;        // [E] or null
@@ -126,7 +131,8 @@ struct DecodeParams {
 // Shared memory after the 1024-aligned weight ring and B buffer.
 struct DecodeCtl {
     uint64_t full[DF_MAX_STAGES], empty[DF_MAX_STAGES];
-    uint64_t accf[2], acce[2], xready, bready, drain;
+    uint64_t hfull[DF_MAX_STAGES], hempty[DF_MAX_STAGES];
+    uint64_t accf[2], acce[2], xready, xfree, drain;
     int abort_flag;
     uint32_t tmem;
     int last;
@@ -142,8 +148,15 @@ struct DecodeCtl {
 __host__ __device__ inline uint32_t df_bbuf_bytes(int nb_max, int kc_max) {
     return static_cast<uint32_t>(nb_max) * DF_B_BLOCK + static_cast<uint32_t>(kc_max) * 512u;
 }
+// The B buffer holds x's operand during the gate/up work and the H ring (one
+// slot per weight stage) during the down work.
+__host__ __device__ inline uint32_t df_bregion_bytes(int stages, int nb_max, int kc_max) {
+    const uint32_t a = df_bbuf_bytes(nb_max, kc_max), b = static_cast<uint32_t>(stages) * DF_HSLOT;
+    return a > b ? a : b;
+}
 __host__ inline size_t df_smem_bytes(int stages, int nb_max, int kc_max) {
-    return 1024 + static_cast<size_t>(stages) * DF_STAGE + df_bbuf_bytes(nb_max, kc_max) + sizeof(DecodeCtl) + 16;
+    return 1024 + static_cast<size_t>(stages) * DF_STAGE + df_bregion_bytes(stages, nb_max, kc_max) +
+           sizeof(DecodeCtl) + 16;
 }
 
 // Bytes of the down item j (chunks 2j and 2j+1 of feature tile ft): contiguous in the tiled layout.
@@ -168,7 +181,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
     const uint32_t bsf = bbuf + static_cast<uint32_t>(p.nb_max) * DF_B_BLOCK;    // B scale atoms
     uint8_t* bbuf_ptr = base_ptr + static_cast<size_t>(p.stages) * DF_STAGE;
     uint8_t* bsf_ptr = bbuf_ptr + static_cast<size_t>(p.nb_max) * DF_B_BLOCK;
-    DecodeCtl& C = *reinterpret_cast<DecodeCtl*>(bsf_ptr + static_cast<size_t>(p.kc_max) * 512);
+    DecodeCtl& C = *reinterpret_cast<DecodeCtl*>(bbuf_ptr + df_bregion_bytes(p.stages, p.nb_max, p.kc_max));
     volatile int* abort_flag = &C.abort_flag;
     const int S = p.stages;
     auto full_bar = [&](int s) { return smem_u32(&C.full[s]); };
@@ -188,8 +201,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             mbar_init(smem_u32(&C.accf[b]), 1);
             mbar_init(smem_u32(&C.acce[b]), DF_EPI_WARPS);
         }
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_u32(&C.hfull[s]), 1);
+            mbar_init(smem_u32(&C.hempty[s]), 1);   // the MMA commit of the H slot
+        }
         mbar_init(smem_u32(&C.xready), 1);
-        mbar_init(smem_u32(&C.bready), 1);
+        mbar_init(smem_u32(&C.xfree), 1);
         mbar_init(smem_u32(&C.drain), 1);
         C.abort_flag = 0;
         C.last = 0;
@@ -505,7 +522,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
     } else if (warp == 1) {
         // -------------------------------------------------------------- MMA issuer
         int s = 0, sfs = 0, buf = 0;
-        uint32_t ph = 0, bph = 0;
+        uint32_t ph = 0;
         uint32_t eph[2] = {0u, 0u};
         bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.xready), 0, abort_flag, p.status, p.timeout_ns));
         // gate/up tiles
@@ -548,17 +565,16 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             tc_commit_warp(smem_u32(&C.accf[buf]));
             buf ^= 1;
         }
-        // down pieces
+        // down pieces: item k of this CTA takes weight stage s (the producer's
+        // sequence) and H slot k % S (the H issuer's sequence)
         long jt = d_lo;
+        int hs = 0;
+        uint32_t hph = 0;
         while (ok && jt < d_hi) {
             const int i = static_cast<int>(jt / (F_dn * NP));
             const int ft = static_cast<int>((jt % (F_dn * NP)) / NP);
             const long piece_end = min(d_hi, static_cast<long>(i) * F_dn * NP + static_cast<long>(ft + 1) * NP);
             const int rf = min(128, d - ft * 128);
-            const int pc0 = 2 * static_cast<int>(jt % NP);   // first K chunk of the piece
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.bready), bph, abort_flag, p.status, p.timeout_ns));
-            if (!ok) break;
-            bph ^= 1u;
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.acce[buf]), eph[buf] ^ 1u, abort_flag, p.status,
                                                            p.timeout_ns));
             if (!ok) break;
@@ -569,9 +585,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             for (; jt < piece_end; ++jt) {
                 const int j = static_cast<int>(jt % NP);
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), ph, abort_flag, p.status, p.timeout_ns));
+                if (ok)
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.hfull[hs]), hph, abort_flag, p.status,
+                                                                   p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t ws = ring + s * DF_STAGE;
+                const uint32_t hsl = bbuf + hs * DF_HSLOT;
                 const uint32_t sfc = tmem + DF_SF_COL0 + DF_SF_SLOT_COLS * sfs;
                 uint32_t off = 0;
                 for (int hc = 0; hc < 2; ++hc) {
@@ -580,7 +600,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                     const int nbc = p.Mdn.blocks_in_chunk(c);
                     const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16);
                     tc_cp_sf_warp(sfc + 4 * hc, desc_noswz(ws + off + codes_b, 0, 128));
-                    tc_cp_sf_warp(sfc + 8 + 4 * hc, desc_noswz(bsf + (c - pc0) * 512u, 0, 128));
+                    tc_cp_sf_warp(sfc + 8 + 4 * hc, desc_noswz(hsl + DF_HSLOT_CODES + hc * 512u, 0, 128));
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (2 * h < nbc) {
@@ -588,15 +608,16 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                             first = false;
                             const uint32_t id = idesc | idesc_sf_ids(2u * h);
                             const uint64_t ad = desc_noswz(ws + off + 2 * h * rf * 16, rf * 16, 128);
-                            const uint64_t bd =
-                                desc_noswz(bbuf + (4 * (c - pc0) + 2 * h) * DF_B_BLOCK, DF_B_BLOCK, 128);
+                            const uint64_t bd = desc_noswz(hsl + (4 * hc + 2 * h) * DF_B_BLOCK, DF_B_BLOCK, 128);
                             mma_mxf4_warp(d0, ad, bd, id, sfc + 4 * hc, sfc + 8 + 4 * hc, acc);
                         }
                     }
                     off += codes_b + 512u;
                 }
                 tc_commit_warp(empty_bar(s));
+                tc_commit_warp(smem_u32(&C.hempty[hs]));
                 if (++s == S) { s = 0; ph ^= 1u; }
+                if (++hs == S) { hs = 0; hph ^= 1u; }
                 if (++sfs == DF_SF_SLOTS) sfs = 0;
             }
             if (!ok) break;
@@ -606,7 +627,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
         tc_commit_warp(smem_u32(&C.drain));
         if (lane == 0) mbar_wait_drain(smem_u32(&C.drain), 0, 200000000ull);
         __syncwarp();
-    } else {
+    } else if (warp < DF_HWARP) {
         // -------------------------------------------------------------- epilogue warps
         const int et = tid - 64;                 // 0 .. 255
         const int q = warp & 3;                  // TMEM lane quarter (hardware rule: warp % 4)
@@ -688,95 +709,101 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
                 }
             }
             tc_fence_before();
+            // this warp's part of the tile's H is written: stamp it (each lane that
+            // stored fences its own stores first)
+            if (lane < 4) __threadfence();
             __syncwarp();
-            if (w_ok && lane == 0) mbar_arrive(smem_u32(&C.acce[buf]));
+            if (w_ok && lane == 0) {
+                mbar_arrive(smem_u32(&C.acce[buf]));
+                atomicExch(&p.hdone[(static_cast<size_t>(i) * F_gu + ft) * DF_EPI_WARPS + (warp - 2)], epoch + 1u);
+            }
             buf ^= 1;
             // every epilogue thread takes the same decision (no thread is left waiting)
             ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
-            if (!ok) break;
-            if (et == 0) {
-                __threadfence();
-                atomicExch(&p.hdone[i * F_gu + ft], epoch + 1u);
-            }
         }
+        // the x operand is no longer read (every gate/up MMA has completed): the
+        // H issuer may reuse its space
+        if (et == 0) mbar_arrive(smem_u32(&C.xfree));
 
-        // down pieces: wait for H, copy it in, combine
+        // down pieces: y_acc[t] += w[t, e] D for the tokens routed to the piece's expert
         long jt = d_lo;
-        int pend_buf = -1, pend_i = 0, pend_ft = 0, pend_rf = 0;
-        auto drain_pending = [&]() {
-            // the pending piece's MMAs have completed (its accumulator-full phase was waited)
-            if (32 * q < pend_rf && 8 * hh < T) {
-                const uint32_t d0 = tmem + static_cast<uint32_t>(pend_buf * DF_ACC_COLS);
+        while (ok && jt < d_hi) {
+            const int i = static_cast<int>(jt / (F_dn * NP));
+            const int ft = static_cast<int>((jt % (F_dn * NP)) / NP);
+            const long piece_end = min(d_hi, static_cast<long>(i) * F_dn * NP + static_cast<long>(ft + 1) * NP);
+            const int rf = min(128, d - ft * 128);
+            const bool w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[buf]), fph[buf], abort_flag,
+                                                                         p.status, p.timeout_ns));
+            fph[buf] ^= 1u;
+            tc_fence_after();
+            if (w_ok && 32 * q < rf && 8 * hh < T) {
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf * DF_ACC_COLS);
                 float o[8];
                 load_acc(d0, o);
-                const int n = pend_ft * 128 + 32 * q + lane;
-                if (32 * q + lane < pend_rf) {
+                const int n = ft * 128 + 32 * q + lane;
+                if (32 * q + lane < rf) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const int t = 8 * hh + j;
-                        const float w = t < T ? C.selw[pend_i][t] : 0.f;
+                        const float w = t < T ? C.selw[i][t] : 0.f;
                         if (w != 0.f) atomicAdd(yacc + static_cast<size_t>(t) * d + n, w * o[j]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&C.acce[pend_buf]));
-            pend_buf = -1;
-        };
-        while (ok && jt < d_hi) {
-            const int i = static_cast<int>(jt / (F_dn * NP));
-            const int ft = static_cast<int>((jt % (F_dn * NP)) / NP);
-            const long piece_end = min(d_hi, static_cast<long>(i) * F_dn * NP + static_cast<long>(ft + 1) * NP);
-            const int rf = min(128, d - ft * 128);
-            const int c0 = 2 * static_cast<int>(jt % NP);
-            const int c1 = min(KC_dn, 2 * static_cast<int>((piece_end - 1) % NP) + 2);
-            // H of features [128 c0, 128 c1) written (gate/up feature tiles c0 .. c1-1
-            // stamped): one thread polls the stamps in turn (they share a line or two)
-            bool w_ok = true;
-            if (et == 0)
-                for (int ft_g = c0; ft_g < c1 && w_ok; ++ft_g)
-                    w_ok = spin_until_reached(&p.hdone[i * F_gu + ft_g], epoch + 1u, abort_flag, p.status,
-                                              p.timeout_ns);
-            // the previous down piece's MMAs must be done before its operand is overwritten
-            if (pend_buf >= 0) {
-                w_ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag,
-                                                                 p.status, p.timeout_ns)) && w_ok;
-                fph[pend_buf] ^= 1u;
-                tc_fence_after();
-            }
+            if (w_ok && lane == 0) mbar_arrive(smem_u32(&C.acce[buf]));
+            buf ^= 1;
             ok = named_barrier_and(1, DF_EPI_THREADS, w_ok);
+            jt = piece_end;
+        }
+    } else {
+        // -------------------------------------------------------------- H issuer
+        // For down item k of this CTA (H slot k % S): once the slot is free and
+        // the gate/up tiles of its two K chunks are stamped by all their
+        // epilogue warps, copy that part of the expert's H operand (codes of 8
+        // blocks, 2 scale atoms) into the slot; hfull completes on the bytes.
+        int hs = 0;
+        uint32_t hph = 0;
+        int hpend[DF_MAX_STAGES];
+        for (int i = 0; i < DF_MAX_STAGES; ++i) hpend[i] = -1;
+        bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.xready), 0, abort_flag, p.status, p.timeout_ns));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.xfree), 0, abort_flag, p.status, p.timeout_ns));
+        for (long jt = d_lo; jt < d_hi && ok; ++jt) {
+            const int i = static_cast<int>(jt / (F_dn * NP));
+            const int j = static_cast<int>(jt % NP);
+            const int c0 = 2 * j, c1 = min(KC_dn, c0 + 2);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&C.hempty[hs]), hph ^ 1u, abort_flag, p.status,
+                                                           p.timeout_ns));
             if (!ok) break;
-            // the piece's range of the expert's H operand into shared memory (bready
-            // completes on the bytes)
-            if (et == 0) {
-                __threadfence();   // acquire side of the stamps the other threads read
+            if (lane < (c1 - c0) * DF_EPI_WARPS) {
+                // lane l polls the stamp of warp l % 8 of gate/up tile c0 + l / 8
+                const int ft_g = c0 + lane / DF_EPI_WARPS, wq = lane % DF_EPI_WARPS;
+                ok = spin_until_reached(&p.hdone[(static_cast<size_t>(i) * F_gu + ft_g) * DF_EPI_WARPS + wq], epoch + 1u,
+                                        abort_flag, p.status, p.timeout_ns);
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (lane == 0) {
+                __threadfence();
                 fence_proxy_async_global();
                 const uint8_t* hcodes = p.hq + i * p.hq_stride;
                 const uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;
                 const int b0 = 4 * c0, b1 = min(4 * c1, nb_f);
                 const uint32_t cb = static_cast<uint32_t>(b1 - b0) * DF_B_BLOCK, ab = static_cast<uint32_t>(c1 - c0) * 512u;
-                mbar_arrive_expect_tx(smem_u32(&C.bready), cb + ab);
-                bulk_g2s(bbuf, hcodes + static_cast<size_t>(b0) * DF_B_BLOCK, cb, smem_u32(&C.bready));
-                bulk_g2s(bsf, hatoms + static_cast<size_t>(c0) * 512, ab, smem_u32(&C.bready));
+                const uint32_t hsl = bbuf + hs * DF_HSLOT;
+                mbar_arrive_expect_tx(smem_u32(&C.hfull[hs]), cb + ab);
+                bulk_g2s(hsl, hcodes + static_cast<size_t>(b0) * DF_B_BLOCK, cb, smem_u32(&C.hfull[hs]));
+                bulk_g2s(hsl + DF_HSLOT_CODES, hatoms + static_cast<size_t>(c0) * 512, ab, smem_u32(&C.hfull[hs]));
             }
-            if (pend_buf >= 0) drain_pending();
-            pend_buf = buf;
-            pend_i = i;
-            pend_ft = ft;
-            pend_rf = rf;
-            buf ^= 1;
-            jt = piece_end;
+            hpend[hs] = static_cast<int>(hph);
+            if (++hs == S) { hs = 0; hph ^= 1u; }
         }
-        if (ok && pend_buf >= 0) {
-            const bool w_ok =
-                mbar_wait_bounded(smem_u32(&C.accf[pend_buf]), fph[pend_buf], abort_flag, p.status, p.timeout_ns);
-            if (__all_sync(0xffffffffu, w_ok)) {
-                fph[pend_buf] ^= 1u;
-                tc_fence_after();
-                drain_pending();
-            }
-        }
+        // copies still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int i = 0; i < S; ++i)
+                if (hpend[i] >= 0) mbar_wait_drain(smem_u32(&C.hfull[i]), static_cast<uint32_t>(hpend[i]), 200000000ull);
+        __syncwarp();
     }
 
     // ---- finish: free tensor memory; the last CTA writes y

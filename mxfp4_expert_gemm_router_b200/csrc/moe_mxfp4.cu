@@ -496,7 +496,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
             if (oe != cudaSuccess) return fail(MOE_ERR_CUDA);
             if (per_sm >= 1) {
                 const size_t ya_bytes_df = sizeof(float) * 2 * DF_MAX_T * static_cast<size_t>(d);
-                const size_t stamp_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu;
+                const size_t stamp_bytes = sizeof(uint32_t) * h->df_max_touched * h->F_gu * DF_EPI_WARPS;
                 const size_t xq_bytes = static_cast<size_t>(d / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_gu) * 512;
                 h->df_hq_stride = static_cast<size_t>(f / 32) * DF_B_BLOCK + static_cast<size_t>(h->KC_dn) * 512;
                 A dfa[] = {
