@@ -785,7 +785,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             if (lane == 0) {
-                __threadfence();
+                // the stamps were read with acquire loads; order them before the
+                // async-proxy reads of the copy
                 fence_proxy_async_global();
                 const uint8_t* hcodes = p.hq + i * p.hq_stride;
                 const uint8_t* hatoms = hcodes + static_cast<size_t>(nb_f) * DF_B_BLOCK;

@@ -52,8 +52,8 @@ template <> struct Raw8<float> {
 // transposed [64 k][128 tokens] and the router chunk [64 k][32 experts], fp32;
 // the top-k tail reuses it for the scores of 32 tokens [32][E + 1].
 constexpr int ROUTER_ETILE = 32;
-constexpr int ROUTER_MAX_SPLITS = 16;
-constexpr int ROUTER_SUB = 32;   // tokens per pass of the top-k tail
+constexpr int ROUTER_MAX_SPLITS = 8;
+constexpr int ROUTER_SUB = 32;   // tokens per pass of the top-k tail at E = 256 (more when E is smaller)
 __host__ __device__ constexpr size_t router_smem_bytes() {
     return sizeof(float) * (static_cast<size_t>(ROUTER_KCHUNK) * ROUTER_TOKENS +
                             static_cast<size_t>(ROUTER_KCHUNK) * ROUTER_ETILE);
@@ -362,32 +362,55 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     if (tid < ntok) {
         double inv = 1.0;
         if (norm) {
+            double pq[ROUTER_MAX_SPLITS];
+#pragma unroll
+            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
+                pq[sp] = sp < a.S ? __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid) : 0.0;
             double sq = 0.0;
-            for (int sp = 0; sp < a.S; ++sp) sq += __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid);
+#pragma unroll
+            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sq += pq[sp];
             inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
             a.inv_rms[t0 + tid] = static_cast<float>(inv);
         }
         inv_s[tid] = inv;
     }
     const size_t pstride = static_cast<size_t>(a.T) * E;
-    for (int sub = 0; sub < ntok; sub += ROUTER_SUB) {
-        const int nsub = min(ROUTER_SUB, ntok - sub);
+    // tokens per pass: as many as the scores [sub][E + 1] fit in the staging
+    // space (128 at E = 32, 64 at E = 128, 32 at E = 256)
+    int sub_n = static_cast<int>(router_smem_bytes() / (sizeof(float) * (E + 1))) & ~31;
+    sub_n = min(ROUTER_TOKENS, max(ROUTER_SUB, sub_n));
+    for (int sub = 0; sub < ntok; sub += sub_n) {
+        const int nsub = min(sub_n, ntok - sub);
         __syncthreads();
-        // scores = partials summed in split order (deterministic), x inverse RMS, + bias
-        for (int i = tid; i < nsub * E; i += ROUTER_THREADS) {
-            const int tl = i / E, e = i % E;
-            const double* pp = a.part + static_cast<size_t>(t0 + sub + tl) * E + e;
-            double sv = 0.0;
-            for (int sp = 0; sp < a.S; ++sp) sv += __ldcg(pp + sp * pstride);
-            if (norm) sv *= inv_s[sub + tl];
-            if (a.bias) sv += a.bias[e];
-            lg[tl * (E + 1) + e] = static_cast<float>(sv);
+        // scores = partials summed in split order (deterministic), x inverse RMS,
+        // + bias; four scores per thread at a time, all their partials in flight
+        for (int i0 = tid; i0 < nsub * E; i0 += 4 * ROUTER_THREADS) {
+            double pv[4][ROUTER_MAX_SPLITS];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                const double* pp = a.part + static_cast<size_t>(t0 + sub + i / E) * E + i % E;
+#pragma unroll
+                for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
+                    pv[m][sp] = (i < nsub * E && sp < a.S) ? __ldcg(pp + sp * pstride) : 0.0;
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                if (i < nsub * E) {
+                    double sv = 0.0;
+#pragma unroll
+                    for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sv += pv[m][sp];
+                    const int tl = i / E, e = i % E;
+                    if (norm) sv *= inv_s[sub + tl];
+                    if (a.bias) sv += a.bias[e];
+                    lg[tl * (E + 1) + e] = static_cast<float>(sv);
+                }
+            }
         }
         __syncthreads();
-        // top-k + softmax: warp w handles tokens sub + 4w .. sub + 4w + 3
-        for (int j = 0; j < 4; ++j) {
-            const int tl = warp * 4 + j;
-            if (tl >= nsub) break;
+        // top-k + softmax: warp w handles tokens sub + w, sub + w + 8, ...
+        for (int tl = warp; tl < nsub; tl += ROUTER_THREADS / 32) {
             const float* row = lg + tl * (E + 1);
             uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
             float sel_v[MAX_TOPK];
