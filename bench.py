@@ -78,7 +78,7 @@ def algorithmic_work(cfg: mi.MoeConfig, T: int, touched: int):
     out = {
         "router_topk_schedule": {"bytes": T * d * act + E * d * act + rows * 8, "flops": 2.0 * T * d * E},
         "gate_up_swiglu": {"bytes": gu_w + rows * d * op_bytes + rows * f * op_bytes, "flops": 4.0 * rows * d * f},
-        "down_combine": {"bytes": dn_w + rows * f * op_bytes + T * d * 4, "flops": 2.0 * rows * d * f},
+        "down": {"bytes": dn_w + rows * f * op_bytes + rows * d * act, "flops": 2.0 * rows * d * f},
         "layer": {"bytes": gu_w + dn_w + 2 * T * d * act + E * d * act, "flops": 6.0 * rows * d * f + 2.0 * T * d * E},
     }
     # the fused decode kernel (at most 16 tokens) is the whole layer in one launch
@@ -497,7 +497,7 @@ def main():
         stages[name] = sum(vals) / len(vals)
     work = algorithmic_work(cfg, cfg.T, r["touched"])
     peaks = measured_peaks()
-    dominant = max(("gate_up_swiglu", "down_combine", "router_topk_schedule", "fused_decode"),
+    dominant = max(("gate_up_swiglu", "down", "router_topk_schedule", "fused_decode"),
                    key=lambda n: stages.get(n, 0.0))
     dur_s = stages[dominant] / 1e3
     roof = roofline(work[dominant], dur_s, peaks, dominant)

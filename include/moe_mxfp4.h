@@ -237,8 +237,9 @@ moe_status_t moe_mxfp4_set_profiling(moe_mxfp4_t* h, int32_t enable);
 /* Stage names in the order moe_mxfp4_kernel_times reports them. */
 #define MOE_NUM_STAGES 7
 /* 0 router + top-k + softmax + grouping schedule, 1 gather into grouped rows,
- * 2 gate/up + SwiGLU, 3 H encoding (three MXFP4 terms), 4 down + weighted combine,
- * 5 output cast, 6 the fused decode kernel (forwards of at most 16 tokens).  Synchronises;
+ * 2 gate/up + SwiGLU, 3 H encoding (three MXFP4 terms), 4 down (weighted row
+ * outputs), 5 combine of each token's k rows into y, 6 the fused decode kernel
+ * (forwards of at most 16 tokens).  Synchronises;
  * writes the last profiled forward's durations in ms (0 for stages that did
  * not run) into ms[0..min(n, MOE_NUM_STAGES)). */
 moe_status_t moe_mxfp4_kernel_times(moe_mxfp4_t* h, float* ms, int32_t n);

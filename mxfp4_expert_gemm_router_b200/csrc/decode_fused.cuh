@@ -180,7 +180,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) decode_fused_kernel(const Decod
     const uint32_t bbuf = base + static_cast<uint32_t>(p.stages) * DF_STAGE;      // B codes
     const uint32_t bsf = bbuf + static_cast<uint32_t>(p.nb_max) * DF_B_BLOCK;    // B scale atoms
     uint8_t* bbuf_ptr = base_ptr + static_cast<size_t>(p.stages) * DF_STAGE;
-    uint8_t* bsf_ptr = bbuf_ptr + static_cast<size_t>(p.nb_max) * DF_B_BLOCK;
     DecodeCtl& C = *reinterpret_cast<DecodeCtl*>(bbuf_ptr + df_bregion_bytes(p.stages, p.nb_max, p.kc_max));
     volatile int* abort_flag = &C.abort_flag;
     const int S = p.stages;

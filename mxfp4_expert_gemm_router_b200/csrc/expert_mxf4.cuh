@@ -28,8 +28,9 @@
 //     B operand; with a K split, fp32 partials are added into GU instead (and
 //     h_encode_kernel encodes H).
 //   MODE 1 (down): per stage the down chunk (8704 bytes), one accumulator;
-//     epilogue: y[token, f] += w_row * d, red.add into the fp32 output
-//     accumulator (the weighted scatter-combine).
+//     epilogue: the row's weighted output w_row * d, stored once per grouped
+//     row (combine_out_kernel sums a token's k rows), or, when K is split,
+//     red.add into the fp32 output accumulator.
 //
 // Persistent kernel: one CTA per SM, units (expert | token tile, first row,
 // valid rows, feature tile | K split) taken round-robin from a device-built
@@ -43,6 +44,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "mxq.cuh"
 #include "quantize.cuh"
@@ -77,7 +79,9 @@ struct MxgParams {
     uint32_t idesc;           // M = 128, N = BN (or 3 * BN stacked), without scale-factor ids
     GroupedOperand Hd;        // MODE 0 output: H as the down GEMM's B operand
     float* GU;                // MODE 0 split partials [rows][2N]
-    float* yacc;              // MODE 1 output accumulator [T][N]
+    float* yacc;              // MODE 1, K split: output accumulator [T][N] (scatter-add)
+    void* obuf;               // MODE 1, K not split: weighted output of each grouped row [rows][N], act dtype
+    int obuf_bf16;            // obuf element type: 1 bf16, 0 fp32
     const int32_t* row_token; // MODE 1
     const float* row_weight;  // MODE 1
     int* status;
@@ -330,6 +334,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
             }
             fph[buf] ^= 1u;
             tc_fence_after();
+            bool released = false;   // the accumulator went back to the MMA warp early
             if (warp_rows) {
                 const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
                 // accumulators of token columns r0 .. r0 + 7 for this lane's feature
@@ -362,18 +367,38 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                     }
                 };
                 if (MODE == 0 && nsplit == 1) {
-                    // groups of 32 tokens alternate between the quarter's two warps
+                    // Groups of 32 tokens alternate between the quarter's two warps
+                    // (at most two groups each, BN <= 128).  First H of both groups
+                    // is read out of the accumulator into registers, which then goes
+                    // back to the MMA warp; the transposes and the encodes of H run
+                    // while the next unit's MMAs do.
+                    float hreg[2][32];
+#pragma unroll
+                    for (int gi = 0; gi < 2; ++gi) {
+                        const int g0 = 32 * hh + 64 * gi;
+#pragma unroll
+                        for (int s8 = 0; s8 < 32; s8 += 8) {
+                            if (g0 + s8 < nvalid) {
+                                float gs[8], us[8];
+                                load8(g0 + s8, gs, us);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) hreg[gi][s8 + j] = swish_f(gs[j]) * us[j];
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acce_bar(buf));
+                    released = true;
                     float* ht = htile_all + (warp - 2) * 32 * MXG_HT_STRIDE;
                     const int blk = 4 * ft + q;
                     uint8_t* atoms = scale_atom_base(p.Hd, tile, ft);
-                    for (int g0 = 32 * hh; g0 < nvalid; g0 += 64) {
-                        for (int s8 = 0; s8 < 32 && g0 + s8 < nvalid; s8 += 8) {
-                            float gs[8], us[8];
-                            load8(g0 + s8, gs, us);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                ht[(s8 + j) * MXG_HT_STRIDE + lane] = swish_f(gs[j]) * us[j];
-                        }
+                    for (int gi = 0; gi < 2; ++gi) {
+                        const int g0 = 32 * hh + 64 * gi;
+                        if (g0 >= nvalid) break;
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) ht[c * MXG_HT_STRIDE + lane] = hreg[gi][c];
                         __syncwarp();
                         const int r = g0 + lane;   // this lane's token: one 32-feature block of H
                         if (r < nvalid) {
@@ -406,19 +431,29 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                                     float* gu = p.GU + static_cast<size_t>(rr) * 2 * p.N;
                                     atomicAdd(gu + n, gs[j]);
                                     atomicAdd(gu + p.N + n, us[j]);
-                                } else {
+                                } else if (nsplit > 1) {
                                     const int tok = p.row_token[rr];
                                     if (MOE_IN_BOUNDS(tok >= 0 && tok < p.T, p.status))
                                         atomicAdd(p.yacc + static_cast<size_t>(tok) * p.N + n, gs[j] * p.row_weight[rr]);
+                                } else {
+                                    // the row's whole output: stored once, summed per token by the combine
+                                    const float o = gs[j] * p.row_weight[rr];
+                                    if (p.obuf_bf16)
+                                        static_cast<__nv_bfloat16*>(p.obuf)[static_cast<size_t>(rr) * p.N + n] =
+                                            __float2bfloat16_rn(o);
+                                    else
+                                        static_cast<float*>(p.obuf)[static_cast<size_t>(rr) * p.N + n] = o;
                                 }
                             }
                         }
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(buf));
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce_bar(buf));
+            }
             if (++buf == NACC) buf = 0;
         }
     }

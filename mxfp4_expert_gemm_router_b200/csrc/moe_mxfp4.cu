@@ -17,8 +17,9 @@
 //                        SwiGLU epilogue encoding H as three MXFP4 terms for the
 //                        down GEMM (fp32 partials instead when K is split)
 //   h_encode_kernel      only when the gate/up GEMM may split K: SwiGLU + encoding
-//   expert_mxf4<1>       down GEMM, routing-weighted scatter-combine epilogue
-//   cast_out_kernel      fp32 accumulator -> bf16 output (bf16 layers only)
+//   expert_mxf4<1>       down GEMM: each grouped row's weighted output stored
+//                        once (a fp32 scatter-add when K is split)
+//   combine_out_kernel   y = (x) + the sum of each token's k rows, in slot order
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -104,7 +105,9 @@ struct moe_mxfp4 {
     uint8_t* sfh = nullptr;    // scale atoms of Hq per (token tile, K chunk)
     size_t sfx_bytes = 0, sfh_bytes = 0, xq_bytes = 0, hq_bytes = 0;
     float* GU = nullptr;
-    float* yacc = nullptr;
+    float* yacc = nullptr;      // fp32 output accumulator (down GEMM with split K)
+    void* obuf = nullptr;       // weighted output of each grouped row (down GEMM without split K)
+    int32_t* pair_row = nullptr;  // grouped row of each (token, slot) pair
     int* status = nullptr;
     void* x_stage = nullptr;
     void* y_stage = nullptr;
@@ -208,7 +211,7 @@ static void free_all(moe_mxfp4* h) {
                     h->idx_ws, h->w_ws, h->hist,
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
-                    h->GU, h->yacc, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
+                    h->GU, h->yacc, h->obuf, h->pair_row, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
                     h->df_state, h->df_part, h->df_part_ss, h->df_yacc, h->df_xq, h->df_hq, h->df_hdone};
     for (void* p : ptrs)
         if (p) cudaFree(p);
@@ -344,7 +347,7 @@ const char* moe_mxfp4_status_string(moe_status_t s) {
 
 const char* moe_mxfp4_stage_name(int32_t stage) {
     static const char* names[MOE_NUM_STAGES] = {"router_topk_schedule", "gather", "gate_up_swiglu",
-                                                 "h_encode", "down_combine", "cast_out", "fused_decode"};
+                                                 "h_encode", "down", "combine_out", "fused_decode"};
     return (stage >= 0 && stage < MOE_NUM_STAGES) ? names[stage] : "unknown";
 }
 
@@ -441,6 +444,8 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->sfh), h->sfh_bytes},
         {reinterpret_cast<void**>(&h->GU), sizeof(float) * h->gu_rows * 2 * f},
         {reinterpret_cast<void**>(&h->yacc), sizeof(float) * static_cast<size_t>(c.max_tokens) * d},
+        {&h->obuf, TK * d * static_cast<size_t>(h->act_bytes)},
+        {reinterpret_cast<void**>(&h->pair_row), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->status), sizeof(int) * 4},
         {&h->x_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
         {&h->y_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
@@ -678,7 +683,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     int32_t* idx = topk_idx ? topk_idx : h->idx_ws;
     float* wts = topk_w ? topk_w : h->w_ws;
     const bool bf16 = c.act_dtype == MOE_DTYPE_BF16;
-    float* acc = bf16 ? h->yacc : static_cast<float*>(y);
+    float* acc = h->yacc;
     const bool prof = h->prof;
     for (int i = 0; i < MOE_NUM_STAGES; ++i) h->stage_ran[i] = false;
     // While the stream is being captured into a CUDA graph, the stage events
@@ -814,7 +819,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
                    h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0,
-                   tiles_cap, h->status);
+                   tiles_cap, h->status, h->pair_row);
         launch_pdl(pdl, encode_rows_kernel<__nv_bfloat16>, egrid, dim3(ENC_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), gam, static_cast<const float*>(h->inv_rms),
                    static_cast<const int32_t*>(h->row_token), static_cast<const int4*>(h->units_gu),
@@ -825,7 +830,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
                    BN, h->row_token, h->row_weight, h->row_slot, h->GU, 2 * f, acc,
-                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status);
+                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status, h->pair_row);
         launch_pdl(pdl, encode_rows_kernel<float>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
                    gam, static_cast<const float*>(h->inv_rms), static_cast<const int32_t*>(h->row_token),
                    static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T,
@@ -893,17 +898,29 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.sfb = h->sfh;
     dp.GU = nullptr;
     dp.yacc = acc;
+    dp.obuf = h->obuf;
+    dp.obuf_bf16 = bf16 ? 1 : 0;
     dp.skip_first_copy = 0;
     launch_pdl(pdl, expert_mxf4_kernel<1>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages), stream,
                h->tm_h[BN / 16 - 1], dp);
     h->stage_ran[4] = true;
-    // 5: output cast
+    // 5: the output: the sum of each token's k rows (+ x), or the cast accumulator
     mark(5);
-    if (bf16) {
-        const size_t n4 = static_cast<size_t>(T) * d / 4;
-        const int blocks = static_cast<int>(std::min<size_t>(4 * static_cast<size_t>(h->nsm), (n4 + 255) / 256));
-        launch_pdl(pdl, cast_out_kernel, dim3(std::max(1, blocks)), dim3(256), 0, stream, static_cast<const float*>(h->yacc),
-                   static_cast<__nv_bfloat16*>(y), n4);
+    {
+        const size_t n8 = static_cast<size_t>(T) * d / 8;
+        const int blocks = static_cast<int>(
+            std::min<size_t>(4 * static_cast<size_t>(h->nsm), (n8 + COMBINE_THREADS - 1) / COMBINE_THREADS));
+        if (bf16)
+            launch_pdl(pdl, combine_out_kernel<__nv_bfloat16>, dim3(std::max(1, blocks)), dim3(COMBINE_THREADS), 0,
+                       stream, static_cast<const __nv_bfloat16*>(h->obuf), static_cast<const int32_t*>(h->pair_row),
+                       static_cast<const float*>(h->yacc), static_cast<const __nv_bfloat16*>(x),
+                       static_cast<__nv_bfloat16*>(y), T, d, k, h->residual ? 1 : 0,
+                       static_cast<const int32_t*>(h->sched));
+        else
+            launch_pdl(pdl, combine_out_kernel<float>, dim3(std::max(1, blocks)), dim3(COMBINE_THREADS), 0, stream,
+                       static_cast<const float*>(h->obuf), static_cast<const int32_t*>(h->pair_row),
+                       static_cast<const float*>(h->yacc), static_cast<const float*>(x), static_cast<float*>(y), T, d,
+                       k, h->residual ? 1 : 0, static_cast<const int32_t*>(h->sched));
         h->stage_ran[5] = true;
     }
     mark(6);

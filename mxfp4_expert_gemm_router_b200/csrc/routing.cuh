@@ -530,11 +530,11 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
 // within its router tile), so the rows of an expert are in (token, slot)
 // order; the row's place in the expert's token tiles is (tile_base[e] +
 // (row - offsets[e]) / BN, (row - offsets[e]) % BN).  One thread per pair
-// records each row's token, routing weight and tile slot.  All threads then
-// initialise the tokens' rows of the fp32 output accumulator for the down
-// GEMM's scatter-add (to x itself when the block's residual is fused, else to
-// zero) and, when the gate/up GEMM splits K, clear the pairs' fp32
-// partial-sum rows.
+// records each row's token, routing weight and tile slot, and the pair's row.
+// When the down GEMM splits K, all threads then initialise the tokens' rows
+// of the fp32 output accumulator for its scatter-add (to x itself when the
+// block's residual is fused, else to zero); when the gate/up GEMM splits K,
+// they clear the pairs' fp32 partial-sum rows.
 constexpr int ROWS_TOKENS = 8;
 constexpr int ROWS_THREADS = 256;
 template <typename TA>
@@ -544,7 +544,7 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
             const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
             int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
             float* __restrict__ GU, int gu_ld, float* __restrict__ yacc, const int32_t* __restrict__ sched,
-            int residual, int tiles_cap, int* status) {
+            int residual, int tiles_cap, int* status, int32_t* __restrict__ pair_row) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ int pos_s[ROWS_TOKENS * MAX_TOPK];
@@ -564,12 +564,16 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
                 row_token[pos] = t;
                 row_weight[pos] = w[p];
                 row_slot[pos] = tl * BN + loc % BN;
+                pair_row[p] = pos;
                 pos_s[tid] = pos;
             }
         }
     }
-    // output accumulator rows: x (residual) or zero
+    // output accumulator rows: x (residual) or zero -- only when the down GEMM
+    // splits K and adds partial sums (otherwise each grouped row's output is
+    // stored once and combine_out_kernel sums them)
     const int d4 = d / 4;
+    if (sched[SCHED_SPLIT_DN] > 1)
     for (int i = tid; i < nt * d4; i += ROWS_THREADS) {
         const int t = t0 + i / d4, c4 = i % d4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -705,18 +709,74 @@ h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int B
     }
 }
 
-// fp32 accumulator -> bf16 output, 4 elements per thread-iteration.
-__global__ void cast_out_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ y, size_t n4) {
+// The layer output.  When the down GEMM did not split K, each grouped row's
+// weighted expert output w_j (H_row . W_down) was stored once (act dtype);
+// y[t] = (x[t] with the residual) + the sum of token t's k rows, added in
+// slot order j = 0 .. k-1 in fp32 (deterministic).  When it split K, the
+// outputs were added into the fp32 accumulator (which started at x with the
+// residual): y = that accumulator, cast.  One thread per 8 consecutive
+// features of a token (16-byte loads and stores for bf16).
+constexpr int COMBINE_THREADS = 256;
+template <typename TA> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+        const uint4 q = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+template <> struct Vec8<float> {
+    static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+        const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    static __device__ __forceinline__ void store(float* p, const float (&v)[8]) {
+        reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+};
+template <typename TA>
+__global__ void __launch_bounds__(COMBINE_THREADS)
+combine_out_kernel(const TA* __restrict__ obuf, const int32_t* __restrict__ pair_row, const float* __restrict__ yacc,
+                   const TA* __restrict__ x, TA* __restrict__ y, int T, int d, int k, int residual,
+                   const int32_t* __restrict__ sched) {
     pdl_wait();
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const float4 v = reinterpret_cast<const float4*>(acc)[i];
-        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
-        __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
-        uint2 o;
-        o.x = *reinterpret_cast<uint32_t*>(&a);
-        o.y = *reinterpret_cast<uint32_t*>(&b);
-        reinterpret_cast<uint2*>(y)[i] = o;
+    const int d8 = d / 8;
+    const bool split = sched[SCHED_SPLIT_DN] > 1;
+    for (long i = blockIdx.x * static_cast<long>(COMBINE_THREADS) + threadIdx.x; i < static_cast<long>(T) * d8;
+         i += static_cast<long>(gridDim.x) * COMBINE_THREADS) {
+        const int t = static_cast<int>(i / d8), c = static_cast<int>(i % d8) * 8;
+        float v[8];
+        if (split) {
+            Vec8<float>::load(yacc + static_cast<size_t>(t) * d + c, v);
+        } else {
+            if (residual) {
+                Vec8<TA>::load(x + static_cast<size_t>(t) * d + c, v);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = 0.f;
+            }
+            for (int j = 0; j < k; ++j) {
+                float o[8];
+                Vec8<TA>::load(obuf + static_cast<size_t>(pair_row[static_cast<size_t>(t) * k + j]) * d + c, o);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] += o[q];
+            }
+        }
+        Vec8<TA>::store(y + static_cast<size_t>(t) * d + c, v);
     }
 }
 
