@@ -75,7 +75,7 @@ struct MxgParams {
     int stages;
     int nacc;                 // accumulator buffers (1 or 2)
     const uint8_t* sfb;       // B operand scale atoms [tiles][K chunks][3][512]
-    int stacked;              // 1: the three terms are N = 3 * BN rows of one MMA (3 * BN <= 128)
+    int stacked;              // 1: the three terms are N = 3 * BN rows of one MMA (3 * BN <= 192)
     uint32_t idesc;           // M = 128, N = BN (or 3 * BN stacked), without scale-factor ids
     GroupedOperand Hd;        // MODE 0 output: H as the down GEMM's B operand
     float* GU;                // MODE 0 split partials [rows][2N]
@@ -111,11 +111,17 @@ __device__ __forceinline__ bool mxg_unit_ok(const MxgParams& p, const int4& U, i
 __host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
 __host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
 constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
-// Stacked terms for small tiles: one MMA per K step reads the weight tile once
-// (separate per-term MMAs would read it three times); needs 3 * BN <= 128.
-__host__ __device__ constexpr bool mxg_stacked(int BN) { return MXQ_TERMS * BN <= 128; }
-// B scale atoms per stage: one (all terms' rows in one atom) when stacked, else one per term.
-__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN) { return mxg_stacked(BN) ? 512u : MXG_SFB_BYTES; }
+// Stacked terms: one MMA per K step and matrix, N = 3 * BN, reads the weight
+// tile from shared memory once (separate per-term MMAs read it three times,
+// which makes shared-memory bandwidth, not the tensor pipe, the limit);
+// needs 3 * BN <= 192 so that the gate and up accumulators (2 x 192 columns)
+// and the scale-factor slots fit in tensor memory.
+__host__ __device__ constexpr bool mxg_stacked(int BN) { return MXQ_TERMS * BN <= 192; }
+// B scale atoms per stage: stacked, the operand rows t * BN + r in one atom per
+// 128 rows (one or two); per term, one atom per term.
+__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN) {
+    return mxg_stacked(BN) ? 512u * ((MXQ_TERMS * BN + 127) / 128) : MXG_SFB_BYTES;
+}
 __host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
     return mxg_w_stage(mode) + mxg_b_bytes(BN) + mxg_sfb_stage(BN);
 }
@@ -268,8 +274,10 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
                 if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
                 if (p.stacked) {
-                    // one MMA per K step and matrix: N = 3 * BN rows (term-major), one B scale atom
+                    // one MMA per K step and matrix: N = 3 * BN rows (term-major); the B
+                    // scales of rows 0..127 in columns 8..11, of rows 128.. in 12..15
                     tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
+                    if (NB3 > 128) tc_cp_sf_warp(sfc + 12, desc_noswz(ss + 512, 0, 128));
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         if (2 * i < nbc) {

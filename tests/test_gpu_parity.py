@@ -142,7 +142,7 @@ def test_e128_layer_parity():
 
 
 @pytest.mark.parametrize("d,f_", [(192, 320), (96, 160)])
-@pytest.mark.parametrize("bn", [16, 48, 112, 128])
+@pytest.mark.parametrize("bn", [16, 48, 64, 112, 128])
 def test_every_token_tile_on_ragged_shapes(d, f_, bn):
     """Token tiles from 16 to 128 rows (one or two accumulator buffers) on
     shapes with a short last feature tile (64 or 32 rows), a short last K
