@@ -64,14 +64,15 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- per-kernel algorithmic work
 
-def algorithmic_work(cfg: mi.MoeConfig, T: int, touched: int):
+def algorithmic_work(cfg: mi.MoeConfig, T: int, touched: int, act_format: str = "mxf4x3"):
     """Bytes / flops each stage must move / do at minimum (per launch)."""
     d, f, E, k = cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.top_k
     act = 2 if cfg.act_dtype == "bf16" else 4
     mx_bytes_per_param = 17 / 32
     # the grouped activation operands (x rows for gate/up, H rows for down) are
-    # three MXFP4 terms per element
-    op_bytes = MXQ_TERMS * 17 / 32
+    # three MXFP4 terms per element (4 bits + a scale byte per 32), or two
+    # MXFP8 terms (8 bits + a scale byte per 32)
+    op_bytes = MXQ_TERMS * 17 / 32 if act_format == "mxf4x3" else MX8_TERMS * 33 / 32
     gu_w = touched * 2 * d * f * mx_bytes_per_param
     dn_w = touched * d * f * mx_bytes_per_param
     rows = T * k
@@ -191,14 +192,15 @@ def act_tensor(cfg, a, device):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
 
 
-def uses_dependent_launches(cfg: mi.MoeConfig, T: int) -> bool:
+def uses_dependent_launches(cfg: mi.MoeConfig, T: int, act_format: str = "mxf4x3") -> bool:
     """The library launches a forward's kernels with programmatic (dependent)
     launches when it has at most 2048 grouped rows; stage events between the
     kernels would serialise those launches, so such forwards are timed without
     them and their stage times come from a second captured graph.  Forwards of
     at most 16 tokens are one launch (the fused decode kernel): its events sit
-    outside it and ride in the timed graph."""
-    return 16 < T and T * cfg.top_k <= 2048
+    outside it and ride in the timed graph (layers with two-MXFP8-term
+    operands have no fused kernel)."""
+    return (16 < T or act_format == "mxf8x2") and T * cfg.top_k <= 2048
 
 
 def run_ours(args, cfg, rank, world, local_rank):
@@ -208,7 +210,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     T = cfg.T
     import mxfp4_expert_gemm_router_b200 as mx
-    layer, _ = build_layer(cfg, T, mx.token_tile_flag(args.token_tile) if args.token_tile else 0)
+    flags = mx.token_tile_flag(args.token_tile) if args.token_tile else 0
+    if args.act_format == "mxf8x2":
+        flags |= mx.MOE_FLAG_ACT_MXF8X2
+    layer, _ = build_layer(cfg, T, flags)
     x = act_tensor(cfg, mi.draw_x(cfg), dev)
     y = torch.empty_like(x)
     counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
@@ -243,7 +248,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     # Stage events ride inside the timed graph (event-record nodes between the
     # kernels) unless the forward uses dependent launches, which the nodes would
     # serialise; then a second graph with the nodes gives the stage times.
-    stages_in_timed = not uses_dependent_launches(cfg, T)
+    stages_in_timed = not uses_dependent_launches(cfg, T, args.act_format)
     graph = capture(stages_in_timed)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -414,7 +419,8 @@ def config_dict(cfg, args):
             "seed": cfg.seed, "parallelism": f"replicas x{args.gpus}",
             "l2": "256 MB flush written between timed steps (outside each step's event span)",
             "launch": "forward captured once as a CUDA graph, replayed per timed step",
-            "token_tile": getattr(args, "token_tile", 0) or "auto"}
+            "token_tile": getattr(args, "token_tile", 0) or "auto",
+            "act_format": getattr(args, "act_format", "mxf4x3")}
 
 
 # Dense tensor-core rate of the experts' MMA operand type relative to bf16
@@ -423,6 +429,7 @@ def config_dict(cfg, args):
 # the tensor cores execute MXQ_TERMS times the layer's useful FLOPs.
 MMA_KIND = "mxf4"
 MXQ_TERMS = 3
+MX8_TERMS = 2
 MMA_RATE_VS_BF16 = {"f16": 1.0, "f8f6f4": 2.0, "mxf4": 4.0}
 
 
@@ -434,7 +441,8 @@ def roofline(work_k, dur_s, peaks, kernel, mma_kind=None):
     # burst figure: each kernel is timed over a loop of well under a second with
     # the clocks at their maximum (the clock sampler records them)
     tflops_peak = peaks["bf16_tflops"] * MMA_RATE_VS_BF16[kind]
-    terms = MXQ_TERMS if kind == "mxf4" else 1   # MMA flops executed per useful flop
+    # MMA flops executed per useful flop: one MMA per activation term
+    terms = {"mxf4": MXQ_TERMS, "f8f6f4": MX8_TERMS}.get(kind, 1)
     t_tensor = terms * work_k["flops"] / (tflops_peak * 1e12)
     t_hbm = work_k["bytes"] / (peaks["hbm_gbs"] * 1e9)
     if t_tensor > t_hbm:
@@ -462,6 +470,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--act-format", default="mxf4x3", choices=["mxf4x3", "mxf8x2"],
+                    help="activation operand format: three MXFP4 terms (kind::mxf4) or two MXFP8 terms "
+                         "(kind::mxf8f6f4)")
     ap.add_argument("--token-tile", type=int, default=0, choices=[0, 16, 32, 48, 64, 80, 96, 112, 128],
                     help="token rows per expert-GEMM tile (0: chosen per forward)")
     args = ap.parse_args()
@@ -495,12 +506,12 @@ def main():
     for name in r["stage_ms"][0]:
         vals = [s[name] for s in r["stage_ms"]]
         stages[name] = sum(vals) / len(vals)
-    work = algorithmic_work(cfg, cfg.T, r["touched"])
+    work = algorithmic_work(cfg, cfg.T, r["touched"], args.act_format)
     peaks = measured_peaks()
     dominant = max(("gate_up_swiglu", "down", "router_topk_schedule", "fused_decode"),
                    key=lambda n: stages.get(n, 0.0))
     dur_s = stages[dominant] / 1e3
-    roof = roofline(work[dominant], dur_s, peaks, dominant)
+    roof = roofline(work[dominant], dur_s, peaks, dominant, "f8f6f4" if args.act_format == "mxf8x2" else "mxf4")
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peaks["source"]
     roof["algorithmic_per_launch"] = work[dominant]["bytes"] if roof["bound"] == "hbm" else work[dominant]["flops"]
@@ -512,7 +523,10 @@ def main():
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "mxf4: MXFP4 weights as stored x activations as 3 MXFP4 terms, fp32 accumulate",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("mxf4: MXFP4 weights as stored x activations as 3 MXFP4 terms, fp32 accumulate"
+                  if args.act_format == "mxf4x3" else
+                  "mxf8f6f4: MXFP4 weights as stored x activations as 2 MXFP8 (E4M3) terms, fp32 accumulate"),
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) experts quantised to MXFP4)",
         "config": config_dict(cfg, args),
         "roofline": roof,

@@ -67,6 +67,18 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
  * multi-launch path instead; both compute the same layer. */
 #define MOE_FLAG_UNFUSED_DECODE (1u << 12)
 
+/* Activation operand format of the expert GEMMs.  Default: every activation
+ * block (32 values along K: x for gate/up, the SwiGLU output H for down) is a
+ * sum of three MXFP4 terms multiplied with the MXFP4 weights by the block-
+ * scaled FP4 MMA (kind::mxf4).  With this flag it is a sum of two MXFP8 (E4M3)
+ * terms multiplied with the same MXFP4 weights by kind::mxf8f6f4; the weights
+ * are then stored in a padded layout (about 4.5 % more bytes for 2880 x 2880
+ * experts) and forwards of at most 16 tokens take the multi-launch path.  Both
+ * compute the layer of "GPT-OSS-20B : Architecture MoE & Résumé du Model
+ * Card" §3.2/§4 within the same tolerance; export_weights returns the same
+ * canonical codes and scales. */
+#define MOE_FLAG_ACT_MXF8X2 (1u << 13)
+
 /* Test-only: the n-th device allocation of moe_mxfp4_create (n = 1..255 in
  * this field; 0 = off) fails as if cudaMalloc had, so the failure path can be
  * exercised; create then returns MOE_ERR_CUDA having freed everything. */

@@ -25,6 +25,7 @@ MOE_FLAG_TEST_SKIP_FIRST_COPY = 1 << 30
 MOE_FLAG_TOKEN_TILE_SHIFT = 8
 MOE_FLAG_TOKEN_TILE_MASK = 0xF << MOE_FLAG_TOKEN_TILE_SHIFT
 MOE_FLAG_UNFUSED_DECODE = 1 << 12
+MOE_FLAG_ACT_MXF8X2 = 1 << 13
 MOE_FLAG_TEST_FAIL_ALLOC_SHIFT = 16
 MOE_FLAG_TEST_FAIL_ALLOC_MASK = 0xFF << MOE_FLAG_TEST_FAIL_ALLOC_SHIFT
 

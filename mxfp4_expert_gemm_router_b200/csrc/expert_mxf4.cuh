@@ -106,53 +106,75 @@ __device__ __forceinline__ bool mxg_unit_ok(const MxgParams& p, const int4& U, i
 }
 
 // Weight bytes per stage (codes of 128 rows x 4 blocks + one scale atom, per
-// matrix), B bytes per stage (4 blocks x 3 terms x BN rows x 16 B), B scale
-// atoms per stage (one per term), accumulator columns (rounded to 32).
-__host__ __device__ constexpr uint32_t mxg_w_stage(int mode) { return (mode == 0 ? 2u : 1u) * (4u * 128 * 16 + 512); }
-__host__ __device__ constexpr uint32_t mxg_b_bytes(int BN) { return 4u * MXQ_TERMS * BN * 16; }
-constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;
-// Stacked terms: one MMA per K step and matrix, N = 3 * BN, reads the weight
-// tile from shared memory once (separate per-term MMAs read it three times,
+// matrix), B bytes per stage (4 blocks x terms x BN rows x 16 B per 16-byte
+// chunk of a block), B scale atoms per stage (one per term), accumulator
+// columns (rounded to 32).  AF = 1 (two MXFP8 terms): each matrix's codes land
+// padded to 16 KB (16 codes in the low half of every 16 bytes, 128-byte
+// swizzle, 1024-byte aligned), the scale atoms follow all the matrices' codes,
+// and a stage is a whole number of KB.
+__host__ __device__ constexpr int mxg_terms(int af) { return af ? MX8_TERMS : MXQ_TERMS; }
+__host__ __device__ constexpr uint32_t mxg_w_stage(int mode, int af = 0) {
+    return (mode == 0 ? 2u : 1u) * (af ? 16384u + 512u : 4u * 128 * 16 + 512);
+}
+__host__ __device__ constexpr uint32_t mxg_b_bytes(int BN, int af = 0) {
+    return 4u * (af ? 2u : 1u) * mxg_terms(af) * BN * 16;
+}
+constexpr uint32_t MXG_SFB_BYTES = 512u * MXQ_TERMS;   // B atoms per (token tile, chunk) in global memory
+// Stacked terms: one MMA per K step and matrix, N = terms * BN, reads the weight
+// tile from shared memory once (separate per-term MMAs read it once per term,
 // which makes shared-memory bandwidth, not the tensor pipe, the limit);
-// needs 3 * BN <= 192 so that the gate and up accumulators (2 x 192 columns)
-// and the scale-factor slots fit in tensor memory.
-__host__ __device__ constexpr bool mxg_stacked(int BN) { return MXQ_TERMS * BN <= 192; }
+// needs terms * BN <= 192 so that the gate and up accumulators (2 x 192
+// columns) and the scale-factor slots fit in tensor memory.
+__host__ __device__ constexpr bool mxg_stacked(int BN, int af = 0) { return mxg_terms(af) * BN <= 192; }
 // B scale atoms per stage: stacked, the operand rows t * BN + r in one atom per
 // 128 rows (one or two); per term, one atom per term.
-__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN) {
-    return mxg_stacked(BN) ? 512u * ((MXQ_TERMS * BN + 127) / 128) : MXG_SFB_BYTES;
+__host__ __device__ constexpr uint32_t mxg_sfb_stage(int BN, int af = 0) {
+    return mxg_stacked(BN, af) ? 512u * ((mxg_terms(af) * BN + 127) / 128) : 512u * mxg_terms(af);
 }
-__host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN) {
-    return mxg_w_stage(mode) + mxg_b_bytes(BN) + mxg_sfb_stage(BN);
+__host__ __device__ constexpr uint32_t mxg_stage_bytes(int mode, int BN, int af = 0) {
+    return af ? (mxg_w_stage(mode, af) + mxg_b_bytes(BN, af) + mxg_sfb_stage(BN, af) + 1023u) & ~1023u
+              : mxg_w_stage(mode, af) + mxg_b_bytes(BN, af) + mxg_sfb_stage(BN, af);
 }
-__host__ __device__ constexpr int mxg_mat_cols(int BN) {
-    return (((mxg_stacked(BN) ? MXQ_TERMS : 1) * BN + 31) / 32) * 32;
+__host__ __device__ constexpr int mxg_mat_cols(int BN, int af = 0) {
+    return (((mxg_stacked(BN, af) ? mxg_terms(af) : 1) * BN + 31) / 32) * 32;
 }
-__host__ __device__ constexpr int mxg_acc_cols(int mode, int BN) { return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN); }
-__host__ inline int mxg_nacc(int mode, int BN) { return 2 * mxg_acc_cols(mode, BN) <= MXG_SF_COL0 ? 2 : 1; }
+__host__ __device__ constexpr int mxg_acc_cols(int mode, int BN, int af = 0) {
+    return (mode == 0 ? 2 : 1) * mxg_mat_cols(BN, af);
+}
+__host__ inline int mxg_nacc(int mode, int BN, int af = 0) {
+    return 2 * mxg_acc_cols(mode, BN, af) <= MXG_SF_COL0 ? 2 : 1;
+}
 // MODE 0 epilogue tiles: per epilogue warp 32 tokens x 32 features of fp32 H,
 // rows padded to 33 so both the row writes and the column reads are
 // conflict-free.  fp32 keeps H's full range and precision into the encoder.
 constexpr int MXG_HT_STRIDE = 33;
 constexpr uint32_t MXG_HT_BYTES = MXG_EPI_WARPS * 32 * MXG_HT_STRIDE * 4;
 __host__ __device__ constexpr uint32_t mxg_extra_smem(int mode) { return mode == 0 ? MXG_HT_BYTES : 0u; }
-__host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages) {
-    const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN) +
+__host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0) {
+    const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN, af) +
                      (2 * stages + 2 * MXG_MAX_ACC + 1) * 8 + 64 + mxg_extra_smem(mode);
     return b < static_cast<size_t>(MXG_MIN_SMEM) ? static_cast<size_t>(MXG_MIN_SMEM) : b;
 }
 
-template <int MODE>
+// AF = 0: activations as three MXFP4 terms, kind::mxf4 (K = 64 per MMA).
+// AF = 1: activations as two MXFP8 terms, kind::mxf8f6f4 (K = 32 per MMA); the
+// weights (padded form) arrive through tmap_w, a 16U4_ALIGN16B tensor map
+// over the weight array's 8704-byte parts, one 128 x 128 box per matrix and
+// stage, and their scale atoms through bulk copies.
+template <int MODE, int AF = 0>
 __global__ void __launch_bounds__(MXG_THREADS, 1)
-expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p) {
+expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_w,
+                   const MxgParams p) {
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr uint32_t W_STAGE = mxg_w_stage(MODE);
+    constexpr uint32_t W_STAGE = mxg_w_stage(MODE, AF);
+    constexpr int TERMS = mxg_terms(AF);
+    constexpr int NMAT = MODE == 0 ? 2 : 1;
 
-    const int S = p.stages, BN = p.BN, NB3 = MXQ_TERMS * p.BN;
-    const uint32_t b_bytes = mxg_b_bytes(BN);
-    const uint32_t sf_bytes = mxg_sfb_stage(BN);                   // atoms used per stage
-    const uint32_t stage_bytes = mxg_stage_bytes(MODE, BN);
+    const int S = p.stages, BN = p.BN, NB3 = TERMS * p.BN;
+    const uint32_t b_bytes = mxg_b_bytes(BN, AF);
+    const uint32_t sf_bytes = mxg_sfb_stage(BN, AF);               // atoms used per stage
+    const uint32_t stage_bytes = mxg_stage_bytes(MODE, BN, AF);
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t bar0 = base + S * stage_bytes;                 // barriers (8-byte aligned)
@@ -166,7 +188,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 16);
     float* htile_all = reinterpret_cast<float*>(ctl + 64);     // MODE 0 epilogue tiles
-    const int mat_cols = mxg_mat_cols(BN);
+    const int mat_cols = mxg_mat_cols(BN, AF);
     const int acc_cols = (MODE == 0 ? 2 : 1) * mat_cols;
     const int NACC = p.nacc;
 
@@ -187,7 +209,10 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
         tmem_alloc(smem_u32(tmem_slot), MXG_TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_b);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_b);
+        if (AF) prefetch_tmap(&tmap_w);
+    }
     pdl_launch_dependents();
     tc_fence_before();
     __syncthreads();
@@ -224,6 +249,24 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 if (!ok) break;
                 if (skip) {
                     skip = false;  // test hook: this stage is never filled
+                } else if (AF) {
+                    // per matrix: the 128 x 128 code box (8192 global bytes, padded to
+                    // 16 KB in shared memory) and its scale atom
+                    const uint32_t st = w_sm(s);
+                    mbar_arrive_expect_tx_warp(full_bar(s), NMAT * (8192u + 512u) + b_bytes + sf_bytes);
+                    const size_t off = static_cast<size_t>(e) * expert_bytes + p.M.chunk_offset(ft, c, rf);
+                    const int part = static_cast<int>(off / TiledMatrix::PAD_MAT);
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m) {
+                        tma_load_3d_warp(st + 16384u * m, &tmap_w, 0, 0, part + m, full_bar(s));
+                        bulk_g2s_warp(st + 16384u * NMAT + 512u * m, p.wpack + off + m * TiledMatrix::PAD_MAT + 8192,
+                                      512u, full_bar(s));
+                    }
+                    // rows U.y .. U.y + BN - 1 of every (16-byte chunk, term)
+                    tma_load_3d_warp(st + W_STAGE, &tmap_b, 2 * U.y, 0, 8 * c, full_bar(s));
+                    bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * MXG_SFB_BYTES,
+                                  sf_bytes, full_bar(s));
+                    pend_ph[s] = static_cast<int>(ph);
                 } else {
                     const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
                     const uint32_t st = w_sm(s);
@@ -267,6 +310,53 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 if (!ok) break;
                 tc_fence_after();
                 const int nbc = p.M.blocks_in_chunk(c);
+                if constexpr (AF == 1) {
+                    // one MMA per block (K = 32, scale byte i); A from the padded,
+                    // swizzled 16 KB tile of each matrix, B [8 chunks][2 terms][BN][16 B]
+                    const uint32_t ws = w_sm(s), bs = ws + W_STAGE, ss = bs + b_bytes;
+                    const uint32_t wsf = ws + 16384u * NMAT;
+                    const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
+                    tc_cp_sf_warp(sfc, desc_noswz(wsf, 0, 128));
+                    if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(wsf + 512, 0, 128));
+                    if (p.stacked) {
+                        tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
+                        if (NB3 > 128) tc_cp_sf_warp(sfc + 12, desc_noswz(ss + 512, 0, 128));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            if (i < nbc) {
+                                const uint32_t acc = (c > c0 || i > 0) ? 1u : 0u;
+                                const uint32_t id = p.idesc | idesc_sf_ids(static_cast<uint32_t>(i));
+                                const uint64_t bd = desc_noswz(bs + 2 * i * NB3 * 16, NB3 * 16, 128);
+                                mma_mxf8f6f4_warp(d0, desc_sw128(ws + 32 * i), bd, id, sfc, sfc + 8, acc);
+                                if (MODE == 0)
+                                    mma_mxf8f6f4_warp(d0 + mat_cols, desc_sw128(ws + 16384 + 32 * i), bd, id, sfc + 4,
+                                                      sfc + 8, acc);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < TERMS; ++t) tc_cp_sf_warp(sfc + 8 + 4 * t, desc_noswz(ss + 512 * t, 0, 128));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            if (i < nbc) {
+                                const uint32_t id = p.idesc | idesc_sf_ids(static_cast<uint32_t>(i));
+#pragma unroll
+                                for (int t = 0; t < TERMS; ++t) {
+                                    const uint32_t acc = (c > c0 || i > 0 || t > 0) ? 1u : 0u;
+                                    const uint64_t bd = desc_noswz(bs + (2 * i * TERMS + t) * BN * 16, NB3 * 16, 128);
+                                    mma_mxf8f6f4_warp(d0, desc_sw128(ws + 32 * i), bd, id, sfc, sfc + 8 + 4 * t, acc);
+                                    if (MODE == 0)
+                                        mma_mxf8f6f4_warp(d0 + mat_cols, desc_sw128(ws + 16384 + 32 * i), bd, id,
+                                                          sfc + 4, sfc + 8 + 4 * t, acc);
+                                }
+                            }
+                        }
+                    }
+                    tc_commit_warp(empty_bar(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    if (++sfs == MXG_SF_SLOTS) sfs = 0;
+                    continue;
+                }
                 const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16);
                 const uint32_t mat_b = codes_b + 512u;
                 const uint32_t ws = w_sm(s), bs = ws + W_STAGE, ss = bs + b_bytes;
@@ -348,19 +438,24 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                 // accumulators of token columns r0 .. r0 + 7 for this lane's feature
                 auto load8 = [&](int r0, float (&gs)[8], float (&us)[8]) {
                     if (p.stacked) {
-                        // the three term columns of each token are BN apart: add them
-                        uint32_t g[MXQ_TERMS][8], v[MXQ_TERMS][8];
+                        // the term columns of each token are BN apart: add them
+                        uint32_t g[TERMS][8], v[TERMS][8];
 #pragma unroll
-                        for (int t = 0; t < MXQ_TERMS; ++t) {
+                        for (int t = 0; t < TERMS; ++t) {
                             tmem_ld8(d0 + t * BN + r0, g[t]);
                             if (MODE == 0) tmem_ld8(d0 + mat_cols + t * BN + r0, v[t]);
                         }
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            gs[j] = __uint_as_float(g[0][j]) + __uint_as_float(g[1][j]) + __uint_as_float(g[2][j]);
-                            us[j] = MODE == 0 ? __uint_as_float(v[0][j]) + __uint_as_float(v[1][j]) + __uint_as_float(v[2][j])
-                                              : 0.f;
+                            float a = 0.f, b = 0.f;
+#pragma unroll
+                            for (int t = 0; t < TERMS; ++t) {
+                                a += __uint_as_float(g[t][j]);
+                                if (MODE == 0) b += __uint_as_float(v[t][j]);
+                            }
+                            gs[j] = a;
+                            us[j] = b;
                         }
                     } else {
                         uint32_t g[8], v[8];
@@ -413,16 +508,11 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const MxgParams p
                             float hv[32];
 #pragma unroll
                             for (int c = 0; c < 32; ++c) hv[c] = ht[lane * MXG_HT_STRIDE + c];
-                            uint4 codes[MXQ_TERMS];
                             uint32_t sb[MXQ_TERMS];
-                            mxq_block_thread(hv, codes, sb);
+                            act_encode_store<AF>(hv, p.Hd.codes, p.Hd.R, blk, row0 + r, sb);
 #pragma unroll
-                            for (int t = 0; t < MXQ_TERMS; ++t) {
-                                *reinterpret_cast<uint4*>(
-                                    p.Hd.codes + ((static_cast<size_t>(blk) * MXQ_TERMS + t) * p.Hd.R + row0 + r) * 16) =
-                                    codes[t];
+                            for (int t = 0; t < TERMS; ++t)
                                 atoms[sf_atom_offset(t * p.Hd.term_rows + r, q)] = static_cast<uint8_t>(sb[t]);
-                            }
                         }
                         __syncwarp();
                     }

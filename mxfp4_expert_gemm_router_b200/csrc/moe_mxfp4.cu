@@ -69,6 +69,7 @@ struct moe_mxfp4 {
     int act_bytes = 2;
     int KC_gu = 0, KC_dn = 0, F_gu = 0, F_dn = 0;
     int TK = 0, nblk_max = 0, max_units = 0, gu_rows = 0;
+    int af = 0;                // activation operand format: 0 three MXFP4 terms, 1 two MXFP8 terms
     size_t part_elems = 0;
     // weights
     uint8_t* w_gu = nullptr;   // tiled gate+up
@@ -117,6 +118,7 @@ struct moe_mxfp4 {
     CUtensorMap tm_x[BN_OPTIONS];
     CUtensorMap tm_h[BN_OPTIONS];
     bool tm_ok[BN_OPTIONS] = {};
+    CUtensorMap tm_wgu{}, tm_wdn{};   // two-MXFP8-term layers: the padded weights as 16U4_ALIGN16B boxes
     // fused decode path (forwards of at most DF_MAX_T tokens)
     bool df_ok = false, last_fused = false;
     int df_stages = 0, df_S = 0, df_nb_max = 0, df_kc_max = 0, df_max_touched = 0;
@@ -248,6 +250,7 @@ static size_t max_tile_atoms(size_t TK, int E) { return (TK / 16 + E) * MXQ_TERM
 static TiledMatrix tiled(moe_mxfp4* h, int which) {
     const auto& c = h->cfg;
     TiledMatrix M;
+    M.padded = h->af;
     if (which < 2) {
         M.base = h->w_gu;
         M.N = c.d_ff;
@@ -312,6 +315,10 @@ static cudaError_t ensure_kernel_attrs(int dev) {
         return e;
     if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
         return e;
+    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
+        return e;
+    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
+        return e;
     if ((e = set_router_smem<float>(rsm))) return e;
     if ((e = set_router_smem<__nv_bfloat16>(rsm))) return e;
     if ((e = cudaFuncSetAttribute(decode_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -324,9 +331,9 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     return cudaSuccess;
 }
 
-static int stages_for(int mode, int BN) {
+static int stages_for(int mode, int BN, int af) {
     const size_t budget = 227 * 1024 - 1024 - 512 - mxg_extra_smem(mode);
-    int s = static_cast<int>(budget / mxg_stage_bytes(mode, BN));
+    int s = static_cast<int>(budget / mxg_stage_bytes(mode, BN, af));
     return std::max(2, std::min(MXG_MAX_STAGES, s));
 }
 
@@ -362,6 +369,8 @@ int64_t moe_mxfp4_expert_weight_bytes(const moe_mxfp4_config_t* cfg) {
 }
 
 uint64_t moe_mxfp4_launch_count(const moe_mxfp4_t* h) { return h ? h->launches : 0; }
+
+static moe_status_t make_weight_tmaps(moe_mxfp4* h);
 
 moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) {
     if (!cfg || !out) return MOE_ERR_INVALID_ARG;
@@ -409,8 +418,11 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
     if (!h->expert_done) return fail(MOE_ERR_CUDA);
 
     const size_t TK = h->TK;
-    h->xq_bytes = static_cast<size_t>(d / 32) * MXQ_TERMS * TK * 16;
-    h->hq_bytes = static_cast<size_t>(f / 32) * MXQ_TERMS * TK * 16;
+    h->af = (c.flags & MOE_FLAG_ACT_MXF8X2) ? 1 : 0;
+    // operand codes per row and block: 3 terms x 16 B, or 2 terms x 32 B
+    const size_t block_code_bytes = h->af ? 2 * 32 : MXQ_TERMS * 16;
+    h->xq_bytes = static_cast<size_t>(d / 32) * block_code_bytes * TK;
+    h->hq_bytes = static_cast<size_t>(f / 32) * block_code_bytes * TK;
     h->sfx_bytes = max_tile_atoms(TK, E) * h->KC_gu * 512;
     h->sfh_bytes = max_tile_atoms(TK, E) * h->KC_dn * 512;
     const size_t gu_bytes = static_cast<size_t>(E) * tiled(h, 0).expert_bytes();
@@ -473,6 +485,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         return fail(MOE_ERR_CUDA);
 
     if (ensure_kernel_attrs(h->dev) != cudaSuccess) return fail(MOE_ERR_CUDA);
+    if (h->af && make_weight_tmaps(h) != MOE_OK) return fail(MOE_ERR_CUDA);
 
     // fused decode path: one persistent grid for forwards of at most DF_MAX_T
     // tokens, when its shared-memory plan fits (the whole-K B operand plus at
@@ -486,7 +499,9 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         // the router's scratch (2 x 16 x K chunks doubles) and logits live in the ring
         const size_t router_scratch = 2 * DF_MAX_T * sizeof(double) * ((d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK);
         const size_t logits = DF_MAX_T * sizeof(float) * (E + 1);
-        if (h->df_stages >= 2 && std::max(router_scratch, logits) <= static_cast<size_t>(h->df_stages) * DF_STAGE) {
+        // (the fused kernel reads three-MXFP4-term operands only)
+        if (!h->af && h->df_stages >= 2 &&
+            std::max(router_scratch, logits) <= static_cast<size_t>(h->df_stages) * DF_STAGE) {
             h->df_smem = df_smem_bytes(h->df_stages, h->df_nb_max, h->df_kc_max);
             const int kch = (d + ROUTER_KCHUNK - 1) / ROUTER_KCHUNK;
             h->df_S = std::max(1, std::min(h->nsm / E, kch));
@@ -631,12 +646,14 @@ moe_status_t moe_mxfp4_export_weights(const moe_mxfp4_t* hc, int32_t which, uint
     return cuda_status(cudaGetLastError());
 }
 
-// 3-D maps over the three-term operands [K/32 blocks][3 terms][TK rows x 16 B],
-// read as 8-byte elements so that the innermost box dimension is one
-// contiguous run of BN rows (BN * 16 bytes): box {2 BN, 3 terms, 4 blocks}
-// lands in shared memory as [4 blocks][3 terms][BN rows][16 B], the
+// 3-D maps over the activation operands, read as 8-byte elements so that the
+// innermost box dimension is one contiguous run of BN rows (BN * 16 bytes).
+// Three MXFP4 terms, [K/32 blocks][3 terms][TK rows x 16 B]: box {2 BN, 3
+// terms, 4 blocks} lands in shared memory as [4 blocks][3 terms][BN rows][16 B].
+// Two MXFP8 terms, [K/16 chunks][2 terms][TK rows x 16 B]: box {2 BN, 2 terms,
+// 8 chunks} lands as [8 chunks][2 terms][BN rows][16 B].  Either is the
 // unswizzled K-major layout of each term's operand.  Rows past TK and blocks
-// past K/32 read as zeros.
+// past K read as zeros.
 static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
     const int i = BN / 16 - 1;
     if (h->tm_ok[i]) return MOE_OK;
@@ -644,11 +661,12 @@ static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
     if (!enc) return MOE_ERR_CUDA;
     const auto& c = h->cfg;
     const cuuint64_t R = static_cast<cuuint64_t>(h->TK);
+    const cuuint32_t terms = h->af ? 2 : MXQ_TERMS, cpb = h->af ? 2 : 1;
     for (int which = 0; which < 2; ++which) {
-        const cuuint64_t nb = (which == 0 ? c.d_model : c.d_ff) / 32;
-        cuuint64_t dims[3] = {2 * R, MXQ_TERMS, nb};
-        cuuint64_t strides[2] = {R * 16, R * 16 * MXQ_TERMS};
-        cuuint32_t box[3] = {static_cast<cuuint32_t>(2 * BN), MXQ_TERMS, 4};
+        const cuuint64_t nch = (which == 0 ? c.d_model : c.d_ff) / 32 * cpb;
+        cuuint64_t dims[3] = {2 * R, terms, nch};
+        cuuint64_t strides[2] = {R * 16, R * 16 * terms};
+        cuuint32_t box[3] = {static_cast<cuuint32_t>(2 * BN), terms, 4 * cpb};
         cuuint32_t estr[3] = {1, 1, 1};
         CUresult r = enc(which == 0 ? &h->tm_x[i] : &h->tm_h[i], CU_TENSOR_MAP_DATA_TYPE_UINT64, 3,
                          which == 0 ? static_cast<void*>(h->Xq) : static_cast<void*>(h->Hq), dims, strides, box, estr,
@@ -657,6 +675,29 @@ static moe_status_t ensure_tmaps(moe_mxfp4* h, int BN) {
         if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
     }
     h->tm_ok[i] = true;
+    return MOE_OK;
+}
+
+// Two-MXFP8-term layers keep the weights in the padded form: parts of 8704
+// bytes (codes [128 rows][64 B] + a scale atom).  The map views the array as
+// {128 four-bit elements, 128 rows, parts} with the 16U4_ALIGN16B type and the
+// 128-byte swizzle: a {128, 128, 1} box is one matrix's codes of a chunk,
+// landing as the 16 KB padded, swizzled A operand of kind::mxf8f6f4.
+static moe_status_t make_weight_tmaps(moe_mxfp4* h) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    for (int which = 0; which < 2; ++which) {
+        const TiledMatrix M = tiled(h, which == 0 ? 0 : 2);
+        const cuuint64_t parts = static_cast<cuuint64_t>(h->cfg.n_experts) * M.expert_bytes() / TiledMatrix::PAD_MAT;
+        cuuint64_t dims[3] = {128, 128, parts};
+        cuuint64_t strides[2] = {64, TiledMatrix::PAD_MAT};
+        cuuint32_t box[3] = {128, 128, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = enc(which == 0 ? &h->tm_wgu : &h->tm_wdn, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, M.base, dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    }
     return MOE_OK;
 }
 
@@ -804,7 +845,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     // 1: gather into grouped rows
     mark(1);
     const bool pdl = static_cast<long>(T) * k <= h->gu_rows;
-    const bool stacked = mxg_stacked(BN);
+    const int af = h->af;
+    const bool stacked = mxg_stacked(BN, af);
     GroupedOperand Xop{h->Xq, h->sfx, h->TK, h->KC_gu, stacked ? BN : 128};
     GroupedOperand Hop{h->Hq, h->sfh, h->TK, h->KC_dn, stacked ? BN : 128};
     const float* gam = h->use_norm ? h->gamma : nullptr;
@@ -820,7 +862,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
                    h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0,
                    tiles_cap, h->status, h->pair_row);
-        launch_pdl(pdl, encode_rows_kernel<__nv_bfloat16>, egrid, dim3(ENC_THREADS), 0, stream,
+        launch_pdl(pdl, af ? encode_rows_kernel<__nv_bfloat16, 1> : encode_rows_kernel<__nv_bfloat16, 0>, egrid, dim3(ENC_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), gam, static_cast<const float*>(h->inv_rms),
                    static_cast<const int32_t*>(h->row_token), static_cast<const int4*>(h->units_gu),
                    static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T, h->status);
@@ -831,7 +873,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
                    BN, h->row_token, h->row_weight, h->row_slot, h->GU, 2 * f, acc,
                    static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status, h->pair_row);
-        launch_pdl(pdl, encode_rows_kernel<float>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
+        launch_pdl(pdl, af ? encode_rows_kernel<float, 1> : encode_rows_kernel<float, 0>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
                    gam, static_cast<const float*>(h->inv_rms), static_cast<const int32_t*>(h->row_token),
                    static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T,
                    h->status);
@@ -848,11 +890,12 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.N = f;
     gp.K = d;
     gp.BN = BN;
-    gp.stages = stages_for(0, BN);
-    gp.nacc = mxg_nacc(0, BN);
+    gp.stages = stages_for(0, BN, af);
+    gp.nacc = mxg_nacc(0, BN, af);
     gp.sfb = h->sfx;
     gp.stacked = stacked ? 1 : 0;
-    gp.idesc = idesc_mxf4(128, (stacked ? MXQ_TERMS : 1) * BN);
+    gp.idesc = af ? idesc_mxf8f6f4_e2m1_e4m3(128, (stacked ? MX8_TERMS : 1) * BN)
+                  : idesc_mxf4(128, (stacked ? MXQ_TERMS : 1) * BN);
     gp.Hd = Hop;
     gp.GU = h->GU;
     gp.yacc = nullptr;
@@ -865,8 +908,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.T = T;
     gp.tiles_cap = tiles_cap;
     const int grid = h->nsm;
-    launch_pdl(pdl, expert_mxf4_kernel<0>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(0, BN, gp.stages), stream,
-               h->tm_x[BN / 16 - 1], gp);
+    launch_pdl(pdl, af ? expert_mxf4_kernel<0, 1> : expert_mxf4_kernel<0, 0>, dim3(grid), dim3(MXG_THREADS),
+               mxg_smem_bytes(0, BN, gp.stages, af), stream, h->tm_x[BN / 16 - 1], h->tm_wgu, gp);
     h->stage_ran[2] = true;
     // 3: split-K finish (a no-op unless the schedule split K): SwiGLU + H encoding.
     // The schedule splits the gate/up K only for at most gu_rows grouped rows,
@@ -880,7 +923,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     if (may_split) {
         const long items = static_cast<long>(T) * k * (f / 32);
         const int blocks = static_cast<int>((items + HENC_THREADS - 1) / HENC_THREADS);
-        launch_pdl(pdl, h_encode_kernel, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const float*>(h->GU),
+        launch_pdl(pdl, af ? h_encode_kernel<1> : h_encode_kernel<0>, dim3(blocks), dim3(HENC_THREADS), 0, stream, static_cast<const float*>(h->GU),
                    Hop, f, BN, static_cast<const int32_t*>(h->row_slot), static_cast<const int32_t*>(h->sched), tiles_cap,
                    h->status);
         h->stage_ran[3] = true;
@@ -893,16 +936,16 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.M = tiled(h, 2);
     dp.N = d;
     dp.K = f;
-    dp.stages = stages_for(1, BN);
-    dp.nacc = mxg_nacc(1, BN);
+    dp.stages = stages_for(1, BN, af);
+    dp.nacc = mxg_nacc(1, BN, af);
     dp.sfb = h->sfh;
     dp.GU = nullptr;
     dp.yacc = acc;
     dp.obuf = h->obuf;
     dp.obuf_bf16 = bf16 ? 1 : 0;
     dp.skip_first_copy = 0;
-    launch_pdl(pdl, expert_mxf4_kernel<1>, dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages), stream,
-               h->tm_h[BN / 16 - 1], dp);
+    launch_pdl(pdl, af ? expert_mxf4_kernel<1, 1> : expert_mxf4_kernel<1, 0>, dim3(grid), dim3(MXG_THREADS),
+               mxg_smem_bytes(1, BN, dp.stages, af), stream, h->tm_h[BN / 16 - 1], h->tm_wdn, dp);
     h->stage_ran[4] = true;
     // 5: the output: the sum of each token's k rows (+ x), or the cast accumulator
     mark(5);

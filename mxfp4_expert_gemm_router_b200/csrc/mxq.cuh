@@ -120,4 +120,102 @@ __device__ __forceinline__ void mxq_block_warp(float v, uint32_t (&w)[MXQ_TERMS]
     }
 }
 
+
+// ---------------------------------------------------------------- 2 x MXFP8
+// The alternative operand format: a block of 32 values as q1 + q2, two MXFP8
+// terms (E4M3 elements: 4 exponent and 3 mantissa bits, largest finite 448;
+// one E8M0 scale per term and block), read by the kind::mxf8f6f4 MMA against
+// the same MXFP4 weights.  Scale rule of a term: the smallest power of two
+// 2^e with max|v| <= 448 * 2^e (no element saturates); elements round to the
+// nearest E4M3 value with ties to even (the hardware conversion).  Two terms
+// keep about eight significant bits per element.
+//
+// Operand codes in global memory: [K/16 chunks][2 terms][R rows][16 B], chunk
+// 2b + j holding elements 16j .. 16j+15 of block b (one byte per element);
+// the scale atoms are laid out as for the three-term format (atom t per term,
+// or rows t * BN + r when the terms are stacked).
+constexpr int MX8_TERMS = 2;
+
+// Exponent e of a term whose largest magnitude has bits `amax_bits`: amax =
+// m 2^E0 with m in [1, 2); e = E0 - 8 when m <= 1.75, else E0 - 7.  -127 for
+// zero or subnormal amax.
+__device__ __forceinline__ int mx8_exp(uint32_t amax_bits) {
+    const int ex = static_cast<int>(amax_bits >> 23);
+    if (ex == 0) return -127;
+    const int e = ex - 135 + ((amax_bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : e;
+}
+
+// One thread encodes one block of 32 values (v is overwritten with the final
+// residual).  codes[t][j] = the 16 code bytes of chunk j of term t.
+__device__ __forceinline__ void mx8_block_thread(float (&v)[32], uint4 (&codes)[MX8_TERMS][2],
+                                                 uint32_t (&sbyte)[MX8_TERMS]) {
+#pragma unroll
+    for (int t = 0; t < MX8_TERMS; ++t) {
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+        const int e = mx8_exp(__float_as_uint(am));
+        sbyte[t] = static_cast<uint32_t>(e + 127);
+        const float inv = mxq_inv(e), sc = mxq_scale(e);
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t pair = e4m3x2_from_f32(v[2 * i] * inv, v[2 * i + 1] * inv);
+            if (i & 1)
+                w[i >> 1] |= pair << 16;
+            else
+                w[i >> 1] = pair;
+            if (t + 1 < MX8_TERMS) {
+                const uint32_t h2 = e4m3x2_to_f16x2(pair);
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+                v[2 * i] -= f.x * sc;
+                v[2 * i + 1] -= f.y * sc;
+            }
+        }
+        codes[t][0] = make_uint4(w[0], w[1], w[2], w[3]);
+        codes[t][1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
+// Activation operand formats: AF = 0, three MXFP4 terms (16 code bytes per
+// block and term); AF = 1, two MXFP8 terms (32 bytes per block and term).
+template <int AF> struct ActFormat;
+template <> struct ActFormat<0> {
+    static constexpr int TERMS = MXQ_TERMS;
+    static constexpr int CPB = 1;   // 16-byte chunks per block and term
+};
+template <> struct ActFormat<1> {
+    static constexpr int TERMS = MX8_TERMS;
+    static constexpr int CPB = 2;
+};
+
+// Encode one block b (32 values along K) of operand row `row` in format AF:
+// the codes go to `codes` ([K/32 * CPB chunks][TERMS][R][16 B]), the scale
+// bytes to sb[0 .. TERMS-1].
+template <int AF>
+__device__ __forceinline__ void act_encode_store(float (&v)[32], uint8_t* codes, int R, int b, int row,
+                                                 uint32_t (&sb)[MXQ_TERMS]) {
+    if constexpr (AF == 0) {
+        uint4 c[MXQ_TERMS];
+        mxq_block_thread(v, c, sb);
+#pragma unroll
+        for (int t = 0; t < MXQ_TERMS; ++t)
+            *reinterpret_cast<uint4*>(codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * R + row) * 16) = c[t];
+    } else {
+        uint4 c[MX8_TERMS][2];
+        uint32_t s2[MX8_TERMS];
+        mx8_block_thread(v, c, s2);
+        sb[0] = s2[0];
+        sb[1] = s2[1];
+        sb[2] = 0u;
+#pragma unroll
+        for (int t = 0; t < MX8_TERMS; ++t)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                *reinterpret_cast<uint4*>(codes + ((static_cast<size_t>(2 * b + j) * MX8_TERMS + t) * R + row) * 16) =
+                    c[t][j];
+    }
+}
+
 }  // namespace moe

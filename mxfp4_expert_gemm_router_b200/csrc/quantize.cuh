@@ -24,6 +24,16 @@
 // padding where a tile has fewer than 128 rows or a chunk fewer than 4 blocks
 // (0.26 % for the 2880 x 2880 experts).  Padding bytes stay zero (a finite
 // scale, 2^-127).
+//
+// Padded form (the layers whose activations are two MXFP8 terms, read by the
+// kind::mxf8f6f4 MMA): every tile has 128 rows and every chunk 4 blocks (zero
+// padding), and a matrix's part of a chunk is codes [128 rows][64 B] (row-major:
+// the row's 128 elements of the chunk) + the same scale atom, 8704 bytes.
+// All parts have one size, so the array is a 3-D tensor {128 elements, 128
+// rows, parts} that a tensor map of the 16U4_ALIGN16B type reads, writing
+// each group of 16 codes into the low half of 16 bytes of shared memory: the
+// layout that MMA kind wants for E2M1.  Padding costs 2.2 % rows and 2.2 %
+// blocks for the 2880 x 2880 experts.
 #pragma once
 #include <cstdint>
 
@@ -34,24 +44,29 @@ struct TiledMatrix {
     int N, K;        // rows, contraction length (K % 32 == 0)
     int NM;          // matrices interleaved per chunk (2: gate+up, 1: down)
     int sub;         // which matrix of the chunk this one is (0 or 1)
+    int padded;      // 1: the row-major, padded form (below), 0: the compact form
     static constexpr int BPC = 4;   // 32-blocks per chunk
+    static constexpr size_t PAD_MAT = 128 * 64 + 512;   // padded form: one matrix's part of a chunk
     __host__ __device__ int nb() const { return K / 32; }
     __host__ __device__ int chunks() const { return (nb() + BPC - 1) / BPC; }
     __host__ __device__ int tiles() const { return (N + 127) / 128; }
     __host__ __device__ int blocks_in_chunk(int c) const { return min(BPC, nb() - c * BPC); }
     // bytes of one matrix's part of a chunk: codes + one scale atom
     __host__ __device__ size_t mat_bytes(int c, int rf) const {
-        return static_cast<size_t>(blocks_in_chunk(c)) * rf * 16 + 512;
+        return padded ? PAD_MAT : static_cast<size_t>(blocks_in_chunk(c)) * rf * 16 + 512;
     }
     __host__ __device__ size_t chunk_bytes(int c, int rf) const { return NM * mat_bytes(c, rf); }
     __host__ __device__ size_t tile_offset(int ft) const {
+        if (padded) return static_cast<size_t>(ft) * chunks() * NM * PAD_MAT;
         return static_cast<size_t>(ft) * NM * (static_cast<size_t>(128) * 16 * nb() + 512 * static_cast<size_t>(chunks()));
     }
     // byte offset, within one expert, of feature tile ft's chunk c (all NM matrices)
     __host__ __device__ size_t chunk_offset(int ft, int c, int rf) const {
+        if (padded) return tile_offset(ft) + static_cast<size_t>(c) * NM * PAD_MAT;
         return tile_offset(ft) + static_cast<size_t>(c) * NM * (static_cast<size_t>(BPC) * rf * 16 + 512);
     }
     __host__ __device__ size_t expert_bytes() const {
+        if (padded) return static_cast<size_t>(tiles()) * chunks() * NM * PAD_MAT;
         return static_cast<size_t>(NM) *
                (static_cast<size_t>(N) * 16 * nb() + 512 * static_cast<size_t>(chunks()) * tiles());
     }
@@ -62,8 +77,14 @@ struct TiledMatrix {
         const int c = b / BPC, h = b % BPC;
         const int nbc = blocks_in_chunk(c);
         const size_t base_m = chunk_offset(ft, c, rf) + static_cast<size_t>(sub) * mat_bytes(c, rf);
-        code_off = base_m + static_cast<size_t>(h * rf + r) * 16;
-        scale_off = base_m + static_cast<size_t>(nbc) * rf * 16 + 16 * (r & 31) + 4 * (r >> 5) + h;
+        const size_t sf = 16 * (r & 31) + 4 * (r >> 5) + h;
+        if (padded) {
+            code_off = base_m + static_cast<size_t>(r) * 64 + h * 16;
+            scale_off = base_m + 128 * 64 + sf;
+        } else {
+            code_off = base_m + static_cast<size_t>(h * rf + r) * 16;
+            scale_off = base_m + static_cast<size_t>(nbc) * rf * 16 + sf;
+        }
     }
 };
 

@@ -513,7 +513,7 @@ template <> struct BlockLoader<float> {
 
 // Where the grouped operands live.
 struct GroupedOperand {
-    uint8_t* codes;   // [K/32][3][R][16]
+    uint8_t* codes;   // three MXFP4 terms [K/32][3][R][16 B]; two MXFP8 terms [K/16][2][R][16 B]
     uint8_t* scales;  // [tiles][KC][3 atoms][512]
     int R;            // row capacity
     int KC;           // chunks of 128 along K
@@ -604,12 +604,13 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
 // CTAs running together read one 128-wide column slice of x, which stays in
 // L2 while every tile that needs it reads it.  Thread r encodes blocks
 // 4c .. 4c+3 of the tile's row r (x of its token, times gamma / rms(x) with
-// the pre-norm) as three MXFP4 terms: the codes go straight to global memory
+// the pre-norm) in the operand format AF (three MXFP4 or two MXFP8 terms):
+// the codes go straight to global memory
 // (consecutive threads, consecutive rows: coalesced), the scale bytes into a
 // shared-memory copy of the tile's scale atoms, which the CTA then writes
 // whole (rows past the tile's valid rows get zero scale bytes).
 constexpr int ENC_THREADS = 128;
-template <typename TA>
+template <typename TA, int AF>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, const float* __restrict__ inv_rms,
                    const int32_t* __restrict__ row_token, const int4* __restrict__ units_gu,
@@ -648,15 +649,11 @@ encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, co
                     v[4 * i + 3] *= g.w * r;
                 }
             }
-            uint4 codes[MXQ_TERMS];
             uint32_t sb[MXQ_TERMS];
-            mxq_block_thread(v, codes, sb);
+            act_encode_store<AF>(v, X.codes, X.R, b, row, sb);
 #pragma unroll
-            for (int tt = 0; tt < MXQ_TERMS; ++tt) {
-                *reinterpret_cast<uint4*>(X.codes + ((static_cast<size_t>(b) * MXQ_TERMS + tt) * X.R + row) * 16) =
-                    codes[tt];
+            for (int tt = 0; tt < ActFormat<AF>::TERMS; ++tt)
                 atoms[sf_atom_offset(tt * X.term_rows + tid, q)] = static_cast<uint8_t>(sb[tt]);
-            }
         }
     }
     __syncthreads();
@@ -671,9 +668,10 @@ constexpr int HENC_THREADS = 128;
 // Split-K finish of the gate/up GEMM (only when the schedule split K): one
 // thread per (grouped row, 32-feature block), consecutive threads taking
 // consecutive blocks of a row, applies SwiGLU to the fp32 partial sums of g
-// and u and encodes the block of H as three MXFP4 terms into the down GEMM's
-// B operand (16 code bytes per term, one scale byte per term into the scale
+// and u and encodes the block of H (format AF) into the down GEMM's
+// B operand (the codes of each term, one scale byte per term into the scale
 // atom of the row's token tile).
+template <int AF>
 __global__ void __launch_bounds__(HENC_THREADS)
 h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
                 const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched, int tiles_cap, int* status) {
@@ -698,15 +696,12 @@ h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int B
         v[4 * i + 2] = swish_f(gg.z) * uu.z;
         v[4 * i + 3] = swish_f(gg.w) * uu.w;
     }
-    uint4 codes[MXQ_TERMS];
     uint32_t sb[MXQ_TERMS];
-    mxq_block_thread(v, codes, sb);
+    act_encode_store<AF>(v, Hd.codes, Hd.R, b, row, sb);
     uint8_t* atoms = scale_atom_base(Hd, tile, b >> 2);
 #pragma unroll
-    for (int t = 0; t < MXQ_TERMS; ++t) {
-        *reinterpret_cast<uint4*>(Hd.codes + ((static_cast<size_t>(b) * MXQ_TERMS + t) * Hd.R + row) * 16) = codes[t];
+    for (int t = 0; t < ActFormat<AF>::TERMS; ++t)
         atoms[sf_atom_offset(t * Hd.term_rows + rloc, b & 3)] = static_cast<uint8_t>(sb[t]);
-    }
 }
 
 // The layer output.  When the down GEMM did not split K, each grouped row's

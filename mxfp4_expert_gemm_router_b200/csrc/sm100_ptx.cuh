@@ -260,6 +260,21 @@ __device__ __forceinline__ void mma_mxf4_warp(uint32_t d_tmem, uint64_t a_desc, 
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
         : "memory");
 }
+// As mma_mxf4_warp with kind::mxf8f6f4 (32-element block scaling): here A is
+// E2M1 in the 16-byte-padded shared-memory form (16 codes in the low 8 bytes
+// of every 16), B is E4M3; the instruction consumes K = 32, one scale byte per
+// row chosen by the sf ids (0..3).
+__device__ __forceinline__ void mma_mxf8f6f4_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
 // Copy one 512-byte scale-factor atom (32 rows x 16 B) from shared memory to 4
 // tensor-memory columns of lanes 0..31, replicated to the four lane quarters.
 // Warp-collective; ordered with the tcgen05.mma instructions the same thread issues.
@@ -289,6 +304,21 @@ __host__ __device__ constexpr uint64_t desc_noswz(uint32_t saddr, uint32_t lbo, 
     return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (static_cast<uint64_t>(1) << 46);
 }
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of
+// 128 B, 8-row groups of 1024 B (the group must start 1024-byte aligned), the
+// 16-byte chunks of row r stored at chunk position (c ^ r % 8).  A K step
+// inside the 128-byte row advances the start address.
+__host__ __device__ constexpr uint64_t desc_sw128(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+           (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+           (static_cast<uint64_t>(2) << 61);
+}
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A E2M1 (format 5), B
+// E4M3 (format 0), E8M0 scales, f32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4_e2m1_e4m3(int M, int N) {
+    return (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
 // Instruction descriptor, kind::mxf4 block-scaled: E2M1 A and B (format 1),
 // E8M0 scales (bit 23), f32 accumulator, both K-major.  The scale-factor ids
 // (bits 4-5 for B, 29-30 for A) are or-ed in per instruction.
@@ -317,6 +347,21 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
         "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}"
         : "=r"(d)
         : "r"(byte));
+    return d;
+}
+
+// Two floats -> two E4M3 codes (lo in the low byte), rounded to nearest even,
+// saturating at +-448 (the largest finite E4M3 value).
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// Two E4M3 codes (low 16 bits) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+    uint32_t d;
+    const uint16_t h = static_cast<uint16_t>(pair);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(h));
     return d;
 }
 

@@ -117,7 +117,7 @@ def test_binding_constants_match_the_header():
              "MOE_ERR_TIMEOUT", "MOE_ERR_BOUNDS", "MOE_DTYPE_F32", "MOE_DTYPE_BF16", "MOE_FLAG_TEST_SKIP_FIRST_COPY",
              "MOE_FLAG_TOKEN_TILE_SHIFT", "MOE_FLAG_TOKEN_TILE_MASK", "MOE_NUM_STAGES",
              "MOE_ROUTE_NOALLOC_MAX_TOKENS", "MOE_ROUTE_NOALLOC_MAX_EXPERTS", "MOE_FLAG_UNFUSED_DECODE",
-             "MOE_FLAG_TEST_FAIL_ALLOC_SHIFT", "MOE_FLAG_TEST_FAIL_ALLOC_MASK"]
+             "MOE_FLAG_TEST_FAIL_ALLOC_SHIFT", "MOE_FLAG_TEST_FAIL_ALLOC_MASK", "MOE_FLAG_ACT_MXF8X2"]
     for n in names:
         assert getattr(mx, n) == hdr[n], n
     # the token-tile flag encodes BN / 16 in its field and rejects other sizes
