@@ -36,6 +36,7 @@
 #include "decode_fused.cuh"
 #include "expert_mxf4.cuh"
 #include "quantize.cuh"
+#include "router_tc.cuh"
 #include "routing.cuh"
 
 using namespace moe;
@@ -118,7 +119,11 @@ struct moe_mxfp4 {
     CUtensorMap tm_x[BN_OPTIONS];
     CUtensorMap tm_h[BN_OPTIONS];
     bool tm_ok[BN_OPTIONS] = {};
-    CUtensorMap tm_wgu{}, tm_wdn{};   // two-MXFP8-term layers: the padded weights as 16U4_ALIGN16B boxes
+    CUtensorMap tm_wgu{}, tm_wdn{};
+    // tensor-core router (bf16 layers): the weight planes and their map
+    __nv_bfloat16* wr_planes = nullptr;   // [3][E][d]: gamma * W_router as hi, mid, lo (with the pre-norm)
+    CUtensorMap tm_wr{};
+    int router_P = 1;                     // planes the map covers (1: W_router itself, 3: the planes)   // two-MXFP8-term layers: the padded weights as 16U4_ALIGN16B boxes
     // fused decode path (forwards of at most DF_MAX_T tokens)
     bool df_ok = false, last_fused = false;
     int df_stages = 0, df_S = 0, df_nb_max = 0, df_kc_max = 0, df_max_touched = 0;
@@ -320,6 +325,13 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
         return e;
     if ((e = set_router_smem<float>(rsm))) return e;
+    {
+        const int tsm = static_cast<int>(rtc_smem_bytes(3));
+        if ((e = cudaFuncSetAttribute(router_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
+        if ((e = cudaFuncSetAttribute(router_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
+        if ((e = cudaFuncSetAttribute(router_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
+        if ((e = cudaFuncSetAttribute(router_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
+    }
     if ((e = set_router_smem<__nv_bfloat16>(rsm))) return e;
     if ((e = cudaFuncSetAttribute(decode_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   227 * 1024)))
@@ -460,6 +472,7 @@ moe_status_t moe_mxfp4_create(const moe_mxfp4_config_t* cfg, moe_mxfp4_t** out) 
         {reinterpret_cast<void**>(&h->pair_row), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->status), sizeof(int) * 4},
         {&h->x_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
+        {reinterpret_cast<void**>(&h->wr_planes), 3 * static_cast<size_t>(E) * d * sizeof(__nv_bfloat16)},
         {&h->y_stage, static_cast<size_t>(c.max_tokens) * d * h->act_bytes},
         {reinterpret_cast<void**>(&h->idx_stage), sizeof(int32_t) * TK},
         {reinterpret_cast<void**>(&h->w_stage), sizeof(float) * TK},
@@ -572,6 +585,38 @@ static moe_status_t quantize_matrix(moe_mxfp4* h, int which, const float* W, int
     return cuda_status(cudaGetLastError());
 }
 
+// The tensor-core router's weight operand (bf16 layers): W_router itself, or
+// with the pre-norm gamma * W_router as three bf16 planes; and its map, a 3-D
+// view {d, E, planes} read in boxes {64, 32, planes} with the 128-byte swizzle.
+static moe_status_t prepare_router_tc(moe_mxfp4* h, cudaStream_t stream) {
+    const auto& c = h->cfg;
+    if (c.act_dtype != MOE_DTYPE_BF16 || !h->router_set) return MOE_OK;
+    const int E = c.n_experts, d = c.d_model;
+    void* src = h->w_router;
+    h->router_P = 1;
+    if (h->use_norm) {
+        const long n = static_cast<long>(E) * d;
+        const int blocks = static_cast<int>(std::min<long>(4L * h->nsm, (n + 255) / 256));
+        router_planes_kernel<<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(h->w_router), h->gamma,
+                                                          h->wr_planes, E, d);
+        h->launches++;
+        MOE_TRY(cudaGetLastError());
+        src = h->wr_planes;
+        h->router_P = 3;
+    }
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return MOE_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E), static_cast<cuuint64_t>(h->router_P)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(E) * d * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(ROUTER_KCHUNK), static_cast<cuuint32_t>(ROUTER_ETILE),
+                         static_cast<cuuint32_t>(h->router_P)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&h->tm_wr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, src, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router, const float* router_bias,
                                   cudaStream_t stream) {
     if (!h || !w_router) return MOE_ERR_INVALID_ARG;
@@ -586,7 +631,7 @@ moe_status_t moe_mxfp4_set_router(moe_mxfp4_t* h, const void* w_router, const fl
     h->has_bias = router_bias != nullptr;
     h->router_set = true;
     h->last_stream = stream;
-    return MOE_OK;
+    return prepare_router_tc(h, stream);
 }
 
 moe_status_t moe_mxfp4_set_norm_residual(moe_mxfp4_t* h, const float* gamma, float eps, int32_t residual,
@@ -599,7 +644,7 @@ moe_status_t moe_mxfp4_set_norm_residual(moe_mxfp4_t* h, const float* gamma, flo
     h->eps = eps;
     h->residual = residual != 0;
     h->last_stream = stream;
-    return MOE_OK;
+    return prepare_router_tc(h, stream);
 }
 
 moe_status_t moe_mxfp4_quantize_expert(moe_mxfp4_t* h, int32_t e, const float* w_gate, const float* w_up,
@@ -835,12 +880,30 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     ra.units_gu = h->units_gu;
     ra.units_dn = h->units_dn;
     ra.sched = h->sched;
-    const size_t rsm = router_smem_bytes();
-    const dim3 rgrid(nblk, ra.S, router_etiles(E));
-    if (bf16)
-        launch_router<__nv_bfloat16>(ra, rgrid, rsm, stream);
-    else
-        launch_router<float>(ra, rgrid, rsm, stream);
+    if (bf16) {
+        // tensor-core scores: x's map is made per call (its pointer and T change)
+        EncodeTiledFn enc = get_encode_fn();
+        if (!enc) return MOE_ERR_CUDA;
+        CUtensorMap tm_x;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(ROUTER_KCHUNK), static_cast<cuuint32_t>(ROUTER_TOKENS)};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+        const int Z = router_etiles(E), P = h->router_P;
+        const dim3 tgrid(static_cast<unsigned>(nblk * ra.S * Z));
+        const size_t tsm = rtc_smem_bytes(P);
+        const int ept = (E + 31) / 32;
+        if (ept <= 1) router_tc_kernel<1><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
+        else if (ept <= 2) router_tc_kernel<2><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
+        else if (ept <= 4) router_tc_kernel<4><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
+        else router_tc_kernel<8><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
+    } else {
+        launch_router<float>(ra, dim3(nblk, ra.S, router_etiles(E)), router_smem_bytes(), stream);
+    }
     h->stage_ran[0] = true;
     // 1: gather into grouped rows
     mark(1);

@@ -212,27 +212,20 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
     }
 }
 
-// Grid (token tiles of 128, S splits of K, expert tiles of 32).  Each CTA
-// accumulates the scores of its 128 tokens x 32 experts over its K range:
-// each thread holds a 4-token x 4-expert register tile, fp32 within a 64-wide
-// K chunk staged in shared memory (bf16 x bf16 products are exact in fp32),
-// fp64 across chunks; the next chunk is loaded into registers while the
-// current one is multiplied.  With the pre-norm the staged router chunk is
-// W_router * gamma (so the scores are of x * gamma) and the sum of x^2 per
-// token is kept (by the expert tile 0 CTAs).  The last CTA of a token tile to
-// finish sums the S partials in split order (deterministic), scales by the
-// inverse RMS, adds the bias, and for 32 tokens at a time selects the top-k
-// with one warp per token by k rounds of warp arg-max (ties to the lower
-// index) and applies the softmax over the k selected scores; it then ranks
-// the tile's (token, slot) pairs within their expert and writes the tile
-// histogram.  The last tile to finish builds the schedule (schedule_block).
-// EPT = experts per lane in the top-k (ceil(E / 32) rounded up to 1, 2, 4, 8).
-template <typename TA, int EPT>
-__global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
-    extern __shared__ __align__(16) float rsm[];
-    float* xs = rsm;                                        // [64 k][128 tokens]
-    float* ws = xs + ROUTER_KCHUNK * ROUTER_TOKENS;         // [64 k][32 experts]
-    float* lg = rsm;                                        // tail: [32 tokens][E + 1]
+// The end of a router launch, run by every CTA once its partial scores (and
+// partial sums of x^2) are written.  The last CTA of a token tile to finish
+// (of `ctas_per_tile`) sums the S partials in split order (deterministic),
+// scales by the inverse RMS, adds the bias, and for up to 128 tokens at a time
+// selects the top-k with one warp per token by k rounds of warp arg-max (ties
+// to the lower index) and applies the softmax over the k selected scores; it
+// then ranks the tile's (token, slot) pairs within their expert and writes the
+// tile histogram.  The last tile to finish builds the schedule
+// (schedule_block).  `lg` (lg_bytes of shared memory) holds the scores of a
+// pass.  EPT = experts per lane in the top-k (ceil(E / 32) rounded up to 1,
+// 2, 4, 8).  Needs ROUTER_THREADS threads.
+template <int EPT>
+__device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int ntiles, int ctas_per_tile, float* lg,
+                                            size_t lg_bytes) {
     __shared__ int hist_s[MAX_EXPERTS];
     __shared__ int es[ROUTER_TOKENS * MAX_TOPK];
     __shared__ int cnt_s[MAX_EXPERTS];
@@ -240,14 +233,166 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
     __shared__ int tb_s[MAX_EXPERTS + 1];
     __shared__ int split_s[2];
     __shared__ int last_s;
-    __shared__ double ss_s[ROUTER_TOKENS];
     __shared__ double inv_s[ROUTER_TOKENS];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int E = a.E, d = a.d, k = a.k;
+    const int t0 = tile * ROUTER_TOKENS;
+    const int ntok = min(ROUTER_TOKENS, a.T - t0);
+    const bool norm = a.gamma != nullptr;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = (atomicAdd(a.tile_cnt + tile, 1) == ctas_per_tile - 1);
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
+
+    for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
+    if (tid < ntok) {
+        double inv = 1.0;
+        if (norm) {
+            double pq[ROUTER_MAX_SPLITS];
+#pragma unroll
+            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
+                pq[sp] = sp < a.S ? __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid) : 0.0;
+            double sq = 0.0;
+#pragma unroll
+            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sq += pq[sp];
+            inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
+            a.inv_rms[t0 + tid] = static_cast<float>(inv);
+        }
+        inv_s[tid] = inv;
+    }
+    const size_t pstride = static_cast<size_t>(a.T) * E;
+    // tokens per pass: as many as the scores [sub][E + 1] fit in the staging
+    // space (128 at E = 32, 64 at E = 128, 32 at E = 256)
+    int sub_n = static_cast<int>(lg_bytes / (sizeof(float) * (E + 1))) & ~31;
+    sub_n = min(ROUTER_TOKENS, max(ROUTER_SUB, sub_n));
+    for (int sub = 0; sub < ntok; sub += sub_n) {
+        const int nsub = min(sub_n, ntok - sub);
+        __syncthreads();
+        // scores = partials summed in split order (deterministic), x inverse RMS,
+        // + bias; four scores per thread at a time, all their partials in flight
+        for (int i0 = tid; i0 < nsub * E; i0 += 4 * ROUTER_THREADS) {
+            double pv[4][ROUTER_MAX_SPLITS];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                const double* pp = a.part + static_cast<size_t>(t0 + sub + i / E) * E + i % E;
+#pragma unroll
+                for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
+                    pv[m][sp] = (i < nsub * E && sp < a.S) ? __ldcg(pp + sp * pstride) : 0.0;
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int i = i0 + m * ROUTER_THREADS;
+                if (i < nsub * E) {
+                    double sv = 0.0;
+#pragma unroll
+                    for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sv += pv[m][sp];
+                    const int tl = i / E, e = i % E;
+                    if (norm) sv *= inv_s[sub + tl];
+                    if (a.bias) sv += a.bias[e];
+                    lg[tl * (E + 1) + e] = static_cast<float>(sv);
+                }
+            }
+        }
+        __syncthreads();
+        // top-k + softmax: warp w handles tokens sub + w, sub + w + 8, ...
+        for (int tl = warp; tl < nsub; tl += ROUTER_THREADS / 32) {
+            const float* row = lg + tl * (E + 1);
+            uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
+            float sel_v[MAX_TOPK];
+            int sel_e[MAX_TOPK];
+            for (int r = 0; r < k; ++r) {
+                float bv = -INFINITY;
+                int be = 0x7FFFFFFF;
+                for (int i = 0; i < EPT; ++i) {
+                    const int e = lane + 32 * i;
+                    if (e < E && !((taken >> i) & 1u)) {
+                        const float v = row[e];
+                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+                }
+                be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                sel_v[r] = bv;
+                sel_e[r] = be;
+            }
+            if (lane == 0) {
+                const float m = sel_v[0];
+                float den = 0.f;
+                for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
+                const float inv = 1.f / den;
+                const int t = t0 + sub + tl;
+                for (int r = 0; r < k; ++r) {
+                    a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
+                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
+                    es[(sub + tl) * k + r] = sel_e[r];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    // stable rank of each pair among the tile's earlier pairs with the same
+    // expert, and the tile histogram: warp 0 walks the pairs in order, 32 at a
+    // time; lanes with the same expert find one another with match_any.
+    if (warp == 0) {
+        for (int p0 = 0; p0 < ntok * k; p0 += 32) {
+            const int p = p0 + lane;
+            const bool valid = p < ntok * k;
+            const int e = valid ? es[p] : -1 - lane;   // idle lanes form groups of their own
+            const unsigned grp = __match_any_sync(0xffffffffu, e);
+            const int before = __popc(grp & ((1u << lane) - 1u));
+            if (valid) a.local_rank[static_cast<size_t>(t0) * k + p] = hist_s[e] + before;
+            __syncwarp();
+            if (valid && before == 0) hist_s[e] += __popc(grp);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += ROUTER_THREADS) a.hist[static_cast<size_t>(tile) * E + e] = hist_s[e];
+
+    // the last tile builds the schedule
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = (atomicAdd(a.glob_cnt, 1) == ntiles - 1);
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    if (tid == 0) *a.glob_cnt = 0;
+    schedule_block(a, ntiles, cnt_s, off_s, tb_s, split_s);
+}
+
+// Grid (token tiles of 128, S splits of K, expert tiles of 32).  Each CTA
+// accumulates the scores of its 128 tokens x 32 experts over its K range on
+// the CUDA cores: each thread holds a 4-token x 4-expert register tile, fp32
+// within a 64-wide K chunk staged in shared memory (products of bf16 or fp32
+// inputs), fp64 across chunks; the next chunk is loaded into registers while
+// the current one is multiplied.  With the pre-norm the staged router chunk is
+// W_router * gamma (so the scores are of x * gamma) and the sum of x^2 per
+// token is kept (by the expert tile 0 CTAs).  router_tail finishes.  The
+// layers with bf16 activations use router_tc_kernel (tensor cores) instead;
+// this kernel serves fp32 activations and the no-allocation entry point.
+template <typename TA, int EPT>
+__global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
+    extern __shared__ __align__(16) float rsm[];
+    float* xs = rsm;                                        // [64 k][128 tokens]
+    float* ws = xs + ROUTER_KCHUNK * ROUTER_TOKENS;         // [64 k][32 experts]
+    float* lg = rsm;                                        // tail: [32 tokens][E + 1]
+    __shared__ double ss_s[ROUTER_TOKENS];
 
     pdl_launch_dependents();
     const TA* x = static_cast<const TA*>(a.x);
     const TA* wr = static_cast<const TA*>(a.wr);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int E = a.E, d = a.d, k = a.k;
+    const int tid = threadIdx.x;
+    const int E = a.E, d = a.d;
     const int tile = blockIdx.x, split = blockIdx.y, e0 = blockIdx.z * ROUTER_ETILE;
     const int ntiles = gridDim.x;
     const int t0 = tile * ROUTER_TOKENS;
@@ -350,135 +495,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
         __syncthreads();
         if (tid < ROUTER_TOKENS && xt < ntok) a.part_ss[static_cast<size_t>(split) * a.T + t0 + xt] = ss + ss_s[xt];
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = (atomicAdd(a.tile_cnt + tile, 1) == a.S * static_cast<int>(gridDim.z) - 1);
-    __syncthreads();
-    if (!last_s) return;
-    __threadfence();
-    if (tid == 0) a.tile_cnt[tile] = 0;  // ready for the next launch
-
-    for (int e = tid; e < E; e += ROUTER_THREADS) hist_s[e] = 0;
-    if (tid < ntok) {
-        double inv = 1.0;
-        if (norm) {
-            double pq[ROUTER_MAX_SPLITS];
-#pragma unroll
-            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
-                pq[sp] = sp < a.S ? __ldcg(a.part_ss + static_cast<size_t>(sp) * a.T + t0 + tid) : 0.0;
-            double sq = 0.0;
-#pragma unroll
-            for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sq += pq[sp];
-            inv = 1.0 / sqrt(sq / static_cast<double>(d) + static_cast<double>(a.eps));
-            a.inv_rms[t0 + tid] = static_cast<float>(inv);
-        }
-        inv_s[tid] = inv;
-    }
-    const size_t pstride = static_cast<size_t>(a.T) * E;
-    // tokens per pass: as many as the scores [sub][E + 1] fit in the staging
-    // space (128 at E = 32, 64 at E = 128, 32 at E = 256)
-    int sub_n = static_cast<int>(router_smem_bytes() / (sizeof(float) * (E + 1))) & ~31;
-    sub_n = min(ROUTER_TOKENS, max(ROUTER_SUB, sub_n));
-    for (int sub = 0; sub < ntok; sub += sub_n) {
-        const int nsub = min(sub_n, ntok - sub);
-        __syncthreads();
-        // scores = partials summed in split order (deterministic), x inverse RMS,
-        // + bias; four scores per thread at a time, all their partials in flight
-        for (int i0 = tid; i0 < nsub * E; i0 += 4 * ROUTER_THREADS) {
-            double pv[4][ROUTER_MAX_SPLITS];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int i = i0 + m * ROUTER_THREADS;
-                const double* pp = a.part + static_cast<size_t>(t0 + sub + i / E) * E + i % E;
-#pragma unroll
-                for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp)
-                    pv[m][sp] = (i < nsub * E && sp < a.S) ? __ldcg(pp + sp * pstride) : 0.0;
-            }
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const int i = i0 + m * ROUTER_THREADS;
-                if (i < nsub * E) {
-                    double sv = 0.0;
-#pragma unroll
-                    for (int sp = 0; sp < ROUTER_MAX_SPLITS; ++sp) sv += pv[m][sp];
-                    const int tl = i / E, e = i % E;
-                    if (norm) sv *= inv_s[sub + tl];
-                    if (a.bias) sv += a.bias[e];
-                    lg[tl * (E + 1) + e] = static_cast<float>(sv);
-                }
-            }
-        }
-        __syncthreads();
-        // top-k + softmax: warp w handles tokens sub + w, sub + w + 8, ...
-        for (int tl = warp; tl < nsub; tl += ROUTER_THREADS / 32) {
-            const float* row = lg + tl * (E + 1);
-            uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-            float sel_v[MAX_TOPK];
-            int sel_e[MAX_TOPK];
-            for (int r = 0; r < k; ++r) {
-                float bv = -INFINITY;
-                int be = 0x7FFFFFFF;
-                for (int i = 0; i < EPT; ++i) {
-                    const int e = lane + 32 * i;
-                    if (e < E && !((taken >> i) & 1u)) {
-                        const float v = row[e];
-                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-                    }
-                }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-                }
-                be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                sel_v[r] = bv;
-                sel_e[r] = be;
-            }
-            if (lane == 0) {
-                const float m = sel_v[0];
-                float den = 0.f;
-                for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
-                const float inv = 1.f / den;
-                const int t = t0 + sub + tl;
-                for (int r = 0; r < k; ++r) {
-                    a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
-                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
-                    es[(sub + tl) * k + r] = sel_e[r];
-                }
-            }
-        }
-    }
-    __syncthreads();
-    // stable rank of each pair among the tile's earlier pairs with the same
-    // expert, and the tile histogram: warp 0 walks the pairs in order, 32 at a
-    // time; lanes with the same expert find one another with match_any.
-    if (warp == 0) {
-        for (int p0 = 0; p0 < ntok * k; p0 += 32) {
-            const int p = p0 + lane;
-            const bool valid = p < ntok * k;
-            const int e = valid ? es[p] : -1 - lane;   // idle lanes form groups of their own
-            const unsigned grp = __match_any_sync(0xffffffffu, e);
-            const int before = __popc(grp & ((1u << lane) - 1u));
-            if (valid) a.local_rank[static_cast<size_t>(t0) * k + p] = hist_s[e] + before;
-            __syncwarp();
-            if (valid && before == 0) hist_s[e] += __popc(grp);
-            __syncwarp();
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += ROUTER_THREADS) a.hist[static_cast<size_t>(tile) * E + e] = hist_s[e];
-
-    // the last tile builds the schedule
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = (atomicAdd(a.glob_cnt, 1) == ntiles - 1);
-    __syncthreads();
-    if (!last_s) return;
-    __threadfence();
-    if (tid == 0) *a.glob_cnt = 0;
-    schedule_block(a, ntiles, cnt_s, off_s, tb_s, split_s);
+    router_tail<EPT>(a, tile, ntiles, a.S * static_cast<int>(gridDim.z), lg, router_smem_bytes());
 }
 
 // One 32-element block of a token's activations as floats.
