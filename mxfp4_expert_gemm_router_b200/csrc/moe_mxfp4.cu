@@ -5,17 +5,19 @@
 // decode_fused_kernel (router, both expert GEMMs and the combine in one
 // persistent grid).  Larger forwards are up to seven launches on the caller's
 // stream; no host sync and no allocation either way:
-//   router_kernel        scores (K split over the grid), top-k, softmax over the
-//                        selected scores, per-tile histogram and ranks, zeroing
-//                        of the output rows; its last CTA builds the schedule
-//                        (expert offsets, K splits, unit lists)
-//   rows_kernel          grouped rows (token, weight, tile slot); output
-//                        accumulator initialised (zero, or x for the residual)
-//   encode_rows_kernel   the grouped rows of x encoded as three MXFP4 terms
-//                        (the gate/up GEMM's B operand)
-//   expert_mxf4<0>       gate/up GEMM on block-scaled MXFP4 tensor cores,
-//                        SwiGLU epilogue encoding H as three MXFP4 terms for the
-//                        down GEMM (fp32 partials instead when K is split)
+//   router_tc_kernel     scores on the tensor cores (bf16 layers; router_kernel
+//                        on the CUDA cores for fp32 ones), K split over the grid;
+//                        top-k, softmax over the selected scores, per-tile
+//                        histogram and ranks; its last CTA builds the schedule
+//                        (expert offsets, K splits, unit counts)
+//   rows_kernel          the unit lists; grouped rows (token, weight, tile
+//                        slot); output accumulator initialised when K is split
+//   encode_rows_kernel   the grouped rows of x encoded as the gate/up GEMM's B
+//                        operand (three MXFP4 or two MXFP8 terms)
+//   expert_mxf4<0>       gate/up GEMM on block-scaled tensor cores (kind::mxf4,
+//                        or kind::mxf8f6f4 for two MXFP8 terms), SwiGLU epilogue
+//                        encoding H for the down GEMM (fp32 partials instead
+//                        when K is split)
 //   h_encode_kernel      only when the gate/up GEMM may split K: SwiGLU + encoding
 //   expert_mxf4<1>       down GEMM: each grouped row's weighted output stored
 //                        once (a fp32 scatter-add when K is split)
@@ -219,7 +221,8 @@ static void free_all(moe_mxfp4* h) {
                     h->part, h->counters, h->local_rank, h->offsets, h->tile_base, h->sched, h->units_gu,
                     h->units_dn, h->row_token, h->row_weight, h->row_slot, h->Xq, h->Hq, h->sfx, h->sfh,
                     h->GU, h->yacc, h->obuf, h->pair_row, h->status, h->x_stage, h->y_stage, h->idx_stage, h->w_stage,
-                    h->df_state, h->df_part, h->df_part_ss, h->df_yacc, h->df_xq, h->df_hq, h->df_hdone};
+                    h->df_state, h->df_part, h->df_part_ss, h->df_yacc, h->df_xq, h->df_hq, h->df_hdone,
+                    h->wr_planes};
     for (void* p : ptrs)
         if (p) cudaFree(p);
     for (auto& e : h->ev)
@@ -284,22 +287,14 @@ static int router_splits(int T, int d, int E, int nsm) {
     return std::max(1, std::min(std::min(kch, ROUTER_MAX_SPLITS), want));
 }
 
-// Router launch for the expert count: EPT = experts per lane, 1/2/4/8.
+// CUDA-core router launch (fp32 activations and the no-allocation entry point).
 template <typename TA>
 static void launch_router(const RouterArgs& ra, dim3 grid, size_t smem, cudaStream_t stream) {
-    const int ept = (ra.E + 31) / 32;
-    if (ept <= 1) router_kernel<TA, 1><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
-    else if (ept <= 2) router_kernel<TA, 2><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
-    else if (ept <= 4) router_kernel<TA, 4><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
-    else router_kernel<TA, 8><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
+    router_kernel<TA><<<grid, ROUTER_THREADS, smem, stream>>>(ra);
 }
 template <typename TA>
 static cudaError_t set_router_smem(int bytes) {
-    cudaError_t e;
-    if ((e = cudaFuncSetAttribute(router_kernel<TA, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
-    if ((e = cudaFuncSetAttribute(router_kernel<TA, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
-    if ((e = cudaFuncSetAttribute(router_kernel<TA, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))) return e;
-    return cudaFuncSetAttribute(router_kernel<TA, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return cudaFuncSetAttribute(router_kernel<TA>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
 // The handle's buffers live on the device that was current at create: calls
@@ -327,10 +322,7 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     if ((e = set_router_smem<float>(rsm))) return e;
     {
         const int tsm = static_cast<int>(rtc_smem_bytes(3));
-        if ((e = cudaFuncSetAttribute(router_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
-        if ((e = cudaFuncSetAttribute(router_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
-        if ((e = cudaFuncSetAttribute(router_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
-        if ((e = cudaFuncSetAttribute(router_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
+        if ((e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tsm))) return e;
     }
     if ((e = set_router_smem<__nv_bfloat16>(rsm))) return e;
     if ((e = cudaFuncSetAttribute(decode_fused_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -896,11 +888,7 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
         const int Z = router_etiles(E), P = h->router_P;
         const dim3 tgrid(static_cast<unsigned>(nblk * ra.S * Z));
         const size_t tsm = rtc_smem_bytes(P);
-        const int ept = (E + 31) / 32;
-        if (ept <= 1) router_tc_kernel<1><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
-        else if (ept <= 2) router_tc_kernel<2><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
-        else if (ept <= 4) router_tc_kernel<4><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
-        else router_tc_kernel<8><<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
+        router_tc_kernel<<<tgrid, RTC_THREADS, tsm, stream>>>(tm_x, h->tm_wr, ra, Z, P, h->status, tmo);
     } else {
         launch_router<float>(ra, dim3(nblk, ra.S, router_etiles(E)), router_smem_bytes(), stream);
     }
@@ -924,7 +912,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->hist), static_cast<const int32_t*>(h->offsets),
                    static_cast<const int32_t*>(h->tile_base), T, d, E, k, BN, h->row_token, h->row_weight,
                    h->row_slot, h->GU, 2 * f, acc, static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0,
-                   tiles_cap, h->status, h->pair_row);
+                   tiles_cap, h->status, h->pair_row, h->F_gu, h->F_dn,
+                   h->units_gu, h->units_dn);
         launch_pdl(pdl, af ? encode_rows_kernel<__nv_bfloat16, 1> : encode_rows_kernel<__nv_bfloat16, 0>, egrid, dim3(ENC_THREADS), 0, stream,
                    static_cast<const __nv_bfloat16*>(x), gam, static_cast<const float*>(h->inv_rms),
                    static_cast<const int32_t*>(h->row_token), static_cast<const int4*>(h->units_gu),
@@ -935,7 +924,8 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
                    static_cast<const int32_t*>(h->local_rank), static_cast<const int32_t*>(h->hist),
                    static_cast<const int32_t*>(h->offsets), static_cast<const int32_t*>(h->tile_base), T, d, E, k,
                    BN, h->row_token, h->row_weight, h->row_slot, h->GU, 2 * f, acc,
-                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status, h->pair_row);
+                   static_cast<const int32_t*>(h->sched), h->residual ? 1 : 0, tiles_cap, h->status, h->pair_row, h->F_gu, h->F_dn,
+                   h->units_gu, h->units_dn);
         launch_pdl(pdl, af ? encode_rows_kernel<float, 1> : encode_rows_kernel<float, 0>, egrid, dim3(ENC_THREADS), 0, stream, static_cast<const float*>(x),
                    gam, static_cast<const float*>(h->inv_rms), static_cast<const int32_t*>(h->row_token),
                    static_cast<const int4*>(h->units_gu), static_cast<const int32_t*>(h->sched), h->F_gu, d, Xop, T,

@@ -106,7 +106,6 @@ __global__ void router_planes_kernel(const __nv_bfloat16* __restrict__ wr, const
 // tmap_x: x [T][d] bf16, box {64, 128}, 128-byte swizzle (rows past T read as
 // zeros).  tmap_w: the weight planes [P][E][d] bf16, box {64, 32, P}, landing
 // as P x 32 rows of 128 B (experts past E read as zeros).
-template <int EPT>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                  const RouterArgs a, int Z, int P, int* status, uint64_t timeout_ns) {
@@ -267,7 +266,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
         tmem_dealloc(tmem, 256);
     }
     // the stages are free again: the tail's scores reuse them
-    router_tail<EPT>(a, tile, ntiles, a.S * Z, reinterpret_cast<float*>(smem_raw + (base - raw)),
+    router_tail(a, tile, ntiles, a.S * Z, reinterpret_cast<float*>(smem_raw + (base - raw)),
                      static_cast<size_t>(RTC_STAGES) * SB);
 }
 

@@ -114,26 +114,34 @@ __device__ inline int pick_split(int base, int nsm, int KC) {
 
 // Run by the last router CTA to finish: per-expert totals and per-tile
 // prefixes of the histogram (warp scans over tiles), group offsets and token
-// tile bases (one warp-wide scan over experts), K splits, and the unit lists of
+// tile bases (one warp-wide scan over experts), K splits and the unit counts of
 // both expert GEMMs.  Units are ordered (expert, token tile, feature tile,
-// split); token tiles are numbered consecutively over the experts, so unit u
-// is token tile u / (F S), feature tile (u / S) % F, split u % S, and its
-// expert is found by binary search over the tile bases.
+// split); token tiles are numbered consecutively over the experts.  The unit
+// lists themselves are written by the next kernel (build_units), in parallel.
 __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt, int* off, int* tb, int* split_s) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     for (int e = warp; e < a.E; e += nwarps) {
         int carry = 0;
-        for (int b0 = 0; b0 < ntiles; b0 += 32) {
-            const int b = b0 + lane;
-            const int v = (b < ntiles) ? __ldcg(a.hist + static_cast<size_t>(b) * a.E + e) : 0;
-            int inc = v;
+        // 256 tiles per round: the eight loads of a lane are issued together
+        for (int r0 = 0; r0 < ntiles; r0 += 256) {
+            int v[8];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += n;
+            for (int i = 0; i < 8; ++i) {
+                const int b = r0 + 32 * i + lane;
+                v[i] = (b < ntiles) ? __ldcg(a.hist + static_cast<size_t>(b) * a.E + e) : 0;
             }
-            if (b < ntiles) a.hist[static_cast<size_t>(b) * a.E + e] = carry + inc - v;
-            carry += __shfl_sync(0xffffffffu, inc, 31);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int b = r0 + 32 * i + lane;
+                int inc = v[i];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += n;
+                }
+                if (b < ntiles) a.hist[static_cast<size_t>(b) * a.E + e] = carry + inc - v[i];
+                carry += __shfl_sync(0xffffffffu, inc, 31);
+            }
         }
         if (lane == 0) cnt[e] = carry;
     }
@@ -189,26 +197,39 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
         for (int e = tid; e < a.E; e += blockDim.x) a.counts_out[e] = cnt[e];
     if (a.tile_base)
         for (int e = tid; e < a.E; e += blockDim.x) a.tile_base[e] = tb[e];
-    const int total_tiles = tb[a.E];
-    for (int g = 0; g < 2; ++g) {
-        const int F = g ? a.F_dn : a.F_gu;
-        const int S = split_s[g];
-        int4* units = g ? a.units_dn : a.units_gu;
-        const int nu = min(total_tiles * F * S, a.max_units);
-        for (int u = tid; u < nu; u += blockDim.x) {
-            const int tile = u / (F * S);
-            const int rem = u - tile * F * S;
-            const int ft = rem / S, sp = rem - ft * S;
-            // the last e with tb[e] <= tile: an expert with no tiles shares its base
-            // with the next one, so this e owns the tile
-            int lo = 0, hi = a.E - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (tb[mid] <= tile) lo = mid; else hi = mid - 1;
-            }
-            const int m = tile - tb[lo];
-            units[u] = make_int4(lo | (tile << 8), off[lo] + m * a.BN, min(a.BN, cnt[lo] - m * a.BN), ft | (sp << 16));
-        }
+}
+
+// Unit u of an expert GEMM's list (F feature tiles, S K splits): token tile
+// u / (F S), feature tile (u / S) % F, split u % S; the tile's expert is the
+// last e with tile_base[e] <= tile (an expert with no tiles shares its base
+// with the next one).  {expert | tile << 8, first grouped row, rows, feature
+// tile | split << 16}.
+__device__ __forceinline__ int4 make_unit(int u, int F, int S, int E, int BN, const int32_t* tile_base,
+                                          const int32_t* offsets) {
+    const int tile = u / (F * S);
+    const int rem = u - tile * F * S;
+    const int ft = rem / S, sp = rem - ft * S;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_base[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int m = tile - tile_base[lo];
+    const int cnt = offsets[lo + 1] - offsets[lo];
+    return make_int4(lo | (tile << 8), offsets[lo] + m * BN, min(BN, cnt - m * BN), ft | (sp << 16));
+}
+
+// Both GEMMs' unit lists from the schedule, spread over a whole grid (thread
+// `gtid` of `gthreads`): run by the kernel after the router.
+__device__ inline void build_units(int gtid, int gthreads, const int32_t* sched, int E, int BN, int F_gu, int F_dn,
+                                   const int32_t* tile_base, const int32_t* offsets, int4* units_gu, int4* units_dn) {
+    const int n_gu = sched[SCHED_UNITS_GU], n_dn = sched[SCHED_UNITS_DN];
+    const int S_gu = sched[SCHED_SPLIT_GU], S_dn = sched[SCHED_SPLIT_DN];
+    for (int u = gtid; u < n_gu + n_dn; u += gthreads) {
+        if (u < n_gu)
+            units_gu[u] = make_unit(u, F_gu, S_gu, E, BN, tile_base, offsets);
+        else
+            units_dn[u - n_gu] = make_unit(u - n_gu, F_dn, S_dn, E, BN, tile_base, offsets);
     }
 }
 
@@ -216,14 +237,12 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
 // partial sums of x^2) are written.  The last CTA of a token tile to finish
 // (of `ctas_per_tile`) sums the S partials in split order (deterministic),
 // scales by the inverse RMS, adds the bias, and for up to 128 tokens at a time
-// selects the top-k with one warp per token by k rounds of warp arg-max (ties
-// to the lower index) and applies the softmax over the k selected scores; it
+// selects the top-k (one thread per token; ties to the lower index) and
+// applies the softmax over the k selected scores; it
 // then ranks the tile's (token, slot) pairs within their expert and writes the
 // tile histogram.  The last tile to finish builds the schedule
 // (schedule_block).  `lg` (lg_bytes of shared memory) holds the scores of a
-// pass.  EPT = experts per lane in the top-k (ceil(E / 32) rounded up to 1,
-// 2, 4, 8).  Needs ROUTER_THREADS threads.
-template <int EPT>
+// pass.  Needs ROUTER_THREADS threads.
 __device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int ntiles, int ctas_per_tile, float* lg,
                                             size_t lg_bytes) {
     __shared__ int hist_s[MAX_EXPERTS];
@@ -298,43 +317,49 @@ __device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int n
             }
         }
         __syncthreads();
-        // top-k + softmax: warp w handles tokens sub + w, sub + w + 8, ...
-        for (int tl = warp; tl < nsub; tl += ROUTER_THREADS / 32) {
+        // top-k + softmax: one thread per token, one ascending pass over the
+        // experts keeping the k best sorted by (score desc, index asc); a
+        // candidate displaces an entry only if it is larger, or equal with a
+        // lower index, so ties go to the lower index; a NaN never enters
+        for (int tl = tid; tl < nsub; tl += ROUTER_THREADS) {
             const float* row = lg + tl * (E + 1);
-            uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-            float sel_v[MAX_TOPK];
-            int sel_e[MAX_TOPK];
-            for (int r = 0; r < k; ++r) {
-                float bv = -INFINITY;
-                int be = 0x7FFFFFFF;
-                for (int i = 0; i < EPT; ++i) {
-                    const int e = lane + 32 * i;
-                    if (e < E && !((taken >> i) & 1u)) {
-                        const float v = row[e];
-                        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+            float sv[MAX_TOPK];
+            int se[MAX_TOPK];
+#pragma unroll
+            for (int r = 0; r < MAX_TOPK; ++r) {
+                sv[r] = -INFINITY;
+                se[r] = 0x7FFFFFFF;
+            }
+#pragma unroll 4
+            for (int e = 0; e < E; ++e) {
+                float cv = row[e];
+                int ce = e;
+#pragma unroll
+                for (int r = 0; r < MAX_TOPK; ++r) {
+                    if (r < k && (cv > sv[r] || (cv == sv[r] && ce < se[r]))) {
+                        const float tv = sv[r];
+                        const int te = se[r];
+                        sv[r] = cv;
+                        se[r] = ce;
+                        cv = tv;
+                        ce = te;
                     }
                 }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-                }
-                be = min(be, E - 1);   // a NaN score selects nothing: keep the index in range
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                sel_v[r] = bv;
-                sel_e[r] = be;
             }
-            if (lane == 0) {
-                const float m = sel_v[0];
-                float den = 0.f;
-                for (int r = 0; r < k; ++r) den += expf(sel_v[r] - m);
-                const float inv = 1.f / den;
-                const int t = t0 + sub + tl;
-                for (int r = 0; r < k; ++r) {
-                    a.idx_out[static_cast<size_t>(t) * k + r] = sel_e[r];
-                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sel_v[r] - m) * inv;
-                    es[(sub + tl) * k + r] = sel_e[r];
+            const float m = sv[0];
+            float den = 0.f;
+#pragma unroll
+            for (int r = 0; r < MAX_TOPK; ++r)
+                if (r < k) den += expf(sv[r] - m);
+            const float inv = 1.f / den;
+            const int t = t0 + sub + tl;
+#pragma unroll
+            for (int r = 0; r < MAX_TOPK; ++r) {
+                if (r < k) {
+                    const int e = min(se[r], E - 1);   // a NaN score selects nothing: keep the index in range
+                    a.idx_out[static_cast<size_t>(t) * k + r] = e;
+                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sv[r] - m) * inv;
+                    es[(sub + tl) * k + r] = e;
                 }
             }
         }
@@ -380,7 +405,7 @@ __device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int n
 // token is kept (by the expert tile 0 CTAs).  router_tail finishes.  The
 // layers with bf16 activations use router_tc_kernel (tensor cores) instead;
 // this kernel serves fp32 activations and the no-allocation entry point.
-template <typename TA, int EPT>
+template <typename TA>
 __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs a) {
     extern __shared__ __align__(16) float rsm[];
     float* xs = rsm;                                        // [64 k][128 tokens]
@@ -495,7 +520,7 @@ __global__ void __launch_bounds__(ROUTER_THREADS) router_kernel(const RouterArgs
         __syncthreads();
         if (tid < ROUTER_TOKENS && xt < ntok) a.part_ss[static_cast<size_t>(split) * a.T + t0 + xt] = ss + ss_s[xt];
     }
-    router_tail<EPT>(a, tile, ntiles, a.S * static_cast<int>(gridDim.z), lg, router_smem_bytes());
+    router_tail(a, tile, ntiles, a.S * static_cast<int>(gridDim.z), lg, router_smem_bytes());
 }
 
 // One 32-element block of a token's activations as floats.
@@ -542,7 +567,8 @@ __device__ __forceinline__ uint8_t* scale_atom_base(const GroupedOperand& g, int
     return g.scales + (static_cast<size_t>(tile) * g.KC + chunk) * MXQ_TERMS * 512;
 }
 
-// Grouping, part 1: one CTA per ROWS_TOKENS tokens.  Pair p = t*k + j goes
+// Grouping, part 1: one CTA per ROWS_TOKENS tokens.  The whole grid first
+// writes both expert GEMMs' unit lists (build_units).  Pair p = t*k + j goes
 // to grouped row offsets[e] + (rows of e in earlier router tiles) + (its rank
 // within its router tile), so the rows of an expert are in (token, slot)
 // order; the row's place in the expert's token tiles is (tile_base[e] +
@@ -556,18 +582,20 @@ constexpr int ROWS_TOKENS = 8;
 constexpr int ROWS_THREADS = 256;
 template <typename TA>
 __global__ void __launch_bounds__(ROWS_THREADS)
-rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ w,
-            const int32_t* __restrict__ local_rank, const int32_t* __restrict__ tile_prefix,
-            const int32_t* __restrict__ offsets, const int32_t* __restrict__ tile_base, int T, int d, int E, int k,
+rows_kernel(const TA* __restrict__ x, const int32_t* idx, const float* w, const int32_t* local_rank,
+            const int32_t* tile_prefix, const int32_t* offsets, const int32_t* tile_base, int T, int d, int E, int k,
             int BN, int32_t* __restrict__ row_token, float* __restrict__ row_weight, int32_t* __restrict__ row_slot,
-            float* __restrict__ GU, int gu_ld, float* __restrict__ yacc, const int32_t* __restrict__ sched,
-            int residual, int tiles_cap, int* status, int32_t* __restrict__ pair_row) {
+            float* __restrict__ GU, int gu_ld, float* __restrict__ yacc, const int32_t* sched,
+            int residual, int tiles_cap, int* status, int32_t* __restrict__ pair_row, int F_gu, int F_dn,
+            int4* __restrict__ units_gu, int4* __restrict__ units_dn) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ int pos_s[ROWS_TOKENS * MAX_TOPK];
     const int t0 = blockIdx.x * ROWS_TOKENS;
     const int nt = min(ROWS_TOKENS, T - t0);
     const int tid = threadIdx.x;
+    build_units(blockIdx.x * ROWS_THREADS + tid, gridDim.x * ROWS_THREADS, sched, E, BN, F_gu, F_dn, tile_base, offsets,
+                units_gu, units_dn);
     if (tid < nt * k) {
         const int p = t0 * k + tid;
         const int t = p / k;
@@ -629,9 +657,8 @@ rows_kernel(const TA* __restrict__ x, const int32_t* __restrict__ idx, const flo
 constexpr int ENC_THREADS = 128;
 template <typename TA, int AF>
 __global__ void __launch_bounds__(ENC_THREADS)
-encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, const float* __restrict__ inv_rms,
-                   const int32_t* __restrict__ row_token, const int4* __restrict__ units_gu,
-                   const int32_t* __restrict__ sched, int F_gu, int d, GroupedOperand X, int T, int* status) {
+encode_rows_kernel(const TA* __restrict__ x, const float* __restrict__ gamma, const float* inv_rms,
+                   const int32_t* row_token, const int4* units_gu, const int32_t* sched, int F_gu, int d, GroupedOperand X, int T, int* status) {
     pdl_launch_dependents();
     pdl_wait();
     __shared__ __align__(16) uint8_t atoms[MXQ_TERMS * 512];
@@ -690,8 +717,8 @@ constexpr int HENC_THREADS = 128;
 // atom of the row's token tile).
 template <int AF>
 __global__ void __launch_bounds__(HENC_THREADS)
-h_encode_kernel(const float* __restrict__ GU, GroupedOperand Hd, int d_ff, int BN,
-                const int32_t* __restrict__ row_slot, const int32_t* __restrict__ sched, int tiles_cap, int* status) {
+h_encode_kernel(const float* GU, GroupedOperand Hd, int d_ff, int BN, const int32_t* row_slot, const int32_t* sched,
+                int tiles_cap, int* status) {
     pdl_launch_dependents();
     pdl_wait();
     if (sched[SCHED_SPLIT_GU] <= 1) return;
@@ -762,9 +789,8 @@ template <> struct Vec8<float> {
 };
 template <typename TA>
 __global__ void __launch_bounds__(COMBINE_THREADS)
-combine_out_kernel(const TA* __restrict__ obuf, const int32_t* __restrict__ pair_row, const float* __restrict__ yacc,
-                   const TA* __restrict__ x, TA* __restrict__ y, int T, int d, int k, int residual,
-                   const int32_t* __restrict__ sched) {
+combine_out_kernel(const TA* obuf, const int32_t* pair_row, const float* yacc, const TA* __restrict__ x,
+                   TA* __restrict__ y, int T, int d, int k, int residual, const int32_t* sched) {
     pdl_wait();
     const int d8 = d / 8;
     const bool split = sched[SCHED_SPLIT_DN] > 1;

@@ -65,6 +65,10 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // Wait until the preceding kernel in the stream has completed and its writes
 // are visible; a no-op for a kernel launched without programmatic serialization.
+// Pointers to what the preceding kernels write must not be `const __restrict__`
+// in a kernel that waits here: the compiler may then load through them before
+// the wait (the asm's memory clobber does not cover restrict-qualified data),
+// which, with the kernel launched early, reads values not yet written.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Device-side status word shared with the host: a set of bits.
