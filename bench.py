@@ -517,8 +517,10 @@ def main():
     roof["algorithmic_per_launch"] = work[dominant]["bytes"] if roof["bound"] == "hbm" else work[dominant]["flops"]
     tr = load_traffic_record()
     roof["traffic"] = None
-    if tr and tr.get("source_hash") == kernel_source_hash() and tr.get("config") == cfg.name:
-        roof["traffic"] = tr.get("per_launch_bytes", {}).get(dominant)
+    if tr and tr.get("source_hash") == kernel_source_hash():
+        # per-launch DRAM bytes of this workload's dominant kernel, from its ncu
+        # capture (null when the kernels changed after the capture)
+        roof["traffic"] = tr.get("per_config", {}).get(cfg.name, {}).get(dominant)
     layer_s = r["total_ms"] / 1e3 / args.steps
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
