@@ -132,6 +132,7 @@ __device__ inline void schedule_block(const RouterArgs& a, int ntiles, int* cnt,
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
+                if (r0 + 32 * i >= ntiles) break;   // warp-uniform
                 const int b = r0 + 32 * i + lane;
                 int inc = v[i];
 #pragma unroll
@@ -317,12 +318,19 @@ __device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int n
             }
         }
         __syncthreads();
-        // top-k + softmax: one thread per token, one ascending pass over the
-        // experts keeping the k best sorted by (score desc, index asc); a
-        // candidate displaces an entry only if it is larger, or equal with a
-        // lower index, so ties go to the lower index; a NaN never enters
-        for (int tl = tid; tl < nsub; tl += ROUTER_THREADS) {
-            const float* row = lg + tl * (E + 1);
+        // top-k + softmax: G = 256 / (tokens rounded up to a power of two)
+        // consecutive lanes per token (1 .. 8).  Lane g of a token takes experts
+        // g, g + G, ... in ascending order, keeping its k best sorted by (score
+        // desc, index asc): a candidate displaces an entry only if it is
+        // larger, or equal with a lower index (ties go to the lower index; a
+        // NaN never enters).  The G lists are then merged by k rounds of a
+        // shuffle arg-max over the lanes' heads.
+        int G = 1;
+        while (G < 8 && G * 2 * nsub <= ROUTER_THREADS) G *= 2;
+        const int tl = tid / G, g = tid % G;
+        {
+            const bool active = tl < nsub;
+            const float* row = lg + (active ? tl : 0) * (E + 1);
             float sv[MAX_TOPK];
             int se[MAX_TOPK];
 #pragma unroll
@@ -330,36 +338,67 @@ __device__ __forceinline__ void router_tail(const RouterArgs& a, int tile, int n
                 sv[r] = -INFINITY;
                 se[r] = 0x7FFFFFFF;
             }
+            if (active) {
 #pragma unroll 4
-            for (int e = 0; e < E; ++e) {
-                float cv = row[e];
-                int ce = e;
+                for (int e = g; e < E; e += G) {
+                    float cv = row[e];
+                    int ce = e;
 #pragma unroll
-                for (int r = 0; r < MAX_TOPK; ++r) {
-                    if (r < k && (cv > sv[r] || (cv == sv[r] && ce < se[r]))) {
-                        const float tv = sv[r];
-                        const int te = se[r];
-                        sv[r] = cv;
-                        se[r] = ce;
-                        cv = tv;
-                        ce = te;
+                    for (int r = 0; r < MAX_TOPK; ++r) {
+                        if (r < k && (cv > sv[r] || (cv == sv[r] && ce < se[r]))) {
+                            const float tv = sv[r];
+                            const int te = se[r];
+                            sv[r] = cv;
+                            se[r] = ce;
+                            cv = tv;
+                            ce = te;
+                        }
                     }
                 }
             }
-            const float m = sv[0];
-            float den = 0.f;
-#pragma unroll
-            for (int r = 0; r < MAX_TOPK; ++r)
-                if (r < k) den += expf(sv[r] - m);
-            const float inv = 1.f / den;
-            const int t = t0 + sub + tl;
+            // merge: round r takes the best head over the G lanes; its lane pops it
+            float mv[MAX_TOPK];
+            int me[MAX_TOPK];
 #pragma unroll
             for (int r = 0; r < MAX_TOPK; ++r) {
-                if (r < k) {
-                    const int e = min(se[r], E - 1);   // a NaN score selects nothing: keep the index in range
-                    a.idx_out[static_cast<size_t>(t) * k + r] = e;
-                    a.w_out[static_cast<size_t>(t) * k + r] = expf(sv[r] - m) * inv;
-                    es[(sub + tl) * k + r] = e;
+                float bv = sv[0];
+                int be = se[0];
+                for (int o = 1; o < G; o <<= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    if (ov > bv || (ov == bv && oe < be)) {
+                        bv = ov;
+                        be = oe;
+                    }
+                }
+                mv[r] = bv;
+                me[r] = be;
+                if (se[0] == be) {   // experts are disjoint across the lanes: only the owner pops
+#pragma unroll
+                    for (int i = 0; i + 1 < MAX_TOPK; ++i) {
+                        sv[i] = sv[i + 1];
+                        se[i] = se[i + 1];
+                    }
+                    sv[MAX_TOPK - 1] = -INFINITY;
+                    se[MAX_TOPK - 1] = 0x7FFFFFFF;
+                }
+            }
+            if (active && g == 0) {
+                const float m = mv[0];
+                float den = 0.f;
+#pragma unroll
+                for (int r = 0; r < MAX_TOPK; ++r)
+                    if (r < k) den += expf(mv[r] - m);
+                const float inv = 1.f / den;
+                const int t = t0 + sub + tl;
+#pragma unroll
+                for (int r = 0; r < MAX_TOPK; ++r) {
+                    if (r < k) {
+                        const int e = min(me[r], E - 1);   // a NaN score selects nothing: keep the index in range
+                        a.idx_out[static_cast<size_t>(t) * k + r] = e;
+                        a.w_out[static_cast<size_t>(t) * k + r] = expf(mv[r] - m) * inv;
+                        es[(sub + tl) * k + r] = e;
+                    }
                 }
             }
         }

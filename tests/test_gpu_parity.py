@@ -221,6 +221,29 @@ def test_forward_host_matches_device(layer20b):
     assert np.abs(to_f64(yh) - y_dev).max() <= 1e-2 * np.abs(y_dev).max()
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 40, 200])
+def test_router_ties_go_to_the_lower_index(dtype, T):
+    """Experts 2 and 6 get identical router rows and a bias far above the rest,
+    so every token's two best scores are exactly equal: expert 2 (the lower
+    index) comes first, then 6, with weights 1/2 each.  T = 1, 40 and 200 take
+    the top-k with 8, 4 and 1-2 lanes per token (and two router tiles at 200);
+    fp32 layers score on the CUDA cores, bf16 layers on the tensor cores."""
+    import mxfp4_expert_gemm_router_b200 as mx
+    cfg = mi.MoeConfig("ties", T, 64, 128, 8, 2, dtype)
+    L = GpuLayer(cfg, T, flags=mx.MOE_FLAG_UNFUSED_DECODE)
+    wr = L.wr.copy()
+    wr[6] = wr[2]
+    bias = np.zeros(cfg.n_experts, np.float32)
+    bias[2] = bias[6] = 50.0
+    L.set_router(wr, bias)
+    x = mi.draw_x(cfg)
+    _, idx, w, counts = L.forward(x)
+    assert (idx[:, 0] == 2).all() and (idx[:, 1] == 6).all(), idx[:4]
+    np.testing.assert_allclose(w, 0.5, atol=1e-7)
+    assert counts[2] == T and counts[6] == T and counts.sum() == 2 * T
+
+
 def test_identity_experts_closed_form():
     """W_gate = a I, W_up = b I, W_down = c I (powers of two): y = sum_j w_j c a b x^2 sigma(a x)."""
     import torch
