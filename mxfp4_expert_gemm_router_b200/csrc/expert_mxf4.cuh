@@ -150,8 +150,8 @@ __host__ inline int mxg_nacc(int mode, int BN, int af = 0) {
 constexpr int MXG_HT_STRIDE = 33;
 constexpr uint32_t MXG_HT_BYTES = MXG_EPI_WARPS * 32 * MXG_HT_STRIDE * 4;
 __host__ __device__ constexpr uint32_t mxg_extra_smem(int mode) { return mode == 0 ? MXG_HT_BYTES : 0u; }
-__host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0) {
-    const size_t b = 1024 + static_cast<size_t>(stages) * mxg_stage_bytes(mode, BN, af) +
+__host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0, int cps = 1) {
+    const size_t b = 1024 + static_cast<size_t>(stages) * cps * mxg_stage_bytes(mode, BN, af) +
                      (2 * stages + 2 * MXG_MAX_ACC + 1) * 8 + 64 + mxg_extra_smem(mode);
     return b < static_cast<size_t>(MXG_MIN_SMEM) ? static_cast<size_t>(MXG_MIN_SMEM) : b;
 }
@@ -161,7 +161,10 @@ __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0) 
 // weights (padded form) arrive through tmap_w, a 16U4_ALIGN16B tensor map
 // over the weight array's 8704-byte parts, one 128 x 128 box per matrix and
 // stage, and their scale atoms through bulk copies.
-template <int MODE, int AF = 0>
+// CP2 (MODE 1, AF 0, stacked tiles with 3 * BN <= 128): two K chunks per stage.
+// It is its own instantiation: the larger loop bodies measurably slowed the
+// other down-GEMM configurations when they shared one kernel.
+template <int MODE, int AF = 0, int CP2 = 0>
 __global__ void __launch_bounds__(MXG_THREADS, 1)
 expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_w,
                    const MxgParams p) {
@@ -174,7 +177,9 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
     const int S = p.stages, BN = p.BN, NB3 = TERMS * p.BN;
     const uint32_t b_bytes = mxg_b_bytes(BN, AF);
     const uint32_t sf_bytes = mxg_sfb_stage(BN, AF);               // atoms used per stage
-    const uint32_t stage_bytes = mxg_stage_bytes(MODE, BN, AF);
+    // a stage holds one K chunk of 128, or two (MODE 1 with cps2): [weights][B codes][B atoms],
+    // each region holding the chunks in order
+    const uint32_t stage_bytes = mxg_stage_bytes(MODE, BN, AF) * (CP2 ? 2u : 1u);
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t bar0 = base + S * stage_bytes;                 // barriers (8-byte aligned)
@@ -267,6 +272,21 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                     bulk_g2s_warp(st + W_STAGE + b_bytes, p.sfb + (static_cast<size_t>(tile) * KC + c) * MXG_SFB_BYTES,
                                   sf_bytes, full_bar(s));
                     pend_ph[s] = static_cast<int>(ph);
+                } else if (CP2) {
+                    // chunks c and c + 1 of the feature tile are adjacent (chunk c is full)
+                    const int nch = min(2, c1 - c);
+                    const uint32_t st = w_sm(s);
+                    uint32_t wb = 0;
+                    for (int j = 0; j < nch; ++j) wb += static_cast<uint32_t>(p.M.chunk_bytes(c + j, rf));
+                    mbar_arrive_expect_tx_warp(full_bar(s), wb + nch * (b_bytes + sf_bytes));
+                    bulk_g2s_warp(st, we + p.M.chunk_offset(ft, c, rf), wb, full_bar(s));
+                    for (int j = 0; j < nch; ++j) {
+                        tma_load_3d_warp(st + 2 * W_STAGE + j * b_bytes, &tmap_b, 2 * U.y, 0, 4 * (c + j), full_bar(s));
+                        bulk_g2s_warp(st + 2 * W_STAGE + 2 * b_bytes + j * sf_bytes,
+                                      p.sfb + (static_cast<size_t>(tile) * KC + c + j) * MXG_SFB_BYTES, sf_bytes,
+                                      full_bar(s));
+                    }
+                    pend_ph[s] = static_cast<int>(ph);
                 } else {
                     const uint32_t wb = static_cast<uint32_t>(p.M.chunk_bytes(c, rf));
                     const uint32_t st = w_sm(s);
@@ -279,6 +299,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                     pend_ph[s] = static_cast<int>(ph);
                 }
                 if (++s == S) { s = 0; ph ^= 1u; }
+                if (CP2) ++c;   // the stage took chunk c + 1 as well
             }
         }
         // copies still in flight must land before the CTA exits
@@ -355,6 +376,36 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                     tc_commit_warp(empty_bar(s));
                     if (++s == S) { s = 0; ph ^= 1u; }
                     if (++sfs == MXG_SF_SLOTS) sfs = 0;
+                    continue;
+                }
+                if constexpr (CP2 != 0) {
+                    // two K chunks per stage; tensor-memory columns: A atom of chunk j
+                    // at 4 j, B atom of chunk j at 8 + 4 j (3 * BN <= 128: one atom each)
+                    const int nch = min(2, c1 - c);
+                    const uint32_t ws = w_sm(s), bs = ws + 2 * W_STAGE, ss = bs + 2 * b_bytes;
+                    const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
+                    uint32_t wj = ws;
+                    for (int j = 0; j < nch; ++j) {
+                        const int nbj = p.M.blocks_in_chunk(c + j);
+                        const uint32_t cb = static_cast<uint32_t>(nbj * rf * 16);
+                        tc_cp_sf_warp(sfc + 4 * j, desc_noswz(wj + cb, 0, 128));
+                        tc_cp_sf_warp(sfc + 8 + 4 * j, desc_noswz(ss + j * sf_bytes, 0, 128));
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            if (2 * i < nbj) {
+                                const uint32_t acc = (c > c0 || j > 0 || i > 0) ? 1u : 0u;
+                                const uint32_t id = p.idesc | idesc_sf_ids(2u * i);
+                                const uint64_t ad = desc_noswz(wj + 2 * i * rf * 16, rf * 16, 128);
+                                const uint64_t bd = desc_noswz(bs + j * b_bytes + 2 * i * NB3 * 16, NB3 * 16, 128);
+                                mma_mxf4_warp(d0, ad, bd, id, sfc + 4 * j, sfc + 8 + 4 * j, acc);
+                            }
+                        }
+                        wj += cb + 512u;
+                    }
+                    tc_commit_warp(empty_bar(s));
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    if (++sfs == MXG_SF_SLOTS) sfs = 0;
+                    ++c;   // the stage held chunk c + 1 as well
                     continue;
                 }
                 const uint32_t codes_b = static_cast<uint32_t>(nbc * rf * 16);

@@ -319,6 +319,9 @@ static cudaError_t ensure_kernel_attrs(int dev) {
         return e;
     if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
         return e;
+    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  227 * 1024)))
+        return e;
     if ((e = set_router_smem<float>(rsm))) return e;
     {
         const int tsm = static_cast<int>(rtc_smem_bytes(3));
@@ -335,9 +338,9 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     return cudaSuccess;
 }
 
-static int stages_for(int mode, int BN, int af) {
+static int stages_for(int mode, int BN, int af, int cps = 1) {
     const size_t budget = 227 * 1024 - 1024 - 512 - mxg_extra_smem(mode);
-    int s = static_cast<int>(budget / mxg_stage_bytes(mode, BN, af));
+    int s = static_cast<int>(budget / (static_cast<size_t>(cps) * mxg_stage_bytes(mode, BN, af)));
     return std::max(2, std::min(MXG_MAX_STAGES, s));
 }
 
@@ -989,7 +992,10 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.M = tiled(h, 2);
     dp.N = d;
     dp.K = f;
-    dp.stages = stages_for(1, BN, af);
+    // small stacked tiles: two K chunks (17,408 weight bytes) per down stage, as
+    // many bytes per stage round trip as a gate/up stage
+    const bool cp2 = af == 0 && stacked && MXQ_TERMS * BN <= 128;
+    dp.stages = stages_for(1, BN, af, cp2 ? 2 : 1);
     dp.nacc = mxg_nacc(1, BN, af);
     dp.sfb = h->sfh;
     dp.GU = nullptr;
@@ -997,8 +1003,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.obuf = h->obuf;
     dp.obuf_bf16 = bf16 ? 1 : 0;
     dp.skip_first_copy = 0;
-    launch_pdl(pdl, af ? expert_mxf4_kernel<1, 1> : expert_mxf4_kernel<1, 0>, dim3(grid), dim3(MXG_THREADS),
-               mxg_smem_bytes(1, BN, dp.stages, af), stream, h->tm_h[BN / 16 - 1], h->tm_wdn, dp);
+    launch_pdl(pdl, af ? expert_mxf4_kernel<1, 1> : (cp2 ? expert_mxf4_kernel<1, 0, 1> : expert_mxf4_kernel<1, 0>),
+               dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages, af, cp2 ? 2 : 1), stream,
+               h->tm_h[BN / 16 - 1], h->tm_wdn, dp);
     h->stage_ran[4] = true;
     // 5: the output: the sum of each token's k rows (+ x), or the cast accumulator
     mark(5);
