@@ -161,10 +161,12 @@ __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0, 
 // weights (padded form) arrive through tmap_w, a 16U4_ALIGN16B tensor map
 // over the weight array's 8704-byte parts, one 128 x 128 box per matrix and
 // stage, and their scale atoms through bulk copies.
+// STK: the terms stacked into one MMA (1) or one MMA per term (0).
 // CP2 (MODE 1, AF 0, stacked tiles with 3 * BN <= 128): two K chunks per stage.
-// It is its own instantiation: the larger loop bodies measurably slowed the
-// other down-GEMM configurations when they shared one kernel.
-template <int MODE, int AF = 0, int CP2 = 0>
+// Each is its own instantiation: larger loop bodies measurably slowed the
+// down GEMM when configurations shared one kernel (the loops of the warp
+// roles compete for the instruction cache).
+template <int MODE, int AF, int STK, int CP2 = 0>
 __global__ void __launch_bounds__(MXG_THREADS, 1)
 expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_w,
                    const MxgParams p) {
@@ -339,7 +341,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                     const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
                     tc_cp_sf_warp(sfc, desc_noswz(wsf, 0, 128));
                     if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(wsf + 512, 0, 128));
-                    if (p.stacked) {
+                    if constexpr (STK != 0) {
                         tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
                         if (NB3 > 128) tc_cp_sf_warp(sfc + 12, desc_noswz(ss + 512, 0, 128));
 #pragma unroll
@@ -414,7 +416,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                 const uint32_t sfc = tmem + MXG_SF_COL0 + MXG_SF_SLOT_COLS * sfs;
                 tc_cp_sf_warp(sfc, desc_noswz(ws + codes_b, 0, 128));
                 if (MODE == 0) tc_cp_sf_warp(sfc + 4, desc_noswz(ws + mat_b + codes_b, 0, 128));
-                if (p.stacked) {
+                if constexpr (STK != 0) {
                     // one MMA per K step and matrix: N = 3 * BN rows (term-major); the B
                     // scales of rows 0..127 in columns 8..11, of rows 128.. in 12..15
                     tc_cp_sf_warp(sfc + 8, desc_noswz(ss, 0, 128));
@@ -488,7 +490,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
                 const uint32_t d0 = tmem + lane_addr + static_cast<uint32_t>(buf * acc_cols);
                 // accumulators of token columns r0 .. r0 + 7 for this lane's feature
                 auto load8 = [&](int r0, float (&gs)[8], float (&us)[8]) {
-                    if (p.stacked) {
+                    if constexpr (STK != 0) {
                         // the term columns of each token are BN apart: add them
                         uint32_t g[TERMS][8], v[TERMS][8];
 #pragma unroll

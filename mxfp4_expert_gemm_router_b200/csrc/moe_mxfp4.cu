@@ -311,17 +311,14 @@ static cudaError_t ensure_kernel_attrs(int dev) {
     if (g_attrs_set[dev]) return cudaSuccess;
     const int rsm = static_cast<int>(router_smem_bytes());
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
-        return e;
-    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
-        return e;
-    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
-        return e;
-    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
-        return e;
-    if ((e = cudaFuncSetAttribute(expert_mxf4_kernel<1, 0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  227 * 1024)))
-        return e;
+    const void* gemms[] = {
+        reinterpret_cast<const void*>(expert_mxf4_kernel<0, 0, 0>), reinterpret_cast<const void*>(expert_mxf4_kernel<0, 0, 1>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 0>), reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 1>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 1, 1>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<0, 1, 0>), reinterpret_cast<const void*>(expert_mxf4_kernel<0, 1, 1>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 1, 0>), reinterpret_cast<const void*>(expert_mxf4_kernel<1, 1, 1>)};
+    for (const void* k : gemms)
+        if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024))) return e;
     if ((e = set_router_smem<float>(rsm))) return e;
     {
         const int tsm = static_cast<int>(rtc_smem_bytes(3));
@@ -964,7 +961,9 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.T = T;
     gp.tiles_cap = tiles_cap;
     const int grid = h->nsm;
-    launch_pdl(pdl, af ? expert_mxf4_kernel<0, 1> : expert_mxf4_kernel<0, 0>, dim3(grid), dim3(MXG_THREADS),
+    auto gu_kernel = af ? (stacked ? expert_mxf4_kernel<0, 1, 1> : expert_mxf4_kernel<0, 1, 0>)
+                        : (stacked ? expert_mxf4_kernel<0, 0, 1> : expert_mxf4_kernel<0, 0, 0>);
+    launch_pdl(pdl, gu_kernel, dim3(grid), dim3(MXG_THREADS),
                mxg_smem_bytes(0, BN, gp.stages, af), stream, h->tm_x[BN / 16 - 1], h->tm_wgu, gp);
     h->stage_ran[2] = true;
     // 3: split-K finish (a no-op unless the schedule split K): SwiGLU + H encoding.
@@ -1003,7 +1002,10 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.obuf = h->obuf;
     dp.obuf_bf16 = bf16 ? 1 : 0;
     dp.skip_first_copy = 0;
-    launch_pdl(pdl, af ? expert_mxf4_kernel<1, 1> : (cp2 ? expert_mxf4_kernel<1, 0, 1> : expert_mxf4_kernel<1, 0>),
+    auto dn_kernel = af ? (stacked ? expert_mxf4_kernel<1, 1, 1> : expert_mxf4_kernel<1, 1, 0>)
+                        : (cp2 ? expert_mxf4_kernel<1, 0, 1, 1>
+                               : (stacked ? expert_mxf4_kernel<1, 0, 1> : expert_mxf4_kernel<1, 0, 0>));
+    launch_pdl(pdl, dn_kernel,
                dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages, af, cp2 ? 2 : 1), stream,
                h->tm_h[BN / 16 - 1], h->tm_wdn, dp);
     h->stage_ran[4] = true;
