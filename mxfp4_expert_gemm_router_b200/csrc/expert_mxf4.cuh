@@ -163,10 +163,12 @@ __host__ inline size_t mxg_smem_bytes(int mode, int BN, int stages, int af = 0, 
 // stage, and their scale atoms through bulk copies.
 // STK: the terms stacked into one MMA (1) or one MMA per term (0).
 // CP2 (MODE 1, AF 0, stacked tiles with 3 * BN <= 128): two K chunks per stage.
+// SPL = 0: the schedule cannot split K for this launch (the host proves it from
+// T), so the split-K epilogue paths are left out.
 // Each is its own instantiation: larger loop bodies measurably slowed the
 // down GEMM when configurations shared one kernel (the loops of the warp
 // roles compete for the instruction cache).
-template <int MODE, int AF, int STK, int CP2 = 0>
+template <int MODE, int AF, int STK, int CP2 = 0, int SPL = 1>
 __global__ void __launch_bounds__(MXG_THREADS, 1)
 expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_w,
                    const MxgParams p) {
@@ -230,7 +232,7 @@ expert_mxf4_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_cons
     pdl_wait();
 
     const int num_units = p.sched[MODE == 0 ? SCHED_UNITS_GU : SCHED_UNITS_DN];
-    const int nsplit = p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN];
+    const int nsplit = SPL ? p.sched[MODE == 0 ? SCHED_SPLIT_GU : SCHED_SPLIT_DN] : 1;
     const int KC = p.M.chunks();
     const size_t expert_bytes = p.M.expert_bytes();
 
