@@ -320,7 +320,12 @@ static cudaError_t ensure_kernel_attrs(int dev) {
         reinterpret_cast<const void*>(expert_mxf4_kernel<0, 0, 0, 0, 0>),
         reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 0, 0, 0>),
         reinterpret_cast<const void*>(expert_mxf4_kernel<0, 1, 0, 0, 0>),
-        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 1, 0, 0, 0>)};
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 1, 0, 0, 0>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<0, 0, 1, 0, 0>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 1, 0, 0>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 0, 1, 1, 0>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<0, 1, 1, 0, 0>),
+        reinterpret_cast<const void*>(expert_mxf4_kernel<1, 1, 1, 0, 0>)};
     for (const void* k : gemms)
         if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024))) return e;
     if ((e = set_router_smem<float>(rsm))) return e;
@@ -965,17 +970,18 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     gp.T = T;
     gp.tiles_cap = tiles_cap;
     const int grid = h->nsm;
-    // The schedule splits the gate/up K only for at most gu_rows grouped rows,
-    // and the down K only while ceil(rows / BN) token tiles x its feature tiles
-    // leave SMs idle: beyond either bound the kernel without the split-K
-    // epilogue runs (per-term tiles, the large-batch case).
+    // The schedule splits a GEMM's K only while its units (at least ceil(rows /
+    // BN) token tiles x its feature tiles) leave SMs idle, and the gate/up K
+    // only for at most gu_rows grouped rows: past those bounds the kernel
+    // without the split-K epilogue runs.
     const long rows_all = static_cast<long>(T) * k;
-    const bool gu_nosplit = rows_all > h->gu_rows;
+    const bool gu_nosplit = rows_all > h->gu_rows || ((rows_all + BN - 1) / BN) * h->F_gu >= h->nsm;
     const bool dn_nosplit = ((rows_all + BN - 1) / BN) * h->F_dn >= h->nsm;
-    auto gu_kernel = af ? (stacked ? expert_mxf4_kernel<0, 1, 1>
-                                   : (gu_nosplit ? expert_mxf4_kernel<0, 1, 0, 0, 0> : expert_mxf4_kernel<0, 1, 0>))
-                        : (stacked ? expert_mxf4_kernel<0, 0, 1>
-                                   : (gu_nosplit ? expert_mxf4_kernel<0, 0, 0, 0, 0> : expert_mxf4_kernel<0, 0, 0>));
+    auto gu_kernel =
+        af ? (stacked ? (gu_nosplit ? expert_mxf4_kernel<0, 1, 1, 0, 0> : expert_mxf4_kernel<0, 1, 1>)
+                      : (gu_nosplit ? expert_mxf4_kernel<0, 1, 0, 0, 0> : expert_mxf4_kernel<0, 1, 0>))
+           : (stacked ? (gu_nosplit ? expert_mxf4_kernel<0, 0, 1, 0, 0> : expert_mxf4_kernel<0, 0, 1>)
+                      : (gu_nosplit ? expert_mxf4_kernel<0, 0, 0, 0, 0> : expert_mxf4_kernel<0, 0, 0>));
     launch_pdl(pdl, gu_kernel, dim3(grid), dim3(MXG_THREADS),
                mxg_smem_bytes(0, BN, gp.stages, af), stream, h->tm_x[BN / 16 - 1], h->tm_wgu, gp);
     h->stage_ran[2] = true;
@@ -1015,11 +1021,12 @@ moe_status_t moe_mxfp4_forward(moe_mxfp4_t* h, const void* x, int32_t T, void* y
     dp.obuf = h->obuf;
     dp.obuf_bf16 = bf16 ? 1 : 0;
     dp.skip_first_copy = 0;
-    auto dn_kernel = af ? (stacked ? expert_mxf4_kernel<1, 1, 1>
-                                   : (dn_nosplit ? expert_mxf4_kernel<1, 1, 0, 0, 0> : expert_mxf4_kernel<1, 1, 0>))
-                        : (cp2 ? expert_mxf4_kernel<1, 0, 1, 1>
-                               : (stacked ? expert_mxf4_kernel<1, 0, 1>
-                                          : (dn_nosplit ? expert_mxf4_kernel<1, 0, 0, 0, 0> : expert_mxf4_kernel<1, 0, 0>)));
+    auto dn_kernel =
+        af ? (stacked ? (dn_nosplit ? expert_mxf4_kernel<1, 1, 1, 0, 0> : expert_mxf4_kernel<1, 1, 1>)
+                      : (dn_nosplit ? expert_mxf4_kernel<1, 1, 0, 0, 0> : expert_mxf4_kernel<1, 1, 0>))
+           : (cp2 ? (dn_nosplit ? expert_mxf4_kernel<1, 0, 1, 1, 0> : expert_mxf4_kernel<1, 0, 1, 1>)
+                  : (stacked ? (dn_nosplit ? expert_mxf4_kernel<1, 0, 1, 0, 0> : expert_mxf4_kernel<1, 0, 1>)
+                             : (dn_nosplit ? expert_mxf4_kernel<1, 0, 0, 0, 0> : expert_mxf4_kernel<1, 0, 0>)));
     launch_pdl(pdl, dn_kernel,
                dim3(grid), dim3(MXG_THREADS), mxg_smem_bytes(1, BN, dp.stages, af, cp2 ? 2 : 1), stream,
                h->tm_h[BN / 16 - 1], h->tm_wdn, dp);
