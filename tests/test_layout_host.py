@@ -3,7 +3,9 @@
 tests/layout_check.cu includes the library's layout headers and checks, with
 no kernel and no GPU, that the tiled weight layout (codes and scale atoms per
 feature tile and K chunk) is a bijection with no gaps or overlaps, on the
-2880-wide shapes and on ragged ones, and that the scale-atom byte formula is a
+2880-wide shapes and on ragged ones; that the padded form (two-MXFP8-term
+layers) puts every code and scale byte where the weight tensor map's box of
+the producer's part index finds it; and that the scale-atom byte formula is a
 bijection onto the atoms."""
 import os
 import subprocess
