@@ -73,6 +73,26 @@ def test_roofline_bound_follows_machine_balance():
     assert r4["peak"] == 6400.0
 
 
+def test_roofline_of_the_two_mxfp8_term_variant():
+    """kind::mxf8f6f4 runs at the FP8 rate (2x bf16) and executes one MMA per
+    activation term (two), and its operands carry 2 x 33/32 bytes per element
+    against 3 x 17/32 for three MXFP4 terms."""
+    import bench
+    import moe_inputs as mi
+
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    cfg = mi.CONFIGS["pre4096"]
+    w4 = bench.algorithmic_work(cfg, cfg.T, cfg.n_experts, "mxf4x3")["gate_up_swiglu"]
+    w8 = bench.algorithmic_work(cfg, cfg.T, cfg.n_experts, "mxf8x2")["gate_up_swiglu"]
+    assert w8["flops"] == w4["flops"] and w8["bytes"] > w4["bytes"]
+    rows = cfg.T * cfg.top_k
+    extra = rows * (cfg.d_model + cfg.d_ff) * (2 * 33 / 32 - 3 * 17 / 32)
+    assert abs((w8["bytes"] - w4["bytes"]) - extra) < 1e-6 * extra
+    r = bench.roofline(w8, 1e-3, peaks, "gate_up_swiglu", "f8f6f4")
+    assert r["bound"] == "tensor" and r["peak"] == 3200.0
+    assert abs(r["executed_frac"] - 2 * w8["flops"] / 1e-3 / 1e12 / 3200.0) < 1e-12
+
+
 def test_reference_arm_prints_one_json_line():
     """`bench.py --impl reference` (the oracle on the host cores) keeps the bench
     line's contract: one JSON line with the metric, its value and unit, the
